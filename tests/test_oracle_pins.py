@@ -1,0 +1,371 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+Published known-answer values (tests/golden/), closed forms, library routines
+(torch.nn.functional.embedding_bag / embedding, torch's fp32 -> bf16 conversion),
+brute force on tiny inputs and invariants of the method.  The method is the one in
+"Qwen Brought Back N-Grams. All 51 Billion Parameters of Them." (section "N-grams, of
+all things": hash bigram + trigram context, gather 16 rows, sum, add to the residual)
+with the gate of "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with Heterogeneous
+Memory Prefetch", Key point 1 (h = h + W_g elementwise e_Ngram).
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ngram_inputs as gen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+GAMMA = 0x9E3779B97F4A7C15
+M64 = (1 << 64) - 1
+PAD = oracle.DEFAULT_PAD_ID
+K_BF16 = float.fromhex("0x1.1bc77ap-22")
+K_INT8 = float.fromhex("0x1.1bc5f4p-11")
+
+
+def _kat(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([int(x, 16) for x in line.split()])
+    return rows
+
+
+def _bits_to_f64(bits):
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def _bf16_ulp(v):
+    """Spacing of bf16 values at |v| (8 significant bits; 2^-133 below the normals)."""
+    v = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.where(v > 0, v, 1.0)))
+    return np.where(v > 0, np.exp2(np.maximum(e - 7, -133)), 2.0 ** -133)
+
+
+# --------------------------------------------------------------------------- generators
+def test_splitmix64_known_answers():
+    for seed, *outs in _kat("splitmix64_kat.txt"):
+        assert oracle.splitmix64_outputs(seed, len(outs)) == outs
+
+
+def test_head_seeds_are_successive_splitmix64_outputs():
+    (seed, *outs), = _kat("splitmix64_kat.txt")
+    assert [int(x) for x in oracle.head_seeds(seed, 3)] == outs
+
+
+def test_philox4x32_10_known_answers():
+    for row in _kat("philox4x32_10_kat.txt"):
+        ctr, key, want = row[0:4], row[4:6], row[6:10]
+        assert [int(x) for x in oracle.philox4x32_10(ctr, key)] == want
+
+
+# --------------------------------------------------------------------------- the hash
+def _unxorshift(y, s):
+    x = y
+    for _ in range(64 // s + 1):
+        x = y ^ (x >> s)
+    return x & M64
+
+
+def _splitmix_state_for_output(z):
+    """Invert the splitmix64 output function (xorshifts and odd multipliers are
+    bijections mod 2^64): returns the state whose next() output is z."""
+    z = _unxorshift(z, 31)
+    z = (z * pow(0x94D049BB133111EB, -1, 1 << 64)) & M64
+    z = _unxorshift(z, 27)
+    z = (z * pow(0xBF58476D1CE4E5B9, -1, 1 << 64)) & M64
+    return _unxorshift(z, 30)
+
+
+@pytest.mark.parametrize("head,R", [(0, 20_000_000), (5, 65_536), (8, 1_000_003),
+                                    (15, 4_294_967_291)])
+def test_hash_path_reaches_known_answer(head, R):
+    """Choose base_seed so that seed_head equals the packed key of one context; then
+    key ^ seed = 0 and the row must be splitmix64's first output from 0, mod R."""
+    (_, first_out, *_), = _kat("splitmix64_kat.txt")
+    w2, w1, w0 = 1_500_001, 678_901, 12_345
+    key = ((w1 << 21) | w0) if head < 8 else ((w2 << 42) | (w1 << 21) | w0)
+    state = _splitmix_state_for_output(key)
+    base = (state - (head + 1) * GAMMA) & M64
+    assert int(oracle.head_seeds(base, 16)[head]) == key
+    idx = oracle.indices([[w2, w1, w0]], None, R, base_seed=base, vocab_size=PAD)
+    assert int(idx[2, head]) == first_out % R
+
+
+def test_bigram_heads_ignore_w2_and_trigram_heads_do_not():
+    toks = np.array([[7, 100, 200], [9, 100, 200]], dtype=np.int32)
+    idx = oracle.indices(toks, None, 1 << 30, vocab_size=1000)
+    a, b = idx[2], idx[5]
+    assert np.array_equal(a[:8], b[:8])
+    assert np.all(a[8:] != b[8:])
+    assert len(set(a.tolist())) == 16          # 16 distinct heads on this context
+
+
+def test_power_of_two_R_is_a_mask():
+    toks = gen.zipf_tokens(2, 300, 32_000, seed=11)
+    big = oracle.indices(toks, None, 1 << 31, vocab_size=32_000)
+    for k in (1, 10, 16, 20):
+        small = oracle.indices(toks, None, 1 << k, vocab_size=32_000)
+        assert np.array_equal(small, big & ((1 << k) - 1))
+
+
+def test_repeated_context_gives_identical_rows():
+    toks = np.array([[3, 4, 5, 6, 3, 4, 5, 9, 4, 5]], dtype=np.int32)
+    idx = oracle.indices(toks, None, 65_536, vocab_size=100)
+    assert np.array_equal(idx[2], idx[6])      # (3,4,5) at t=2 and t=6
+    assert np.array_equal(idx[6, :8], idx[9, :8])   # bigram (4,5) again at t=9
+    assert not np.array_equal(idx[6, 8:], idx[9, 8:])
+
+
+# --------------------------------------------------------------------------- boundaries
+def test_pad_history_equivalences():
+    V = 32_000
+    toks = gen.zipf_tokens(1, 64, V, seed=5)
+    full = oracle.indices(toks, None, 65_536, vocab_size=V)
+    # no history == explicit PAD history
+    assert np.array_equal(full, oracle.indices(toks, [[PAD, PAD]], 65_536, vocab_size=V))
+    # writing the pads as tokens reproduces the boundary positions
+    padded = np.concatenate([[[PAD, PAD]], toks], axis=1).astype(np.int32)
+    assert np.array_equal(oracle.indices(padded, None, 65_536, vocab_size=V)[2:], full)
+
+
+def test_chunked_prefill_and_decode_equal_full_prefill():
+    V = 151_936
+    toks = gen.zipf_tokens(1, 40, V, seed=6)
+    full = oracle.indices(toks, None, 20_000_000, vocab_size=V)
+    c1, c2 = toks[:, :17], toks[:, 17:]
+    i1 = oracle.indices(c1, None, 20_000_000, vocab_size=V)
+    i2 = oracle.indices(c2, c1[:, -2:], 20_000_000, vocab_size=V)
+    assert np.array_equal(np.concatenate([i1, i2]), full)
+    ext = np.concatenate([[PAD, PAD], toks[0]])
+    for t in range(toks.shape[1]):
+        step = oracle.indices([[toks[0, t]]], [[ext[t], ext[t + 1]]], 20_000_000, vocab_size=V)
+        assert np.array_equal(step[0], full[t])
+
+
+def test_contexts_do_not_cross_sequences():
+    V = 32_000
+    toks = gen.zipf_tokens(3, 20, V, seed=7)
+    allidx = oracle.indices(toks, None, 65_536, vocab_size=V)
+    for s in range(3):
+        alone = oracle.indices(toks[s:s + 1], None, 65_536, vocab_size=V)
+        assert np.array_equal(allidx[s * 20:(s + 1) * 20], alone)
+
+
+def test_out_of_vocab_tokens_read_as_pad():
+    V = 1000
+    a = oracle.indices([[5, 6, 7]], None, 65_536, vocab_size=V)
+    b = oracle.indices([[5, V + 3, 7]], None, 65_536, vocab_size=V)
+    c = oracle.indices([[5, PAD, 7]], None, 65_536, vocab_size=V)
+    assert np.array_equal(b, c) and not np.array_equal(a, b)
+
+
+def test_empty_batch():
+    assert oracle.indices(np.zeros((0, 5), np.int32), None, 100).shape == (0, 16)
+    out = oracle.forward(np.zeros((2, 0), np.int32), None, np.zeros((0, 8), np.uint16),
+                         np.ones(8, np.float32), R=100, d=8, table_seed=1)
+    assert out.shape == (0, 8)
+
+
+# --------------------------------------------------------------------------- bf16 rounding
+def test_bf16_from_f32_matches_torch_round_to_nearest_even():
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 2**32, size=200_000, dtype=np.uint64).astype(np.uint32)
+    ties = (rng.integers(0, 2**16, size=5000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    bits = np.concatenate([bits, ties, np.array([0, 0x80000000, 0x7F7FFFFF, 0x7F7F8000], np.uint32)])
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]             # finite only
+    f = bits.view(np.float32)
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.bf16_from_f32(x) for x in f[:20000]], dtype=np.uint16)
+    assert np.array_equal(got, want[:20000])
+    got_t = np.array([oracle.bf16_from_f32(x) for x in f[-5004:]], dtype=np.uint16)
+    assert np.array_equal(got_t, want[-5004:])
+
+
+def test_bf16_from_f64_is_nearest_even():
+    rng = np.random.default_rng(1)
+    ys = list(rng.standard_normal(3000) * np.exp2(rng.integers(-40, 40, 3000)))
+    # exact midpoints between neighbouring bf16 values, both parities
+    for m in range(128, 256, 7):
+        for e in (-30, -3, 0, 5):
+            ys.append((m + 0.5) * 2.0 ** (e - 7))
+            ys.append(-(m + 0.5) * 2.0 ** (e - 7))
+    for y in ys:
+        b = oracle.bf16_from_f64(y)
+        v = Fraction(float(_bits_to_f64([b])[0]))
+        nb = [Fraction(float(_bits_to_f64([(b + k) & 0xFFFF])[0])) for k in (-1, 1)]
+        fy = Fraction(y)
+        assert all(abs(fy - v) <= abs(fy - w) for w in nb), y
+        for w in nb:
+            if abs(fy - v) == abs(fy - w):
+                assert b % 2 == 0, y
+
+
+# --------------------------------------------------------------------------- table values
+def test_bf16_table_distribution_closed_form():
+    """C = 2S - 262140, S a sum of four iid U{0..65535}: mean 0, std
+    4 * sqrt((65536^2 - 1) / 12) = 75674.4, so std(C * K) = 0.02, |C| <= 262140."""
+    v = _bits_to_f64(oracle.fill_bf16(gen.TABLE_SEED, 1234, 300, 512)).ravel()
+    n = v.size
+    assert abs(v.mean()) < 4 * 0.02 / np.sqrt(n)
+    assert abs(v.std() / 0.02 - 1) < 0.01
+    assert np.abs(v).max() <= 262140 * K_BF16 * (1 + 2 ** -8)
+    # Irwin-Hall(4) kurtosis = 3 - 6/(5*4) = 2.7
+    kurt = ((v - v.mean()) ** 4).mean() / v.var() ** 2
+    assert abs(kurt - 2.7) < 0.03
+    # columns and rows are independent streams
+    m = v.reshape(300, 512)
+    assert abs(np.corrcoef(m[:, 0::2].ravel(), m[:, 1::2].ravel())[0, 1]) < 0.01
+    assert abs(np.corrcoef(m[:-1].ravel(), m[1:].ravel())[0, 1]) < 0.01
+
+
+def test_int8_table_distribution_closed_form():
+    """q = floor((B - 510) / 4), B a sum of four iid bytes: std(B) = sqrt(4*(256^2-1)/12),
+    mean(q) = -3/8 (floor of quarter steps), range [-128, 127]; row scale in
+    [0.75, 1.25) * K8 with mean K8."""
+    q, s = oracle.fill_int8(gen.TABLE_SEED, 77, 400, 512)
+    qf = q.astype(np.float64).ravel()
+    assert q.min() >= -128 and q.max() <= 127
+    assert abs(qf.mean() + 0.375) < 4 * 37 / np.sqrt(qf.size)
+    var_b = 4 * (256 ** 2 - 1) / 12
+    # var(q) = var(B) / 16 + 5/64 (the dropped quarter steps, uniform on {0, 1/4, 1/2, 3/4})
+    assert abs(qf.std() / np.sqrt(var_b / 16 + 5 / 64) - 1) < 0.01
+    assert np.all(s >= 0.75 * K_INT8) and np.all(s < 1.25 * K_INT8)
+    assert abs(s.mean() / K_INT8 - 1) < 0.02
+
+
+def test_table_is_a_pure_function_of_seed_row_col():
+    a = oracle.fill_bf16(99, 10, 4, 64)
+    b = oracle.fill_bf16(99, 12, 2, 64)
+    assert np.array_equal(a[2:], b)
+    assert oracle.table_bf16(99, 11, 5) == a[1, 5]
+    assert not np.array_equal(a, oracle.fill_bf16(100, 10, 4, 64))
+
+
+# --------------------------------------------------------------------------- the sum
+def _tiny_case(seed=0, n_seq=3, T=17, V=50, R=97, d=24, nb=8, nt=8):
+    rng = np.random.default_rng(seed)
+    toks = rng.integers(0, V, (n_seq, T)).astype(np.int32)
+    res = gen.residual_bf16_bits(n_seq * T, d, seed + 1)
+    g = gen.gate_f32(d, seed + 2)
+    return toks, res, g
+
+
+def _one_hot_sum(idx, E):
+    N, H = idx.shape
+    A = np.zeros((N, E.shape[0]))
+    for t in range(N):
+        for h in range(H):
+            A[t, idx[t, h]] += 1.0          # colliding heads count twice
+    return A @ E
+
+
+@pytest.mark.parametrize("dtype", [oracle.BF16, oracle.INT8])
+def test_brute_force_one_hot_matmul_and_embedding_bag(dtype):
+    R, d, V = 97, 24, 50
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    if dtype == oracle.BF16:
+        E = _bits_to_f64(oracle.fill_bf16(42, 0, R, d)).reshape(R, d)
+    else:
+        q, s = oracle.fill_int8(42, 0, R, d)
+        E = q.astype(np.float64) * s.astype(np.float64)[:, None]
+    out, y, mag, idx = oracle.forward(toks, None, res, g, R=R, d=d, dtype=dtype, table_seed=42,
+                                      acc=oracle.ACC_F64, vocab_size=V, want_aux=True)
+    assert np.array_equal(idx, oracle.indices(toks, None, R, vocab_size=V))
+    e = _one_hot_sum(idx, E)
+    bag = torch.nn.functional.embedding_bag(torch.from_numpy(idx.astype(np.int64)),
+                                            torch.from_numpy(E), mode="sum").numpy()
+    assert np.array_equal(e, bag)
+    r = _bits_to_f64(res).reshape(-1, d)
+    assert np.array_equal(y, r + g.astype(np.float64)[None, :] * e)
+    v = _bits_to_f64(out).reshape(y.shape)
+    assert np.all(np.abs(v - y) <= _bf16_ulp(y) / 2)     # rounded to a nearest bf16
+    assert np.allclose(mag, np.abs(r) + g[None, :] * (np.abs(E)[idx].sum(axis=1)))
+
+
+def test_collisions_count_once_per_head():
+    """R = 2 forces heads to collide: the sum must count every head's row."""
+    toks, res, g = _tiny_case(R=2, d=8, T=5, n_seq=1)
+    E = _bits_to_f64(oracle.fill_bf16(3, 0, 2, 8)).reshape(2, 8)
+    out, y, _, idx = oracle.forward(toks, None, np.zeros_like(res), np.ones(8, np.float32),
+                                    R=2, d=8, table_seed=3, acc=oracle.ACC_F64,
+                                    vocab_size=50, want_aux=True)
+    counts = np.stack([(idx == 0).sum(1), (idx == 1).sum(1)], 1).astype(np.float64)
+    assert np.array_equal(y, counts @ E)
+
+
+def test_single_head_reduces_to_embedding():
+    R, d, V = 1000, 32, 500
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    Eb = oracle.fill_bf16(8, 0, R, d)
+    for nb, nt in ((1, 0), (0, 1)):
+        out, _, _, idx = oracle.forward(toks, None, np.zeros_like(res), np.ones(d, np.float32),
+                                        R=R, d=d, table_seed=8, n_bigram=nb, n_trigram=nt,
+                                        vocab_size=V, want_aux=True)
+        emb = torch.nn.functional.embedding(torch.from_numpy(idx[:, 0].astype(np.int64)),
+                                            torch.from_numpy(Eb.astype(np.int32))).numpy()
+        assert np.array_equal(out, emb.astype(np.uint16))
+
+
+@pytest.mark.parametrize("acc", [oracle.ACC_F32, oracle.ACC_F64])
+def test_zero_gate_returns_residual_bitwise(acc):
+    toks, res, g = _tiny_case()
+    out = oracle.forward(toks, None, res, np.zeros_like(g), R=97, d=24, table_seed=1,
+                         acc=acc, vocab_size=50)
+    assert np.array_equal(out, res.reshape(out.shape))
+
+
+def test_unit_gate_zero_residual_is_fp32_head_order_sum():
+    """r = 0, g = 1: the fp32 reference is bf16(fp32 sum in head order), computed here
+    with torch fp32 adds and torch's bf16 conversion."""
+    R, d, V = 300, 40, 60
+    toks, res, _ = _tiny_case(R=R, d=d, V=V)
+    E32 = torch.from_numpy(_bits_to_f64(oracle.fill_bf16(5, 0, R, d)).reshape(R, d).astype(np.float32))
+    out, _, _, idx = oracle.forward(toks, None, np.zeros_like(res), np.ones(d, np.float32), R=R,
+                                    d=d, table_seed=5, acc=oracle.ACC_F32, vocab_size=V,
+                                    want_aux=True)
+    rows = E32[torch.from_numpy(idx.astype(np.int64))]          # [N][H][d]
+    acc = torch.zeros(rows.shape[0], d, dtype=torch.float32)
+    for h in range(rows.shape[1]):
+        acc = acc + rows[:, h]
+    want = acc.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(out, want)
+
+
+def test_head_order_invariance_fp64_exact_fp32_within_rounding():
+    R, d, V = 500, 32, 80
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    E = _bits_to_f64(oracle.fill_bf16(9, 0, R, d)).reshape(R, d)
+    _, y64, mag, idx = oracle.forward(toks, None, np.zeros_like(res), np.ones(d, np.float32),
+                                      R=R, d=d, table_seed=9, acc=oracle.ACC_F64, vocab_size=V,
+                                      want_aux=True)
+    _, y32, _, _ = oracle.forward(toks, None, np.zeros_like(res), np.ones(d, np.float32), R=R,
+                                  d=d, table_seed=9, acc=oracle.ACC_F32, vocab_size=V,
+                                  want_aux=True)
+    rev = E[idx[:, ::-1]].sum(axis=1)        # reverse head order, fp64 (exact)
+    assert np.array_equal(y64, rev)
+    # fp32 head-order sum: at most 15 roundings of partial sums bounded by sum |E|
+    assert np.all(np.abs(y32 - y64) <= 16 * 2.0 ** -24 * mag)
+
+
+def test_fp32_reference_within_tolerance_of_exact_definition():
+    """The two accumulation modes agree to 1 bf16 ulp except where cancellation brings
+    y close to zero (absolute slack 2^-20 * (|r| + |g| sum |E|))."""
+    w = gen.WORKLOADS["tiny"]
+    inp = gen.make_inputs(w)
+    o32 = oracle.forward(inp["tokens"], None, inp["residual"], inp["gate"], R=w.R, d=w.d,
+                         table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32, vocab_size=w.vocab,
+                         n_threads=4)
+    o64, y64, mag, _ = oracle.forward(inp["tokens"], None, inp["residual"], inp["gate"], R=w.R,
+                                      d=w.d, table_seed=gen.TABLE_SEED, acc=oracle.ACC_F64,
+                                      vocab_size=w.vocab, n_threads=4, want_aux=True)
+    a, b = _bits_to_f64(o32).reshape(y64.shape), _bits_to_f64(o64).reshape(y64.shape)
+    tol = _bf16_ulp(b) + 2.0 ** -20 * mag
+    assert np.all(np.abs(a - b) <= tol)
+    assert np.mean(a == b) > 0.999
