@@ -1,0 +1,415 @@
+"""Benchmark of the hashed n-gram embedding lookup on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the fused kernel forms the
+bigram/trigram contexts, hashes 16 rows per token, gathers and sums them, applies the
+gate and adds the residual ("Qwen Brought Back N-Grams. All 51 Billion Parameters of
+Them.", section "N-grams, of all things"; gate of "Qwen3.8-Flash-Next: A 51B N-gram
+Embedding Table with Heterogeneous Memory Prefetch", Key point 1).
+
+Default workload: the full-size table of the pages (20,000,000 x 2560 bf16, 95.4 GiB in
+HBM) and one 32,768-token prefill of Zipf(1.1) tokens over a 151,936-id vocabulary.
+Prints one JSON line (rank 0).  Under torchrun every rank holds its own table replica
+and its own token batch (weak scaling, no collective on the data path); the time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import ngram_inputs as gen  # noqa: E402
+
+METRIC = "n-gram embed tokens/s and gather GB/s (% of HBM or PCIe H2D roofline), 1 B200"
+UNIT = "tokens/s"
+HEADS = 16
+KERNEL_SOURCES = ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
+                  "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"]
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# --------------------------------------------------------------------------- helpers
+def row_bytes(w) -> int:
+    return 2 * w.d if w.dtype == "bf16" else w.d + 4
+
+
+def algorithmic_bytes(w, n_seq=None, T=None) -> int:
+    """Bytes the method must move per call: 16 rows, the residual read and the output
+    write per token, the token id, the gate once and the history once per sequence."""
+    n_seq = w.n_seq if n_seq is None else n_seq
+    T = w.T if T is None else T
+    N = n_seq * T
+    hist = 8 * n_seq if w.history else 0
+    return N * (HEADS * row_bytes(w) + 2 * 2 * w.d + 4) + 4 * w.d + hist
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel source as it is now (else None)."""
+    p = os.path.join(ROOT, "profiles", "gather_%s.txt" % workload)
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith(" "):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_sha") != kernel_sha():
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while running."""
+
+    def __init__(self, gpu_id: str, period_ms: int = 50):
+        self.gpu_id, self.period_ms = gpu_id, period_ms
+        self.proc, self.path = None, None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + CLOCK_FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms), "-i", self.gpu_id],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) == 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(dev) -> str:
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    bus = getattr(p, "pci_bus_id", None)
+    dom = getattr(p, "pci_domain_id", 0)
+    devid = getattr(p, "pci_device_id", 0)
+    if bus is not None:
+        return "%08X:%02X:%02X.0" % (dom, bus, devid)
+    return str(dev.index or 0)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0):
+    """Time the oracle (test infrastructure; rows regenerated on the fly, the full table
+    cannot be materialised on the host) on a bounded sample of this workload's tokens."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    kw = dict(R=w.R, d=w.d, dtype=oracle.BF16 if w.dtype == "bf16" else oracle.INT8,
+              table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32, n_threads=threads,
+              vocab_size=w.vocab)
+    probe = rng.choice(w.N, size=min(w.N, 4 * threads), replace=False)
+    t0 = time.perf_counter()
+    oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=probe, **kw)
+    per_tok = (time.perf_counter() - t0) / probe.size
+    n = int(max(1, min(w.N, budget_s / max(per_tok, 1e-9))))
+    sel = np.sort(rng.choice(w.N, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sel, **kw)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, w):
+    """The oracle on the host cores, as the reference arm: each step is a bounded
+    sample of the workload's tokens (rank 0 only)."""
+    import oracle  # noqa: F401
+    threads = os.cpu_count() or 1
+    inp = gen.make_inputs(w)
+    total_budget = args.reference_seconds
+    steps, warm = args.steps, args.warmup
+    per_step_budget = total_budget / max(1, steps + warm)
+    _, n_probe, dt_probe = oracle_tokens_per_s(w, inp, min(2.0, per_step_budget), threads)
+    per_tok = dt_probe / n_probe
+    n_step = int(max(1, min(w.N, per_step_budget / per_tok)))
+    rng = np.random.default_rng(7)
+    import oracle as orc
+    kw = dict(R=w.R, d=w.d, dtype=orc.BF16 if w.dtype == "bf16" else orc.INT8,
+              table_seed=gen.TABLE_SEED, acc=orc.ACC_F32, n_threads=threads, vocab_size=w.vocab)
+    sels = [np.sort(rng.choice(w.N, size=n_step, replace=False)) for _ in range(steps + warm)]
+    for i in range(warm):
+        orc.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sels[i], **kw)
+    t0 = time.perf_counter()
+    for i in range(warm, warm + steps):
+        orc.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sels[i], **kw)
+    dt = time.perf_counter() - t0
+    value = n_step * steps / dt
+    sample = "%d of %d tokens per step (rows regenerated from the synthetic-table definition)" % (
+        n_step, w.N)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": 1e3 * dt / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_for(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_for(w, args) -> dict:
+    return {
+        "workload": w.name, "R": w.R, "d": w.d, "table_dtype": w.dtype,
+        "table_gib": round(w.R * row_bytes(w) / 2**30, 2), "n_seq": w.n_seq, "T": w.T,
+        "tokens_per_step_per_gpu": w.N, "heads": "8 bigram + 8 trigram",
+        "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
+        "accumulate": "fp32, head order", "residency": "hbm",
+        "l2": "inputs larger than L2: %.2f GB moved per step vs 126 MB L2; %d token batches "
+              "alternate" % (algorithmic_bytes(w) / 1e9, args.batches),
+        "parallelism": "replicas x%d (tokens sharded, table replicated)" % args.gpus,
+    }
+
+
+def run_ours(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_ngram_b200 as ng
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- table (set-up, untimed): a replica of the whole table on every GPU
+    if w.dtype == "bf16":
+        dtype = ng.NGRAM_BF16
+        table = torch.empty((w.R, w.d), dtype=torch.bfloat16, device=dev)
+        scale = None
+    else:
+        dtype = ng.NGRAM_INT8_ROWSCALE
+        table = torch.empty((w.R, w.d), dtype=torch.int8, device=dev)
+        scale = torch.empty((w.R,), dtype=torch.float32, device=dev)
+    ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
+    hp = ng.ngram_default_hash_params(vocab_size=w.vocab)
+    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
+
+    # ---- inputs: this rank's token batches (distinct seeds per rank and batch)
+    host_tok, host_hist = [], []
+    for b in range(args.batches):
+        host_tok.append(gen.tokens_for(w, gen.TOKEN_SEED + 1000 * rank + b))
+        host_hist.append(gen.history_for(w, gen.HISTORY_SEED + 1000 * rank + b))
+    res_bits = gen.residual_bf16_bits(w.N, w.d, gen.RESIDUAL_SEED + rank)
+    gate_h = gen.gate_f32(w.d)
+    tok_d = [torch.from_numpy(t).to(dev) for t in host_tok]
+    hist_d = [None if h is None else torch.from_numpy(h).to(dev) for h in host_hist]
+    res_cpu = torch.from_numpy(res_bits.view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
+    residual = res_cpu.to(dev)
+    out = torch.empty_like(residual)
+    gate = torch.from_numpy(gate_h).to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        b = i % args.batches
+        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
+
+    # ---- device-resident timing
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id_for(dev)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(K):
+            ev_s[i].record(stream)
+            step(i)
+            ev_e[i].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    kern_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(K))
+    st, info = ng.ngram_get_device_error(ctx)
+    if st != ng.NGRAM_OK:
+        raise SystemExit("device error word set: %s" % info)
+
+    # ---- end to end: pinned host inputs in, result back to the host, every step
+    tok_h = [torch.from_numpy(t).pin_memory() for t in host_tok]
+    hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in host_hist]
+    res_h = res_cpu.pin_memory()
+    out_h = torch.empty_like(res_h).pin_memory()
+    E = max(1, args.e2e_steps)
+
+    def e2e_step(i):
+        b = i % args.batches
+        tok_d[b].copy_(tok_h[b], non_blocking=True)
+        if hist_h[b] is not None:
+            hist_d[b].copy_(hist_h[b], non_blocking=True)
+        residual.copy_(res_h, non_blocking=True)
+        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for i in range(min(3, E)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(E):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = w.N * 4 + (w.n_seq * 8 if w.history else 0) + w.N * w.d * 2
+    d2h = w.N * w.d * 2
+
+    # ---- max over ranks
+    times = torch.tensor([elapsed_ms, kern_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    elapsed_ms, kern_ms, e2e_ms = (float(x) for x in times.tolist())
+    clocks = clk.summary()
+
+    if rank == 0:
+        tokens_total = world * w.N
+        value = tokens_total * K / (elapsed_ms / 1e3)
+        e2e_value = tokens_total * E / (e2e_ms / 1e3)
+        peaks = measured_peaks()
+        bytes_launch = algorithmic_bytes(w)
+        achieved = bytes_launch / (kern_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": config_for(w, args),
+            "gather_gbs": bytes_launch * world * K / (elapsed_ms / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic(w.name),
+                         "kernel": "k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8",
+                         "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
+                         "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": E,
+                    "path": "pinned host tokens+residual -> device, ngram_forward, out -> pinned host"},
+            "clocks": clocks,
+            "gpu_launches": K,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            threads = os.cpu_count() or 1
+            inp = {"tokens": host_tok[0], "history": host_hist[0], "residual": res_bits,
+                   "gate": gate_h}
+            v, n, dt = oracle_tokens_per_s(w, inp, args.cpu_seconds, threads)
+            line["cpu_baseline"] = {
+                "value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": "%d of %d tokens of this workload, %.1f s, rows regenerated from "
+                          "the synthetic-table definition (the 95 GiB table is not on the host)"
+                          % (n, w.N, dt)}
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="full_prefill", choices=sorted(gen.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batches", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = gen.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+    run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

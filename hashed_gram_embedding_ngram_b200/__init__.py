@@ -1,0 +1,22 @@
+"""B200 (sm_100a) hashed n-gram embedding lookup.
+
+For every token the bigram and trigram context is hashed into one large row table,
+16 rows are gathered and summed in fp32, and the sum is added to the residual stream
+through an elementwise gate -- the "storage expert" of "Qwen Brought Back N-Grams.
+All 51 Billion Parameters of Them." (section "N-grams, of all things") with the gate
+of "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with Heterogeneous Memory
+Prefetch", Key point 1.
+
+The compute lives in libngram.so (C ABI in include/ngram.h, CUDA kernels in csrc/);
+this package is its thin ctypes binding.  Importing it fails if the library is not
+built: there is no fallback path.
+"""
+from ._binding import (  # noqa: F401
+    LIB_PATH, Context, HashParams, NgramError, lib,
+    NGRAM_OK, NGRAM_EINVAL, NGRAM_ENOMEM, NGRAM_ECUDA, NGRAM_EUNSUPPORTED, NGRAM_ETIMEOUT,
+    NGRAM_EDEVICE, NGRAM_BF16, NGRAM_INT8_ROWSCALE, NGRAM_RES_HBM, NGRAM_RES_HOST_UVA,
+    NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO, MAX_HEADS, DEFAULT_BASE_SEED, DEFAULT_PAD_ID,
+    ngram_default_hash_params, ngram_init, ngram_forward, ngram_hash_indices,
+    ngram_fill_synthetic, ngram_get_device_error, ngram_last_error, ngram_status_string,
+    ngram_destroy,
+)

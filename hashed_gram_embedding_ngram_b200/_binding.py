@@ -1,0 +1,226 @@
+"""ctypes binding of libngram.so: argument marshalling only.
+
+Each function has the name of the C entry point it calls (include/ngram.h) and does
+nothing but check tensor shapes, dtypes, devices and contiguity, take raw pointers
+and the CUDA stream handle, and turn a non-OK status into an exception.  Every step
+of the lookup runs in the library's kernels; there is no Python or CPU fallback: if
+libngram.so is missing, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libngram.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libngram.so is not built (expected at %s); build it with "
+        "`python hashed_gram_embedding_ngram_b200/build.py`" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ngram_status
+NGRAM_OK, NGRAM_EINVAL, NGRAM_ENOMEM, NGRAM_ECUDA = 0, 1, 2, 3
+NGRAM_EUNSUPPORTED, NGRAM_ETIMEOUT, NGRAM_EDEVICE = 4, 5, 6
+# ngram_dtype
+NGRAM_BF16, NGRAM_INT8_ROWSCALE = 0, 1
+# ngram_residency
+NGRAM_RES_HBM, NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO = 0, 1, 2, 3
+
+MAX_HEADS = 16
+DEFAULT_BASE_SEED = 0x6E6772616D5F7631
+DEFAULT_PAD_ID = 0x1FFFFF
+
+
+class NgramError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s: %s" % (ngram_status_string(status), message))
+        self.status = status
+
+
+class HashParams(ctypes.Structure):
+    _fields_ = [("base_seed", ctypes.c_uint64),
+                ("n_bigram_heads", ctypes.c_uint32),
+                ("n_trigram_heads", ctypes.c_uint32),
+                ("pad_id", ctypes.c_uint32),
+                ("vocab_size", ctypes.c_uint32),
+                ("flags", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+
+_P = ctypes.c_void_p
+_u32, _u64, _i32 = ctypes.c_uint32, ctypes.c_uint64, ctypes.c_int
+
+_lib.ngram_default_hash_params.argtypes = [ctypes.POINTER(HashParams)]
+_lib.ngram_default_hash_params.restype = _i32
+_lib.ngram_init.argtypes = [ctypes.POINTER(_P), _P, _P, _u64, _u32, _i32, _i32,
+                            ctypes.POINTER(HashParams), _u32]
+_lib.ngram_init.restype = _i32
+_lib.ngram_forward.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
+_lib.ngram_forward.restype = _i32
+_lib.ngram_hash_indices.argtypes = [_P, _P, _P, _u32, _u32, _P, _P]
+_lib.ngram_hash_indices.restype = _i32
+_lib.ngram_fill_synthetic.argtypes = [_P, _P, _u64, _u32, _i32, _u64, _P]
+_lib.ngram_fill_synthetic.restype = _i32
+_lib.ngram_get_device_error.argtypes = [_P, _P, _i32]
+_lib.ngram_get_device_error.restype = _i32
+_lib.ngram_last_error.argtypes = []
+_lib.ngram_last_error.restype = ctypes.c_char_p
+_lib.ngram_status_string.argtypes = [_i32]
+_lib.ngram_status_string.restype = ctypes.c_char_p
+_lib.ngram_destroy.argtypes = [_P]
+_lib.ngram_destroy.restype = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libngram.so handle."""
+    return _lib
+
+
+def ngram_status_string(status: int) -> str:
+    return _lib.ngram_status_string(status).decode()
+
+
+def ngram_last_error() -> str:
+    return _lib.ngram_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != NGRAM_OK:
+        raise NgramError(status, ngram_last_error())
+
+
+def ngram_default_hash_params(**overrides) -> HashParams:
+    hp = HashParams()
+    _check(_lib.ngram_default_hash_params(ctypes.byref(hp)))
+    for k, v in overrides.items():
+        setattr(hp, k, v)
+    return hp
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t, name, dtype, device=None, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if device is not None and t.device != device:
+        raise ValueError("%s must be on %s, got %s" % (name, device, t.device))
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got %d" % (name, ndim, t.dim()))
+
+
+class Context:
+    """An ngram_ctx handle; keeps the table tensors alive while it lives."""
+
+    def __init__(self, handle, table, row_scale, R, d, dtype, residency, hp, max_tokens):
+        self.handle = handle
+        self.table, self.row_scale = table, row_scale
+        self.R, self.d, self.dtype, self.residency = R, d, dtype, residency
+        self.hp, self.max_tokens = hp, max_tokens
+        self.n_heads = hp.n_bigram_heads + hp.n_trigram_heads
+
+    def close(self):
+        if self.handle:
+            ngram_destroy(self)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ngram_init(table: torch.Tensor, R: int, d: int, dtype: int = NGRAM_BF16,
+               where: int = NGRAM_RES_HBM, hp: HashParams | None = None,
+               max_tokens: int = 65536, row_scale: torch.Tensor | None = None) -> Context:
+    if hp is None:
+        hp = ngram_default_hash_params()
+    handle = ctypes.c_void_p()
+    _check(_lib.ngram_init(ctypes.byref(handle), _ptr(table), _ptr(row_scale), R, d, dtype,
+                           where, ctypes.byref(hp), max_tokens))
+    return Context(handle.value, table, row_scale, R, d, dtype, where, hp, max_tokens)
+
+
+def ngram_forward(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor,
+                  gate: torch.Tensor, out: torch.Tensor | None = None,
+                  history: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = residual + gate * sum of the 16 hashed rows (bf16).  tokens int32
+    [n_seq][T]; residual bf16 [N][d]; gate fp32 [d]; history int32 [n_seq][2] or None;
+    out bf16 [N][d] (allocated if None; may be residual itself)."""
+    dev = tokens.device
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    n_seq, T = tokens.shape
+    N = n_seq * T
+    _need(residual, "residual", torch.bfloat16, dev)
+    if residual.numel() != N * ctx.d:
+        raise ValueError("residual must hold N * d = %d elements" % (N * ctx.d))
+    _need(gate, "gate", torch.float32, dev)
+    if gate.numel() != ctx.d:
+        raise ValueError("gate must hold d = %d elements" % ctx.d)
+    if history is not None:
+        _need(history, "history", torch.int32, dev, ndim=2)
+        if tuple(history.shape) != (n_seq, 2):
+            raise ValueError("history must be [n_seq][2]")
+    if out is None:
+        out = torch.empty_like(residual)
+    _need(out, "out", torch.bfloat16, dev)
+    if out.numel() != N * ctx.d:
+        raise ValueError("out must hold N * d elements")
+    _check(_lib.ngram_forward(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                              _ptr(residual), _ptr(gate), _ptr(out), _stream(stream)))
+    return out
+
+
+def ngram_hash_indices(ctx: Context, tokens: torch.Tensor, history: torch.Tensor | None = None,
+                       idx_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row indices [N][H] (int32 tensor holding uint32 values) of every token and head."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    n_seq, T = tokens.shape
+    if history is not None:
+        _need(history, "history", torch.int32, tokens.device, ndim=2)
+    if idx_out is None:
+        idx_out = torch.empty((n_seq * T, ctx.n_heads), dtype=torch.int32, device=tokens.device)
+    _need(idx_out, "idx_out", torch.int32, tokens.device)
+    _check(_lib.ngram_hash_indices(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                                   _ptr(idx_out), _stream(stream)))
+    return idx_out
+
+
+def ngram_fill_synthetic(table: torch.Tensor, R: int, d: int, dtype: int = NGRAM_BF16,
+                         seed: int = 0, row_scale: torch.Tensor | None = None,
+                         stream=None) -> None:
+    _check(_lib.ngram_fill_synthetic(_ptr(table), _ptr(row_scale), R, d, dtype,
+                                     seed & (2**64 - 1), _stream(stream)))
+
+
+def ngram_get_device_error(ctx: Context, clear: bool = True):
+    """(status, [flag, position, bad id, 0]); synchronises the device."""
+    info = (ctypes.c_uint32 * 4)()
+    st = _lib.ngram_get_device_error(ctx.handle, info, 1 if clear else 0)
+    if st not in (NGRAM_OK, NGRAM_EDEVICE):
+        _check(st)
+    return st, list(info)
+
+
+def ngram_destroy(ctx: Context) -> None:
+    if ctx.handle:
+        _lib.ngram_destroy(ctx.handle)
+        ctx.handle = None

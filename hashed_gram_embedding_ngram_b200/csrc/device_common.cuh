@@ -1,0 +1,132 @@
+// device_common.cuh -- device helpers of libngram: context formation, the per-head
+// hash, exact remainder by R, Philox4x32-10 and cache-hinted vector loads.
+//
+// The method ("Qwen Brought Back N-Grams. All 51 Billion Parameters of Them.",
+// section "N-grams, of all things"): hash the bigram and trigram context of each
+// token into one table, gather 16 rows.  The pages fix no hash; the one defined
+// here is documented in include/ngram.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace ngram {
+
+constexpr uint64_t kGolden = 0x9E3779B97F4A7C15ull;   // splitmix64 state increment
+constexpr uint32_t kTokenMask = (1u << 21) - 1u;
+
+// splitmix64 output for the state reached by one increment from z (Steele, Lea &
+// Flood, OOPSLA 2014): the mixer with the published constants.
+__host__ __device__ __forceinline__ uint64_t splitmix64_step(uint64_t z) {
+    z += kGolden;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// x mod R for R >= 2 with the Barrett constant m = floor(2^64 / R) (Barrett, CRYPTO
+// '86).  q = floor(x * m / 2^64) is floor(x / R) or one less, so one conditional
+// subtraction gives the exact remainder.  R == 1 is handled by the caller (m = 0).
+__device__ __forceinline__ uint32_t mod_rows(uint64_t x, uint64_t R, uint64_t m) {
+    if (m == 0) return 0u;                       // R == 1
+    uint64_t q = __umul64hi(x, m);
+    uint64_t r = x - q * R;
+    if (r >= R) r -= R;
+    return static_cast<uint32_t>(r);
+}
+
+// Parameters of the hash, passed by value to every kernel that hashes.
+struct HashArgs {
+    uint64_t base_seed;
+    uint64_t R;
+    uint64_t barrett_m;       // floor(2^64 / R), 0 when R == 1
+    uint32_t n_bigram;
+    uint32_t n_heads;         // bigram + trigram, <= 16
+    uint32_t pad_id;
+    uint32_t vocab;
+};
+
+// Device error word: [0] flag, [1] position (bit 31 = history entry), [2] bad id.
+__device__ __forceinline__ void flag_bad_token(uint32_t *err, uint32_t pos, int32_t id) {
+    if (atomicCAS(err, 0u, 1u) == 0u) {
+        err[1] = pos;
+        err[2] = static_cast<uint32_t>(id);
+    }
+}
+
+__device__ __forceinline__ uint32_t checked_token(int32_t w, const HashArgs &a,
+                                                  uint32_t *err, uint32_t pos) {
+    if (w < 0 || static_cast<uint32_t>(w) >= a.vocab) {
+        flag_bad_token(err, pos, w);
+        return a.pad_id;
+    }
+    return static_cast<uint32_t>(w);
+}
+
+// w0 = w_t, w1 = w_{t-1}, w2 = w_{t-2} of flat token `tok` (= s * T + t); earlier
+// positions come from history[s] = {w_-2, w_-1} or PAD.  Never crosses sequences.
+__device__ __forceinline__ void token_context(const int32_t *__restrict__ tokens,
+                                              const int32_t *__restrict__ history,
+                                              uint32_t tok, uint32_t T, const HashArgs &a,
+                                              uint32_t *err, uint32_t &w0, uint32_t &w1,
+                                              uint32_t &w2) {
+    const uint32_t s = tok / T;
+    const uint32_t t = tok - s * T;
+    w0 = checked_token(__ldg(tokens + tok), a, err, tok);
+    uint32_t h_old = a.pad_id, h_new = a.pad_id;
+    if (history != nullptr && t < 2) {
+        h_new = checked_token(__ldg(history + 2 * s + 1), a, err, 0x80000000u | (2 * s + 1));
+        if (t == 0)
+            h_old = checked_token(__ldg(history + 2 * s), a, err, 0x80000000u | (2 * s));
+    }
+    w1 = (t >= 1) ? checked_token(__ldg(tokens + tok - 1), a, err, tok - 1) : h_new;
+    w2 = (t >= 2) ? checked_token(__ldg(tokens + tok - 2), a, err, tok - 2)
+                  : ((t == 1) ? h_new : h_old);
+}
+
+// Row index of head h for context (w0, w1, w2).
+__device__ __forceinline__ uint32_t head_row(uint32_t h, uint32_t w0, uint32_t w1,
+                                             uint32_t w2, const HashArgs &a) {
+    // seed_h = (h+1)-th splitmix64 output from base_seed
+    const uint64_t seed = splitmix64_step(a.base_seed + static_cast<uint64_t>(h) * kGolden);
+    const uint64_t k2 = (static_cast<uint64_t>(w1) << 21) | w0;
+    const uint64_t key = (h < a.n_bigram) ? k2 : ((static_cast<uint64_t>(w2) << 42) | k2);
+    return mod_rows(splitmix64_step(key ^ seed), a.R, a.barrett_m);
+}
+
+// Philox4x32-10 (Salmon, Moraes, Dror & Shaw, SC'11): ten rounds of two 32x32->64
+// multiplies on words 0 and 2, key bumped by the Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// 16-byte read-only load that does not allocate in L1 (rows and residual are read
+// once per use; reuse across tokens is left to L2).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+// bf16 pair in one 32-bit word -> two fp32 values (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 -> bf16 pair (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+}  // namespace ngram

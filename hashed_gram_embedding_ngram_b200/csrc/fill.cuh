@@ -1,0 +1,81 @@
+// fill.cuh -- synthetic table initialisation (set-up, not on the timed path).
+//
+// The pages' table is learned ("Qwen Brought Back N-Grams. All 51 Billion
+// Parameters of Them.", section "N-grams, of all things"); no weights exist here, so
+// element (row, col) is a pure function of (seed, row, col) through Philox4x32-10.
+// The exact mapping is stated in include/ngram.h (ngram_fill_synthetic).
+#pragma once
+
+#include "device_common.cuh"
+
+namespace ngram {
+
+constexpr float kBf16Scale = 0x1.1bc77ap-22f;   // 0.02 / std(2S - 262140)
+constexpr float kInt8Scale = 0x1.1bc5f4p-11f;   // 0.02 / std(q)
+
+// bf16 value from the two Philox words (a, b) of its column parity.
+__device__ __forceinline__ float synth_bf16_value(uint32_t a, uint32_t b) {
+    const int32_t S = static_cast<int32_t>((a & 0xFFFFu) + (a >> 16) + (b & 0xFFFFu) + (b >> 16));
+    const int32_t C = 2 * S - 262140;                     // |C| < 2^24: exact in fp32
+    return __fmul_rn(__int2float_rn(C), kBf16Scale);
+}
+
+// int8 value from one Philox word: (sum of its bytes - 510) >> 2, arithmetic shift.
+__device__ __forceinline__ int32_t synth_int8_value(uint32_t w) {
+    const int32_t sum = static_cast<int32_t>((w & 0xFFu) + ((w >> 8) & 0xFFu) +
+                                             ((w >> 16) & 0xFFu) + (w >> 24));
+    return (sum - 510) >> 2;
+}
+
+// One CTA per row (grid-stride over rows); each thread writes 8 columns (16 bytes)
+// per step, from four Philox calls with counters (col/2, row, 1, 0).
+__global__ void __launch_bounds__(256) k_fill_bf16(uint16_t *__restrict__ table, uint64_t R,
+                                                   uint32_t d, uint32_t k0, uint32_t k1) {
+    const uint32_t nvec = d >> 3;
+    for (uint64_t row = blockIdx.x; row < R; row += gridDim.x) {
+        uint4 *dst = reinterpret_cast<uint4 *>(table + row * d);
+        for (uint32_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+            uint32_t words[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {                // column pair 4v+p: cols 8v+2p, +1
+                const uint4 x = philox4x32_10(
+                    make_uint4(4u * v + p, static_cast<uint32_t>(row), 1u, 0u), k0, k1);
+                words[p] = pack_bf16x2(synth_bf16_value(x.x, x.y), synth_bf16_value(x.z, x.w));
+            }
+            dst[v] = make_uint4(words[0], words[1], words[2], words[3]);
+        }
+    }
+}
+
+// int8 rows: each thread writes 16 columns from four Philox calls with counters
+// (col/4, row, 2, 0); thread 0 of the row also writes the row scale (counter
+// (0, row, 3, 0)).
+__global__ void __launch_bounds__(256) k_fill_int8(int8_t *__restrict__ table,
+                                                   float *__restrict__ row_scale, uint64_t R,
+                                                   uint32_t d, uint32_t k0, uint32_t k1) {
+    const uint32_t nvec = d >> 4;
+    for (uint64_t row = blockIdx.x; row < R; row += gridDim.x) {
+        uint4 *dst = reinterpret_cast<uint4 *>(table + row * d);
+        for (uint32_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+            uint32_t words[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {                // columns 16v+4p .. 16v+4p+3
+                const uint4 x = philox4x32_10(
+                    make_uint4(4u * v + p, static_cast<uint32_t>(row), 2u, 0u), k0, k1);
+                const uint32_t q0 = synth_int8_value(x.x) & 0xFFu;
+                const uint32_t q1 = synth_int8_value(x.y) & 0xFFu;
+                const uint32_t q2 = synth_int8_value(x.z) & 0xFFu;
+                const uint32_t q3 = synth_int8_value(x.w) & 0xFFu;
+                words[p] = q0 | (q1 << 8) | (q2 << 16) | (q3 << 24);
+            }
+            dst[v] = make_uint4(words[0], words[1], words[2], words[3]);
+        }
+        if (threadIdx.x == 0) {
+            const uint4 x = philox4x32_10(make_uint4(0u, static_cast<uint32_t>(row), 3u, 0u), k0, k1);
+            const float t = __fmul_rn(__uint2float_rn(x.x >> 8), 0x1p-25f);
+            row_scale[row] = __fmul_rn(kInt8Scale, __fadd_rn(0.75f, t));
+        }
+    }
+}
+
+}  // namespace ngram

@@ -1,0 +1,148 @@
+// gather.cuh -- the hot path: context -> 16 hashed rows -> fp32 sum -> gate -> residual.
+//
+// "Qwen Brought Back N-Grams. All 51 Billion Parameters of Them.", section "N-grams,
+// of all things": hash the bigram and trigram context into the table, gather 16 rows,
+// sum them into one d-wide vector that is added to the residual stream.  The gate is
+// the elementwise W_g of "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with
+// Heterogeneous Memory Prefetch", Key point 1.
+//
+// Design (HBM-bound gather, no contraction, so no tensor cores):
+//   * One warp owns one (token, group of 32-vector column strips) work item.  Lanes
+//     0..H-1 form the context and hash one head each; the H row indices are then
+//     broadcast with shuffles, so there is no shared memory and no block barrier.
+//   * For each strip a lane owns one 16-byte column vector (8 bf16): it issues all H
+//     row loads (16 x 16 B in flight per lane, 8 KB per warp) plus the residual load
+//     before the first add, then sums in head order 0..H-1 in fp32, applies
+//     y = r + g * acc with separately rounded multiply and add, and stores bf16.
+//   * Work items are dealt to a persistent grid (blocks = SMs x resident blocks);
+//     decode-sized batches split a token's strips across warps for latency, large
+//     batches keep all strips of a token in one warp so the hash is computed once.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace ngram {
+
+struct GatherArgs {
+    HashArgs h;
+    const void *table;          // [R][d] bf16 bits, or int8
+    const float *row_scale;     // [R] (int8)
+    const int32_t *tokens;      // [n_seq][T]
+    const int32_t *history;     // [n_seq][2] or null
+    const uint16_t *residual;   // [N][d] bf16 bits
+    const float *gate;          // [d]
+    uint16_t *out;              // [N][d] bf16 bits (may alias residual)
+    uint32_t *err;              // device error word
+    uint32_t T;
+    uint32_t N;
+    uint32_t d;
+    uint32_t n_strips;          // strips of 32 column vectors per token
+    uint32_t strips_per_item;
+    uint32_t groups_per_token;  // ceil(n_strips / strips_per_item)
+};
+
+// 16-byte load through L2 without L1 allocation; coherent (the residual may be the
+// output buffer of the same launch when the caller works in place).
+__device__ __forceinline__ uint4 ld_na_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Row indices of the warp's token, one head per lane (lanes >= H hold 0).
+__device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t tok,
+                                                  uint32_t lane, uint32_t H) {
+    uint32_t row = 0;
+    if (lane < H) {
+        uint32_t w0, w1, w2;
+        token_context(g.tokens, g.history, tok, g.T, g.h, g.err, w0, w1, w2);
+        row = head_row(lane, w0, w1, w2, g.h);
+    }
+    return row;
+}
+
+template <int kH>   // compile-time head count (16), or 0: runtime g.h.n_heads <= 16
+__global__ void __launch_bounds__(256, 2) k_gather_bf16(const GatherArgs g) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
+    const uint32_t H = kH ? static_cast<uint32_t>(kH) : g.h.n_heads;
+    const uint32_t nvec = g.d >> 3;
+    const uint32_t n_items = g.N * g.groups_per_token;
+    const uint16_t *__restrict__ table = static_cast<const uint16_t *>(g.table);
+
+    for (uint32_t item = warp; item < n_items; item += n_warps) {
+        const uint32_t tok = item / g.groups_per_token;
+        const uint32_t grp = item - tok * g.groups_per_token;
+        const uint32_t my_row = warp_head_row(g, tok, lane, H);
+        uint32_t rows[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);
+
+        const uint32_t s_begin = grp * g.strips_per_item;
+        const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
+        const size_t tok_off = static_cast<size_t>(tok) * g.d;
+        for (uint32_t s = s_begin; s < s_end; ++s) {
+            const uint32_t v = s * 32u + lane;
+            if (v >= nvec) continue;
+            // issue every load of this column vector before the first add
+            uint4 e[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h)
+                if (kH || h < static_cast<int>(H))
+                    e[h] = ld_stream_v4(table + static_cast<size_t>(rows[h]) * g.d + v * 8u);
+            const uint4 r = ld_na_v4(g.residual + tok_off + v * 8u);
+            const float4 ga = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v);
+            const float4 gb = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v + 1u);
+
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                if (kH || h < static_cast<int>(H)) {
+                    acc[0] = __fadd_rn(acc[0], bf16_lo(e[h].x));
+                    acc[1] = __fadd_rn(acc[1], bf16_hi(e[h].x));
+                    acc[2] = __fadd_rn(acc[2], bf16_lo(e[h].y));
+                    acc[3] = __fadd_rn(acc[3], bf16_hi(e[h].y));
+                    acc[4] = __fadd_rn(acc[4], bf16_lo(e[h].z));
+                    acc[5] = __fadd_rn(acc[5], bf16_hi(e[h].z));
+                    acc[6] = __fadd_rn(acc[6], bf16_lo(e[h].w));
+                    acc[7] = __fadd_rn(acc[7], bf16_hi(e[h].w));
+                }
+            }
+            const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float y0 = __fadd_rn(bf16_lo(rw[p]), __fmul_rn(gv[2 * p], acc[2 * p]));
+                const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[2 * p + 1]));
+                o[p] = pack_bf16x2(y0, y1);
+            }
+            *reinterpret_cast<uint4 *>(g.out + tok_off + v * 8u) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// The index step alone: one thread per (token, head).
+__global__ void __launch_bounds__(256) k_hash_indices(const HashArgs a,
+                                                      const int32_t *__restrict__ tokens,
+                                                      const int32_t *__restrict__ history,
+                                                      uint32_t T, uint32_t N, uint32_t *err,
+                                                      uint32_t *__restrict__ idx_out) {
+    const uint32_t H = a.n_heads;
+    const uint32_t total = N * H;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += gridDim.x * blockDim.x) {
+        const uint32_t tok = i / H;
+        const uint32_t h = i - tok * H;
+        uint32_t w0, w1, w2;
+        token_context(tokens, history, tok, T, a, err, w0, w1, w2);
+        idx_out[i] = head_row(h, w0, w1, w2, a);
+    }
+}
+
+}  // namespace ngram

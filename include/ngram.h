@@ -1,0 +1,169 @@
+/*
+ * ngram.h -- C ABI of libngram.so, the B200 (sm_100a) hashed n-gram embedding lookup.
+ *
+ * The operation ("Qwen Brought Back N-Grams. All 51 Billion Parameters of Them.",
+ * section "N-grams, of all things", and its "Key Takeaways"): for every token, hash
+ * the local bigram and trigram context into one table of R rows of width d
+ * (20,000,000 x 2560 in the full model), gather 16 rows, sum them, and add the sum to
+ * the residual stream.  The sum enters through an elementwise gate, as in the
+ * equation of Key point 1 of "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with
+ * Heterogeneous Memory Prefetch":  out = residual + g (elementwise) sum_h E[idx_h].
+ *
+ * Definitions this library fixes where the pages are silent:
+ *   - Context of token t in sequence s (t counted from 0 inside the sequence):
+ *       w0 = w_t,  w1 = w_{t-1},  w2 = w_{t-2}.  Positions before 0 come from
+ *       history[s] = {w_-2, w_-1} (oldest first) when history is non-NULL, else they
+ *       are pad_id.  Contexts never cross from one sequence row into another.
+ *       A token id outside [0, vocab_size) is read as pad_id and flags the device
+ *       error word (see ngram_get_device_error).
+ *   - Keys: bigram k2 = (w1 << 21) | w0, trigram k3 = (w2 << 42) | (w1 << 21) | w0.
+ *   - Heads: h = 0 .. n_bigram_heads-1 hash k2, the next n_trigram_heads hash k3
+ *       (defaults 8 + 8 = the 16 rows per token the pages give).
+ *   - Hash: mix(z) = the splitmix64 output function applied to state z + 0x9E3779B97F4A7C15;
+ *       seed_h = (h+1)-th splitmix64 output from base_seed;
+ *       idx_h  = mix(key ^ seed_h) mod R   (exact 64-bit remainder).
+ *   - Sum: fp32, in head order 0..H-1; colliding heads each contribute their row.
+ *   - Output: y = fp32(residual) + g * sum (separately rounded multiply and add),
+ *       stored as bf16 rounded to nearest even.
+ *
+ * Memory: every pointer argument of the compute calls is a device pointer (or, for
+ * the table in the host-resident modes, a pinned host pointer).  The caller owns
+ * every buffer it passes.  bf16 arrays are passed as uint16_t bit patterns.
+ * Streams: all compute calls are asynchronous on the stream given (NULL = legacy
+ * default stream); the library creates no cross-stream dependency of its own.
+ * Errors: every call returns an ngram_status; invalid arguments are reported before
+ * any CUDA work is issued, and nothing aborts the process.  ngram_last_error() gives
+ * the text of the last failure on the calling thread.
+ */
+#ifndef NGRAM_H_
+#define NGRAM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define NGRAM_API __attribute__((visibility("default")))
+#else
+#define NGRAM_API
+#endif
+
+/* Same underlying type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *ngram_stream_t;
+
+typedef enum {
+    NGRAM_OK = 0,
+    NGRAM_EINVAL = 1,          /* bad argument; nothing was launched */
+    NGRAM_ENOMEM = 2,          /* a device or pinned allocation failed */
+    NGRAM_ECUDA = 3,           /* a CUDA runtime call failed (text in ngram_last_error) */
+    NGRAM_EUNSUPPORTED = 4,    /* valid request this build does not implement */
+    NGRAM_ETIMEOUT = 5,        /* a bounded host-side wait ran out */
+    NGRAM_EDEVICE = 6          /* a kernel flagged bad input (device error word set) */
+} ngram_status;
+
+typedef enum {
+    NGRAM_BF16 = 0,            /* table [R][d] bf16 */
+    NGRAM_INT8_ROWSCALE = 1    /* table [R][d] int8 + row_scale [R] fp32; value = q * scale */
+} ngram_dtype;
+
+typedef enum {
+    NGRAM_RES_HBM = 0,         /* table in this GPU's memory */
+    NGRAM_RES_HOST_UVA = 1,    /* table in pinned host memory, read by the kernel over PCIe */
+    NGRAM_RES_HOST_DMA = 2,    /* table in pinned host memory, rows staged by copy engine */
+    NGRAM_RES_HOST_AUTO = 3    /* host-resident; the faster of UVA / DMA, chosen by timing */
+} ngram_residency;
+
+#define NGRAM_MAX_HEADS 16u
+#define NGRAM_TOKEN_BITS 21u
+#define NGRAM_DEFAULT_BASE_SEED 0x6E6772616D5F7631ull   /* ASCII "ngram_v1" */
+#define NGRAM_DEFAULT_PAD_ID 0x1FFFFFu                   /* 2^21 - 1 */
+
+typedef struct {
+    uint64_t base_seed;        /* head seeds are the splitmix64 outputs from this state */
+    uint32_t n_bigram_heads;   /* default 8 */
+    uint32_t n_trigram_heads;  /* default 8; n_bigram + n_trigram in [1, 16] */
+    uint32_t pad_id;           /* default 2^21 - 1; must be < 2^21 */
+    uint32_t vocab_size;       /* token ids must lie in [0, vocab_size); <= 2^21 - 1 */
+    uint32_t flags;            /* reserved, must be 0 */
+    uint32_t reserved;         /* must be 0 */
+} ngram_hash_params;
+
+typedef struct ngram_ctx ngram_ctx;
+
+/* Fill hp with the defaults: base_seed "ngram_v1", 8 + 8 heads, pad 2^21-1, and
+ * vocab_size 2^21-1.  Returns NGRAM_EINVAL if hp is NULL. */
+NGRAM_API ngram_status ngram_default_hash_params(ngram_hash_params *hp);
+
+/* Create a lookup context on the current CUDA device.
+ *   table      device pointer to [R][d] rows (bf16 bits, or int8), 16-byte aligned;
+ *              not owned, must outlive the context.
+ *   row_scale  device pointer to [R] fp32 (int8 only, else NULL); not owned.
+ *   R          rows, 1 <= R < 2^32.   d: row width, multiple of 8 (bf16) or 16 (int8).
+ *   where      residency of the table (NGRAM_RES_HBM in this build).
+ *   hp         hash parameters (NULL = defaults).
+ *   max_tokens largest n_seq * T a later call may pass (>= 1).
+ * The context owns a 16-byte device error word.  EINVAL on bad arguments (checked
+ * before any CUDA call), EUNSUPPORTED for residencies not built, ECUDA/ENOMEM on
+ * CUDA failures.  On failure *out is set to NULL. */
+NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_scale,
+                        uint64_t R, uint32_t d, ngram_dtype dtype, ngram_residency where,
+                        const ngram_hash_params *hp, uint32_t max_tokens);
+
+/* The fused lookup: for all N = n_seq * T tokens,
+ *   out[t][c] = bf16( residual[t][c] + gate[c] * sum_h table[idx_h(t)][c] ).
+ *   tokens    device int32 [n_seq][T] (row-major).
+ *   history   device int32 [n_seq][2] = {w_-2, w_-1} per sequence, or NULL (PAD).
+ *   residual  device bf16 [N][d], 16-byte aligned.
+ *   gate      device fp32 [d], 16-byte aligned (the static gate W_g).
+ *   out       device bf16 [N][d], 16-byte aligned; may equal residual (in place),
+ *             must not otherwise overlap it.
+ * One kernel launch on stream; N == 0 launches nothing.  EINVAL if N > max_tokens,
+ * a pointer is NULL or misaligned.  Bad token ids are reported asynchronously through
+ * ngram_get_device_error. */
+NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
+                           uint32_t n_seq, uint32_t T, const uint16_t *residual,
+                           const float *gate, uint16_t *out, ngram_stream_t stream);
+
+/* The index step alone: idx_out (device uint32 [N][H], H = heads) receives the row
+ * index of every (token, head), computed exactly as ngram_forward computes them. */
+NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
+                                uint32_t n_seq, uint32_t T, uint32_t *idx_out,
+                                ngram_stream_t stream);
+
+/* Fill a device table with the synthetic values used by the tests and benchmarks
+ * (the pages' table is learned; no weights exist here).  Element (row, col) is a
+ * pure function of (seed, row, col) through Philox4x32-10 (Salmon et al., SC'11):
+ *   bf16: counter (col/2, row, 1, 0), key (seed lo32, seed hi32); words (x0,x1) for
+ *         even col, (x2,x3) for odd; S = sum of their four 16-bit halves;
+ *         value = bf16_rne(float(2S - 262140) * 0x1.1bc77ap-22)   (std 0.02).
+ *   int8: counter (col/4, row, 2, 0), word x[col%4]; q = (sum of its bytes - 510) >> 2;
+ *         row_scale[row] = 0x1.1bc5f4p-11 * (0.75 + (x0 >> 8) * 2^-25) with x0 from
+ *         counter (0, row, 3, 0), each fp32 step rounded separately.
+ * table (and row_scale for int8) are device pointers.  Asynchronous on stream. */
+NGRAM_API ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
+                                  ngram_dtype dtype, uint64_t seed, ngram_stream_t stream);
+
+/* Synchronise the context's device, read and optionally clear its error word.
+ * info (may be NULL) receives {flag, flat position, bad id, 0}; a position with bit
+ * 31 set names history entry (position & 0x7FFFFFFF) = 2*s + j.  Returns NGRAM_OK if
+ * no kernel flagged bad input, NGRAM_EDEVICE if one did. */
+NGRAM_API ngram_status ngram_get_device_error(ngram_ctx *ctx, uint32_t info[4], int clear);
+
+/* Text of the last failure on the calling thread ("" if none). */
+NGRAM_API const char *ngram_last_error(void);
+
+/* Constant name of a status code. */
+NGRAM_API const char *ngram_status_string(ngram_status s);
+
+/* Free the context's own allocations (never the caller's buffers).  NULL is a no-op.
+ * The caller must make sure no work using ctx is still running. */
+NGRAM_API void ngram_destroy(ngram_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NGRAM_H_ */

@@ -56,6 +56,8 @@ WORKLOADS = {
     "full_decode_16": Workload("full_decode_16", 20_000_000, 2560, "bf16", 151_936, 16, 1, history=True),
     "full_decode_64": Workload("full_decode_64", 20_000_000, 2560, "bf16", 151_936, 64, 1, history=True),
     "full_decode_256": Workload("full_decode_256", 20_000_000, 2560, "bf16", 151_936, 256, 1, history=True),
+    # profiling case for full ncu captures: 400k x 2560 bf16 (2 GB), 4 x 2048 Zipf tokens
+    "profile_small": Workload("profile_small", 400_000, 2560, "bf16", 151_936, 4, 2048),
     # 20M x 2560 int8 + fp32 row scale (47.8 GiB), 65,536 uniform tokens (little reuse)
     "int8_uniform": Workload("int8_uniform", 20_000_000, 2560, "int8", 151_936, 16, 4096, tokens="uniform"),
 }

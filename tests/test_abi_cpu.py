@@ -1,0 +1,117 @@
+"""Host-side checks of libngram.so that need no GPU: the library loads, exports every
+entry point include/ngram.h declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import hashed_gram_embedding_ngram_b200 as ng
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ngram.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NGRAM_API\s+[\w\s\*]*?\b(ngram_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("ngram_init", "ngram_forward", "ngram_hash_indices", "ngram_fill_synthetic",
+              "ngram_get_device_error", "ngram_last_error", "ngram_status_string",
+              "ngram_destroy", "ngram_default_hash_params"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ng.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_library_exports_nothing_else():
+    out = os.popen("nm -D --defined-only %s" % ng.LIB_PATH).read().split("\n")
+    exported = sorted(l.split()[-1] for l in out if " T " in l)
+    assert exported == _declared()
+
+
+def test_status_strings():
+    assert ng.ngram_status_string(ng.NGRAM_OK) == "NGRAM_OK"
+    assert ng.ngram_status_string(ng.NGRAM_EDEVICE) == "NGRAM_EDEVICE"
+    assert ng.ngram_status_string(99) == "NGRAM_UNKNOWN"
+
+
+def test_default_hash_params():
+    hp = ng.ngram_default_hash_params()
+    assert (hp.base_seed, hp.n_bigram_heads, hp.n_trigram_heads, hp.pad_id, hp.vocab_size) == (
+        0x6E6772616D5F7631, 8, 8, 0x1FFFFF, 0x1FFFFF)
+
+
+_T = torch.zeros(64, dtype=torch.bfloat16)      # any 16-byte aligned host address
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(R=0), "R must"),
+    (dict(R=2**32), "R must"),
+    (dict(d=12), "d % 8"),
+    (dict(d=0), "d % 8"),
+    (dict(max_tokens=0), "max_tokens"),
+    (dict(hp=dict(n_bigram_heads=9, n_trigram_heads=8)), "heads"),
+    (dict(hp=dict(n_bigram_heads=0, n_trigram_heads=0)), "heads"),
+    (dict(hp=dict(pad_id=1 << 21)), "pad_id"),
+    (dict(hp=dict(vocab_size=1 << 21)), "vocab_size"),
+    (dict(hp=dict(vocab_size=0)), "vocab_size"),
+    (dict(hp=dict(flags=1)), "flags"),
+    (dict(dtype=7), "dtype"),
+    (dict(where=9), "residency"),
+    (dict(dtype=ng.NGRAM_INT8_ROWSCALE, d=32), "row_scale"),
+    (dict(d=264, max_tokens=2**31), "too large"),
+])
+def test_init_rejects_bad_arguments_before_cuda(kw, msg):
+    args = dict(R=1000, d=256, dtype=ng.NGRAM_BF16, where=ng.NGRAM_RES_HBM, max_tokens=16)
+    hpo = kw.pop("hp", None)
+    args.update(kw)
+    hp = ng.ngram_default_hash_params(**(hpo or {}))
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_init(_T, args["R"], args["d"], args["dtype"], args["where"], hp,
+                      args["max_tokens"])
+    assert ei.value.status == ng.NGRAM_EINVAL
+    assert msg in str(ei.value)
+
+
+def test_init_rejects_null_and_misaligned_table():
+    lib = ng.lib()
+    h = ctypes.c_void_p(123)
+    assert lib.ngram_init(ctypes.byref(h), None, None, 10, 8, 0, 0, None, 4) == ng.NGRAM_EINVAL
+    assert h.value is None                                  # *out reset on failure
+    addr = ctypes.c_void_p(_T.data_ptr() + 2)
+    assert lib.ngram_init(ctypes.byref(h), addr, None, 10, 8, 0, 0, None, 4) == ng.NGRAM_EINVAL
+    assert "aligned" in ng.ngram_last_error()
+
+
+def test_valid_init_without_a_gpu_reports_a_cuda_error():
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, None, 16)
+    assert ei.value.status in (ng.NGRAM_ECUDA, ng.NGRAM_ENOMEM)
+
+
+def test_fill_rejects_bad_arguments():
+    with pytest.raises(ng.NgramError):
+        ng.ngram_fill_synthetic(_T, 0, 8, stream=0)
+    with pytest.raises(ng.NgramError):
+        ng.ngram_fill_synthetic(_T, 10, 12, stream=0)
+    with pytest.raises(ng.NgramError):
+        ng.ngram_fill_synthetic(_T, 10, 32, ng.NGRAM_INT8_ROWSCALE, stream=0)   # no row_scale
+
+
+def test_null_context_is_rejected():
+    lib = ng.lib()
+    assert lib.ngram_forward(None, None, None, 1, 1, None, None, None, None) == ng.NGRAM_EINVAL
+    assert lib.ngram_hash_indices(None, None, None, 1, 1, None, None) == ng.NGRAM_EINVAL
+    assert lib.ngram_get_device_error(None, None, 0) == ng.NGRAM_EINVAL
+    lib.ngram_destroy(None)                                 # no-op

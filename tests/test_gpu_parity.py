@@ -1,0 +1,295 @@
+"""GPU parity: libngram.so (through the C ABI) against the CPU oracle, element by element.
+
+Indices and table values must match bit for bit.  Outputs must lie within 1 bf16 ulp
+of the oracle's fp32-accumulated result, and within 1 ulp plus the near-zero slack of
+its exact fp64 result (see parity_helpers).  Sizes: every token at the sizes the
+oracle finishes in seconds (tiny: 512 tokens; mid: all 8192 tokens), sampled tokens at
+the full 20M x 2560 size in the same launch configuration the benchmark times, and the
+edge cases of the method (boundaries, history, collisions, ragged shapes, in place).
+"""
+import numpy as np
+import pytest
+import torch
+
+import ngram_inputs as gen
+import oracle
+import hashed_gram_embedding_ngram_b200 as ng
+from parity_helpers import (N_CPU, TABLES, assert_parity, from_dev_bf16, parity_report,
+                            sample_tokens, to_dev_bf16, to_dev_tokens, workload_on_device)
+
+pytestmark = pytest.mark.gpu
+W = gen.WORKLOADS
+
+
+def _hp(vocab, nb=8, nt=8, **kw):
+    return ng.ngram_default_hash_params(vocab_size=vocab, n_bigram_heads=nb,
+                                        n_trigram_heads=nt, **kw)
+
+
+def _oracle(w, inp, sel=None, acc=oracle.ACC_F32, want_aux=False, **kw):
+    return oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"],
+                          R=w.R, d=w.d, dtype=oracle.BF16 if w.dtype == "bf16" else oracle.INT8,
+                          table_seed=gen.TABLE_SEED, sel=sel, acc=acc, n_threads=N_CPU,
+                          vocab_size=w.vocab, want_aux=want_aux, **kw)
+
+
+def _run(w, dev, inp_dev, ctx, out=None):
+    return ng.ngram_forward(ctx, inp_dev["tokens"], inp_dev["residual"], inp_dev["gate"],
+                            out=out, history=inp_dev["history"])
+
+
+def _ctx_for(w, dev, max_tokens=None):
+    dtype = ng.NGRAM_BF16 if w.dtype == "bf16" else ng.NGRAM_INT8_ROWSCALE
+    table, scale = TABLES.get(w.R, w.d, dtype, gen.TABLE_SEED, dev)
+    return ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, _hp(w.vocab),
+                         max_tokens or w.N, row_scale=scale)
+
+
+def _dummy_ctx(dev, R, d=8, vocab=0x1FFFFF, nb=8, nt=8, max_tokens=1 << 20):
+    """A context whose table is never read (index step only)."""
+    buf = torch.zeros(16, dtype=torch.bfloat16, device=dev)
+    ctx = ng.ngram_init(buf, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(vocab, nb, nt), max_tokens)
+    ctx._keep = buf
+    return ctx
+
+
+# --------------------------------------------------------------------------- table values
+def test_table_bitexact_every_row_tiny(cuda_device):
+    w = W["tiny"]
+    table, _ = TABLES.get(w.R, w.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    got = from_dev_bf16(table)
+    assert np.array_equal(got, oracle.fill_bf16(gen.TABLE_SEED, 0, w.R, w.d))
+
+
+def test_table_bitexact_int8_and_scale(cuda_device):
+    R, d = 3000, 512
+    q = torch.empty((R, d), dtype=torch.int8, device=cuda_device)
+    s = torch.empty((R,), dtype=torch.float32, device=cuda_device)
+    ng.ngram_fill_synthetic(q, R, d, ng.NGRAM_INT8_ROWSCALE, 12345, row_scale=s)
+    wq, ws = oracle.fill_int8(12345, 0, R, d)
+    assert np.array_equal(q.cpu().numpy(), wq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+
+
+# --------------------------------------------------------------------------- indices
+@pytest.mark.parametrize("name", ["tiny", "mid", "full_prefill", "full_decode_1",
+                                  "full_decode_16", "full_decode_64", "full_decode_256",
+                                  "int8_uniform"])
+def test_indices_bitexact(cuda_device, name):
+    w = W[name]
+    inp = gen.make_inputs(w)
+    ctx = _dummy_ctx(cuda_device, w.R, vocab=w.vocab, max_tokens=w.N)
+    got = ng.ngram_hash_indices(ctx, to_dev_tokens(inp["tokens"], cuda_device),
+                                to_dev_tokens(inp["history"], cuda_device))
+    want = oracle.indices(inp["tokens"], inp["history"], w.R, vocab_size=w.vocab)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 1 << 16, 1 << 31, 20_000_000, 4_294_967_291,
+                               4_294_967_295])
+def test_indices_exact_remainder_edge_R(cuda_device, R):
+    toks = gen.zipf_tokens(5, 97, 151_936, seed=21)
+    hist = gen.zipf_tokens(5, 2, 151_936, seed=22)
+    ctx = _dummy_ctx(cuda_device, R, vocab=151_936)
+    got = ng.ngram_hash_indices(ctx, to_dev_tokens(toks, cuda_device), to_dev_tokens(hist, cuda_device))
+    want = oracle.indices(toks, hist, R, vocab_size=151_936)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+
+
+@pytest.mark.parametrize("nb,nt", [(1, 0), (0, 1), (3, 5), (16, 0), (0, 16), (7, 9)])
+def test_indices_head_counts(cuda_device, nb, nt):
+    toks = gen.zipf_tokens(3, 50, 32_000, seed=23)
+    ctx = _dummy_ctx(cuda_device, 65_536, vocab=32_000, nb=nb, nt=nt)
+    got = ng.ngram_hash_indices(ctx, to_dev_tokens(toks, cuda_device))
+    want = oracle.indices(toks, None, 65_536, n_bigram=nb, n_trigram=nt, vocab_size=32_000)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+
+
+# --------------------------------------------------------------------------- forward
+def test_forward_tiny_every_token(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    r32 = assert_parity(got, _oracle(w, inp))
+    want64, _, mag, _ = _oracle(w, inp, acc=oracle.ACC_F64, want_aux=True)
+    assert_parity(got, want64, mag)
+    assert r32["exact"] == r32["n"]          # same operations in the same order
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
+def test_forward_mid_every_token(cuda_device):
+    w = W["mid"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    r = assert_parity(got, _oracle(w, inp))
+    assert r["exact"] == r["n"]
+
+
+def test_forward_full_prefill_sampled(cuda_device):
+    """Full size (20M x 2560, 32,768 tokens) in the benchmark's launch configuration;
+    1,024 sampled tokens (boundaries included) against the oracle."""
+    w = W["full_prefill"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx)).reshape(w.N, w.d)
+    sel = sample_tokens(w, 1024)
+    want, _, mag, idx = _oracle(w, inp, sel=sel, acc=oracle.ACC_F64, want_aux=True)
+    assert_parity(got[sel], want, mag)
+    assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    # the same sampled indices straight from the index step
+    gi = ng.ngram_hash_indices(ctx, dv["tokens"]).cpu().numpy().view(np.uint32)
+    assert np.array_equal(gi[sel], idx)
+
+
+@pytest.mark.parametrize("name", ["full_decode_1", "full_decode_16", "full_decode_64",
+                                  "full_decode_256"])
+def test_forward_full_decode_every_token(cuda_device, name):
+    w = W[name]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    r = assert_parity(got, _oracle(w, inp))
+    assert r["exact"] == r["n"]
+
+
+@pytest.mark.parametrize("d,nb,nt,n_seq,T,hist", [
+    (8, 8, 8, 3, 37, False),       # one column vector: 31 idle lanes per strip
+    (136, 3, 5, 2, 45, True),      # 17 vectors: ragged strip
+    (264, 16, 0, 1, 70, True),     # 33 vectors: a full strip plus one lane
+    (520, 0, 16, 5, 9, False),     # 65 vectors
+    (2568, 8, 8, 2, 33, True),     # 321 vectors: the pages' width plus a ragged tail
+    (256, 1, 0, 4, 16, False),     # single head: an embedding lookup
+])
+def test_forward_ragged_shapes_and_heads(cuda_device, d, nb, nt, n_seq, T, hist):
+    R, V = 4099, 5000
+    w = gen.Workload("ragged", R, d, "bf16", V, n_seq, T, history=hist)
+    inp = gen.make_inputs(w, token_seed=31)
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V, nb, nt), w.N)
+    dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device),
+          "history": to_dev_tokens(inp["history"], cuda_device),
+          "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
+          "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    want = _oracle(w, inp, n_bigram=nb, n_trigram=nt)
+    r = assert_parity(got, want)
+    assert r["exact"] == r["n"]
+
+
+def test_forward_collisions_R2(cuda_device):
+    """R = 2: every token's 16 heads collide on two rows; each head still counts."""
+    R, d, V = 2, 64, 100
+    w = gen.Workload("r2", R, d, "bf16", V, 2, 40)
+    inp = gen.make_inputs(w, token_seed=41)
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device), "history": None,
+          "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
+          "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    assert_parity(got, _oracle(w, inp))
+
+
+def test_forward_large_batch_small_rows(cuda_device):
+    """262,144 tokens (grid-stride loop wraps many times) at d = 256; sampled check."""
+    w = gen.Workload("bigN", 65_536, 256, "bf16", 32_000, 64, 4096)
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx)).reshape(w.N, w.d)
+    sel = sample_tokens(w, 4096)
+    assert_parity(got[sel], _oracle(w, inp, sel=sel))
+
+
+def test_in_place_equals_out_of_place(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    ref = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    buf = dv["residual"].clone()
+    ng.ngram_forward(ctx, dv["tokens"], buf, dv["gate"], out=buf)
+    assert np.array_equal(from_dev_bf16(buf), ref)
+
+
+def test_zero_gate_returns_residual_bitwise(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    out = ng.ngram_forward(ctx, dv["tokens"], dv["residual"], torch.zeros_like(dv["gate"]))
+    assert np.array_equal(from_dev_bf16(out), inp["residual"].reshape(w.N, w.d))
+
+
+def test_chunked_prefill_and_decode_bitexact(cuda_device):
+    """history = the two preceding tokens reproduces the full prefill exactly."""
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    full = from_dev_bf16(_run(w, cuda_device, dv, ctx)).reshape(w.n_seq, w.T, w.d)
+    toks = dv["tokens"]
+    res = dv["residual"].view(w.n_seq, w.T, w.d)
+    c = 50
+    a = ng.ngram_forward(ctx, toks[:, :c].contiguous(), res[:, :c].contiguous().view(-1, w.d), dv["gate"])
+    b = ng.ngram_forward(ctx, toks[:, c:].contiguous(), res[:, c:].contiguous().view(-1, w.d), dv["gate"],
+                         history=toks[:, c - 2:c].contiguous())
+    got = np.concatenate([from_dev_bf16(a).reshape(w.n_seq, c, w.d),
+                          from_dev_bf16(b).reshape(w.n_seq, w.T - c, w.d)], axis=1)
+    assert np.array_equal(got, full)
+    t = 77                                           # one decode step per sequence
+    step = ng.ngram_forward(ctx, toks[:, t:t + 1].contiguous(), res[:, t].contiguous(),
+                            dv["gate"], history=toks[:, t - 2:t].contiguous())
+    assert np.array_equal(from_dev_bf16(step).reshape(w.n_seq, w.d), full[:, t])
+
+
+def test_empty_batch_launches_nothing(cuda_device):
+    w = W["tiny"]
+    ctx = _ctx_for(w, cuda_device)
+    toks = torch.zeros((0, 5), dtype=torch.int32, device=cuda_device)
+    res = torch.zeros((0, w.d), dtype=torch.bfloat16, device=cuda_device)
+    gate = torch.ones(w.d, dtype=torch.float32, device=cuda_device)
+    out = ng.ngram_forward(ctx, toks, res, gate)
+    assert out.numel() == 0
+
+
+def test_argument_errors(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device, max_tokens=100)
+    with pytest.raises(ng.NgramError) as ei:                  # N > max_tokens
+        _run(w, cuda_device, dv, ctx)
+    assert ei.value.status == ng.NGRAM_EINVAL and "max_tokens" in str(ei.value)
+    # every pointer below stays inside its buffer, so even a call that slipped past
+    # the host checks would only touch memory it owns
+    lib = ng.lib()
+    base = dv["residual"].data_ptr()                           # 512 x 256 bf16
+    other = torch.empty((10, w.d), dtype=torch.bfloat16, device=cuda_device)
+    st = lib.ngram_forward(ctx.handle, dv["tokens"].data_ptr(), None, 1, 10, base + 2,
+                           dv["gate"].data_ptr(), other.data_ptr(), None)
+    assert st == ng.NGRAM_EINVAL and "aligned" in ng.ngram_last_error()
+    st = lib.ngram_forward(ctx.handle, dv["tokens"].data_ptr(), None, 1, 10, base,
+                           dv["gate"].data_ptr(), base + 16, None)
+    assert st == ng.NGRAM_EINVAL and "overlaps" in ng.ngram_last_error()
+    torch.cuda.synchronize()
+
+
+def test_bad_token_ids_flag_the_device_error_word(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+    toks = dv["tokens"].clone()
+    toks.view(-1)[300] = w.vocab + 5                          # out of vocabulary
+    out = ng.ngram_forward(ctx, toks, dv["residual"], dv["gate"])
+    st, info = ng.ngram_get_device_error(ctx, clear=True)
+    assert st == ng.NGRAM_EDEVICE and info[0] == 1 and info[2] == w.vocab + 5
+    assert info[1] == 300                                     # the position of the bad id
+    # the bad id reads as PAD: same result as the oracle with PAD there
+    t2 = inp["tokens"].copy()
+    t2.reshape(-1)[300] = oracle.DEFAULT_PAD_ID
+    inp2 = dict(inp, tokens=t2)
+    assert_parity(from_dev_bf16(out), _oracle(w, inp2))
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK   # cleared
+    hist = torch.full((w.n_seq, 2), -1, dtype=torch.int32, device=cuda_device)
+    ng.ngram_forward(ctx, dv["tokens"], dv["residual"], dv["gate"], history=hist)
+    st, info = ng.ngram_get_device_error(ctx, clear=True)
+    assert st == ng.NGRAM_EDEVICE and (info[1] & 0x80000000)
