@@ -162,8 +162,6 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (static_cast<uint64_t>(max_tokens) * n_strips > 0xFFFFFFFFull ||
         static_cast<uint64_t>(max_tokens) * NGRAM_MAX_HEADS > 0xFFFFFFFFull)
         return fail(NGRAM_EINVAL, "max_tokens %u too large for d = %u", max_tokens, d);
-    if (dtype != NGRAM_BF16)
-        return fail(NGRAM_EUNSUPPORTED, "int8 rows are not built yet");
     if (where != NGRAM_RES_HBM)
         return fail(NGRAM_EUNSUPPORTED, "host-resident tables are not built yet");
 
@@ -183,8 +181,11 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     cudaError_t e = cudaGetDevice(&c->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->gather_blocks_per_sm,
-                                                          k_gather_bf16<16>, 256, 0);
+        e = (dtype == NGRAM_BF16)
+                ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->gather_blocks_per_sm,
+                                                                k_gather_bf16<16>, 256, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->gather_blocks_per_sm,
+                                                                k_gather_int8<16>, 256, 0);
     if (e == cudaSuccess) e = cudaMalloc(&c->d_err, 4 * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, 4 * sizeof(uint32_t));
     if (e != cudaSuccess) {
@@ -228,7 +229,8 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
     g.T = T;
     g.N = static_cast<uint32_t>(N);
     g.d = c->d;
-    g.n_strips = (c->d / 8 + 31) / 32;
+    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;
+    g.n_strips = (c->d / cols_per_lane + 31) / 32;
     const uint32_t resident_warps = static_cast<uint32_t>(c->num_sms) * c->gather_blocks_per_sm * 8u;
     // Few tokens: one strip per warp (lowest latency).  Many: a warp keeps its token.
     g.strips_per_item = (static_cast<uint64_t>(N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
@@ -239,12 +241,16 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
     if (blocks > max_blocks) blocks = max_blocks;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (g.h.n_heads == 16)
-        k_gather_bf16<16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(g);
-    else
-        k_gather_bf16<0><<<static_cast<unsigned>(blocks), 256, 0, s>>>(g);
+    const unsigned nb = static_cast<unsigned>(blocks);
+    if (c->dtype == NGRAM_BF16) {
+        if (g.h.n_heads == 16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g);
+        else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
+    } else {
+        if (g.h.n_heads == 16) k_gather_int8<16><<<nb, 256, 0, s>>>(g);
+        else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
+    }
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "k_gather_bf16 launch");
+    if (e != cudaSuccess) return cuda_fail(e, "gather kernel launch");
     return NGRAM_OK;
 }
 

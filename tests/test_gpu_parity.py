@@ -293,3 +293,42 @@ def test_bad_token_ids_flag_the_device_error_word(cuda_device):
     ng.ngram_forward(ctx, dv["tokens"], dv["residual"], dv["gate"], history=hist)
     st, info = ng.ngram_get_device_error(ctx, clear=True)
     assert st == ng.NGRAM_EDEVICE and (info[1] & 0x80000000)
+
+
+# --------------------------------------------------------------------------- int8 rows
+@pytest.mark.parametrize("d,nb,nt,n_seq,T,hist", [
+    (16, 8, 8, 3, 37, False),      # one 16-column vector per row
+    (272, 3, 5, 2, 45, True),      # 17 vectors: ragged strip
+    (528, 16, 0, 1, 70, True),     # 33 vectors
+    (2560, 8, 8, 2, 60, True),     # the pages' width
+    (2576, 0, 16, 3, 11, False),   # 161 vectors: ragged tail
+])
+def test_forward_int8_every_token(cuda_device, d, nb, nt, n_seq, T, hist):
+    R, V = 5003, 7000
+    w = gen.Workload("int8_ragged", R, d, "int8", V, n_seq, T, history=hist)
+    inp = gen.make_inputs(w, token_seed=51)
+    table, scale = TABLES.get(R, d, ng.NGRAM_INT8_ROWSCALE, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_INT8_ROWSCALE, ng.NGRAM_RES_HBM, _hp(V, nb, nt),
+                        w.N, row_scale=scale)
+    dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device),
+          "history": to_dev_tokens(inp["history"], cuda_device),
+          "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
+          "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    r = assert_parity(got, _oracle(w, inp, n_bigram=nb, n_trigram=nt))
+    assert r["exact"] == r["n"]
+    want64, _, mag, _ = _oracle(w, inp, acc=oracle.ACC_F64, want_aux=True, n_bigram=nb,
+                                n_trigram=nt)
+    assert_parity(got, want64, mag)
+
+
+def test_forward_int8_full_sampled(cuda_device):
+    """20M x 2560 int8 + row scales (47.8 GiB), 65,536 uniform tokens; 1,024 sampled."""
+    w = W["int8_uniform"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx)).reshape(w.N, w.d)
+    sel = sample_tokens(w, 1024)
+    r = assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    assert r["exact"] == r["n"]
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
