@@ -31,6 +31,9 @@ NGRAM_BF16, NGRAM_INT8_ROWSCALE = 0, 1
 # ngram_residency
 NGRAM_RES_HBM, NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO = 0, 1, 2, 3
 
+NGRAM_FLAG_DEDUP = 0x1
+NGRAM_FLAG_TMA_STAGING = 0x2
+
 MAX_HEADS = 16
 DEFAULT_BASE_SEED = 0x6E6772616D5F7631
 DEFAULT_PAD_ID = 0x1FFFFF
@@ -74,6 +77,16 @@ _lib.ngram_status_string.argtypes = [_i32]
 _lib.ngram_status_string.restype = ctypes.c_char_p
 _lib.ngram_destroy.argtypes = [_P]
 _lib.ngram_destroy.restype = None
+_lib.ngram_host_alloc.argtypes = [ctypes.POINTER(_P), _u64]
+_lib.ngram_host_alloc.restype = _i32
+_lib.ngram_host_free.argtypes = [_P]
+_lib.ngram_host_free.restype = _i32
+_lib.ngram_set_wait_timeout.argtypes = [_P, _u32]
+_lib.ngram_set_wait_timeout.restype = _i32
+_lib.ngram_auto_choice.argtypes = [_P, _u32, ctypes.POINTER(ctypes.c_int)]
+_lib.ngram_auto_choice.restype = _i32
+_lib.ngram_dedup_rows.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
+_lib.ngram_dedup_rows.restype = _i32
 
 
 def lib() -> ctypes.CDLL:
@@ -224,3 +237,73 @@ def ngram_destroy(ctx: Context) -> None:
     if ctx.handle:
         _lib.ngram_destroy(ctx.handle)
         ctx.handle = None
+
+
+class HostTable:
+    """Pinned, device-mapped host memory from ngram_host_alloc, viewed as a torch CPU
+    tensor (no copy).  The view must not outlive close()."""
+
+    def __init__(self, shape, dtype: torch.dtype):
+        n = 1
+        for x in shape:
+            n *= int(x)
+        self.nbytes = n * torch.empty((), dtype=dtype).element_size()
+        self.ptr = ngram_host_alloc(self.nbytes)
+        buf = (ctypes.c_uint8 * self.nbytes).from_address(self.ptr)
+        self.tensor = torch.frombuffer(buf, dtype=torch.uint8).view(dtype).view(*shape)
+
+    def close(self):
+        if self.ptr:
+            self.tensor = None
+            ngram_host_free(self.ptr)
+            self.ptr = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ngram_host_alloc(nbytes: int) -> int:
+    """Address of nbytes of pinned, device-mapped host memory."""
+    p = ctypes.c_void_p()
+    _check(_lib.ngram_host_alloc(ctypes.byref(p), nbytes))
+    return p.value
+
+
+def ngram_host_free(ptr: int) -> None:
+    _check(_lib.ngram_host_free(ctypes.c_void_p(ptr)))
+
+
+def ngram_set_wait_timeout(ctx: Context, ms: int) -> None:
+    _check(_lib.ngram_set_wait_timeout(ctx.handle, ms))
+
+
+def ngram_auto_choice(ctx: Context, n_tokens: int) -> int:
+    w = ctypes.c_int()
+    _check(_lib.ngram_auto_choice(ctx.handle, n_tokens, ctypes.byref(w)))
+    return w.value
+
+
+def ngram_dedup_rows(ctx: Context, tokens: torch.Tensor, history: torch.Tensor | None = None,
+                     uniq_out=None, inv_out=None, count_out=None, stream=None):
+    """(uniq [N*H], inv [N*H], count [1]) int32 tensors holding uint32 values: the
+    batch's distinct rows in order of first appearance (entries [0, count)) and the
+    inverse map."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    n_seq, T = tokens.shape
+    M = n_seq * T * ctx.n_heads
+    dev = tokens.device
+    if history is not None:
+        _need(history, "history", torch.int32, dev, ndim=2)
+    if uniq_out is None:
+        uniq_out = torch.empty(M, dtype=torch.int32, device=dev)
+    if inv_out is None:
+        inv_out = torch.empty(M, dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(_lib.ngram_dedup_rows(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                                 _ptr(uniq_out), _ptr(inv_out), _ptr(count_out),
+                                 _stream(stream)))
+    return uniq_out, inv_out, count_out

@@ -27,7 +27,7 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo",
-    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden,-fopenmp",
     "-Xptxas", "-v",
     "-shared",
 ]
@@ -59,7 +59,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *_sources()]
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *_sources(), "-lgomp"]
     p = subprocess.run(cmd, capture_output=True, text=True)
     with open(os.path.join(BUILD_DIR, "ptxas.txt"), "w") as f:
         f.write(" ".join(cmd) + "\n" + p.stdout + p.stderr)

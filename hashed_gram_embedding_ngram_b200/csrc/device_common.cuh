@@ -110,12 +110,22 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 }
 
 // 16-byte read-only load that does not allocate in L1 (rows and residual are read
-// once per use; reuse across tokens is left to L2).
+// once per use; reuse across tokens is left to L2).  NGRAM_ROW_LOAD_HINT = 1 (default)
+// adds an L2 256-byte prefetch hint, measured ~0.3% faster on the full-size gather.
+#ifndef NGRAM_ROW_LOAD_HINT
+#define NGRAM_ROW_LOAD_HINT 1
+#endif
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     uint4 r;
+#if NGRAM_ROW_LOAD_HINT == 1
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+#else
     asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
+#endif
     return r;
 }
 

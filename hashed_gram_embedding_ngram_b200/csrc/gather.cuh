@@ -32,6 +32,7 @@ struct GatherArgs {
     const uint16_t *residual;   // [N][d] bf16 bits
     const float *gate;          // [d]
     uint16_t *out;              // [N][d] bf16 bits (may alias residual)
+    const uint32_t *row_ids;    // [N][H] precomputed row ids into `table`, or null (hash)
     uint32_t *err;              // device error word
     uint32_t T;
     uint32_t N;
@@ -51,20 +52,30 @@ __device__ __forceinline__ uint4 ld_na_v4(const void *p) {
     return r;
 }
 
-// Row indices of the warp's token, one head per lane (lanes >= H hold 0).
+// Row indices of the warp's token, one head per lane (lanes >= H hold 0): hashed
+// from the context, or read from precomputed ids (dedup'ed / staged paths, where
+// `table` is the staging buffer and row_ids the inverse map).
 __device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t tok,
                                                   uint32_t lane, uint32_t H) {
     uint32_t row = 0;
     if (lane < H) {
-        uint32_t w0, w1, w2;
-        token_context(g.tokens, g.history, tok, g.T, g.h, g.err, w0, w1, w2);
-        row = head_row(lane, w0, w1, w2, g.h);
+        if (g.row_ids != nullptr) {
+            row = __ldg(g.row_ids + static_cast<size_t>(tok) * H + lane);
+        } else {
+            uint32_t w0, w1, w2;
+            token_context(g.tokens, g.history, tok, g.T, g.h, g.err, w0, w1, w2);
+            row = head_row(lane, w0, w1, w2, g.h);
+        }
     }
     return row;
 }
 
+#ifndef NGRAM_LDG_MIN_BLOCKS          // resident CTAs per SM the register budget targets
+#define NGRAM_LDG_MIN_BLOCKS 2
+#endif
+
 template <int kH>   // compile-time head count (16), or 0: runtime g.h.n_heads <= 16
-__global__ void __launch_bounds__(256, 2) k_gather_bf16(const GatherArgs g) {
+__global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const GatherArgs g) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;

@@ -1,13 +1,18 @@
 // ngram_api.cu -- host side of libngram.so: argument checks, context, launches.
 //
 // Every entry point validates its arguments before touching CUDA and reports through
-// an ngram_status; nothing here aborts the process.  All compute is asynchronous on
-// the caller's stream.  The operation and the definitions it follows are stated in
+// an ngram_status; nothing here aborts the process.  Compute is asynchronous on the
+// caller's stream, except where a residency mode needs the host in the loop (DMA
+// staging, the first AUTO call of a batch-size bucket); those waits are bounded and
+// return NGRAM_ETIMEOUT.  The operation and its definitions are stated in
 // include/ngram.h.
+#include <algorithm>
+#include <chrono>
+#include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <cstdarg>
 #include <string>
+#include <thread>
 
 #include <cuda_runtime.h>
 
@@ -15,23 +20,72 @@
 #include "device_common.cuh"
 #include "fill.cuh"
 #include "gather.cuh"
+#include "gather_bulk.cuh"
+#include "dedup.cuh"
 
 using namespace ngram;
 
+// Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
+//   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
+//     strips of a token run on 10 warps at once (455 us) instead of one warp walking
+//     them (470 us); the 16 hashes are recomputed per strip, which the issue slots absorb.
+//   The TMA-staged kernel (NGRAM_FLAG_TMA_STAGING) measured 522-895 us depending on
+//     chunk and ring depth; its tunables are below.
+#ifndef NGRAM_SPI_ALWAYS_ONE
+#define NGRAM_SPI_ALWAYS_ONE 1
+#endif
+#ifndef NGRAM_BULK_CHUNK_COLS           // columns per work item of the bulk kernel
+#define NGRAM_BULK_CHUNK_COLS 1280
+#endif
+#ifndef NGRAM_BULK_SMEM_BYTES           // shared memory per CTA for the stage ring
+#define NGRAM_BULK_SMEM_BYTES (100 * 1024)
+#endif
+#ifndef NGRAM_BULK_CTAS_PER_SM
+#define NGRAM_BULK_CTAS_PER_SM 2
+#endif
+#ifndef NGRAM_UVA_CTAS_PER_SM           // host-resident (UVA) gather grid, CTAs per SM
+#define NGRAM_UVA_CTAS_PER_SM 2
+#endif
+#ifndef NGRAM_DMA_CHUNK_BYTES           // host gather -> H2D pipelining granularity
+#define NGRAM_DMA_CHUNK_BYTES (8u << 20)
+#endif
+
 struct ngram_ctx {
-    const void *table;
+    const void *table;          // caller's pointer (device, or host for host residency)
+    const void *table_dev;      // device-visible alias used by kernels (UVA), or table
     const float *row_scale;
+    const float *row_scale_dev;
     uint64_t R;
     uint32_t d;
+    uint32_t row_bytes;         // 2d (bf16) or d (int8)
     ngram_dtype dtype;
     ngram_residency where;
     ngram_hash_params hp;
+    uint32_t H;
     uint32_t max_tokens;
     uint64_t barrett_m;
     int device;
     int num_sms;
     int gather_blocks_per_sm;
-    uint32_t *d_err;            // 4 words, owned
+    int bulk_smem_set;
+    uint32_t wait_ms;           // bound of every host-side wait
+    uint32_t *d_err;            // 4 words
+    // dedup scratch, sized for max_tokens (allocated on first use)
+    uint32_t dd_cap;            // entries (max_tokens * H)
+    uint32_t dd_pcap;           // hash-table slots (power of two >= 2 * dd_cap)
+    uint32_t *d_idx, *d_slot, *d_pos, *d_inv, *d_uniq, *d_keys, *d_first, *d_uid, *d_bsum, *d_count;
+    // staging of unique rows (HBM dedup, DMA), sized for dd_cap rows
+    uint8_t *d_stage;
+    float *d_stage_scale;
+    uint8_t *h_stage;           // pinned (DMA)
+    float *h_stage_scale;
+    uint32_t *h_uniq;           // pinned (DMA)
+    uint32_t *h_count;          // pinned (DMA)
+    cudaEvent_t ev_sync;        // D2H of the unique-row list
+    cudaEvent_t ev_stage_free;  // last H2D of the previous DMA call
+    int stage_in_use;
+    cudaEvent_t ev_t0, ev_t1;   // AUTO timing
+    int auto_choice[33];        // per ceil(log2 N): 0 undecided, else ngram_residency
 };
 
 namespace {
@@ -53,7 +107,25 @@ ngram_status cuda_fail(cudaError_t e, const char *what) {
                 cudaGetErrorString(e), cudaGetErrorName(e));
 }
 
+#define NG_CUDA(call, what)                                  \
+    do {                                                     \
+        cudaError_t e_ = (call);                             \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what);   \
+    } while (0)
+
+#define NG_CHECK(expr)                                       \
+    do {                                                     \
+        ngram_status s_ = (expr);                            \
+        if (s_ != NGRAM_OK) return s_;                       \
+    } while (0)
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint32_t ceil_log2(uint64_t x) {
+    uint32_t k = 0;
+    while ((1ull << k) < x) ++k;
+    return k;
+}
 
 ngram_status check_hash_params(const ngram_hash_params &hp) {
     const uint32_t H = hp.n_bigram_heads + hp.n_trigram_heads;
@@ -65,8 +137,8 @@ ngram_status check_hash_params(const ngram_hash_params &hp) {
         return fail(NGRAM_EINVAL, "pad_id %u does not fit in %u bits", hp.pad_id, NGRAM_TOKEN_BITS);
     if (hp.vocab_size == 0 || hp.vocab_size > kTokenMask)
         return fail(NGRAM_EINVAL, "vocab_size must be in [1, 2^21 - 1], got %u", hp.vocab_size);
-    if (hp.flags != 0 || hp.reserved != 0)
-        return fail(NGRAM_EINVAL, "flags/reserved must be 0");
+    if ((hp.flags & ~NGRAM_FLAGS_KNOWN) != 0 || hp.reserved != 0)
+        return fail(NGRAM_EINVAL, "unknown flags 0x%x / reserved must be 0", hp.flags);
     return NGRAM_OK;
 }
 
@@ -76,13 +148,12 @@ HashArgs hash_args(const ngram_ctx *c) {
     a.R = c->R;
     a.barrett_m = c->barrett_m;
     a.n_bigram = c->hp.n_bigram_heads;
-    a.n_heads = c->hp.n_bigram_heads + c->hp.n_trigram_heads;
+    a.n_heads = c->H;
     a.pad_id = c->hp.pad_id;
     a.vocab = c->hp.vocab_size;
     return a;
 }
 
-// Common checks of the token batch of one call.
 ngram_status check_batch(const ngram_ctx *c, const int32_t *tokens, uint32_t n_seq, uint32_t T,
                          uint64_t *N_out) {
     if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
@@ -94,10 +165,313 @@ ngram_status check_batch(const ngram_ctx *c, const int32_t *tokens, uint32_t n_s
                     static_cast<unsigned long long>(N), c->max_tokens);
     if (tokens == nullptr) return fail(NGRAM_EINVAL, "tokens is NULL");
     int cur = -1;
-    cudaError_t e = cudaGetDevice(&cur);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    NG_CUDA(cudaGetDevice(&cur), "cudaGetDevice");
     if (cur != c->device)
         return fail(NGRAM_EINVAL, "current device %d is not the context's device %d", cur, c->device);
+    return NGRAM_OK;
+}
+
+// Wait for an event with the context's bound; the GPU is never waited on without one.
+ngram_status wait_event(const ngram_ctx *c, cudaEvent_t ev, const char *what) {
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t e = cudaEventQuery(ev);
+        if (e == cudaSuccess) return NGRAM_OK;
+        if (e != cudaErrorNotReady) return cuda_fail(e, what);
+        const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                            std::chrono::steady_clock::now() - t0).count();
+        if (ms > static_cast<long long>(c->wait_ms))
+            return fail(NGRAM_ETIMEOUT, "%s: no completion within %u ms", what, c->wait_ms);
+        std::this_thread::yield();
+    }
+}
+
+void free_all(ngram_ctx *c) {
+    uint32_t *dev32[] = {c->d_err, c->d_idx, c->d_slot, c->d_pos, c->d_inv, c->d_uniq,
+                         c->d_keys, c->d_first, c->d_uid, c->d_bsum, c->d_count};
+    for (uint32_t *p : dev32)
+        if (p) cudaFree(p);
+    if (c->d_stage) cudaFree(c->d_stage);
+    if (c->d_stage_scale) cudaFree(c->d_stage_scale);
+    if (c->h_stage) cudaFreeHost(c->h_stage);
+    if (c->h_stage_scale) cudaFreeHost(c->h_stage_scale);
+    if (c->h_uniq) cudaFreeHost(c->h_uniq);
+    if (c->h_count) cudaFreeHost(c->h_count);
+    cudaEvent_t evs[] = {c->ev_sync, c->ev_stage_free, c->ev_t0, c->ev_t1};
+    for (cudaEvent_t e : evs)
+        if (e) cudaEventDestroy(e);
+}
+
+// ---------------------------------------------------------------- scratch on first use
+ngram_status ensure_dedup_scratch(ngram_ctx *c) {
+    if (c->d_idx) return NGRAM_OK;
+    const uint32_t M = c->dd_cap, P = c->dd_pcap, NB = (M + kScanBlock - 1) / kScanBlock;
+    NG_CUDA(cudaMalloc(&c->d_idx, M * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_slot, M * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_pos, M * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_inv, M * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_uniq, M * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_keys, P * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_first, P * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_uid, P * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_bsum, NB * 4ull), "dedup scratch");
+    NG_CUDA(cudaMalloc(&c->d_count, 4), "dedup scratch");
+    return NGRAM_OK;
+}
+
+ngram_status ensure_device_stage(ngram_ctx *c) {
+    if (c->d_stage) return NGRAM_OK;
+    NG_CUDA(cudaMalloc(&c->d_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging");
+    if (c->dtype == NGRAM_INT8_ROWSCALE)
+        NG_CUDA(cudaMalloc(&c->d_stage_scale, c->dd_cap * 4ull), "staging");
+    return NGRAM_OK;
+}
+
+ngram_status ensure_host_stage(ngram_ctx *c) {
+    if (c->h_stage) return NGRAM_OK;
+    NG_CHECK(ensure_device_stage(c));
+    NG_CUDA(cudaHostAlloc(&c->h_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes,
+                          cudaHostAllocPortable), "pinned staging");
+    if (c->dtype == NGRAM_INT8_ROWSCALE)
+        NG_CUDA(cudaHostAlloc(&c->h_stage_scale, c->dd_cap * 4ull, cudaHostAllocPortable),
+                "pinned staging");
+    NG_CUDA(cudaHostAlloc(&c->h_uniq, c->dd_cap * 4ull, cudaHostAllocPortable), "pinned staging");
+    NG_CUDA(cudaHostAlloc(&c->h_count, 4, cudaHostAllocPortable), "pinned staging");
+    NG_CUDA(cudaEventCreateWithFlags(&c->ev_sync, cudaEventDisableTiming), "cudaEventCreate");
+    NG_CUDA(cudaEventCreateWithFlags(&c->ev_stage_free, cudaEventDisableTiming), "cudaEventCreate");
+    return NGRAM_OK;
+}
+
+// ---------------------------------------------------------------- launch helpers
+GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t *history,
+                       uint32_t T, uint32_t N, const uint16_t *residual, const float *gate,
+                       uint16_t *out) {
+    GatherArgs g;
+    g.h = hash_args(c);
+    g.table = c->table_dev;
+    g.row_scale = c->row_scale_dev;
+    g.tokens = tokens;
+    g.history = history;
+    g.residual = residual;
+    g.gate = gate;
+    g.out = out;
+    g.row_ids = nullptr;
+    g.err = c->d_err;
+    g.T = T;
+    g.N = N;
+    g.d = c->d;
+    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;
+    g.n_strips = (c->d / cols_per_lane + 31) / 32;
+    g.strips_per_item = g.n_strips;
+    g.groups_per_token = 1;
+    return g;
+}
+
+// The TMA-staged bf16 gather: work items are (token, column chunk); S stages of
+// (H + 1) row chunks each fill the shared-memory budget.
+ngram_status launch_bulk(ngram_ctx *c, GatherArgs &g, cudaStream_t s) {
+    BulkPlan p;
+    uint32_t chunk = NGRAM_BULK_CHUNK_COLS < c->d ? NGRAM_BULK_CHUNK_COLS : c->d;
+    chunk = (chunk + 7u) & ~7u;
+    p.chunk_cols = chunk;
+    p.n_chunks = (c->d + chunk - 1) / chunk;
+    const uint32_t H = g.h.n_heads;
+    p.stage_bytes = ((H + 1u) * chunk * 2u + 127u) & ~127u;
+    uint32_t stages = (NGRAM_BULK_SMEM_BYTES - 128u) / p.stage_bytes;
+    if (stages > kBulkMaxStages) stages = kBulkMaxStages;
+    if (stages < 2) return fail(NGRAM_EUNSUPPORTED, "bulk gather: stage of %u bytes too large", p.stage_bytes);
+    p.stages = stages;
+    const uint32_t smem = stages * p.stage_bytes + 128u;      // + alignment slack
+    uint32_t threads = ((chunk / 8u) + 31u) & ~31u;
+    if (threads > 512u) threads = 512u;
+    const uint64_t items = static_cast<uint64_t>(g.N) * p.n_chunks;
+    uint64_t grid = static_cast<uint64_t>(c->num_sms) * NGRAM_BULK_CTAS_PER_SM;
+    if (grid > items) grid = items;
+    if (!c->bulk_smem_set) {
+        NG_CUDA(cudaFuncSetAttribute(k_gather_bf16_bulk<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     NGRAM_BULK_SMEM_BYTES), "cudaFuncSetAttribute (bulk gather)");
+        NG_CUDA(cudaFuncSetAttribute(k_gather_bf16_bulk<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     NGRAM_BULK_SMEM_BYTES), "cudaFuncSetAttribute (bulk gather)");
+        c->bulk_smem_set = 1;
+    }
+    if (H == 16) k_gather_bf16_bulk<16><<<static_cast<unsigned>(grid), threads, smem, s>>>(g, p);
+    else k_gather_bf16_bulk<0><<<static_cast<unsigned>(grid), threads, smem, s>>>(g, p);
+    NG_CUDA(cudaGetLastError(), "k_gather_bf16_bulk launch");
+    return NGRAM_OK;
+}
+
+// The register gather (bf16 or int8); ctas_per_sm bounds the persistent grid.
+ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint32_t ctas_per_sm) {
+    const uint32_t resident_warps = static_cast<uint32_t>(c->num_sms) * ctas_per_sm * 8u;
+    g.strips_per_item = (NGRAM_SPI_ALWAYS_ONE ||
+                         static_cast<uint64_t>(g.N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
+    g.groups_per_token = (g.n_strips + g.strips_per_item - 1) / g.strips_per_item;
+    const uint64_t items = static_cast<uint64_t>(g.N) * g.groups_per_token;
+    const uint64_t max_blocks = static_cast<uint64_t>(c->num_sms) * ctas_per_sm;
+    uint64_t blocks = (items + 7) / 8;
+    if (blocks > max_blocks) blocks = max_blocks;
+    const unsigned nb = static_cast<unsigned>(blocks);
+    if (c->dtype == NGRAM_BF16) {
+        if (g.h.n_heads == 16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g);
+        else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
+    } else {
+        if (g.h.n_heads == 16) k_gather_int8<16><<<nb, 256, 0, s>>>(g);
+        else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
+    }
+    NG_CUDA(cudaGetLastError(), "gather kernel launch");
+    return NGRAM_OK;
+}
+
+unsigned grid_for(const ngram_ctx *c, uint64_t work, uint32_t per_block) {
+    uint64_t b = (work + per_block - 1) / per_block;
+    const uint64_t cap = static_cast<uint64_t>(c->num_sms) * 8;
+    if (b > cap) b = cap;
+    if (b == 0) b = 1;
+    return static_cast<unsigned>(b);
+}
+
+ngram_status launch_hash(ngram_ctx *c, const int32_t *tokens, const int32_t *history, uint32_t T,
+                         uint32_t N, uint32_t *idx_out, cudaStream_t s) {
+    const HashArgs a = hash_args(c);
+    k_hash_indices<<<grid_for(c, static_cast<uint64_t>(N) * a.n_heads, 256), 256, 0, s>>>(
+        a, tokens, history, T, N, c->d_err, idx_out);
+    NG_CUDA(cudaGetLastError(), "k_hash_indices launch");
+    return NGRAM_OK;
+}
+
+// Dedup idx[M] (device) into uniq/inv/count (device) with the context's scratch.
+ngram_status launch_dedup(ngram_ctx *c, const uint32_t *idx, uint32_t M, uint32_t *uniq,
+                          uint32_t *inv, uint32_t *count, cudaStream_t s) {
+    const uint32_t log2p = std::max<uint32_t>(10u, ceil_log2(2ull * M));
+    const uint32_t P = 1u << log2p;
+    const uint32_t NB = (M + kScanBlock - 1) / kScanBlock;
+    NG_CUDA(cudaMemsetAsync(c->d_keys, 0xFF, P * 4ull, s), "dedup clear");
+    NG_CUDA(cudaMemsetAsync(c->d_first, 0xFF, P * 4ull, s), "dedup clear");
+    const unsigned gm = grid_for(c, M, 256);
+    k_dedup_insert<<<gm, 256, 0, s>>>(idx, M, c->d_keys, c->d_first, c->d_slot, log2p);
+    k_dedup_scan_local<<<NB, 256, 0, s>>>(c->d_slot, c->d_first, M, c->d_pos, c->d_bsum);
+    k_dedup_scan_blocks<<<1, 1024, 0, s>>>(c->d_bsum, NB, count);
+    k_dedup_emit<<<gm, 256, 0, s>>>(idx, c->d_slot, c->d_first, c->d_pos, c->d_bsum, M, uniq, c->d_uid);
+    k_dedup_inverse<<<gm, 256, 0, s>>>(c->d_slot, c->d_uid, M, inv);
+    NG_CUDA(cudaGetLastError(), "dedup launch");
+    return NGRAM_OK;
+}
+
+// ---------------------------------------------------------------- forward paths
+struct Call {
+    const int32_t *tokens, *history;
+    uint32_t T, N;
+    const uint16_t *residual;
+    const float *gate;
+    uint16_t *out;
+    cudaStream_t s;
+};
+
+ngram_status forward_direct(ngram_ctx *c, const Call &k, uint32_t ctas_per_sm) {
+    GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
+    if ((c->hp.flags & NGRAM_FLAG_TMA_STAGING) && c->dtype == NGRAM_BF16 && c->where == NGRAM_RES_HBM)
+        return launch_bulk(c, g, k.s);
+    return launch_gather(c, g, k.s, ctas_per_sm);
+}
+
+// hash -> dedup -> compact the unique rows into HBM staging -> gather from staging.
+ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
+    NG_CHECK(ensure_dedup_scratch(c));
+    NG_CHECK(ensure_device_stage(c));
+    const uint32_t M = k.N * c->H;
+    NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
+    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
+    k_compact_rows<<<grid_for(c, M * 32ull, 256), 256, 0, k.s>>>(
+        static_cast<const uint8_t *>(c->table_dev), c->row_scale_dev, c->d_uniq, c->d_count,
+        c->row_bytes, c->d_stage, c->d_stage_scale);
+    NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
+    GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
+    g.table = c->d_stage;
+    g.row_scale = c->d_stage_scale;
+    g.row_ids = c->d_inv;
+    return launch_gather(c, g, k.s, static_cast<uint32_t>(c->gather_blocks_per_sm));
+}
+
+// Host-resident, copy-engine path: the unique rows are compacted by host threads
+// into pinned staging and moved to HBM by cudaMemcpyAsync in chunks (the copy of
+// chunk i overlaps the host gather of chunk i+1), then gathered from HBM.
+ngram_status forward_dma(ngram_ctx *c, const Call &k) {
+    NG_CHECK(ensure_dedup_scratch(c));
+    NG_CHECK(ensure_host_stage(c));
+    const uint32_t M = k.N * c->H;
+    NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
+    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
+    if (c->stage_in_use) NG_CHECK(wait_event(c, c->ev_stage_free, "DMA: previous staging copy"));
+    NG_CUDA(cudaMemcpyAsync(c->h_count, c->d_count, 4, cudaMemcpyDeviceToHost, k.s), "D2H count");
+    NG_CUDA(cudaMemcpyAsync(c->h_uniq, c->d_uniq, M * 4ull, cudaMemcpyDeviceToHost, k.s), "D2H rows");
+    NG_CUDA(cudaEventRecord(c->ev_sync, k.s), "cudaEventRecord");
+    NG_CHECK(wait_event(c, c->ev_sync, "DMA: unique-row list"));
+    const uint32_t U = *c->h_count;
+    if (U > M) return fail(NGRAM_ECUDA, "DMA: unique count %u exceeds %u entries", U, M);
+    for (uint32_t u = 0; u < U; ++u)        // host threads read the table: check every row id
+        if (c->h_uniq[u] >= c->R)
+            return fail(NGRAM_ECUDA, "DMA: row id %u out of range %llu", c->h_uniq[u],
+                        static_cast<unsigned long long>(c->R));
+    const uint8_t *table = static_cast<const uint8_t *>(c->table);
+    const uint32_t rb = c->row_bytes;
+    const uint32_t chunk_rows = std::max<uint32_t>(1u, NGRAM_DMA_CHUNK_BYTES / rb);
+    for (uint32_t r0 = 0; r0 < U; r0 += chunk_rows) {
+        const uint32_t r1 = std::min(U, r0 + chunk_rows);
+#pragma omp parallel for schedule(static) if (r1 - r0 >= 256)
+        for (int64_t u = r0; u < static_cast<int64_t>(r1); ++u) {
+            memcpy(c->h_stage + static_cast<size_t>(u) * rb,
+                   table + static_cast<size_t>(c->h_uniq[u]) * rb, rb);
+            if (c->h_stage_scale) c->h_stage_scale[u] = c->row_scale[c->h_uniq[u]];
+        }
+        NG_CUDA(cudaMemcpyAsync(c->d_stage + static_cast<size_t>(r0) * rb,
+                                c->h_stage + static_cast<size_t>(r0) * rb,
+                                static_cast<size_t>(r1 - r0) * rb, cudaMemcpyHostToDevice, k.s),
+                "H2D staging");
+    }
+    if (c->h_stage_scale && U > 0)
+        NG_CUDA(cudaMemcpyAsync(c->d_stage_scale, c->h_stage_scale, U * 4ull, cudaMemcpyHostToDevice, k.s),
+                "H2D scales");
+    NG_CUDA(cudaEventRecord(c->ev_stage_free, k.s), "cudaEventRecord");
+    c->stage_in_use = 1;
+    GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
+    g.table = c->d_stage;
+    g.row_scale = c->d_stage_scale;
+    g.row_ids = c->d_inv;
+    return launch_gather(c, g, k.s, static_cast<uint32_t>(c->gather_blocks_per_sm));
+}
+
+ngram_status forward_uva(ngram_ctx *c, const Call &k) {
+    const uint32_t per_sm = std::min<uint32_t>(NGRAM_UVA_CTAS_PER_SM, c->gather_blocks_per_sm);
+    return forward_direct(c, k, per_sm);
+}
+
+// AUTO: the first call of each batch-size bucket runs and times both host modes
+// (both write the same output), keeps the faster, and later calls use it.
+ngram_status forward_auto(ngram_ctx *c, const Call &k) {
+    const uint32_t b = ceil_log2(k.N);
+    if (c->auto_choice[b] == NGRAM_RES_HOST_UVA) return forward_uva(c, k);
+    if (c->auto_choice[b] == NGRAM_RES_HOST_DMA) return forward_dma(c, k);
+    if (!c->ev_t0) {
+        NG_CUDA(cudaEventCreate(&c->ev_t0), "cudaEventCreate");
+        NG_CUDA(cudaEventCreate(&c->ev_t1), "cudaEventCreate");
+    }
+    float t_uva = 0.f, t_dma = 0.f;
+    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
+    NG_CHECK(forward_uva(c, k));
+    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
+    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: UVA timing"));
+    NG_CUDA(cudaEventElapsedTime(&t_uva, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
+    const auto h0 = std::chrono::steady_clock::now();
+    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
+    NG_CHECK(forward_dma(c, k));
+    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
+    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: DMA timing"));
+    // the DMA path blocks the host while it stages rows: count wall time from its start
+    const float wall =
+        std::chrono::duration<float, std::milli>(std::chrono::steady_clock::now() - h0).count();
+    NG_CUDA(cudaEventElapsedTime(&t_dma, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
+    t_dma = std::max(t_dma, wall);
+    c->auto_choice[b] = (t_dma < t_uva) ? NGRAM_RES_HOST_DMA : NGRAM_RES_HOST_UVA;
     return NGRAM_OK;
 }
 
@@ -132,6 +506,20 @@ const char *ngram_status_string(ngram_status s) {
     return "NGRAM_UNKNOWN";
 }
 
+ngram_status ngram_host_alloc(void **out, uint64_t bytes) {
+    if (out == nullptr) return fail(NGRAM_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (bytes == 0) return fail(NGRAM_EINVAL, "bytes must be > 0");
+    NG_CUDA(cudaHostAlloc(out, bytes, cudaHostAllocMapped | cudaHostAllocPortable), "cudaHostAlloc");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_host_free(void *p) {
+    if (p == nullptr) return NGRAM_OK;
+    NG_CUDA(cudaFreeHost(p), "cudaFreeHost");
+    return NGRAM_OK;
+}
+
 ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_scale, uint64_t R,
                         uint32_t d, ngram_dtype dtype, ngram_residency where,
                         const ngram_hash_params *hp, uint32_t max_tokens) {
@@ -156,28 +544,36 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (max_tokens == 0) return fail(NGRAM_EINVAL, "max_tokens must be >= 1");
     ngram_hash_params p;
     if (hp != nullptr) p = *hp; else ngram_default_hash_params(&p);
-    ngram_status st = check_hash_params(p);
-    if (st != NGRAM_OK) return st;
+    NG_CHECK(check_hash_params(p));
+    const uint32_t H = p.n_bigram_heads + p.n_trigram_heads;
     const uint32_t n_strips = (d / 8 + 31) / 32;
     if (static_cast<uint64_t>(max_tokens) * n_strips > 0xFFFFFFFFull ||
-        static_cast<uint64_t>(max_tokens) * NGRAM_MAX_HEADS > 0xFFFFFFFFull)
+        static_cast<uint64_t>(max_tokens) * NGRAM_MAX_HEADS > (1ull << 30))
         return fail(NGRAM_EINVAL, "max_tokens %u too large for d = %u", max_tokens, d);
-    if (where != NGRAM_RES_HBM)
-        return fail(NGRAM_EUNSUPPORTED, "host-resident tables are not built yet");
+    if ((p.flags & NGRAM_FLAG_DEDUP) && where != NGRAM_RES_HBM)
+        return fail(NGRAM_EINVAL, "NGRAM_FLAG_DEDUP applies to HBM residency (host modes dedup on their own)");
 
     // ---- CUDA from here on
     ngram_ctx *c = new ngram_ctx();
+    memset(c, 0, sizeof(*c));
     c->table = table;
+    c->table_dev = table;
     c->row_scale = row_scale;
+    c->row_scale_dev = row_scale;
     c->R = R;
     c->d = d;
+    c->row_bytes = (dtype == NGRAM_BF16) ? 2u * d : d;
     c->dtype = dtype;
     c->where = where;
     c->hp = p;
+    c->H = H;
     c->max_tokens = max_tokens;
     c->barrett_m = (R == 1) ? 0ull
                             : static_cast<uint64_t>((static_cast<unsigned __int128>(1) << 64) / R);
-    c->d_err = nullptr;
+    c->wait_ms = 10000;
+    c->dd_cap = max_tokens * H;
+    c->dd_pcap = 1u << std::max<uint32_t>(10u, ceil_log2(2ull * c->dd_cap));
+    ngram_status st = NGRAM_OK;
     cudaError_t e = cudaGetDevice(&c->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess)
@@ -188,14 +584,43 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
                                                                 k_gather_int8<16>, 256, 0);
     if (e == cudaSuccess) e = cudaMalloc(&c->d_err, 4 * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, 4 * sizeof(uint32_t));
-    if (e != cudaSuccess) {
-        ngram_status s = cuda_fail(e, "ngram_init");
-        if (c->d_err) cudaFree(c->d_err);
+    if (e != cudaSuccess) st = cuda_fail(e, "ngram_init");
+    if (st == NGRAM_OK && where != NGRAM_RES_HBM) {
+        cudaPointerAttributes attr;
+        e = cudaPointerGetAttributes(&attr, table);
+        if (e != cudaSuccess) {
+            st = cuda_fail(e, "cudaPointerGetAttributes(table)");
+        } else if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+            st = fail(NGRAM_EINVAL, "host residency needs a host table, got device memory");
+        } else if (where != NGRAM_RES_HOST_DMA) {
+            // UVA / AUTO: the kernel reads the table itself, so it must be pinned and mapped
+            if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr)
+                st = fail(NGRAM_EINVAL, "UVA needs pinned, mapped host memory (ngram_host_alloc)");
+            else
+                c->table_dev = attr.devicePointer;
+            if (st == NGRAM_OK && row_scale != nullptr) {
+                e = cudaPointerGetAttributes(&attr, row_scale);
+                if (e != cudaSuccess || attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr)
+                    st = fail(NGRAM_EINVAL, "UVA needs row_scale in pinned, mapped host memory");
+                else
+                    c->row_scale_dev = static_cast<const float *>(attr.devicePointer);
+            }
+        }
+    }
+    if (st != NGRAM_OK) {
+        free_all(c);
         delete c;
-        return s;
+        return st;
     }
     if (c->gather_blocks_per_sm < 1) c->gather_blocks_per_sm = 1;
     *out = c;
+    return NGRAM_OK;
+}
+
+ngram_status ngram_set_wait_timeout(ngram_ctx *c, uint32_t ms) {
+    if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
+    if (ms == 0) return fail(NGRAM_EINVAL, "timeout must be > 0 ms");
+    c->wait_ms = ms;
     return NGRAM_OK;
 }
 
@@ -203,8 +628,8 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
                            uint32_t n_seq, uint32_t T, const uint16_t *residual, const float *gate,
                            uint16_t *out, ngram_stream_t stream) {
     uint64_t N = 0;
-    ngram_status st = check_batch(c, tokens, n_seq, T, &N);
-    if (st != NGRAM_OK || N == 0) return st;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (N == 0) return NGRAM_OK;
     if (residual == nullptr || gate == nullptr || out == nullptr)
         return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
     if (!aligned16(residual) || !aligned16(gate) || !aligned16(out))
@@ -215,42 +640,24 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
         if (a < b + bytes && b < a + bytes)
             return fail(NGRAM_EINVAL, "out overlaps residual without being equal to it");
     }
-
-    GatherArgs g;
-    g.h = hash_args(c);
-    g.table = c->table;
-    g.row_scale = c->row_scale;
-    g.tokens = tokens;
-    g.history = history;
-    g.residual = residual;
-    g.gate = gate;
-    g.out = out;
-    g.err = c->d_err;
-    g.T = T;
-    g.N = static_cast<uint32_t>(N);
-    g.d = c->d;
-    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;
-    g.n_strips = (c->d / cols_per_lane + 31) / 32;
-    const uint32_t resident_warps = static_cast<uint32_t>(c->num_sms) * c->gather_blocks_per_sm * 8u;
-    // Few tokens: one strip per warp (lowest latency).  Many: a warp keeps its token.
-    g.strips_per_item = (static_cast<uint64_t>(N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
-    g.groups_per_token = (g.n_strips + g.strips_per_item - 1) / g.strips_per_item;
-    const uint64_t items = N * g.groups_per_token;
-    const uint64_t max_blocks = static_cast<uint64_t>(c->num_sms) * c->gather_blocks_per_sm;
-    uint64_t blocks = (items + 7) / 8;
-    if (blocks > max_blocks) blocks = max_blocks;
-
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned nb = static_cast<unsigned>(blocks);
-    if (c->dtype == NGRAM_BF16) {
-        if (g.h.n_heads == 16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g);
-        else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
-    } else {
-        if (g.h.n_heads == 16) k_gather_int8<16><<<nb, 256, 0, s>>>(g);
-        else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
+    const Call k{tokens, history, T, static_cast<uint32_t>(N), residual, gate, out,
+                 reinterpret_cast<cudaStream_t>(stream)};
+    switch (c->where) {
+        case NGRAM_RES_HBM:
+            if (c->hp.flags & NGRAM_FLAG_DEDUP) return forward_dedup_hbm(c, k);
+            return forward_direct(c, k, static_cast<uint32_t>(c->gather_blocks_per_sm));
+        case NGRAM_RES_HOST_UVA: return forward_uva(c, k);
+        case NGRAM_RES_HOST_DMA: return forward_dma(c, k);
+        case NGRAM_RES_HOST_AUTO: return forward_auto(c, k);
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "gather kernel launch");
+    return fail(NGRAM_EINVAL, "bad residency");
+}
+
+ngram_status ngram_auto_choice(const ngram_ctx *c, uint32_t n_tokens, int *where_out) {
+    if (c == nullptr || where_out == nullptr) return fail(NGRAM_EINVAL, "ctx / where_out is NULL");
+    if (n_tokens == 0) return fail(NGRAM_EINVAL, "n_tokens must be > 0");
+    const int ch = c->auto_choice[ceil_log2(n_tokens)];
+    *where_out = ch ? ch : -1;
     return NGRAM_OK;
 }
 
@@ -258,19 +665,29 @@ ngram_status ngram_hash_indices(ngram_ctx *c, const int32_t *tokens, const int32
                                 uint32_t n_seq, uint32_t T, uint32_t *idx_out,
                                 ngram_stream_t stream) {
     uint64_t N = 0;
-    ngram_status st = check_batch(c, tokens, n_seq, T, &N);
-    if (st != NGRAM_OK || N == 0) return st;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (N == 0) return NGRAM_OK;
     if (idx_out == nullptr) return fail(NGRAM_EINVAL, "idx_out is NULL");
-    const HashArgs a = hash_args(c);
-    const uint64_t total = N * a.n_heads;
-    uint64_t blocks = (total + 255) / 256;
-    const uint64_t cap = static_cast<uint64_t>(c->num_sms) * 8;
-    if (blocks > cap) blocks = cap;
-    k_hash_indices<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        a, tokens, history, T, static_cast<uint32_t>(N), c->d_err, idx_out);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "k_hash_indices launch");
-    return NGRAM_OK;
+    return launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), idx_out,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+ngram_status ngram_dedup_rows(ngram_ctx *c, const int32_t *tokens, const int32_t *history,
+                              uint32_t n_seq, uint32_t T, uint32_t *uniq_out, uint32_t *inv_out,
+                              uint32_t *count_out, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (uniq_out == nullptr || inv_out == nullptr || count_out == nullptr)
+        return fail(NGRAM_EINVAL, "uniq_out, inv_out and count_out must be non-NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        NG_CUDA(cudaMemsetAsync(count_out, 0, 4, s), "cudaMemsetAsync");
+        return NGRAM_OK;
+    }
+    NG_CHECK(ensure_dedup_scratch(c));
+    const uint32_t M = static_cast<uint32_t>(N) * c->H;
+    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
+    return launch_dedup(c, c->d_idx, M, uniq_out, inv_out, count_out, s);
 }
 
 ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
@@ -285,40 +702,56 @@ ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uin
     if (dtype != NGRAM_BF16 && dtype != NGRAM_INT8_ROWSCALE)
         return fail(NGRAM_EINVAL, "unknown dtype %d", static_cast<int>(dtype));
     int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "ngram_fill_synthetic");
+    NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    NG_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute");
+    // a pinned, mapped host table is written through its device alias
+    void *dst = table;
+    float *dst_scale = row_scale;
+    cudaPointerAttributes attr;
+    NG_CUDA(cudaPointerGetAttributes(&attr, table), "cudaPointerGetAttributes(table)");
+    if (attr.type == cudaMemoryTypeHost) {
+        if (attr.devicePointer == nullptr) return fail(NGRAM_EINVAL, "host table is not mapped");
+        dst = attr.devicePointer;
+        if (row_scale != nullptr) {
+            NG_CUDA(cudaPointerGetAttributes(&attr, row_scale), "cudaPointerGetAttributes(row_scale)");
+            if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr)
+                return fail(NGRAM_EINVAL, "host table needs a mapped host row_scale");
+            dst_scale = static_cast<float *>(attr.devicePointer);
+        }
+    } else if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) {
+        return fail(NGRAM_EINVAL, "table must be device memory or pinned, mapped host memory");
+    }
     uint64_t blocks = static_cast<uint64_t>(sms) * 8;
     if (blocks > R) blocks = R;
     const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == NGRAM_BF16)
-        k_fill_bf16<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<uint16_t *>(table), R, d, k0, k1);
+        k_fill_bf16<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<uint16_t *>(dst), R, d, k0, k1);
     else
-        k_fill_int8<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<int8_t *>(table), row_scale, R, d, k0, k1);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "k_fill launch");
+        k_fill_int8<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<int8_t *>(dst), dst_scale, R, d, k0, k1);
+    NG_CUDA(cudaGetLastError(), "k_fill launch");
     return NGRAM_OK;
 }
 
 ngram_status ngram_get_device_error(ngram_ctx *c, uint32_t info[4], int clear) {
     if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
     uint32_t h[4] = {0, 0, 0, 0};
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e == cudaSuccess) e = cudaMemcpy(h, c->d_err, sizeof(h), cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess && clear) e = cudaMemset(c->d_err, 0, sizeof(h));
-    if (e != cudaSuccess) return cuda_fail(e, "ngram_get_device_error");
+    NG_CUDA(cudaDeviceSynchronize(), "ngram_get_device_error");
+    NG_CUDA(cudaMemcpy(h, c->d_err, sizeof(h), cudaMemcpyDeviceToHost), "ngram_get_device_error");
+    if (clear) NG_CUDA(cudaMemset(c->d_err, 0, sizeof(h)), "ngram_get_device_error");
     if (info != nullptr) memcpy(info, h, sizeof(h));
-    if (h[0] != 0)
+    if (h[0] == 1)
         return fail(NGRAM_EDEVICE, "token id %d out of [0, %u) at %s %u", static_cast<int32_t>(h[2]),
                     c->hp.vocab_size, (h[1] & 0x80000000u) ? "history entry" : "flat position",
                     h[1] & 0x7FFFFFFFu);
+    if (h[0] != 0)
+        return fail(NGRAM_EDEVICE, "a kernel wait ran past its deadline (code %u)", h[0]);
     return NGRAM_OK;
 }
 
 void ngram_destroy(ngram_ctx *c) {
     if (c == nullptr) return;
-    if (c->d_err) cudaFree(c->d_err);
+    free_all(c);
     delete c;
 }
 

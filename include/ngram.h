@@ -76,6 +76,17 @@ typedef enum {
     NGRAM_RES_HOST_AUTO = 3    /* host-resident; the faster of UVA / DMA, chosen by timing */
 } ngram_residency;
 
+/* HBM residency only: dedup the batch's rows first (ngram_dedup_rows), copy each
+ * distinct row once into an HBM staging buffer, and gather from staging through the
+ * inverse map.  Same results bit for bit.  Staging (max_tokens * H rows) and the dedup
+ * scratch are allocated by the first call that needs them. */
+#define NGRAM_FLAG_DEDUP 0x1u
+/* Stage the bf16 rows through shared memory with TMA bulk copies (cp.async.bulk into
+ * an mbarrier ring) instead of register loads.  Same results bit for bit; measured
+ * slower on B200 (522-895 us vs 455 us on the full-size gather), kept for comparison. */
+#define NGRAM_FLAG_TMA_STAGING 0x2u
+#define NGRAM_FLAGS_KNOWN (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING)
+
 #define NGRAM_MAX_HEADS 16u
 #define NGRAM_TOKEN_BITS 21u
 #define NGRAM_DEFAULT_BASE_SEED 0x6E6772616D5F7631ull   /* ASCII "ngram_v1" */
@@ -87,7 +98,7 @@ typedef struct {
     uint32_t n_trigram_heads;  /* default 8; n_bigram + n_trigram in [1, 16] */
     uint32_t pad_id;           /* default 2^21 - 1; must be < 2^21 */
     uint32_t vocab_size;       /* token ids must lie in [0, vocab_size); <= 2^21 - 1 */
-    uint32_t flags;            /* reserved, must be 0 */
+    uint32_t flags;            /* NGRAM_FLAG_* bits, default 0 */
     uint32_t reserved;         /* must be 0 */
 } ngram_hash_params;
 
@@ -97,17 +108,37 @@ typedef struct ngram_ctx ngram_ctx;
  * vocab_size 2^21-1.  Returns NGRAM_EINVAL if hp is NULL. */
 NGRAM_API ngram_status ngram_default_hash_params(ngram_hash_params *hp);
 
+/* Pinned host memory the GPU can read directly (cudaHostAlloc, mapped + portable), for a
+ * host-resident table ("Which is why the offload matters more than the parameter
+ * count" on the aibacon page: rows parked in pinned host memory, gathered over unified
+ * addressing).  ngram_fill_synthetic can fill it.  Free with ngram_host_free. */
+NGRAM_API ngram_status ngram_host_alloc(void **out, uint64_t bytes);
+NGRAM_API ngram_status ngram_host_free(void *p);
+
 /* Create a lookup context on the current CUDA device.
- *   table      device pointer to [R][d] rows (bf16 bits, or int8), 16-byte aligned;
- *              not owned, must outlive the context.
- *   row_scale  device pointer to [R] fp32 (int8 only, else NULL); not owned.
+ *   table      the [R][d] rows (bf16 bits, or int8), 16-byte aligned; not owned, must
+ *              outlive the context.  Device memory for NGRAM_RES_HBM; pinned, mapped
+ *              host memory (ngram_host_alloc) for HOST_UVA and HOST_AUTO; any host
+ *              memory for HOST_DMA (host threads read it).
+ *   row_scale  [R] fp32 (int8 only, else NULL), in the same kind of memory; not owned.
  *   R          rows, 1 <= R < 2^32.   d: row width, multiple of 8 (bf16) or 16 (int8).
- *   where      residency of the table (NGRAM_RES_HBM in this build).
+ *   where      residency of the table:
+ *              HBM       one fused kernel per call;
+ *              HOST_UVA  the same kernel reads the rows from host memory over PCIe;
+ *              HOST_DMA  rows are deduplicated on the GPU, the distinct rows are copied
+ *                        by host threads into pinned staging and moved to HBM by the
+ *                        copy engine in 8 MB chunks (copy and host gather overlap),
+ *                        then gathered from HBM; the call blocks the host until the
+ *                        rows are staged (bounded wait, see ngram_set_wait_timeout);
+ *              HOST_AUTO the first call of each batch-size bucket (ceil(log2 N)) runs
+ *                        and times both UVA and DMA (synchronously), later calls use
+ *                        the faster (ngram_auto_choice reports it).
  *   hp         hash parameters (NULL = defaults).
  *   max_tokens largest n_seq * T a later call may pass (>= 1).
- * The context owns a 16-byte device error word.  EINVAL on bad arguments (checked
- * before any CUDA call), EUNSUPPORTED for residencies not built, ECUDA/ENOMEM on
- * CUDA failures.  On failure *out is set to NULL. */
+ * The context owns a 16-byte device error word; dedup scratch and staging buffers are
+ * allocated by the first call that needs them.  EINVAL on bad arguments (checked
+ * before any CUDA call, except the memory-kind checks of host residency),
+ * ECUDA/ENOMEM on CUDA failures.  On failure *out is set to NULL. */
 NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_scale,
                         uint64_t R, uint32_t d, ngram_dtype dtype, ngram_residency where,
                         const ngram_hash_params *hp, uint32_t max_tokens);
@@ -127,13 +158,38 @@ NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, cons
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
                            const float *gate, uint16_t *out, ngram_stream_t stream);
 
+/* Bound, in milliseconds, of every host-side wait of the context (default 10,000).  A
+ * wait that runs out returns NGRAM_ETIMEOUT; work already enqueued stays enqueued and
+ * the context stays usable once the stream drains. */
+NGRAM_API ngram_status ngram_set_wait_timeout(ngram_ctx *ctx, uint32_t ms);
+
+/* Residency HOST_AUTO picked for batches of n_tokens (its ceil(log2) bucket):
+ * NGRAM_RES_HOST_UVA or NGRAM_RES_HOST_DMA, or -1 while undecided. */
+NGRAM_API ngram_status ngram_auto_choice(const ngram_ctx *ctx, uint32_t n_tokens, int *where_out);
+
+/* Per-batch row dedup (the optional dedup step): with idx the [N][H] row indices of
+ * the batch (as ngram_hash_indices computes them), writes
+ *   uniq_out  device uint32 [N*H]: the distinct rows, in order of first appearance in
+ *             idx, in entries [0, U);
+ *   inv_out   device uint32 [N*H]: inv[i] = position of idx[i]'s row in uniq, so that
+ *             uniq[inv[i]] == idx[i] for every entry (colliding heads keep their own);
+ *   count_out device uint32 [1]: U.
+ * The result is a pure function of the batch.  Several kernel launches on stream; the
+ * context's scratch (allocated on first use, ~24 bytes per entry of max_tokens * H) is
+ * reused by every call, so calls on one context must not overlap on the GPU. */
+NGRAM_API ngram_status ngram_dedup_rows(ngram_ctx *ctx, const int32_t *tokens,
+                                        const int32_t *history, uint32_t n_seq, uint32_t T,
+                                        uint32_t *uniq_out, uint32_t *inv_out,
+                                        uint32_t *count_out, ngram_stream_t stream);
+
 /* The index step alone: idx_out (device uint32 [N][H], H = heads) receives the row
  * index of every (token, head), computed exactly as ngram_forward computes them. */
 NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
                                 uint32_t n_seq, uint32_t T, uint32_t *idx_out,
                                 ngram_stream_t stream);
 
-/* Fill a device table with the synthetic values used by the tests and benchmarks
+/* Fill a table (device memory, or pinned mapped host memory written through its
+ * device alias) with the synthetic values used by the tests and benchmarks
  * (the pages' table is learned; no weights exist here).  Element (row, col) is a
  * pure function of (seed, row, col) through Philox4x32-10 (Salmon et al., SC'11):
  *   bf16: counter (col/2, row, 1, 0), key (seed lo32, seed hi32); words (x0,x1) for
@@ -142,14 +198,15 @@ NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens,
  *   int8: counter (col/4, row, 2, 0), word x[col%4]; q = (sum of its bytes - 510) >> 2;
  *         row_scale[row] = 0x1.1bc5f4p-11 * (0.75 + (x0 >> 8) * 2^-25) with x0 from
  *         counter (0, row, 3, 0), each fp32 step rounded separately.
- * table (and row_scale for int8) are device pointers.  Asynchronous on stream. */
+ * Asynchronous on stream. */
 NGRAM_API ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
                                   ngram_dtype dtype, uint64_t seed, ngram_stream_t stream);
 
 /* Synchronise the context's device, read and optionally clear its error word.
- * info (may be NULL) receives {flag, flat position, bad id, 0}; a position with bit
- * 31 set names history entry (position & 0x7FFFFFFF) = 2*s + j.  Returns NGRAM_OK if
- * no kernel flagged bad input, NGRAM_EDEVICE if one did. */
+ * info (may be NULL) receives {code, flat position, bad id, 0}.  Code 1: a token id was
+ * out of range (a position with bit 31 set names history entry (position & 0x7FFFFFFF)
+ * = 2*s + j).  Code 2: a kernel wait ran past its 1 s deadline (TMA-staged gather).
+ * Returns NGRAM_OK if no kernel flagged anything, NGRAM_EDEVICE if one did. */
 NGRAM_API ngram_status ngram_get_device_error(ngram_ctx *ctx, uint32_t info[4], int clear);
 
 /* Text of the last failure on the calling thread ("" if none). */

@@ -180,6 +180,25 @@ def indices(tokens, history, R, *, base_seed=DEFAULT_BASE_SEED, n_bigram=8, n_tr
     return out
 
 
+def unique_rows(idx):
+    """Per-batch dedup of the gathered rows (the optional dedup step of the lookup):
+    the distinct row ids of the flattened [N][H] index array in order of first
+    appearance, and for every entry the position of its row in that list.  Every entry
+    keeps its own inverse slot, so colliding heads still contribute once each."""
+    flat = np.asarray(idx, dtype=np.uint32).ravel()
+    where = {}
+    uniq = []
+    inv = np.empty(flat.size, dtype=np.uint32)
+    for i, r in enumerate(flat.tolist()):
+        u = where.get(r)
+        if u is None:
+            u = len(uniq)
+            where[r] = u
+            uniq.append(r)
+        inv[i] = u
+    return np.array(uniq, dtype=np.uint32), inv
+
+
 def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_seed=None,
             table=None, table_i8=None, row_scale=None, sel=None, acc=ACC_F32, n_threads=1,
             base_seed=DEFAULT_BASE_SEED, n_bigram=8, n_trigram=8, pad_id=DEFAULT_PAD_ID,

@@ -64,7 +64,7 @@ _T = torch.zeros(64, dtype=torch.bfloat16)      # any 16-byte aligned host addre
     (dict(hp=dict(pad_id=1 << 21)), "pad_id"),
     (dict(hp=dict(vocab_size=1 << 21)), "vocab_size"),
     (dict(hp=dict(vocab_size=0)), "vocab_size"),
-    (dict(hp=dict(flags=1)), "flags"),
+    (dict(hp=dict(flags=0x100)), "flags"),
     (dict(dtype=7), "dtype"),
     (dict(where=9), "residency"),
     (dict(dtype=ng.NGRAM_INT8_ROWSCALE, d=32), "row_scale"),
@@ -115,3 +115,22 @@ def test_null_context_is_rejected():
     assert lib.ngram_hash_indices(None, None, None, 1, 1, None, None) == ng.NGRAM_EINVAL
     assert lib.ngram_get_device_error(None, None, 0) == ng.NGRAM_EINVAL
     lib.ngram_destroy(None)                                 # no-op
+
+
+def test_new_entry_points_reject_bad_arguments():
+    lib = ng.lib()
+    assert lib.ngram_set_wait_timeout(None, 10) == ng.NGRAM_EINVAL
+    w = ctypes.c_int()
+    assert lib.ngram_auto_choice(None, 1, ctypes.byref(w)) == ng.NGRAM_EINVAL
+    assert lib.ngram_dedup_rows(None, None, None, 1, 1, None, None, None, None) == ng.NGRAM_EINVAL
+    p = ctypes.c_void_p(5)
+    assert lib.ngram_host_alloc(ctypes.byref(p), 0) == ng.NGRAM_EINVAL and p.value is None
+    assert lib.ngram_host_alloc(None, 16) == ng.NGRAM_EINVAL
+    assert lib.ngram_host_free(None) == ng.NGRAM_OK
+
+
+def test_dedup_flag_is_for_hbm_only():
+    hp = ng.ngram_default_hash_params(flags=ng.NGRAM_FLAG_DEDUP)
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_DMA, hp, 16)
+    assert ei.value.status == ng.NGRAM_EINVAL and "HBM" in str(ei.value)

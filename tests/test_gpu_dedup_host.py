@@ -1,0 +1,233 @@
+"""GPU parity of the per-batch row dedup and of the host-resident table modes.
+
+Dedup: the distinct rows (in order of first appearance) and the inverse map must equal
+the oracle's exactly.  Residency: HBM, HBM + dedup staging, host UVA, host DMA and
+host AUTO must give bit-identical outputs (the analogue of the offload on/off output
+check on the aibacon page, section "Which is why the offload matters more than the
+parameter count"), and those outputs must match the oracle.  The host waits of the DMA
+mode are bounded: a stream kept busy past the bound makes the call return
+NGRAM_ETIMEOUT and leaves the context usable.
+"""
+import numpy as np
+import pytest
+import torch
+
+import ngram_inputs as gen
+import oracle
+import hashed_gram_embedding_ngram_b200 as ng
+from parity_helpers import (N_CPU, TABLES, assert_parity, from_dev_bf16, sample_tokens,
+                            to_dev_bf16, to_dev_tokens, workload_on_device)
+
+pytestmark = pytest.mark.gpu
+W = gen.WORKLOADS
+
+
+def _hp(vocab, nb=8, nt=8, **kw):
+    return ng.ngram_default_hash_params(vocab_size=vocab, n_bigram_heads=nb,
+                                        n_trigram_heads=nt, **kw)
+
+
+def _dummy_ctx(dev, R, vocab, max_tokens, nb=8, nt=8):
+    buf = torch.zeros(16, dtype=torch.bfloat16, device=dev)
+    ctx = ng.ngram_init(buf, R, 8, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(vocab, nb, nt), max_tokens)
+    ctx._keep = buf
+    return ctx
+
+
+# --------------------------------------------------------------------------- dedup
+@pytest.mark.parametrize("name", ["tiny", "mid", "full_prefill", "full_decode_1",
+                                  "full_decode_256", "int8_uniform"])
+def test_dedup_rows_equal_oracle(cuda_device, name):
+    w = W[name]
+    inp = gen.make_inputs(w)
+    ctx = _dummy_ctx(cuda_device, w.R, w.vocab, w.N)
+    u, v, c = ng.ngram_dedup_rows(ctx, to_dev_tokens(inp["tokens"], cuda_device),
+                                  to_dev_tokens(inp["history"], cuda_device))
+    U = int(c.item())
+    idx = oracle.indices(inp["tokens"], inp["history"], w.R, vocab_size=w.vocab)
+    wu, wv = oracle.unique_rows(idx)
+    assert U == wu.size
+    assert np.array_equal(u[:U].cpu().numpy().view(np.uint32), wu)
+    assert np.array_equal(v.cpu().numpy().view(np.uint32), wv)
+
+
+@pytest.mark.parametrize("R,nb,nt", [(1, 8, 8), (2, 8, 8), (3, 3, 5), (65_536, 16, 0), (65_536, 1, 0)])
+def test_dedup_rows_collisions_and_heads(cuda_device, R, nb, nt):
+    toks = gen.zipf_tokens(3, 77, 500, seed=71)
+    ctx = _dummy_ctx(cuda_device, R, 500, toks.size, nb, nt)
+    u, v, c = ng.ngram_dedup_rows(ctx, to_dev_tokens(toks, cuda_device))
+    idx = oracle.indices(toks, None, R, n_bigram=nb, n_trigram=nt, vocab_size=500)
+    wu, wv = oracle.unique_rows(idx)
+    U = int(c.item())
+    assert U == wu.size
+    assert np.array_equal(u[:U].cpu().numpy().view(np.uint32), wu)
+    assert np.array_equal(v.cpu().numpy().view(np.uint32), wv)
+
+
+def test_dedup_rows_repeat_calls_and_empty(cuda_device):
+    """Scratch is reused across calls of different sizes; an empty batch gives 0."""
+    ctx = _dummy_ctx(cuda_device, 20_000_000, 151_936, 8192)
+    for n_seq, T, seed in ((8, 1024, 1), (1, 3, 2), (4, 500, 3), (8, 1024, 1)):
+        toks = gen.zipf_tokens(n_seq, T, 151_936, seed=seed)
+        u, v, c = ng.ngram_dedup_rows(ctx, to_dev_tokens(toks, cuda_device))
+        wu, wv = oracle.unique_rows(oracle.indices(toks, None, 20_000_000, vocab_size=151_936))
+        assert int(c.item()) == wu.size
+        assert np.array_equal(v.cpu().numpy().view(np.uint32), wv)
+    u, v, c = ng.ngram_dedup_rows(ctx, torch.zeros((0, 4), dtype=torch.int32, device=cuda_device))
+    assert int(c.item()) == 0
+
+
+# --------------------------------------------------------------------------- staged gathers
+def _forward(ctx, dv):
+    return ng.ngram_forward(ctx, dv["tokens"], dv["residual"], dv["gate"], history=dv["history"])
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid", "full_decode_64"])
+def test_hbm_dedup_staging_bitexact(cuda_device, name):
+    w = W[name]
+    inp, dv = workload_on_device(w, cuda_device)
+    table, _ = TABLES.get(w.R, w.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    plain = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(w.vocab), w.N)
+    dd = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM,
+                       _hp(w.vocab, flags=ng.NGRAM_FLAG_DEDUP), w.N)
+    a = from_dev_bf16(_forward(plain, dv))
+    b = from_dev_bf16(_forward(dd, dv))
+    assert np.array_equal(a, b)
+    assert ng.ngram_get_device_error(dd)[0] == ng.NGRAM_OK
+
+
+def test_hbm_dedup_staging_int8(cuda_device):
+    R, d, V = 5003, 272, 7000
+    w = gen.Workload("i8dd", R, d, "int8", V, 3, 50, history=True)
+    inp = gen.make_inputs(w, token_seed=81)
+    table, scale = TABLES.get(R, d, ng.NGRAM_INT8_ROWSCALE, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_INT8_ROWSCALE, ng.NGRAM_RES_HBM,
+                        _hp(V, flags=ng.NGRAM_FLAG_DEDUP), w.N, row_scale=scale)
+    dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device),
+          "history": to_dev_tokens(inp["history"], cuda_device),
+          "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
+          "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
+    got = from_dev_bf16(_forward(ctx, dv))
+    want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
+                          dtype=oracle.INT8, table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32,
+                          n_threads=N_CPU, vocab_size=V)
+    r = assert_parity(got, want)
+    assert r["exact"] == r["n"]
+
+
+# --------------------------------------------------------------------------- host residency
+class _HostFixture:
+    """A synthetic table in pinned, mapped host memory plus the same table in HBM."""
+
+    def __init__(self, dev, R, d, dtype):
+        self.R, self.d, self.dtype = R, d, dtype
+        if dtype == ng.NGRAM_BF16:
+            self.host = ng.HostTable((R, d), torch.bfloat16)
+            self.host_scale = None
+        else:
+            self.host = ng.HostTable((R, d), torch.int8)
+            self.host_scale = ng.HostTable((R,), torch.float32)
+        ng.ngram_fill_synthetic(self.host.tensor, R, d, dtype, gen.TABLE_SEED,
+                                row_scale=None if self.host_scale is None else self.host_scale.tensor)
+        torch.cuda.synchronize()
+
+    def ctx(self, where, vocab, max_tokens, **kw):
+        return ng.ngram_init(self.host.tensor, self.R, self.d, self.dtype, where, _hp(vocab, **kw),
+                             max_tokens, row_scale=None if self.host_scale is None else self.host_scale.tensor)
+
+    def close(self):
+        self.host.close()
+        if self.host_scale is not None:
+            self.host_scale.close()
+
+
+@pytest.fixture(scope="module")
+def host_bf16(cuda_device):
+    TABLES.drop()
+    f = _HostFixture(cuda_device, 400_000, 2560, ng.NGRAM_BF16)
+    yield f
+    f.close()
+
+
+def test_host_table_fill_equals_device_fill(cuda_device, host_bf16):
+    dev_table, _ = TABLES.get(host_bf16.R, host_bf16.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    rows = np.array([0, 1, 12345, host_bf16.R - 1])
+    got = host_bf16.host.tensor[torch.from_numpy(rows)].view(torch.int16).numpy()
+    want = dev_table[torch.from_numpy(rows).to(cuda_device)].view(torch.int16).cpu().numpy()
+    assert np.array_equal(got, want)
+    assert np.array_equal(got.view(np.uint16), oracle.rows_bf16(gen.TABLE_SEED, rows, host_bf16.d))
+
+
+@pytest.mark.parametrize("n_seq,T,hist", [(1, 1, True), (16, 1, True), (256, 1, True),
+                                          (2, 700, False), (1, 4096, False)])
+def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
+    R, d, V = host_bf16.R, host_bf16.d, 151_936
+    w = gen.Workload("host", R, d, "bf16", V, n_seq, T, history=hist)
+    inp, dv = workload_on_device(w, cuda_device, token_seed=90 + n_seq)
+    dev_table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    hbm = ng.ngram_init(dev_table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    ref = from_dev_bf16(_forward(hbm, dv))
+    for where in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA, ng.NGRAM_RES_HOST_AUTO):
+        ctx = host_bf16.ctx(where, V, w.N)
+        for _ in range(2):                       # second call reuses the staging buffers
+            got = from_dev_bf16(_forward(ctx, dv))
+            assert np.array_equal(got, ref), where
+        assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+        if where == ng.NGRAM_RES_HOST_AUTO:
+            assert ng.ngram_auto_choice(ctx, w.N) in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA)
+        ctx.close()
+    sel = sample_tokens(w, 256)
+    want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
+                          table_seed=gen.TABLE_SEED, sel=sel, acc=oracle.ACC_F32, n_threads=N_CPU,
+                          vocab_size=V)
+    assert_parity(ref.reshape(w.N, d)[sel], want)
+
+
+def test_host_int8_modes(cuda_device):
+    R, d, V = 50_000, 512, 9000
+    f = _HostFixture(cuda_device, R, d, ng.NGRAM_INT8_ROWSCALE)
+    try:
+        w = gen.Workload("hosti8", R, d, "int8", V, 4, 33, history=True)
+        inp, dv = workload_on_device(w, cuda_device, token_seed=7)
+        want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R,
+                              d=d, dtype=oracle.INT8, table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32,
+                              n_threads=N_CPU, vocab_size=V)
+        for where in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA):
+            ctx = f.ctx(where, V, w.N)
+            r = assert_parity(from_dev_bf16(_forward(ctx, dv)), want)
+            assert r["exact"] == r["n"]
+            ctx.close()
+    finally:
+        f.close()
+
+
+def test_dma_wait_is_bounded(cuda_device, host_bf16):
+    """A stream kept busy past the bound: the DMA call returns NGRAM_ETIMEOUT instead of
+    waiting; once the stream drains, the context works and gives the right bits."""
+    R, d, V = host_bf16.R, host_bf16.d, 151_936
+    w = gen.Workload("host_to", R, d, "bf16", V, 4, 64)
+    inp, dv = workload_on_device(w, cuda_device, token_seed=5)
+    ctx = host_bf16.ctx(ng.NGRAM_RES_HOST_DMA, V, w.N)
+    ref = from_dev_bf16(_forward(ctx, dv))
+    ng.ngram_set_wait_timeout(ctx, 50)
+    torch.cuda._sleep(int(1.5e9))                 # ~1 s of GPU busy-wait (bounded)
+    with pytest.raises(ng.NgramError) as ei:
+        _forward(ctx, dv)
+    assert ei.value.status == ng.NGRAM_ETIMEOUT
+    torch.cuda.synchronize()
+    ng.ngram_set_wait_timeout(ctx, 10_000)
+    assert np.array_equal(from_dev_bf16(_forward(ctx, dv)), ref)
+
+
+def test_host_residency_argument_checks(cuda_device, host_bf16):
+    dev_table, _ = TABLES.get(1000, 64, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    with pytest.raises(ng.NgramError) as ei:       # device memory is not a host table
+        ng.ngram_init(dev_table, 1000, 64, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_UVA, _hp(1000), 8)
+    assert ei.value.status == ng.NGRAM_EINVAL
+    pageable = torch.zeros((1000, 64), dtype=torch.bfloat16)
+    with pytest.raises(ng.NgramError) as ei:       # UVA needs pinned, mapped memory
+        ng.ngram_init(pageable, 1000, 64, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_UVA, _hp(1000), 8)
+    assert ei.value.status == ng.NGRAM_EINVAL
+    # DMA reads the table with host threads: pageable memory is accepted
+    ctx = ng.ngram_init(pageable, 1000, 64, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_DMA, _hp(1000), 8)
+    ctx.close()

@@ -154,6 +154,7 @@ def test_forward_full_decode_every_token(cuda_device, name):
     assert r["exact"] == r["n"]
 
 
+@pytest.mark.parametrize("flags", [0, ng.NGRAM_FLAG_TMA_STAGING])
 @pytest.mark.parametrize("d,nb,nt,n_seq,T,hist", [
     (8, 8, 8, 3, 37, False),       # one column vector: 31 idle lanes per strip
     (136, 3, 5, 2, 45, True),      # 17 vectors: ragged strip
@@ -162,12 +163,14 @@ def test_forward_full_decode_every_token(cuda_device, name):
     (2568, 8, 8, 2, 33, True),     # 321 vectors: the pages' width plus a ragged tail
     (256, 1, 0, 4, 16, False),     # single head: an embedding lookup
 ])
-def test_forward_ragged_shapes_and_heads(cuda_device, d, nb, nt, n_seq, T, hist):
+def test_forward_ragged_shapes_and_heads(cuda_device, d, nb, nt, n_seq, T, hist, flags):
+    """Both bf16 gathers: register loads (default) and TMA bulk staging (flag)."""
     R, V = 4099, 5000
     w = gen.Workload("ragged", R, d, "bf16", V, n_seq, T, history=hist)
     inp = gen.make_inputs(w, token_seed=31)
     table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
-    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V, nb, nt), w.N)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM,
+                        _hp(V, nb, nt, flags=flags), w.N)
     dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device),
           "history": to_dev_tokens(inp["history"], cuda_device),
           "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
@@ -332,3 +335,17 @@ def test_forward_int8_full_sampled(cuda_device):
     r = assert_parity(got[sel], _oracle(w, inp, sel=sel))
     assert r["exact"] == r["n"]
     assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
+def test_tma_staging_matches_register_gather_full_size(cuda_device):
+    """The TMA-staged gather on the full table equals the default gather bit for bit."""
+    w = W["full_prefill"]
+    inp, dv = workload_on_device(w, cuda_device)
+    table, _ = TABLES.get(w.R, w.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    a = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(w.vocab), w.N)
+    b = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM,
+                      _hp(w.vocab, flags=ng.NGRAM_FLAG_TMA_STAGING), w.N)
+    oa = _run(w, cuda_device, dv, a)
+    ob = _run(w, cuda_device, dv, b)
+    assert torch.equal(oa.view(torch.int16), ob.view(torch.int16))
+    assert ng.ngram_get_device_error(b)[0] == ng.NGRAM_OK

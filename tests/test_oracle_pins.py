@@ -369,3 +369,27 @@ def test_fp32_reference_within_tolerance_of_exact_definition():
     tol = _bf16_ulp(b) + 2.0 ** -20 * mag
     assert np.all(np.abs(a - b) <= tol)
     assert np.mean(a == b) > 0.999
+
+
+# --------------------------------------------------------------------------- dedup
+def test_unique_rows_against_numpy_unique():
+    """First-appearance order and inverse map agree with numpy.unique (library) and
+    reconstruct every entry."""
+    toks = gen.zipf_tokens(4, 300, 2000, seed=61)
+    idx = oracle.indices(toks, None, 5000, vocab_size=2000)
+    uniq, inv = oracle.unique_rows(idx)
+    flat = idx.ravel()
+    u_sorted, first, _ = np.unique(flat, return_index=True, return_inverse=True)
+    order = np.argsort(first, kind="stable")
+    assert np.array_equal(uniq, u_sorted[order])
+    assert np.array_equal(uniq[inv], flat)
+    assert len(set(uniq.tolist())) == uniq.size == u_sorted.size
+    # the inverse of each first occurrence is increasing: 0, 1, 2, ...
+    assert np.array_equal(inv[np.sort(first)], np.arange(uniq.size))
+
+
+def test_unique_rows_keeps_colliding_heads():
+    idx = np.array([[3, 3, 3, 7], [7, 3, 9, 9]], dtype=np.uint32)
+    uniq, inv = oracle.unique_rows(idx)
+    assert uniq.tolist() == [3, 7, 9]
+    assert inv.tolist() == [0, 0, 0, 1, 1, 0, 2, 2]
