@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <thread>
 
@@ -677,13 +678,14 @@ ngram_status ngram_dedup_rows(ngram_ctx *c, const int32_t *tokens, const int32_t
                               uint32_t *count_out, ngram_stream_t stream) {
     uint64_t N = 0;
     NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
-    if (uniq_out == nullptr || inv_out == nullptr || count_out == nullptr)
-        return fail(NGRAM_EINVAL, "uniq_out, inv_out and count_out must be non-NULL");
+    if (count_out == nullptr) return fail(NGRAM_EINVAL, "count_out is NULL");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (N == 0) {
+    if (N == 0) {                               // empty batch: U = 0, nothing else written
         NG_CUDA(cudaMemsetAsync(count_out, 0, 4, s), "cudaMemsetAsync");
         return NGRAM_OK;
     }
+    if (uniq_out == nullptr || inv_out == nullptr)
+        return fail(NGRAM_EINVAL, "uniq_out and inv_out must be non-NULL");
     NG_CHECK(ensure_dedup_scratch(c));
     const uint32_t M = static_cast<uint32_t>(N) * c->H;
     NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
@@ -756,3 +758,4 @@ void ngram_destroy(ngram_ctx *c) {
 }
 
 }  // extern "C"
+

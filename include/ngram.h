@@ -173,7 +173,7 @@ NGRAM_API ngram_status ngram_auto_choice(const ngram_ctx *ctx, uint32_t n_tokens
  *             idx, in entries [0, U);
  *   inv_out   device uint32 [N*H]: inv[i] = position of idx[i]'s row in uniq, so that
  *             uniq[inv[i]] == idx[i] for every entry (colliding heads keep their own);
- *   count_out device uint32 [1]: U.
+ *   count_out device uint32 [1]: U (an empty batch writes 0 and may pass NULL arrays).
  * The result is a pure function of the batch.  Several kernel launches on stream; the
  * context's scratch (allocated on first use, ~24 bytes per entry of max_tokens * H) is
  * reused by every call, so calls on one context must not overlap on the GPU. */

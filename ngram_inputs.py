@@ -38,6 +38,7 @@ class Workload:
     T: int
     tokens: str = "zipf"   # "zipf" or "uniform"
     history: bool = False  # decode / chunked prefill pass the two preceding tokens
+    residency: str = "hbm" # "hbm" or "host" (table in pinned host memory)
 
     @property
     def N(self) -> int:
@@ -56,6 +57,12 @@ WORKLOADS = {
     "full_decode_16": Workload("full_decode_16", 20_000_000, 2560, "bf16", 151_936, 16, 1, history=True),
     "full_decode_64": Workload("full_decode_64", 20_000_000, 2560, "bf16", 151_936, 64, 1, history=True),
     "full_decode_256": Workload("full_decode_256", 20_000_000, 2560, "bf16", 151_936, 256, 1, history=True),
+    # same table in pinned host memory: decode steps and an 8192-token prefill
+    "host_decode_1": Workload("host_decode_1", 20_000_000, 2560, "bf16", 151_936, 1, 1, history=True, residency="host"),
+    "host_decode_16": Workload("host_decode_16", 20_000_000, 2560, "bf16", 151_936, 16, 1, history=True, residency="host"),
+    "host_decode_64": Workload("host_decode_64", 20_000_000, 2560, "bf16", 151_936, 64, 1, history=True, residency="host"),
+    "host_decode_256": Workload("host_decode_256", 20_000_000, 2560, "bf16", 151_936, 256, 1, history=True, residency="host"),
+    "host_prefill": Workload("host_prefill", 20_000_000, 2560, "bf16", 151_936, 1, 8192, residency="host"),
     # profiling case for full ncu captures: 400k x 2560 bf16 (2 GB), 4 x 2048 Zipf tokens
     "profile_small": Workload("profile_small", 400_000, 2560, "bf16", 151_936, 4, 2048),
     # 20M x 2560 int8 + fp32 row scale (47.8 GiB), 65,536 uniform tokens (little reuse)
