@@ -759,3 +759,108 @@ void ngram_destroy(ngram_ctx *c) {
 
 }  // extern "C"
 
+// ------------------------------------------------------------------------------------
+// Dedup without any device allocation.
+//
+// Some callers cannot call cudaMalloc: a serving process whose device memory was handed
+// in full to another allocator at start-up (a cudaMalloc there fails, or carves memory
+// out of a pool that is accounted for elsewhere), or a latency-critical loop that
+// cannot afford the implicit device synchronisation an allocation may cause.  They
+// cannot create an ngram_ctx either (it owns a device error word), so this entry point
+// takes the hash parameters directly and keeps all of its scratch in one file-scope
+// device array, sized for at most kNoAllocMaxEntries (token, head) entries.
+//
+// Layout of the array (32-bit words): idx | slot | pos [E each], keys | first | uid
+// [P each], block sums [E / 1024], error word [4].
+// ------------------------------------------------------------------------------------
+namespace {
+
+constexpr uint32_t kNoAllocMaxEntries = 65536u;                   // 4096 tokens x 16 heads
+constexpr uint32_t kNoAllocSlots = 2u * kNoAllocMaxEntries;        // hash-table slots
+constexpr uint32_t kNoAllocBlocks = kNoAllocMaxEntries / kScanBlock;
+constexpr size_t kNoAllocWords = 3ull * kNoAllocMaxEntries + 3ull * kNoAllocSlots + kNoAllocBlocks + 4;
+
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocWords];
+
+// Device address of g_noalloc_scratch per device, looked up once per device.
+std::mutex g_noalloc_mu;
+uint32_t *g_noalloc_addr[256] = {nullptr};
+
+ngram_status noalloc_scratch(uint32_t **out) {
+    int dev = -1;
+    NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= 256) return fail(NGRAM_EUNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        NG_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(noalloc scratch)");
+        g_noalloc_addr[dev] = static_cast<uint32_t *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return NGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, uint64_t R,
+                                                  const int32_t *tokens, const int32_t *history,
+                                                  uint32_t n_seq, uint32_t T, uint32_t *uniq_out,
+                                                  uint32_t *inv_out, uint32_t *count_out,
+                                                  ngram_stream_t stream) {
+    if (R == 0 || R > 0xFFFFFFFFull) return fail(NGRAM_EINVAL, "R must be in [1, 2^32 - 1]");
+    ngram_hash_params p;
+    if (hp != nullptr) p = *hp; else ngram_default_hash_params(&p);
+    NG_CHECK(check_hash_params(p));
+    if (count_out == nullptr) return fail(NGRAM_EINVAL, "count_out is NULL");
+    const uint32_t H = p.n_bigram_heads + p.n_trigram_heads;
+    const uint64_t N = static_cast<uint64_t>(n_seq) * T;
+    if (N * H > kNoAllocMaxEntries)
+        return fail(NGRAM_EINVAL,
+                    "ngram_dedup_rows_noalloc: %llu tokens x %u heads exceed its fixed scratch of %u "
+                    "entries; use ngram_dedup_rows", static_cast<unsigned long long>(N), H,
+                    kNoAllocMaxEntries);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        NG_CUDA(cudaMemsetAsync(count_out, 0, 4, s), "cudaMemsetAsync");
+        return NGRAM_OK;
+    }
+    if (tokens == nullptr || uniq_out == nullptr || inv_out == nullptr)
+        return fail(NGRAM_EINVAL, "tokens, uniq_out and inv_out must be non-NULL");
+    uint32_t *base = nullptr;
+    NG_CHECK(noalloc_scratch(&base));
+    const uint32_t E = kNoAllocMaxEntries, P = kNoAllocSlots;
+    uint32_t *idx = base, *slot = base + E, *pos = base + 2 * E;
+    uint32_t *keys = base + 3 * E, *first = keys + P, *uid = first + P;
+    uint32_t *bsum = uid + P, *err = bsum + kNoAllocBlocks;
+
+    const uint32_t M = static_cast<uint32_t>(N) * H;
+    const uint32_t log2p = std::max<uint32_t>(10u, ceil_log2(2ull * M));   // <= log2(P)
+    const uint32_t NB = (M + kScanBlock - 1) / kScanBlock;
+    int dev = 0, sms = 0;
+    NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    NG_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute");
+    uint64_t gm = (M + 255) / 256;
+    if (gm > static_cast<uint64_t>(sms) * 8) gm = static_cast<uint64_t>(sms) * 8;
+
+    HashArgs a;
+    a.base_seed = p.base_seed;
+    a.R = R;
+    a.barrett_m = (R == 1) ? 0ull : static_cast<uint64_t>((static_cast<unsigned __int128>(1) << 64) / R);
+    a.n_bigram = p.n_bigram_heads;
+    a.n_heads = H;
+    a.pad_id = p.pad_id;
+    a.vocab = p.vocab_size;
+    // the array keeps the previous call's contents: reset what must start cleared
+    NG_CUDA(cudaMemsetAsync(err, 0, 16, s), "noalloc clear");
+    NG_CUDA(cudaMemsetAsync(keys, 0xFF, (1ull << log2p) * 4, s), "noalloc clear");
+    NG_CUDA(cudaMemsetAsync(first, 0xFF, (1ull << log2p) * 4, s), "noalloc clear");
+    k_hash_indices<<<static_cast<unsigned>(gm), 256, 0, s>>>(a, tokens, history, T,
+                                                              static_cast<uint32_t>(N), err, idx);
+    k_dedup_insert<<<static_cast<unsigned>(gm), 256, 0, s>>>(idx, M, keys, first, slot, log2p);
+    k_dedup_scan_local<<<NB, 256, 0, s>>>(slot, first, M, pos, bsum);
+    k_dedup_scan_blocks<<<1, 1024, 0, s>>>(bsum, NB, count_out);
+    k_dedup_emit<<<static_cast<unsigned>(gm), 256, 0, s>>>(idx, slot, first, pos, bsum, M, uniq_out, uid);
+    k_dedup_inverse<<<static_cast<unsigned>(gm), 256, 0, s>>>(slot, uid, M, inv_out);
+    NG_CUDA(cudaGetLastError(), "ngram_dedup_rows_noalloc launch");
+    return NGRAM_OK;
+}

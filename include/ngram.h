@@ -182,6 +182,31 @@ NGRAM_API ngram_status ngram_dedup_rows(ngram_ctx *ctx, const int32_t *tokens,
                                         uint32_t *uniq_out, uint32_t *inv_out,
                                         uint32_t *count_out, ngram_stream_t stream);
 
+/* ngram_dedup_rows for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call; it exists for users of this library.  Callers that cannot
+ * call cudaMalloc include a serving process whose device memory was handed in full to
+ * another allocator at start-up, and a latency-critical loop that cannot accept the
+ * device synchronisation an allocation may cause.  They cannot create an ngram_ctx
+ * either (the context owns a device error word), so this call takes the hash
+ * parameters (NULL = defaults) and the row count R directly.  Its outputs are exactly
+ * those of ngram_dedup_rows.
+ *   Allocation: none.  All scratch lives in one static device array of 2.25 MiB that
+ *     every GPU which loads libngram.so holds until the process exits.
+ *   Limit: n_seq * T * heads <= 65,536 entries (4,096 tokens at 16 heads); larger
+ *     batches return NGRAM_EINVAL with a message naming the limit.
+ *   Set-up: the first call on each device looks the array's device address up (with
+ *     that device current); make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array and leaves its contents
+ *     behind; the call clears what must start empty.  Calls that overlap on the GPU
+ *     (other streams, other host threads) race on the array: serialise them.
+ *   Bad token ids read as PAD, as in ngram_forward, but are not reported (there is no
+ *     context to hold the error word). */
+NGRAM_API ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, uint64_t R,
+                                                const int32_t *tokens, const int32_t *history,
+                                                uint32_t n_seq, uint32_t T, uint32_t *uniq_out,
+                                                uint32_t *inv_out, uint32_t *count_out,
+                                                ngram_stream_t stream);
+
 /* The index step alone: idx_out (device uint32 [N][H], H = heads) receives the row
  * index of every (token, head), computed exactly as ngram_forward computes them. */
 NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
