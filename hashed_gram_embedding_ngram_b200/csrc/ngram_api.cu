@@ -44,8 +44,12 @@ using namespace ngram;
 #ifndef NGRAM_BULK_CTAS_PER_SM
 #define NGRAM_BULK_CTAS_PER_SM 2
 #endif
-#ifndef NGRAM_UVA_CTAS_PER_SM           // host-resident (UVA) gather grid, CTAs per SM
-#define NGRAM_UVA_CTAS_PER_SM 2
+// NGRAM_UVA_CTAS: CTAs of the host-resident (UVA) gather.  8 CTAs (512 KB of row loads
+//   in flight) already saturate PCIe (51.4 GB/s, 0.93 of measured H2D, for the same
+//   8192-token prefill as 296 CTAs) and leave 140 SMs to the work beside the lookup: a
+//   bf16 4096x2560x2560 GEMM on another stream keeps 1166 TFLOP/s vs 667 with 296 CTAs.
+#ifndef NGRAM_UVA_CTAS
+#define NGRAM_UVA_CTAS 8
 #endif
 #ifndef NGRAM_DMA_CHUNK_BYTES           // host gather -> H2D pipelining granularity
 #define NGRAM_DMA_CHUNK_BYTES (8u << 20)
@@ -301,14 +305,13 @@ ngram_status launch_bulk(ngram_ctx *c, GatherArgs &g, cudaStream_t s) {
     return NGRAM_OK;
 }
 
-// The register gather (bf16 or int8); ctas_per_sm bounds the persistent grid.
-ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint32_t ctas_per_sm) {
-    const uint32_t resident_warps = static_cast<uint32_t>(c->num_sms) * ctas_per_sm * 8u;
+// The register gather (bf16 or int8); max_blocks bounds the persistent grid.
+ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t max_blocks) {
+    const uint64_t resident_warps = max_blocks * 8u;
     g.strips_per_item = (NGRAM_SPI_ALWAYS_ONE ||
                          static_cast<uint64_t>(g.N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
     g.groups_per_token = (g.n_strips + g.strips_per_item - 1) / g.strips_per_item;
     const uint64_t items = static_cast<uint64_t>(g.N) * g.groups_per_token;
-    const uint64_t max_blocks = static_cast<uint64_t>(c->num_sms) * ctas_per_sm;
     uint64_t blocks = (items + 7) / 8;
     if (blocks > max_blocks) blocks = max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
@@ -368,11 +371,16 @@ struct Call {
     cudaStream_t s;
 };
 
-ngram_status forward_direct(ngram_ctx *c, const Call &k, uint32_t ctas_per_sm) {
+// All SMs, every resident CTA: the grid of the HBM-resident gathers.
+uint64_t full_grid(const ngram_ctx *c) {
+    return static_cast<uint64_t>(c->num_sms) * static_cast<uint64_t>(c->gather_blocks_per_sm);
+}
+
+ngram_status forward_direct(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     if ((c->hp.flags & NGRAM_FLAG_TMA_STAGING) && c->dtype == NGRAM_BF16 && c->where == NGRAM_RES_HBM)
         return launch_bulk(c, g, k.s);
-    return launch_gather(c, g, k.s, ctas_per_sm);
+    return launch_gather(c, g, k.s, max_blocks);
 }
 
 // hash -> dedup -> compact the unique rows into HBM staging -> gather from staging.
@@ -390,7 +398,7 @@ ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
     g.table = c->d_stage;
     g.row_scale = c->d_stage_scale;
     g.row_ids = c->d_inv;
-    return launch_gather(c, g, k.s, static_cast<uint32_t>(c->gather_blocks_per_sm));
+    return launch_gather(c, g, k.s, full_grid(c));
 }
 
 // Host-resident, copy-engine path: the unique rows are compacted by host threads
@@ -438,12 +446,13 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
     g.table = c->d_stage;
     g.row_scale = c->d_stage_scale;
     g.row_ids = c->d_inv;
-    return launch_gather(c, g, k.s, static_cast<uint32_t>(c->gather_blocks_per_sm));
+    return launch_gather(c, g, k.s, full_grid(c));
 }
 
+// UVA: the same kernel reading host rows over PCIe.  A bounded grid suffices to keep
+// PCIe busy and leaves the other SMs to whatever runs beside the lookup.
 ngram_status forward_uva(ngram_ctx *c, const Call &k) {
-    const uint32_t per_sm = std::min<uint32_t>(NGRAM_UVA_CTAS_PER_SM, c->gather_blocks_per_sm);
-    return forward_direct(c, k, per_sm);
+    return forward_direct(c, k, std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c)));
 }
 
 // AUTO: the first call of each batch-size bucket runs and times both host modes
@@ -646,7 +655,7 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
     switch (c->where) {
         case NGRAM_RES_HBM:
             if (c->hp.flags & NGRAM_FLAG_DEDUP) return forward_dedup_hbm(c, k);
-            return forward_direct(c, k, static_cast<uint32_t>(c->gather_blocks_per_sm));
+            return forward_direct(c, k, full_grid(c));
         case NGRAM_RES_HOST_UVA: return forward_uva(c, k);
         case NGRAM_RES_HOST_DMA: return forward_dma(c, k);
         case NGRAM_RES_HOST_AUTO: return forward_auto(c, k);
