@@ -37,8 +37,13 @@ import ngram_inputs as gen  # noqa: E402
 METRIC = "n-gram embed tokens/s and gather GB/s (% of HBM or PCIe H2D roofline), 1 B200"
 UNIT = "tokens/s"
 HEADS = 16
-KERNEL_SOURCES = ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
-                  "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"]
+KERNEL_SOURCES = {   # the source files each timed kernel is built from
+    "bf16": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
+             "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
+    "int8": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
+             "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
+             "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
+}
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -68,15 +73,15 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_sha() -> str:
+def kernel_sha(dtype: str = "bf16") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[dtype]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, dtype: str = "bf16"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     kernel source as it is now (else None)."""
     p = os.path.join(ROOT, "profiles", "gather_%s.txt" % workload)
@@ -88,7 +93,7 @@ def profiled_traffic(workload: str):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("kernel_sha") != kernel_sha():
+    if kv.get("kernel_sha") != kernel_sha(dtype):
         return None
     try:
         return float(kv["traffic_bytes_per_launch"])
@@ -158,6 +163,27 @@ def gpu_id_for(dev) -> str:
     return str(dev.index or 0)
 
 
+# --------------------------------------------------------------------------- ranks
+def rank_seeds(rank: int, batch: int):
+    """(token seed, history seed) of one rank's batch: every rank draws its own tokens."""
+    return gen.TOKEN_SEED + 1000 * rank + batch, gen.HISTORY_SEED + 1000 * rank + batch
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings (ms) over all ranks; a plain list back."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_tokens_per_s(world: int, tokens_per_rank: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (elapsed_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- CPU oracle
 def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0):
     """Time the oracle (test infrastructure; rows regenerated on the fly, the full table
@@ -224,10 +250,11 @@ def config_for(w, args) -> dict:
         "table_gib": round(w.R * row_bytes(w) / 2**30, 2), "n_seq": w.n_seq, "T": w.T,
         "tokens_per_step_per_gpu": w.N, "heads": "8 bigram + 8 trigram",
         "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
-        "accumulate": "fp32, head order", "residency": "hbm",
+        "accumulate": "fp32, head order", "residency": "hbm", "variant": args.variant,
         "l2": "inputs larger than L2: %.2f GB moved per step vs 126 MB L2; %d token batches "
               "alternate" % (algorithmic_bytes(w) / 1e9, args.batches),
         "parallelism": "replicas x%d (tokens sharded, table replicated)" % args.gpus,
+        "launch": args.launch,
     }
 
 
@@ -263,14 +290,16 @@ def run_ours(args, w):
         table = torch.empty((w.R, w.d), dtype=torch.int8, device=dev)
         scale = torch.empty((w.R,), dtype=torch.float32, device=dev)
     ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
-    hp = ng.ngram_default_hash_params(vocab_size=w.vocab)
+    flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING}[args.variant]
+    hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
 
     # ---- inputs: this rank's token batches (distinct seeds per rank and batch)
     host_tok, host_hist = [], []
     for b in range(args.batches):
-        host_tok.append(gen.tokens_for(w, gen.TOKEN_SEED + 1000 * rank + b))
-        host_hist.append(gen.history_for(w, gen.HISTORY_SEED + 1000 * rank + b))
+        ts, hs = rank_seeds(rank, b)
+        host_tok.append(gen.tokens_for(w, ts))
+        host_hist.append(gen.history_for(w, hs))
     res_bits = gen.residual_bf16_bits(w.N, w.d, gen.RESIDUAL_SEED + rank)
     gate_h = gen.gate_f32(w.d)
     tok_d = [torch.from_numpy(t).to(dev) for t in host_tok]
@@ -281,36 +310,60 @@ def run_ours(args, w):
     gate = torch.from_numpy(gate_h).to(dev)
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def step(i, s=None):
         b = i % args.batches
-        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
+        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b],
+                         stream=s if s is not None else stream)
 
-    # ---- device-resident timing
+    # ---- device-resident timing.  Eager: one launch per step, CUDA events around each
+    # launch.  Graph: G steps captured once into a CUDA graph and replayed, events around
+    # each replay (decode-sized launches are otherwise bound by the Python launch path).
+    launch = args.launch if args.launch != "auto" else ("graph" if w.N <= 1024 else "eager")
+    G = 100
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     K = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    graph = None
+    if launch == "graph":
+        K = max(G, (K + G - 1) // G * G)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for i in range(G):
+                step(i, cap)
+        graph.replay()
+        torch.cuda.synchronize()
+    n_ev = K if graph is None else K // G
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id_for(dev)) as clk:
         barrier()
         torch.cuda.synchronize()
         t0.record(stream)
-        for i in range(K):
+        for i in range(n_ev):
             ev_s[i].record(stream)
-            step(i)
+            if graph is None:
+                step(i)
+            else:
+                graph.replay()
             ev_e[i].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = t0.elapsed_time(t1)
-    kern_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(K))
+    kern_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(n_ev))
+    if graph is not None:
+        kern_ms /= G                          # per step inside the graph (kernel + gap)
+        del graph
     st, info = ng.ngram_get_device_error(ctx)
     if st != ng.NGRAM_OK:
         raise SystemExit("device error word set: %s" % info)
 
-    # ---- end to end: pinned host inputs in, result back to the host, every step
+    # ---- end to end through the host-buffer call: every step moves its tokens and
+    # residual from pinned host memory to the device and its output back to the host
+    # (ngram_forward_host pipelines the copies with the gather in ~8 MB chunks)
     tok_h = [torch.from_numpy(t).pin_memory() for t in host_tok]
     hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in host_hist]
     res_h = res_cpu.pin_memory()
@@ -319,12 +372,16 @@ def run_ours(args, w):
 
     def e2e_step(i):
         b = i % args.batches
-        tok_d[b].copy_(tok_h[b], non_blocking=True)
-        if hist_h[b] is not None:
-            hist_d[b].copy_(hist_h[b], non_blocking=True)
-        residual.copy_(res_h, non_blocking=True)
-        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
-        out_h.copy_(out, non_blocking=True)
+        if args.variant == "default":
+            ng.ngram_forward_host(ctx, tok_h[b], res_h, gate, out=out_h, history=hist_h[b],
+                                  stream=stream)
+        else:                                 # staged variants: copy in, forward, copy out
+            tok_d[b].copy_(tok_h[b], non_blocking=True)
+            if hist_h[b] is not None:
+                hist_d[b].copy_(hist_h[b], non_blocking=True)
+            residual.copy_(res_h, non_blocking=True)
+            ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
+            out_h.copy_(out, non_blocking=True)
 
     for i in range(min(3, E)):
         e2e_step(i)
@@ -342,16 +399,12 @@ def run_ours(args, w):
     d2h = w.N * w.d * 2
 
     # ---- max over ranks
-    times = torch.tensor([elapsed_ms, kern_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    elapsed_ms, kern_ms, e2e_ms = (float(x) for x in times.tolist())
+    elapsed_ms, kern_ms, e2e_ms = max_over_ranks([elapsed_ms, kern_ms, e2e_ms], world, dev)
     clocks = clk.summary()
 
     if rank == 0:
-        tokens_total = world * w.N
-        value = tokens_total * K / (elapsed_ms / 1e3)
-        e2e_value = tokens_total * E / (e2e_ms / 1e3)
+        value = weak_scaling_tokens_per_s(world, w.N, K, elapsed_ms)
+        e2e_value = weak_scaling_tokens_per_s(world, w.N, E, e2e_ms)
         peaks = measured_peaks()
         bytes_launch = algorithmic_bytes(w)
         achieved = bytes_launch / (kern_ms / 1e3) / 1e9
@@ -359,19 +412,24 @@ def run_ours(args, w):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": config_for(w, args),
+            "config": dict(config_for(w, args), launch=launch),
             "gather_gbs": bytes_launch * world * K / (elapsed_ms / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic(w.name),
-                         "kernel": "k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8",
+                         "traffic": profiled_traffic(w.name, w.dtype) if args.variant == "default" else None,
+                         "kernel": {"default": "k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8<16>",
+                                    "tma": "k_gather_bf16_bulk<16>",
+                                    "dedup": "hash + dedup + compact + gather (8 kernels)"}[args.variant],
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E,
-                    "path": "pinned host tokens+residual -> device, ngram_forward, out -> pinned host"},
+                    "path": ("ngram_forward_host: pinned host tokens + residual in, bf16 out "
+                             "back to pinned host, chunked H2D / gather / D2H on 3 streams")
+                    if args.variant == "default" else
+                            "pinned host tokens + residual -> device, ngram_forward, out -> pinned host"},
             "clocks": clocks,
-            "gpu_launches": K,
+            "gpu_launches": K * {"default": 1, "tma": 1, "dedup": 8}[args.variant],
         }
         if world == 1 and not args.no_cpu_baseline:
             threads = os.cpu_count() or 1
@@ -538,6 +596,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
+                    help="eager launches, or 100-step CUDA graphs (auto: graph for N <= 1024)")
+    ap.add_argument("--variant", default="default", choices=["default", "dedup", "tma"],
+                    help="HBM path: fused gather (default), dedup + staged gather, TMA staging")
     ap.add_argument("--host-workloads", default="host_decode_1,host_decode_16,host_decode_64,"
                                                 "host_decode_256,host_prefill")
     ap.add_argument("--host-steps", type=int, default=200)

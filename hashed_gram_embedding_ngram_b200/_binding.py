@@ -77,6 +77,8 @@ _lib.ngram_status_string.argtypes = [_i32]
 _lib.ngram_status_string.restype = ctypes.c_char_p
 _lib.ngram_destroy.argtypes = [_P]
 _lib.ngram_destroy.restype = None
+_lib.ngram_forward_host.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
+_lib.ngram_forward_host.restype = _i32
 _lib.ngram_host_alloc.argtypes = [ctypes.POINTER(_P), _u64]
 _lib.ngram_host_alloc.restype = _i32
 _lib.ngram_host_free.argtypes = [_P]
@@ -199,6 +201,36 @@ def ngram_forward(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor,
         raise ValueError("out must hold N * d elements")
     _check(_lib.ngram_forward(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
                               _ptr(residual), _ptr(gate), _ptr(out), _stream(stream)))
+    return out
+
+
+def ngram_forward_host(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor,
+                       gate: torch.Tensor, out: torch.Tensor | None = None,
+                       history: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """ngram_forward with tokens, history, residual and out in host (CPU, ideally pinned)
+    memory and the gate on the device.  Returns out; it is complete once `stream` (the
+    current stream by default) is synchronised."""
+    cpu = torch.device("cpu")
+    _need(tokens, "tokens", torch.int32, cpu, ndim=2)
+    n_seq, T = tokens.shape
+    N = n_seq * T
+    _need(residual, "residual", torch.bfloat16, cpu)
+    if residual.numel() != N * ctx.d:
+        raise ValueError("residual must hold N * d = %d elements" % (N * ctx.d))
+    _need(gate, "gate", torch.float32)
+    if gate.device.type != "cuda" or gate.numel() != ctx.d:
+        raise ValueError("gate must be a CUDA tensor of d = %d elements" % ctx.d)
+    if history is not None:
+        _need(history, "history", torch.int32, cpu, ndim=2)
+        if tuple(history.shape) != (n_seq, 2):
+            raise ValueError("history must be [n_seq][2]")
+    if out is None:
+        out = torch.empty_like(residual, pin_memory=True)
+    _need(out, "out", torch.bfloat16, cpu)
+    if out.numel() != N * ctx.d:
+        raise ValueError("out must hold N * d elements")
+    _check(_lib.ngram_forward_host(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                                   _ptr(residual), _ptr(gate), _ptr(out), _stream(stream)))
     return out
 
 

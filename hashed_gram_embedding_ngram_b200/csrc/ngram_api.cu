@@ -21,6 +21,7 @@
 #include "device_common.cuh"
 #include "fill.cuh"
 #include "gather.cuh"
+#include "gather_int8.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
 
@@ -91,6 +92,12 @@ struct ngram_ctx {
     int stage_in_use;
     cudaEvent_t ev_t0, ev_t1;   // AUTO timing
     int auto_choice[33];        // per ceil(log2 N): 0 undecided, else ngram_residency
+    // ngram_forward_host: device copies of the host inputs, double-buffered chunks
+    int32_t *hp_tok, *hp_hist;
+    uint16_t *hp_res[2], *hp_out[2];
+    uint32_t hp_chunk;          // tokens per chunk
+    cudaStream_t hp_s[3];       // H2D, compute, D2H
+    cudaEvent_t hp_entry, hp_h2d[2], hp_kdone[2], hp_d2h[2];
 };
 
 namespace {
@@ -202,9 +209,16 @@ void free_all(ngram_ctx *c) {
     if (c->h_stage_scale) cudaFreeHost(c->h_stage_scale);
     if (c->h_uniq) cudaFreeHost(c->h_uniq);
     if (c->h_count) cudaFreeHost(c->h_count);
-    cudaEvent_t evs[] = {c->ev_sync, c->ev_stage_free, c->ev_t0, c->ev_t1};
+    cudaEvent_t evs[] = {c->ev_sync, c->ev_stage_free, c->ev_t0, c->ev_t1, c->hp_entry,
+                         c->hp_h2d[0], c->hp_h2d[1], c->hp_kdone[0], c->hp_kdone[1],
+                         c->hp_d2h[0], c->hp_d2h[1]};
     for (cudaEvent_t e : evs)
         if (e) cudaEventDestroy(e);
+    void *bufs[] = {c->hp_tok, c->hp_hist, c->hp_res[0], c->hp_res[1], c->hp_out[0], c->hp_out[1]};
+    for (void *p : bufs)
+        if (p) cudaFree(p);
+    for (cudaStream_t s : c->hp_s)
+        if (s) cudaStreamDestroy(s);
 }
 
 // ---------------------------------------------------------------- scratch on first use
@@ -247,6 +261,32 @@ ngram_status ensure_host_stage(ngram_ctx *c) {
     return NGRAM_OK;
 }
 
+#ifndef NGRAM_HOST_CHUNK_BYTES          // residual bytes per pipelined chunk (host buffers)
+#define NGRAM_HOST_CHUNK_BYTES (8u << 20)
+#endif
+
+ngram_status ensure_host_path(ngram_ctx *c) {
+    if (c->hp_tok) return NGRAM_OK;
+    const uint64_t row = 2ull * c->d;
+    uint64_t chunk = NGRAM_HOST_CHUNK_BYTES / row;
+    if (chunk < 1) chunk = 1;
+    if (chunk > c->max_tokens) chunk = c->max_tokens;
+    c->hp_chunk = static_cast<uint32_t>(chunk);
+    NG_CUDA(cudaMalloc(&c->hp_tok, c->max_tokens * 4ull), "host-path buffers");
+    NG_CUDA(cudaMalloc(&c->hp_hist, c->max_tokens * 8ull), "host-path buffers");
+    for (int b = 0; b < 2; ++b) {
+        NG_CUDA(cudaMalloc(&c->hp_res[b], chunk * row), "host-path buffers");
+        NG_CUDA(cudaMalloc(&c->hp_out[b], chunk * row), "host-path buffers");
+        NG_CUDA(cudaEventCreateWithFlags(&c->hp_h2d[b], cudaEventDisableTiming), "cudaEventCreate");
+        NG_CUDA(cudaEventCreateWithFlags(&c->hp_kdone[b], cudaEventDisableTiming), "cudaEventCreate");
+        NG_CUDA(cudaEventCreateWithFlags(&c->hp_d2h[b], cudaEventDisableTiming), "cudaEventCreate");
+    }
+    NG_CUDA(cudaEventCreateWithFlags(&c->hp_entry, cudaEventDisableTiming), "cudaEventCreate");
+    for (int i = 0; i < 3; ++i)
+        NG_CUDA(cudaStreamCreateWithFlags(&c->hp_s[i], cudaStreamNonBlocking), "cudaStreamCreate");
+    return NGRAM_OK;
+}
+
 // ---------------------------------------------------------------- launch helpers
 GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t *history,
                        uint32_t T, uint32_t N, const uint16_t *residual, const float *gate,
@@ -264,6 +304,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.err = c->d_err;
     g.T = T;
     g.N = N;
+    g.tok_begin = 0;
     g.d = c->d;
     const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;
     g.n_strips = (c->d / cols_per_lane + 31) / 32;
@@ -661,6 +702,64 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
         case NGRAM_RES_HOST_AUTO: return forward_auto(c, k);
     }
     return fail(NGRAM_EINVAL, "bad residency");
+}
+
+ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int32_t *history_h,
+                                uint32_t n_seq, uint32_t T, const uint16_t *residual_h,
+                                const float *gate, uint16_t *out_h, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens_h, n_seq, T, &N));
+    if (N == 0) return NGRAM_OK;
+    if (residual_h == nullptr || gate == nullptr || out_h == nullptr)
+        return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
+    if (!aligned16(gate)) return fail(NGRAM_EINVAL, "gate must be 16-byte aligned");
+    if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING)) ||
+        (c->where != NGRAM_RES_HBM && c->where != NGRAM_RES_HOST_UVA))
+        return fail(NGRAM_EUNSUPPORTED,
+                    "ngram_forward_host pipelines the fused gather: HBM or HOST_UVA residency, no flags");
+    NG_CHECK(ensure_host_path(c));
+    cudaStream_t caller = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t sh = c->hp_s[0], sk = c->hp_s[1], sd = c->hp_s[2];
+    const uint64_t row = 2ull * c->d;
+    const uint64_t max_blocks = (c->where == NGRAM_RES_HOST_UVA)
+        ? std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c)) : full_grid(c);
+    // order after the caller's earlier work, and after this context's previous call
+    NG_CUDA(cudaEventRecord(c->hp_entry, caller), "cudaEventRecord");
+    NG_CUDA(cudaStreamWaitEvent(sh, c->hp_entry, 0), "cudaStreamWaitEvent");
+    for (int b = 0; b < 2; ++b) NG_CUDA(cudaStreamWaitEvent(sh, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
+    NG_CUDA(cudaMemcpyAsync(c->hp_tok, tokens_h, N * 4, cudaMemcpyHostToDevice, sh), "H2D tokens");
+    if (history_h)
+        NG_CUDA(cudaMemcpyAsync(c->hp_hist, history_h, n_seq * 8ull, cudaMemcpyHostToDevice, sh),
+                "H2D history");
+    GatherArgs g = gather_args(c, c->hp_tok, history_h ? c->hp_hist : nullptr, T, 0, nullptr, gate,
+                               nullptr);
+    uint32_t chunk_i = 0;
+    for (uint64_t t0 = 0; t0 < N; t0 += c->hp_chunk, ++chunk_i) {
+        const uint32_t b = chunk_i & 1u;
+        const uint32_t n = static_cast<uint32_t>(std::min<uint64_t>(c->hp_chunk, N - t0));
+        // H2D of the chunk's residual once the kernel two chunks back has read the buffer
+        NG_CUDA(cudaStreamWaitEvent(sh, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
+        NG_CUDA(cudaMemcpyAsync(c->hp_res[b], residual_h + t0 * c->d, n * row, cudaMemcpyHostToDevice, sh),
+                "H2D residual");
+        NG_CUDA(cudaEventRecord(c->hp_h2d[b], sh), "cudaEventRecord");
+        // the gather, once its residual is in and the D2H two chunks back has drained out
+        NG_CUDA(cudaStreamWaitEvent(sk, c->hp_h2d[b], 0), "cudaStreamWaitEvent");
+        NG_CUDA(cudaStreamWaitEvent(sk, c->hp_d2h[b], 0), "cudaStreamWaitEvent");
+        g.tok_begin = static_cast<uint32_t>(t0);
+        g.N = n;
+        g.residual = c->hp_res[b];
+        g.out = c->hp_out[b];
+        NG_CHECK(launch_gather(c, g, sk, max_blocks));
+        NG_CUDA(cudaEventRecord(c->hp_kdone[b], sk), "cudaEventRecord");
+        // D2H of the chunk's output
+        NG_CUDA(cudaStreamWaitEvent(sd, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
+        NG_CUDA(cudaMemcpyAsync(out_h + t0 * c->d, c->hp_out[b], n * row, cudaMemcpyDeviceToHost, sd),
+                "D2H out");
+        NG_CUDA(cudaEventRecord(c->hp_d2h[b], sd), "cudaEventRecord");
+    }
+    // the caller's stream resumes once the last output chunk is on the host
+    NG_CUDA(cudaStreamWaitEvent(caller, c->hp_d2h[(chunk_i - 1) & 1u], 0), "cudaStreamWaitEvent");
+    return NGRAM_OK;
 }
 
 ngram_status ngram_auto_choice(const ngram_ctx *c, uint32_t n_tokens, int *where_out) {

@@ -207,6 +207,25 @@ NGRAM_API ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, uin
                                                 uint32_t *inv_out, uint32_t *count_out,
                                                 ngram_stream_t stream);
 
+/* ngram_forward with the per-token inputs and the output in HOST memory (the weights --
+ * table and gate -- stay resident on the device).  The batch is cut into chunks of about
+ * 8 MB of residual; three internal streams overlap the host->device copy of chunk i+1,
+ * the gather of chunk i and the device->host copy of chunk i-1, so PCIe carries input
+ * and output at the same time.
+ *   tokens_h   host int32 [n_seq][T]; history_h host int32 [n_seq][2] or NULL;
+ *   residual_h host bf16 [N][d];  gate: DEVICE fp32 [d];  out_h: host bf16 [N][d], must
+ *   not overlap residual_h.  Pinned host memory gives the overlap; pageable memory works
+ *   but its copies do not overlap.
+ * Ordering: starts after the work already on `stream`; `stream` waits for the last
+ * output chunk, so synchronising `stream` means out_h is complete.  Host buffers must
+ * stay valid until then.  HBM or HOST_UVA residency without flags, else
+ * NGRAM_EUNSUPPORTED.  The device copies of the inputs (max_tokens tokens, two chunks
+ * of residual and output) are allocated by the first call. */
+NGRAM_API ngram_status ngram_forward_host(ngram_ctx *ctx, const int32_t *tokens_h,
+                                          const int32_t *history_h, uint32_t n_seq, uint32_t T,
+                                          const uint16_t *residual_h, const float *gate,
+                                          uint16_t *out_h, ngram_stream_t stream);
+
 /* The index step alone: idx_out (device uint32 [N][H], H = heads) receives the row
  * index of every (token, head), computed exactly as ngram_forward computes them. */
 NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,

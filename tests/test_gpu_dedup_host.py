@@ -175,6 +175,13 @@ def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
         assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
         if where == ng.NGRAM_RES_HOST_AUTO:
             assert ng.ngram_auto_choice(ctx, w.N) in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA)
+        if where == ng.NGRAM_RES_HOST_UVA:       # host table and host activations together
+            t = torch.from_numpy(inp["tokens"]).pin_memory()
+            h = None if inp["history"] is None else torch.from_numpy(inp["history"]).pin_memory()
+            r = torch.from_numpy(inp["residual"].view(np.int16)).view(torch.bfloat16).view(w.N, d)
+            o = ng.ngram_forward_host(ctx, t, r.pin_memory(), dv["gate"], history=h)
+            torch.cuda.current_stream().synchronize()
+            assert np.array_equal(o.view(torch.int16).numpy().view(np.uint16), ref)
         ctx.close()
     sel = sample_tokens(w, 256)
     want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,

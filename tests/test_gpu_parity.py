@@ -349,3 +349,57 @@ def test_tma_staging_matches_register_gather_full_size(cuda_device):
     ob = _run(w, cuda_device, dv, b)
     assert torch.equal(oa.view(torch.int16), ob.view(torch.int16))
     assert ng.ngram_get_device_error(b)[0] == ng.NGRAM_OK
+
+
+# --------------------------------------------------------------------------- host buffers
+def _host_inputs(inp, w, pinned=True):
+    t = torch.from_numpy(np.ascontiguousarray(inp["tokens"]))
+    h = None if inp["history"] is None else torch.from_numpy(np.ascontiguousarray(inp["history"]))
+    r = torch.from_numpy(inp["residual"].view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
+    if pinned:
+        t, r = t.pin_memory(), r.pin_memory()
+        h = None if h is None else h.pin_memory()
+    return t, h, r
+
+
+@pytest.mark.parametrize("name", ["tiny", "full_prefill", "full_decode_256", "full_decode_1"])
+def test_forward_host_buffers_equal_device_forward(cuda_device, name):
+    """Chunked, three-stream pipeline over host buffers: the same bits as the device
+    call, including contexts that straddle chunk boundaries of one long sequence."""
+    w = W[name]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    ref = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    t, h, r = _host_inputs(inp, w)
+    out = ng.ngram_forward_host(ctx, t, r, dv["gate"], history=h)
+    torch.cuda.current_stream().synchronize()
+    assert np.array_equal(out.view(torch.int16).numpy().view(np.uint16), ref)
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
+def test_forward_host_back_to_back_and_pageable(cuda_device):
+    """Consecutive calls reuse the double buffers; pageable host memory also works."""
+    w = W["mid"]
+    table, _ = TABLES.get(w.R, w.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(w.vocab), w.N)
+    outs, refs = [], []
+    for seed, pinned in ((11, True), (12, True), (13, False)):
+        inp, dv = workload_on_device(w, cuda_device, token_seed=seed)
+        refs.append(from_dev_bf16(_run(w, cuda_device, dv, ctx)))
+        t, h, r = _host_inputs(inp, w, pinned)
+        outs.append(ng.ngram_forward_host(ctx, t, r, dv["gate"], history=h))
+    torch.cuda.current_stream().synchronize()
+    for o, ref in zip(outs, refs):
+        assert np.array_equal(o.view(torch.int16).numpy().view(np.uint16), ref)
+
+
+def test_forward_host_rejects_staged_modes(cuda_device):
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    table, _ = TABLES.get(w.R, w.d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, w.R, w.d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM,
+                        _hp(w.vocab, flags=ng.NGRAM_FLAG_DEDUP), w.N)
+    t, h, r = _host_inputs(inp, w)
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_forward_host(ctx, t, r, dv["gate"])
+    assert ei.value.status == ng.NGRAM_EUNSUPPORTED
