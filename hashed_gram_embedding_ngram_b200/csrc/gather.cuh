@@ -12,8 +12,9 @@
 //     broadcast with shuffles, so there is no shared memory and no block barrier.
 //   * For each strip a lane owns one 16-byte column vector (8 bf16): it issues all H
 //     row loads (16 x 16 B in flight per lane, 8 KB per warp) plus the residual load
-//     before the first add, then sums in head order 0..H-1 in fp32, applies
-//     y = r + g * acc with separately rounded multiply and add, and stores bf16.
+//     before the first add, then sums in head order 0..H-1 in fp32 (packed pairs of
+//     columns, each rounded like a scalar add), applies y = r + g * acc with separately
+//     rounded multiply and add, and stores bf16.
 //   * Work items are dealt to a persistent grid (blocks = SMs x resident blocks);
 //     decode-sized batches split a token's strips across warps for latency, large
 //     batches keep all strips of a token in one warp so the hash is computed once.
@@ -111,29 +112,28 @@ __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const
             const float4 ga = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v);
             const float4 gb = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v + 1u);
 
-            float acc[8];
+            // acc[p] holds columns (2p, 2p+1): packed pair adds round each lane exactly as
+            // the scalar head-order sum
+            float2 acc[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int p = 0; p < 4; ++p) acc[p] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
                 if (kH || h < static_cast<int>(H)) {
-                    acc[0] = __fadd_rn(acc[0], bf16_lo(e[h].x));
-                    acc[1] = __fadd_rn(acc[1], bf16_hi(e[h].x));
-                    acc[2] = __fadd_rn(acc[2], bf16_lo(e[h].y));
-                    acc[3] = __fadd_rn(acc[3], bf16_hi(e[h].y));
-                    acc[4] = __fadd_rn(acc[4], bf16_lo(e[h].z));
-                    acc[5] = __fadd_rn(acc[5], bf16_hi(e[h].z));
-                    acc[6] = __fadd_rn(acc[6], bf16_lo(e[h].w));
-                    acc[7] = __fadd_rn(acc[7], bf16_hi(e[h].w));
+                    acc[0] = add2(acc[0], bf16x2(e[h].x));
+                    acc[1] = add2(acc[1], bf16x2(e[h].y));
+                    acc[2] = add2(acc[2], bf16x2(e[h].z));
+                    acc[3] = add2(acc[3], bf16x2(e[h].w));
                 }
             }
+            // y = r + (g * acc): the product is rounded on its own (scalar, never fused)
             const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
             const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
             uint32_t o[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                const float y0 = __fadd_rn(bf16_lo(rw[p]), __fmul_rn(gv[2 * p], acc[2 * p]));
-                const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[2 * p + 1]));
+                const float y0 = __fadd_rn(bf16_lo(rw[p]), __fmul_rn(gv[2 * p], acc[p].x));
+                const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[p].y));
                 o[p] = pack_bf16x2(y0, y1);
             }
             *reinterpret_cast<uint4 *>(g.out + tok_off + v * 8u) = make_uint4(o[0], o[1], o[2], o[3]);

@@ -11,17 +11,15 @@
 
 namespace ngram {
 
-// int8 byte j (0..3) of word w -> exact fp32 value.  The sign bit is flipped (q + 128
-// in [0, 255]), the byte is placed in the mantissa of 2^23 with one byte permute, and
+// Exact int8 -> fp32: the sign bit of each byte is flipped (q + 128 in [0, 255]), one byte
+// permute places the byte in the mantissa of 2^23 (the float 2^23 + 128 + q), and
 // 2^23 + 128 is subtracted; every step is exact.
-__device__ __forceinline__ float int8_at(uint32_t biased, uint32_t j) {
-    return __fsub_rn(__uint_as_float(__byte_perm(biased, 0x4B000000u, 0x7540u + j)), 8388736.0f);
-}
 
 // int8 rows with one fp32 scale per row: value = q * scale[row].  A lane owns 16
 // columns (one 16-byte vector of the row); the per-row scales are loaded once per token
-// by the hashing lanes and broadcast with the row indices.  Sum per head in order:
-// acc = acc + (q * s), each step rounded separately, then the same bf16 epilogue.
+// by the hashing lanes and broadcast with the row indices.  Sum per head in order with
+// one fused multiply-add per head, acc = fma(q, s, acc) (one rounding per head), then
+// the same bf16 epilogue as the bf16 rows.
 template <int kH>
 __global__ void __launch_bounds__(256, 2) k_gather_int8(const GatherArgs g) {
     const uint32_t lane = threadIdx.x & 31u;
@@ -58,32 +56,41 @@ __global__ void __launch_bounds__(256, 2) k_gather_int8(const GatherArgs g) {
             const uint4 r0 = ld_na_v4(g.residual + tok_off + v * 16u);
             const uint4 r1 = ld_na_v4(g.residual + tok_off + v * 16u + 8u);
 
-            float acc[16];
+            // acc[k] holds columns (2k, 2k+1); per head, acc = fma(q, s, acc) on both lanes
+            float2 acc[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 8; ++j) acc[j] = make_float2(0.0f, 0.0f);
+            const float2 bias = make_float2(8388736.0f, 8388736.0f);       // 2^23 + 128
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
                 if (kH || h < static_cast<int>(H)) {
                     const uint32_t wv[4] = {e[h].x ^ 0x80808080u, e[h].y ^ 0x80808080u,
                                             e[h].z ^ 0x80808080u, e[h].w ^ 0x80808080u};
+                    const float2 s2 = make_float2(sc[h], sc[h]);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            acc[4 * k + j] = __fadd_rn(acc[4 * k + j],
-                                                       __fmul_rn(int8_at(wv[k], j), sc[h]));
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 lo = sub2(make_float2(
+                            __uint_as_float(__byte_perm(wv[k], 0x4B000000u, 0x7540u)),
+                            __uint_as_float(__byte_perm(wv[k], 0x4B000000u, 0x7541u))), bias);
+                        const float2 hi = sub2(make_float2(
+                            __uint_as_float(__byte_perm(wv[k], 0x4B000000u, 0x7542u)),
+                            __uint_as_float(__byte_perm(wv[k], 0x4B000000u, 0x7543u))), bias);
+                        acc[2 * k] = fma2(lo, s2, acc[2 * k]);
+                        acc[2 * k + 1] = fma2(hi, s2, acc[2 * k + 1]);
+                    }
                 }
             }
             const float4 *gp = reinterpret_cast<const float4 *>(g.gate) + 4u * v;
             const float4 g0 = __ldg(gp), g1 = __ldg(gp + 1), g2 = __ldg(gp + 2), g3 = __ldg(gp + 3);
+            // y = r + (g * acc): the product is rounded on its own (scalar, never fused)
             const float gv[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w,
                                   g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
             const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
             uint32_t o[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const float y0 = __fadd_rn(bf16_lo(rw[p]), __fmul_rn(gv[2 * p], acc[2 * p]));
-                const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[2 * p + 1]));
+                const float y0 = __fadd_rn(bf16_lo(rw[p]), __fmul_rn(gv[2 * p], acc[p].x));
+                const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[p].y));
                 o[p] = pack_bf16x2(y0, y1);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(g.out + tok_off + v * 16u);

@@ -65,6 +65,8 @@ WORKLOADS = {
     "host_prefill": Workload("host_prefill", 20_000_000, 2560, "bf16", 151_936, 1, 8192, residency="host"),
     # profiling case for full ncu captures: 400k x 2560 bf16 (2 GB), 4 x 2048 Zipf tokens
     "profile_small": Workload("profile_small", 400_000, 2560, "bf16", 151_936, 4, 2048),
+    # profiling case for the int8 gather: 1M x 2560 int8 (2.4 GiB), 16 x 1024 uniform tokens
+    "profile_int8": Workload("profile_int8", 1_000_000, 2560, "int8", 151_936, 16, 1024, tokens="uniform"),
     # 20M x 2560 int8 + fp32 row scale (47.8 GiB), 65,536 uniform tokens (little reuse)
     "int8_uniform": Workload("int8_uniform", 20_000_000, 2560, "int8", 151_936, 16, 4096, tokens="uniform"),
 }

@@ -36,10 +36,12 @@
  *   ORACLE_ACC_F64 -- the plain definition.  The 16 products/values are summed in
  *                     double (exact for these operands), gate and add in double, and
  *                     the result is rounded once to bf16 (round to nearest even).
- *   ORACLE_ACC_F32 -- the fp32-accumulated reference: fp32 sum in head order 0..H-1,
- *                     then a separately rounded fp32 multiply by g and fp32 add of the
- *                     residual, then bf16 round to nearest even.  Build with
- *                     -ffp-contract=off so no step is fused.
+ *   ORACLE_ACC_F32 -- the fp32-accumulated reference: fp32 sum in head order 0..H-1
+ *                     (bf16 rows: acc = acc + E; int8 rows: acc = fmaf(q, s, acc), one
+ *                     correctly rounded fused multiply-add per head), then a separately
+ *                     rounded fp32 multiply by g and fp32 add of the residual, then bf16
+ *                     round to nearest even.  Build with -ffp-contract=off so that no
+ *                     step other than the explicit fmaf is fused.
  */
 #include <stdint.h>
 #include <stddef.h>
@@ -312,20 +314,23 @@ int oracle_indices(const int32_t *tokens, const int32_t *history, uint32_t n_seq
  *   n_threads > 1 splits the token loop across OpenMP threads (per-token work and
  *   arithmetic are unchanged).
  * ---------------------------------------------------------------------------------- */
+/* Element (row, col) of the table: bf16 value v (q = v, s = 1 is not used), or the
+ * int8 pair (q, s).  Returns the exact value in double. */
 static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
                         const float *scale, uint64_t seed, uint64_t row, uint32_t col,
-                        uint32_t d, int acc_mode, float *as_f32)
+                        uint32_t d, float *v_or_q, float *s_out)
 {
     if (dtype == ORACLE_BF16) {
         uint16_t b = table_bf16 ? table_bf16[row * d + col] : oracle_table_bf16(seed, row, col);
         float f = oracle_f32_from_bf16(b);
-        *as_f32 = f;
+        *v_or_q = f;
+        *s_out = 1.0f;
         return (double)f;
     } else {
         int8_t q = table_i8 ? table_i8[row * d + col] : oracle_table_int8(seed, row, col);
         float sc = scale ? scale[row] : oracle_row_scale(seed, row);
-        *as_f32 = (float)q * sc;                   /* fp32 product, rounded */
-        (void)acc_mode;
+        *v_or_q = (float)q;                        /* exact */
+        *s_out = sc;
         return (double)q * (double)sc;             /* exact in double */
     }
 }
@@ -362,11 +367,14 @@ int oracle_forward(int dtype, const uint16_t *table_bf16, const int8_t *table_i8
             float r32 = oracle_f32_from_bf16(residual[flat * d + c]);
             float g32 = gate[c];
             for (h = 0; h < H; h++) {
-                float e32;
+                float v, sc;
                 double e64 = row_value(dtype, table_bf16, table_i8, row_scale, table_seed,
-                                       idx[h], c, d, acc_mode, &e32);
+                                       idx[h], c, d, &v, &sc);
                 acc64 += e64;
-                acc32 = acc32 + e32;               /* fp32, head order */
+                if (dtype == ORACLE_BF16)
+                    acc32 = acc32 + v;             /* fp32, head order */
+                else
+                    acc32 = fmaf(v, sc, acc32);    /* q * s + acc, one rounding per head */
                 mag += fabs(e64);
             }
             if (acc_mode == ORACLE_ACC_F64) {

@@ -393,3 +393,34 @@ def test_unique_rows_keeps_colliding_heads():
     uniq, inv = oracle.unique_rows(idx)
     assert uniq.tolist() == [3, 7, 9]
     assert inv.tolist() == [0, 0, 0, 1, 1, 0, 2, 2]
+
+
+# --------------------------------------------------------------------------- int8 fp32 mode
+def test_fmaf_is_correctly_rounded():
+    """The oracle's int8 fp32 accumulation is one fmaf per head; check that the C
+    library's fmaf returns the float nearest to the exact a * b + c."""
+    import ctypes
+    import random
+    libm = ctypes.CDLL("libm.so.6")
+    libm.fmaf.restype = ctypes.c_float
+    libm.fmaf.argtypes = [ctypes.c_float] * 3
+    rng = random.Random(3)
+    for _ in range(5000):
+        a, b, c = (float(np.float32(rng.uniform(-1, 1) * 2.0 ** rng.randint(-30, 30)))
+                   for _ in range(3))
+        exact = Fraction(a) * Fraction(b) + Fraction(c)
+        f = np.float32(libm.fmaf(a, b, c))
+        for nb in (np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf))):
+            assert abs(Fraction(float(f)) - exact) <= abs(Fraction(float(nb)) - exact)
+
+
+def test_int8_fp32_mode_within_tolerance_of_exact():
+    R, d, V = 3000, 64, 500
+    toks, res, g = _tiny_case(R=R, d=d, V=V, n_seq=4, T=40)
+    o32 = oracle.forward(toks, None, res, g, R=R, d=d, dtype=oracle.INT8, table_seed=17,
+                         acc=oracle.ACC_F32, vocab_size=V)
+    o64, y64, mag, _ = oracle.forward(toks, None, res, g, R=R, d=d, dtype=oracle.INT8,
+                                      table_seed=17, acc=oracle.ACC_F64, vocab_size=V,
+                                      want_aux=True)
+    a, b = _bits_to_f64(o32).reshape(y64.shape), _bits_to_f64(o64).reshape(y64.shape)
+    assert np.all(np.abs(a - b) <= _bf16_ulp(b) + 2.0 ** -20 * mag)
