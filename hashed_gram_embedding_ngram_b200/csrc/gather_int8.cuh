@@ -34,25 +34,29 @@ __global__ void __launch_bounds__(256, 2) k_gather_int8(const GatherArgs g) {
         const uint32_t tok = item / g.groups_per_token;
         const uint32_t grp = item - tok * g.groups_per_token;
         const uint32_t my_row = warp_head_row(g, tok, lane, H);
+        // the scale load is issued here but first used after the row loads are in flight
         const float my_scale = (lane < H) ? __ldg(g.row_scale + my_row) : 0.0f;
         uint32_t rows[16];
-        float sc[16];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);
-            sc[h] = __shfl_sync(0xFFFFFFFFu, my_scale, h);
-        }
+        for (int h = 0; h < 16; ++h) rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);
         const uint32_t s_begin = grp * g.strips_per_item;
         const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
         const size_t tok_off = static_cast<size_t>(tok) * g.d;
         for (uint32_t s = s_begin; s < s_end; ++s) {
             const uint32_t v = s * 32u + lane;
-            if (v >= nvec) continue;
+            const bool active = v < nvec;             // the last strip may be ragged
             uint4 e[16];
+            if (active) {
 #pragma unroll
-            for (int h = 0; h < 16; ++h)
-                if (kH || h < static_cast<int>(H))
-                    e[h] = ld_stream_v4(table + static_cast<size_t>(rows[h]) * g.d + v * 16u);
+                for (int h = 0; h < 16; ++h)
+                    if (kH || h < static_cast<int>(H))
+                        e[h] = ld_stream_v4(table + static_cast<size_t>(rows[h]) * g.d + v * 16u);
+            }
+            // every lane takes part in the shuffles, after the row loads are issued
+            float sc[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) sc[h] = __shfl_sync(0xFFFFFFFFu, my_scale, h);
+            if (!active) continue;
             const uint4 r0 = ld_na_v4(g.residual + tok_off + v * 16u);
             const uint4 r1 = ld_na_v4(g.residual + tok_off + v * 16u + 8u);
 
