@@ -290,7 +290,9 @@ def run_ours(args, w):
         table = torch.empty((w.R, w.d), dtype=torch.int8, device=dev)
         scale = torch.empty((w.R,), dtype=torch.float32, device=dev)
     ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
-    flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING}[args.variant]
+    flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING,
+             "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER}[args.variant]
+    grouped = args.variant == "sort" or (args.variant == "default" and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
     hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
 
@@ -417,9 +419,10 @@ def run_ours(args, w):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": profiled_traffic(w.name, w.dtype) if args.variant == "default" else None,
-                         "kernel": {"default": "k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8<16>",
-                                    "tma": "k_gather_bf16_bulk<16>",
-                                    "dedup": "hash + dedup + compact + gather (8 kernels)"}[args.variant],
+                         "kernel": ("hash + dedup + compact + gather (8 kernels)" if args.variant == "dedup"
+                                    else "k_gather_bf16_bulk<16>" if args.variant == "tma"
+                                    else ("grouped order (3 kernels) + " if grouped else "")
+                                    + ("k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8<16>")),
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -429,7 +432,7 @@ def run_ours(args, w):
                     if args.variant == "default" else
                             "pinned host tokens + residual -> device, ngram_forward, out -> pinned host"},
             "clocks": clocks,
-            "gpu_launches": K * {"default": 1, "tma": 1, "dedup": 8}[args.variant],
+            "gpu_launches": K * (8 if args.variant == "dedup" else 4 if grouped else 1),
         }
         if world == 1 and not args.no_cpu_baseline:
             threads = os.cpu_count() or 1
@@ -598,8 +601,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
                     help="eager launches, or 100-step CUDA graphs (auto: graph for N <= 1024)")
-    ap.add_argument("--variant", default="default", choices=["default", "dedup", "tma"],
-                    help="HBM path: fused gather (default), dedup + staged gather, TMA staging")
+    ap.add_argument("--variant", default="default",
+                    choices=["default", "dedup", "tma", "sort", "batch_order"],
+                    help="HBM path: library default (grouped order from 16,384 tokens), dedup + "
+                         "staged gather, TMA staging, always grouped, always batch order")
     ap.add_argument("--host-workloads", default="host_decode_1,host_decode_16,host_decode_64,"
                                                 "host_decode_256,host_prefill")
     ap.add_argument("--host-steps", type=int, default=200)

@@ -33,6 +33,9 @@ NGRAM_RES_HBM, NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO = 0, 
 
 NGRAM_FLAG_DEDUP = 0x1
 NGRAM_FLAG_TMA_STAGING = 0x2
+NGRAM_FLAG_SORT = 0x4
+NGRAM_FLAG_BATCH_ORDER = 0x8
+NGRAM_SORT_MIN_TOKENS = 16384
 
 MAX_HEADS = 16
 DEFAULT_BASE_SEED = 0x6E6772616D5F7631

@@ -34,6 +34,7 @@ struct GatherArgs {
     const float *gate;          // [d]
     uint16_t *out;              // [N][d] bf16 bits (may alias residual)
     const uint32_t *row_ids;    // [N][H] precomputed row ids into `table`, or null (hash)
+    const uint32_t *perm;       // [N] processing order of the tokens, or null (batch order)
     uint32_t *err;              // device error word
     uint32_t T;
     uint32_t N;                 // tokens of this launch: flat tokens [tok_begin, tok_begin + N)
@@ -89,8 +90,9 @@ __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const
     const uint16_t *__restrict__ table = static_cast<const uint16_t *>(g.table);
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {
-        const uint32_t tok = item / g.groups_per_token;
-        const uint32_t grp = item - tok * g.groups_per_token;
+        const uint32_t pos = item / g.groups_per_token;
+        const uint32_t grp = item - pos * g.groups_per_token;
+        const uint32_t tok = g.perm ? __ldg(g.perm + pos) : pos;
         const uint32_t my_row = warp_head_row(g, tok, lane, H);
         uint32_t rows[16];
 #pragma unroll

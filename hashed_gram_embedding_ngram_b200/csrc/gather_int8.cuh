@@ -31,8 +31,9 @@ __global__ void __launch_bounds__(256, 2) k_gather_int8(const GatherArgs g) {
     const int8_t *__restrict__ table = static_cast<const int8_t *>(g.table);
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {
-        const uint32_t tok = item / g.groups_per_token;
-        const uint32_t grp = item - tok * g.groups_per_token;
+        const uint32_t pos = item / g.groups_per_token;
+        const uint32_t grp = item - pos * g.groups_per_token;
+        const uint32_t tok = g.perm ? __ldg(g.perm + pos) : pos;
         const uint32_t my_row = warp_head_row(g, tok, lane, H);
         // the scale load is issued here but first used after the row loads are in flight
         const float my_scale = (lane < H) ? __ldg(g.row_scale + my_row) : 0.0f;

@@ -24,6 +24,7 @@
 #include "gather_int8.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
+#include "order.cuh"
 
 using namespace ngram;
 
@@ -98,6 +99,8 @@ struct ngram_ctx {
     uint32_t hp_chunk;          // tokens per chunk
     cudaStream_t hp_s[3];       // H2D, compute, D2H
     cudaEvent_t hp_entry, hp_h2d[2], hp_kdone[2], hp_d2h[2];
+    // NGRAM_FLAG_SORT: bucket of each token, bucket counts / cursors, processing order
+    uint32_t *so_bucket, *so_hist, *so_perm;
 };
 
 namespace {
@@ -214,7 +217,8 @@ void free_all(ngram_ctx *c) {
                          c->hp_d2h[0], c->hp_d2h[1]};
     for (cudaEvent_t e : evs)
         if (e) cudaEventDestroy(e);
-    void *bufs[] = {c->hp_tok, c->hp_hist, c->hp_res[0], c->hp_res[1], c->hp_out[0], c->hp_out[1]};
+    void *bufs[] = {c->hp_tok, c->hp_hist, c->hp_res[0], c->hp_res[1], c->hp_out[0], c->hp_out[1],
+                    c->so_bucket, c->so_hist, c->so_perm};
     for (void *p : bufs)
         if (p) cudaFree(p);
     for (cudaStream_t s : c->hp_s)
@@ -301,6 +305,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.gate = gate;
     g.out = out;
     g.row_ids = nullptr;
+    g.perm = nullptr;
     g.err = c->d_err;
     g.T = T;
     g.N = N;
@@ -492,8 +497,41 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
 
 // UVA: the same kernel reading host rows over PCIe.  A bounded grid suffices to keep
 // PCIe busy and leaves the other SMs to whatever runs beside the lookup.
+// Whether an HBM batch of N tokens is gathered in grouped order: always with
+// NGRAM_FLAG_SORT, never with NGRAM_FLAG_BATCH_ORDER or TMA staging, else from
+// NGRAM_SORT_MIN_TOKENS tokens on.
+bool grouped_order(const ngram_ctx *c, uint32_t N) {
+    const uint32_t f = c->hp.flags;
+    if (f & NGRAM_FLAG_SORT) return true;
+    if (f & (NGRAM_FLAG_BATCH_ORDER | NGRAM_FLAG_TMA_STAGING)) return false;
+    return N >= NGRAM_SORT_MIN_TOKENS;
+}
+
+// Grouped order: tokens grouped by bigram context (counting sort on a 13-bit hash),
+// then the fused gather walks them in that order.  Same outputs; repeated rows run back
+// to back so L2 serves the repeats.
+ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
+    if (!c->so_perm) {
+        NG_CUDA(cudaMalloc(&c->so_bucket, c->max_tokens * 4ull), "order scratch");
+        NG_CUDA(cudaMalloc(&c->so_hist, kOrderBuckets * 4ull), "order scratch");
+        NG_CUDA(cudaMalloc(&c->so_perm, c->max_tokens * 4ull), "order scratch");
+    }
+    const HashArgs a = hash_args(c);
+    const unsigned gn = grid_for(c, k.N, 256);
+    NG_CUDA(cudaMemsetAsync(c->so_hist, 0, kOrderBuckets * 4ull, k.s), "order clear");
+    k_order_count<<<gn, 256, 0, k.s>>>(k.tokens, k.history, k.T, k.N, a, c->d_err, c->so_bucket, c->so_hist);
+    k_order_scan<<<1, 1024, 0, k.s>>>(c->so_hist);
+    k_order_scatter<<<gn, 256, 0, k.s>>>(c->so_bucket, k.N, c->so_hist, c->so_perm);
+    NG_CUDA(cudaGetLastError(), "order launch");
+    GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
+    g.perm = c->so_perm;
+    return launch_gather(c, g, k.s, max_blocks);
+}
+
 ngram_status forward_uva(ngram_ctx *c, const Call &k) {
-    return forward_direct(c, k, std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c)));
+    const uint64_t blocks = std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c));
+    if (c->hp.flags & NGRAM_FLAG_SORT) return forward_sorted(c, k, blocks);
+    return forward_direct(c, k, blocks);
 }
 
 // AUTO: the first call of each batch-size bucket runs and times both host modes
@@ -603,6 +641,11 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
         return fail(NGRAM_EINVAL, "max_tokens %u too large for d = %u", max_tokens, d);
     if ((p.flags & NGRAM_FLAG_DEDUP) && where != NGRAM_RES_HBM)
         return fail(NGRAM_EINVAL, "NGRAM_FLAG_DEDUP applies to HBM residency (host modes dedup on their own)");
+    if ((p.flags & NGRAM_FLAG_SORT) && where != NGRAM_RES_HBM && where != NGRAM_RES_HOST_UVA)
+        return fail(NGRAM_EINVAL, "NGRAM_FLAG_SORT applies to HBM and HOST_UVA residency");
+    if ((p.flags & NGRAM_FLAG_SORT) &&
+        (p.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_BATCH_ORDER)))
+        return fail(NGRAM_EINVAL, "NGRAM_FLAG_SORT does not combine with DEDUP, TMA_STAGING or BATCH_ORDER");
 
     // ---- CUDA from here on
     ngram_ctx *c = new ngram_ctx();
@@ -696,6 +739,7 @@ ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *h
     switch (c->where) {
         case NGRAM_RES_HBM:
             if (c->hp.flags & NGRAM_FLAG_DEDUP) return forward_dedup_hbm(c, k);
+            if (grouped_order(c, k.N)) return forward_sorted(c, k, full_grid(c));
             return forward_direct(c, k, full_grid(c));
         case NGRAM_RES_HOST_UVA: return forward_uva(c, k);
         case NGRAM_RES_HOST_DMA: return forward_dma(c, k);
@@ -713,7 +757,7 @@ ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int
     if (residual_h == nullptr || gate == nullptr || out_h == nullptr)
         return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
     if (!aligned16(gate)) return fail(NGRAM_EINVAL, "gate must be 16-byte aligned");
-    if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING)) ||
+    if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT)) ||  // chunks keep batch order
         (c->where != NGRAM_RES_HBM && c->where != NGRAM_RES_HOST_UVA))
         return fail(NGRAM_EUNSUPPORTED,
                     "ngram_forward_host pipelines the fused gather: HBM or HOST_UVA residency, no flags");

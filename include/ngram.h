@@ -85,7 +85,20 @@ typedef enum {
  * an mbarrier ring) instead of register loads.  Same results bit for bit; measured
  * slower on B200 (522-895 us vs 455 us on the full-size gather), kept for comparison. */
 #define NGRAM_FLAG_TMA_STAGING 0x2u
-#define NGRAM_FLAGS_KNOWN (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING)
+/* Grouped order: before the gather, group the batch's tokens by bigram context
+ * (counting sort on a 13-bit hash of (w_{t-1}, w_t): 3 small kernels and a memset, ~11 us)
+ * and gather in that order, so tokens that read the same rows run back to back and L2
+ * serves the repeats.  Same results bit for bit.  Scratch (8 bytes per max_tokens + 32 KB)
+ * is allocated by the first call that groups.
+ *   HBM residency groups by default when N >= NGRAM_SORT_MIN_TOKENS (measured on B200
+ *   with Zipf tokens: break-even near 12,288 tokens, 3-6% faster from 16,384 up).
+ *   NGRAM_FLAG_SORT groups every batch (HBM or HOST_UVA); NGRAM_FLAG_BATCH_ORDER never
+ *   groups. */
+#define NGRAM_FLAG_SORT 0x4u
+#define NGRAM_FLAG_BATCH_ORDER 0x8u
+#define NGRAM_SORT_MIN_TOKENS 16384u
+#define NGRAM_FLAGS_KNOWN (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT | \
+                           NGRAM_FLAG_BATCH_ORDER)
 
 #define NGRAM_MAX_HEADS 16u
 #define NGRAM_TOKEN_BITS 21u

@@ -134,3 +134,14 @@ def test_dedup_flag_is_for_hbm_only():
     with pytest.raises(ng.NgramError) as ei:
         ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_DMA, hp, 16)
     assert ei.value.status == ng.NGRAM_EINVAL and "HBM" in str(ei.value)
+
+
+def test_sort_flag_combinations_rejected():
+    for where, flags in ((ng.NGRAM_RES_HOST_DMA, ng.NGRAM_FLAG_SORT),
+                         (ng.NGRAM_RES_HBM, ng.NGRAM_FLAG_SORT | ng.NGRAM_FLAG_DEDUP),
+                         (ng.NGRAM_RES_HBM, ng.NGRAM_FLAG_SORT | ng.NGRAM_FLAG_TMA_STAGING),
+                         (ng.NGRAM_RES_HBM, ng.NGRAM_FLAG_SORT | ng.NGRAM_FLAG_BATCH_ORDER)):
+        with pytest.raises(ng.NgramError) as ei:
+            ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, where,
+                          ng.ngram_default_hash_params(flags=flags), 16)
+        assert ei.value.status == ng.NGRAM_EINVAL

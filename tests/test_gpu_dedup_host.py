@@ -167,15 +167,16 @@ def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
     dev_table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
     hbm = ng.ngram_init(dev_table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
     ref = from_dev_bf16(_forward(hbm, dv))
-    for where in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA, ng.NGRAM_RES_HOST_AUTO):
-        ctx = host_bf16.ctx(where, V, w.N)
+    for where, flags in ((ng.NGRAM_RES_HOST_UVA, 0), (ng.NGRAM_RES_HOST_DMA, 0),
+                         (ng.NGRAM_RES_HOST_AUTO, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT)):
+        ctx = host_bf16.ctx(where, V, w.N, flags=flags)
         for _ in range(2):                       # second call reuses the staging buffers
             got = from_dev_bf16(_forward(ctx, dv))
             assert np.array_equal(got, ref), where
         assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
         if where == ng.NGRAM_RES_HOST_AUTO:
             assert ng.ngram_auto_choice(ctx, w.N) in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA)
-        if where == ng.NGRAM_RES_HOST_UVA:       # host table and host activations together
+        if where == ng.NGRAM_RES_HOST_UVA and not flags:   # host table and host activations
             t = torch.from_numpy(inp["tokens"]).pin_memory()
             h = None if inp["history"] is None else torch.from_numpy(inp["history"]).pin_memory()
             r = torch.from_numpy(inp["residual"].view(np.int16)).view(torch.bfloat16).view(w.N, d)

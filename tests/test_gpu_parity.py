@@ -403,3 +403,40 @@ def test_forward_host_rejects_staged_modes(cuda_device):
     with pytest.raises(ng.NgramError) as ei:
         ng.ngram_forward_host(ctx, t, r, dv["gate"])
     assert ei.value.status == ng.NGRAM_EUNSUPPORTED
+
+
+# --------------------------------------------------------------------------- grouped order
+@pytest.mark.parametrize("name", ["tiny", "mid", "full_prefill", "full_decode_1",
+                                  "full_decode_256", "int8_uniform"])
+def test_sort_flag_is_bit_identical(cuda_device, name):
+    """Tokens processed grouped by bigram context give exactly the batch-order output;
+    the default (grouped from NGRAM_SORT_MIN_TOKENS tokens) agrees with both."""
+    w = W[name]
+    inp, dv = workload_on_device(w, cuda_device)
+    dtype = ng.NGRAM_BF16 if w.dtype == "bf16" else ng.NGRAM_INT8_ROWSCALE
+    table, scale = TABLES.get(w.R, w.d, dtype, gen.TABLE_SEED, cuda_device)
+    ctxs = [ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, _hp(w.vocab, flags=f), w.N,
+                          row_scale=scale)
+            for f in (ng.NGRAM_FLAG_BATCH_ORDER, ng.NGRAM_FLAG_SORT, 0)]
+    ref = _run(w, cuda_device, dv, ctxs[0])
+    for ctx in ctxs[1:]:
+        for _ in range(2):                   # scratch reuse across calls
+            got = _run(w, cuda_device, dv, ctx)
+            assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+        assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
+def test_sort_flag_ragged_heads(cuda_device):
+    R, d, V = 4099, 136, 300                # small vocabulary: many repeated contexts
+    w = gen.Workload("ragged_sort", R, d, "bf16", V, 3, 211, history=True)
+    inp = gen.make_inputs(w, token_seed=77)
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM,
+                        _hp(V, 3, 5, flags=ng.NGRAM_FLAG_SORT), w.N)
+    dv = {"tokens": to_dev_tokens(inp["tokens"], cuda_device),
+          "history": to_dev_tokens(inp["history"], cuda_device),
+          "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
+          "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
+    got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    r = assert_parity(got, _oracle(w, inp, n_bigram=3, n_trigram=5))
+    assert r["exact"] == r["n"]
