@@ -139,10 +139,11 @@ NGRAM_API ngram_status ngram_host_free(void *p);
  *              HBM       one fused kernel per call;
  *              HOST_UVA  the same kernel reads the rows from host memory over PCIe;
  *              HOST_DMA  rows are deduplicated on the GPU, the distinct rows are copied
- *                        by host threads into pinned staging and moved to HBM by the
- *                        copy engine in 8 MB chunks (copy and host gather overlap),
- *                        then gathered from HBM; the call blocks the host until the
- *                        rows are staged (bounded wait, see ngram_set_wait_timeout);
+ *                        by host threads (OpenMP: OMP_NUM_THREADS / OMP_WAIT_POLICY
+ *                        apply) into pinned staging and moved to HBM by the copy engine
+ *                        in 8 MB chunks (copy and host gather overlap), then gathered
+ *                        from HBM; the call blocks the host until the rows are staged
+ *                        (bounded wait, see ngram_set_wait_timeout);
  *              HOST_AUTO the first call of each batch-size bucket (ceil(log2 N)) runs
  *                        and times both UVA and DMA (synchronously), later calls use
  *                        the faster (ngram_auto_choice reports it).
