@@ -57,6 +57,13 @@ using namespace ngram;
 #define NGRAM_DMA_CHUNK_BYTES (8u << 20)
 #endif
 
+// ngram_forward_host pipeline (measured, 32,768-token prefill, pinned host buffers): 16 MB
+// chunks on 3 streams 4.20 ms; 8 MB on 2 streams 4.27-4.48 ms; 4 MB 4.6-5.2 ms; a thinner
+// gather grid does not help.  The copies alone, both directions, take 3.50 ms.
+#ifndef NGRAM_HOST_BUFFERS              // pipeline streams of ngram_forward_host
+#define NGRAM_HOST_BUFFERS 3
+#endif
+
 struct ngram_ctx {
     const void *table;          // caller's pointer (device, or host for host residency)
     const void *table_dev;      // device-visible alias used by kernels (UVA), or table
@@ -95,10 +102,12 @@ struct ngram_ctx {
     int auto_choice[33];        // per ceil(log2 N): 0 undecided, else ngram_residency
     // ngram_forward_host: device copies of the host inputs, double-buffered chunks
     int32_t *hp_tok, *hp_hist;
-    uint16_t *hp_res[2], *hp_out[2];
+    uint16_t *hp_res[NGRAM_HOST_BUFFERS], *hp_out[NGRAM_HOST_BUFFERS];
     uint32_t hp_chunk;          // tokens per chunk
-    cudaStream_t hp_s[3];       // H2D, compute, D2H
-    cudaEvent_t hp_entry, hp_h2d[2], hp_kdone[2], hp_d2h[2];
+    cudaStream_t hp_s[NGRAM_HOST_BUFFERS];   // pipeline streams, one chunk buffer pair each
+    cudaEvent_t hp_entry;
+    cudaEvent_t hp_h2d[NGRAM_HOST_BUFFERS];   // [0]: tokens uploaded
+    cudaEvent_t hp_d2h[NGRAM_HOST_BUFFERS];   // end of each stream's part of the last call
     // NGRAM_FLAG_SORT: bucket of each token, bucket counts / cursors, processing order
     uint32_t *so_bucket, *so_hist, *so_perm;
 };
@@ -212,13 +221,17 @@ void free_all(ngram_ctx *c) {
     if (c->h_stage_scale) cudaFreeHost(c->h_stage_scale);
     if (c->h_uniq) cudaFreeHost(c->h_uniq);
     if (c->h_count) cudaFreeHost(c->h_count);
-    cudaEvent_t evs[] = {c->ev_sync, c->ev_stage_free, c->ev_t0, c->ev_t1, c->hp_entry,
-                         c->hp_h2d[0], c->hp_h2d[1], c->hp_kdone[0], c->hp_kdone[1],
-                         c->hp_d2h[0], c->hp_d2h[1]};
+    cudaEvent_t evs[] = {c->ev_sync, c->ev_stage_free, c->ev_t0, c->ev_t1, c->hp_entry};
     for (cudaEvent_t e : evs)
         if (e) cudaEventDestroy(e);
-    void *bufs[] = {c->hp_tok, c->hp_hist, c->hp_res[0], c->hp_res[1], c->hp_out[0], c->hp_out[1],
-                    c->so_bucket, c->so_hist, c->so_perm};
+    for (int b = 0; b < NGRAM_HOST_BUFFERS; ++b) {
+        cudaEvent_t pe[] = {c->hp_h2d[b], c->hp_d2h[b]};
+        for (cudaEvent_t e : pe)
+            if (e) cudaEventDestroy(e);
+        if (c->hp_res[b]) cudaFree(c->hp_res[b]);
+        if (c->hp_out[b]) cudaFree(c->hp_out[b]);
+    }
+    void *bufs[] = {c->hp_tok, c->hp_hist, c->so_bucket, c->so_hist, c->so_perm};
     for (void *p : bufs)
         if (p) cudaFree(p);
     for (cudaStream_t s : c->hp_s)
@@ -266,7 +279,7 @@ ngram_status ensure_host_stage(ngram_ctx *c) {
 }
 
 #ifndef NGRAM_HOST_CHUNK_BYTES          // residual bytes per pipelined chunk (host buffers)
-#define NGRAM_HOST_CHUNK_BYTES (8u << 20)
+#define NGRAM_HOST_CHUNK_BYTES (16u << 20)
 #endif
 
 ngram_status ensure_host_path(ngram_ctx *c) {
@@ -278,15 +291,14 @@ ngram_status ensure_host_path(ngram_ctx *c) {
     c->hp_chunk = static_cast<uint32_t>(chunk);
     NG_CUDA(cudaMalloc(&c->hp_tok, c->max_tokens * 4ull), "host-path buffers");
     NG_CUDA(cudaMalloc(&c->hp_hist, c->max_tokens * 8ull), "host-path buffers");
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NGRAM_HOST_BUFFERS; ++b) {
         NG_CUDA(cudaMalloc(&c->hp_res[b], chunk * row), "host-path buffers");
         NG_CUDA(cudaMalloc(&c->hp_out[b], chunk * row), "host-path buffers");
         NG_CUDA(cudaEventCreateWithFlags(&c->hp_h2d[b], cudaEventDisableTiming), "cudaEventCreate");
-        NG_CUDA(cudaEventCreateWithFlags(&c->hp_kdone[b], cudaEventDisableTiming), "cudaEventCreate");
         NG_CUDA(cudaEventCreateWithFlags(&c->hp_d2h[b], cudaEventDisableTiming), "cudaEventCreate");
     }
     NG_CUDA(cudaEventCreateWithFlags(&c->hp_entry, cudaEventDisableTiming), "cudaEventCreate");
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < NGRAM_HOST_BUFFERS; ++i)
         NG_CUDA(cudaStreamCreateWithFlags(&c->hp_s[i], cudaStreamNonBlocking), "cudaStreamCreate");
     return NGRAM_OK;
 }
@@ -762,47 +774,47 @@ ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int
         return fail(NGRAM_EUNSUPPORTED,
                     "ngram_forward_host pipelines the fused gather: HBM or HOST_UVA residency, no flags");
     NG_CHECK(ensure_host_path(c));
+    constexpr int S = NGRAM_HOST_BUFFERS;
     cudaStream_t caller = reinterpret_cast<cudaStream_t>(stream);
-    cudaStream_t sh = c->hp_s[0], sk = c->hp_s[1], sd = c->hp_s[2];
     const uint64_t row = 2ull * c->d;
     const uint64_t max_blocks = (c->where == NGRAM_RES_HOST_UVA)
         ? std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c)) : full_grid(c);
-    // order after the caller's earlier work, and after this context's previous call
+    // every pipeline stream starts after the caller's earlier work; stream 0 uploads the
+    // tokens once the previous call's kernels (on every stream) have stopped reading them
     NG_CUDA(cudaEventRecord(c->hp_entry, caller), "cudaEventRecord");
-    NG_CUDA(cudaStreamWaitEvent(sh, c->hp_entry, 0), "cudaStreamWaitEvent");
-    for (int b = 0; b < 2; ++b) NG_CUDA(cudaStreamWaitEvent(sh, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
-    NG_CUDA(cudaMemcpyAsync(c->hp_tok, tokens_h, N * 4, cudaMemcpyHostToDevice, sh), "H2D tokens");
+    for (int i = 0; i < S; ++i) NG_CUDA(cudaStreamWaitEvent(c->hp_s[i], c->hp_entry, 0), "cudaStreamWaitEvent");
+    for (int i = 1; i < S; ++i) NG_CUDA(cudaStreamWaitEvent(c->hp_s[0], c->hp_d2h[i], 0), "cudaStreamWaitEvent");
+    NG_CUDA(cudaMemcpyAsync(c->hp_tok, tokens_h, N * 4, cudaMemcpyHostToDevice, c->hp_s[0]), "H2D tokens");
     if (history_h)
-        NG_CUDA(cudaMemcpyAsync(c->hp_hist, history_h, n_seq * 8ull, cudaMemcpyHostToDevice, sh),
+        NG_CUDA(cudaMemcpyAsync(c->hp_hist, history_h, n_seq * 8ull, cudaMemcpyHostToDevice, c->hp_s[0]),
                 "H2D history");
+    NG_CUDA(cudaEventRecord(c->hp_h2d[0], c->hp_s[0]), "cudaEventRecord");
+    for (int i = 1; i < S; ++i) NG_CUDA(cudaStreamWaitEvent(c->hp_s[i], c->hp_h2d[0], 0), "cudaStreamWaitEvent");
     GatherArgs g = gather_args(c, c->hp_tok, history_h ? c->hp_hist : nullptr, T, 0, nullptr, gate,
                                nullptr);
+    // chunk i runs on stream i % S, start to end: H2D residual -> gather -> D2H out.  The
+    // S streams overlap each other's copies in both directions; stream order alone makes
+    // a stream's buffers safe to reuse.
     uint32_t chunk_i = 0;
     for (uint64_t t0 = 0; t0 < N; t0 += c->hp_chunk, ++chunk_i) {
-        const uint32_t b = chunk_i & 1u;
+        const int b = static_cast<int>(chunk_i % S);
+        cudaStream_t st = c->hp_s[b];
         const uint32_t n = static_cast<uint32_t>(std::min<uint64_t>(c->hp_chunk, N - t0));
-        // H2D of the chunk's residual once the kernel two chunks back has read the buffer
-        NG_CUDA(cudaStreamWaitEvent(sh, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
-        NG_CUDA(cudaMemcpyAsync(c->hp_res[b], residual_h + t0 * c->d, n * row, cudaMemcpyHostToDevice, sh),
+        NG_CUDA(cudaMemcpyAsync(c->hp_res[b], residual_h + t0 * c->d, n * row, cudaMemcpyHostToDevice, st),
                 "H2D residual");
-        NG_CUDA(cudaEventRecord(c->hp_h2d[b], sh), "cudaEventRecord");
-        // the gather, once its residual is in and the D2H two chunks back has drained out
-        NG_CUDA(cudaStreamWaitEvent(sk, c->hp_h2d[b], 0), "cudaStreamWaitEvent");
-        NG_CUDA(cudaStreamWaitEvent(sk, c->hp_d2h[b], 0), "cudaStreamWaitEvent");
         g.tok_begin = static_cast<uint32_t>(t0);
         g.N = n;
         g.residual = c->hp_res[b];
         g.out = c->hp_out[b];
-        NG_CHECK(launch_gather(c, g, sk, max_blocks));
-        NG_CUDA(cudaEventRecord(c->hp_kdone[b], sk), "cudaEventRecord");
-        // D2H of the chunk's output
-        NG_CUDA(cudaStreamWaitEvent(sd, c->hp_kdone[b], 0), "cudaStreamWaitEvent");
-        NG_CUDA(cudaMemcpyAsync(out_h + t0 * c->d, c->hp_out[b], n * row, cudaMemcpyDeviceToHost, sd),
+        NG_CHECK(launch_gather(c, g, st, max_blocks));
+        NG_CUDA(cudaMemcpyAsync(out_h + t0 * c->d, c->hp_out[b], n * row, cudaMemcpyDeviceToHost, st),
                 "D2H out");
-        NG_CUDA(cudaEventRecord(c->hp_d2h[b], sd), "cudaEventRecord");
     }
-    // the caller's stream resumes once the last output chunk is on the host
-    NG_CUDA(cudaStreamWaitEvent(caller, c->hp_d2h[(chunk_i - 1) & 1u], 0), "cudaStreamWaitEvent");
+    // the caller's stream resumes once every stream's last output chunk is on the host
+    for (int i = 0; i < S; ++i) {
+        NG_CUDA(cudaEventRecord(c->hp_d2h[i], c->hp_s[i]), "cudaEventRecord");
+        NG_CUDA(cudaStreamWaitEvent(caller, c->hp_d2h[i], 0), "cudaStreamWaitEvent");
+    }
     return NGRAM_OK;
 }
 

@@ -223,9 +223,9 @@ NGRAM_API ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, uin
 
 /* ngram_forward with the per-token inputs and the output in HOST memory (the weights --
  * table and gate -- stay resident on the device).  The batch is cut into chunks of about
- * 8 MB of residual; three internal streams overlap the host->device copy of chunk i+1,
- * the gather of chunk i and the device->host copy of chunk i-1, so PCIe carries input
- * and output at the same time.
+ * 16 MB of residual dealt round-robin to three internal streams; each stream copies its
+ * chunk in, gathers it and copies it out, and the streams overlap each other, so PCIe
+ * carries input and output at the same time.
  *   tokens_h   host int32 [n_seq][T]; history_h host int32 [n_seq][2] or NULL;
  *   residual_h host bf16 [N][d];  gate: DEVICE fp32 [d];  out_h: host bf16 [N][d], must
  *   not overlap residual_h.  Pinned host memory gives the overlap; pageable memory works
