@@ -466,6 +466,73 @@ def measure_h2d_gbs(dev, nbytes=1 << 30, reps=10) -> float:
     return best
 
 
+def prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B):
+    """Prefetch pattern on the host-resident table: step i runs its compute (g stand-in
+    GEMMs) and its lookup from HBM staging on the main stream while batch i+1's rows are
+    staged from host memory on a side stream.  Compared with the same steps doing the
+    UVA lookup inline, and with the compute alone."""
+    import math
+
+    import torch
+    side = torch.cuda.Stream()
+    hp = ng.ngram_default_hash_params(vocab_size=w.vocab)
+    ctx = ng.ngram_init(ht.tensor, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_UVA, hp, w.N)
+    bt = []
+    for b in range(2):
+        inp = gen.make_inputs(w, token_seed=500 + b)
+        bt.append((torch.from_numpy(inp["tokens"]).to(dev),
+                   None if inp["history"] is None else torch.from_numpy(inp["history"]).to(dev)))
+    res = torch.from_numpy(gen.residual_bf16_bits(w.N, d).view(np.int16)).view(torch.bfloat16).view(w.N, d).to(dev)
+    gate = torch.from_numpy(gen.gate_f32(d)).to(dev)
+    out = torch.empty_like(res)
+    K = max(5, min(100, int(5e4 / w.N)))
+
+    def timed(fn, n):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main_s)
+        for i in range(n):
+            fn(i)
+        b.record(main_s)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    for i in range(2):
+        ng.ngram_prefetch(ctx, i, *bt[i], stream=main_s)
+    pf_ms = timed(lambda i: ng.ngram_prefetch(ctx, i % 2, *bt[i % 2], stream=main_s), K)
+    st_ms = timed(lambda i: ng.ngram_forward_staged(ctx, i % 2, res, gate, out=out, stream=main_s), K)
+    g = max(1, math.ceil(pf_ms / gemm_ms))
+
+    def compute():
+        for _ in range(g):
+            torch.matmul(A, B)
+
+    comp_ms = timed(lambda i: compute(), K)
+    inline_ms = timed(lambda i: (compute(), ng.ngram_forward(ctx, bt[i % 2][0], res, gate, out=out,
+                                                             history=bt[i % 2][1], stream=main_s)), K)
+    ev_pf = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_used = [torch.cuda.Event(), torch.cuda.Event()]
+    ng.ngram_prefetch(ctx, 0, *bt[0], stream=main_s)
+    ev_pf[0].record(main_s)
+
+    def step(i):
+        cur, nxt = i % 2, (i + 1) % 2
+        side.wait_event(ev_used[nxt])             # the slot's previous lookup is done
+        ng.ngram_prefetch(ctx, nxt, *bt[nxt], stream=side)
+        ev_pf[nxt].record(side)
+        compute()
+        main_s.wait_event(ev_pf[cur])
+        ng.ngram_forward_staged(ctx, cur, res, gate, out=out, stream=main_s)
+        ev_used[cur].record(main_s)
+
+    piped_ms = timed(step, K)
+    ctx.close()
+    return {"prefetch_ms": pf_ms, "staged_lookup_ms": st_ms, "gemms_per_step": g,
+            "compute_only_ms": comp_ms, "step_inline_uva_ms": inline_ms,
+            "step_prefetched_ms": piped_ms,
+            "lookup_on_critical_path_ms": piped_ms - comp_ms}
+
+
 def run_host(args):
     """Host-resident table: the 20M x 2560 bf16 table pinned in host memory, each host
     workload timed in UVA, DMA and AUTO residency, alone and overlapped with a stand-in
@@ -570,6 +637,7 @@ def run_host(args):
                 entry[mname]["choice"] = {ng.NGRAM_RES_HOST_UVA: "uva", ng.NGRAM_RES_HOST_DMA: "dma"}.get(
                     ng.ngram_auto_choice(ctx, w.N), "undecided")
             ctx.close()
+        entry["prefetch"] = prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B)
         report[name] = entry
     head = names[-1]
     best = report[head]["auto"]

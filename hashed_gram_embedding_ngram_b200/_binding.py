@@ -36,6 +36,7 @@ NGRAM_FLAG_TMA_STAGING = 0x2
 NGRAM_FLAG_SORT = 0x4
 NGRAM_FLAG_BATCH_ORDER = 0x8
 NGRAM_SORT_MIN_TOKENS = 16384
+NGRAM_STAGE_SLOTS = 2
 
 MAX_HEADS = 16
 DEFAULT_BASE_SEED = 0x6E6772616D5F7631
@@ -82,6 +83,10 @@ _lib.ngram_destroy.argtypes = [_P]
 _lib.ngram_destroy.restype = None
 _lib.ngram_forward_host.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
 _lib.ngram_forward_host.restype = _i32
+_lib.ngram_prefetch.argtypes = [_P, _u32, _P, _P, _u32, _u32, _P]
+_lib.ngram_prefetch.restype = _i32
+_lib.ngram_forward_staged.argtypes = [_P, _u32, _P, _P, _P, _P]
+_lib.ngram_forward_staged.restype = _i32
 _lib.ngram_host_alloc.argtypes = [ctypes.POINTER(_P), _u64]
 _lib.ngram_host_alloc.restype = _i32
 _lib.ngram_host_free.argtypes = [_P]
@@ -342,3 +347,27 @@ def ngram_dedup_rows(ctx: Context, tokens: torch.Tensor, history: torch.Tensor |
                                  _ptr(uniq_out), _ptr(inv_out), _ptr(count_out),
                                  _stream(stream)))
     return uniq_out, inv_out, count_out
+
+
+def ngram_prefetch(ctx: Context, slot: int, tokens: torch.Tensor, history: torch.Tensor | None = None,
+                   stream=None) -> None:
+    """Stage the distinct rows of this batch in HBM slot `slot` (asynchronous)."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    n_seq, T = tokens.shape
+    if history is not None:
+        _need(history, "history", torch.int32, tokens.device, ndim=2)
+    _check(_lib.ngram_prefetch(ctx.handle, slot, _ptr(tokens), _ptr(history), n_seq, T,
+                               _stream(stream)))
+
+
+def ngram_forward_staged(ctx: Context, slot: int, residual: torch.Tensor, gate: torch.Tensor,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """ngram_forward for the batch staged in `slot`, gathering from HBM staging."""
+    _need(residual, "residual", torch.bfloat16)
+    _need(gate, "gate", torch.float32, residual.device)
+    if out is None:
+        out = torch.empty_like(residual)
+    _need(out, "out", torch.bfloat16, residual.device)
+    _check(_lib.ngram_forward_staged(ctx.handle, slot, _ptr(residual), _ptr(gate), _ptr(out),
+                                     _stream(stream)))
+    return out

@@ -60,6 +60,9 @@ using namespace ngram;
 // ngram_forward_host pipeline (measured, 32,768-token prefill, pinned host buffers): 16 MB
 // chunks on 3 streams 4.20 ms; 8 MB on 2 streams 4.27-4.48 ms; 4 MB 4.6-5.2 ms; a thinner
 // gather grid does not help.  The copies alone, both directions, take 3.50 ms.
+#ifndef NGRAM_STAGE_SLOTS               // staged batches ngram_prefetch keeps in HBM
+#define NGRAM_STAGE_SLOTS 2
+#endif
 #ifndef NGRAM_HOST_BUFFERS              // pipeline streams of ngram_forward_host
 #define NGRAM_HOST_BUFFERS 3
 #endif
@@ -110,6 +113,15 @@ struct ngram_ctx {
     cudaEvent_t hp_d2h[NGRAM_HOST_BUFFERS];   // end of each stream's part of the last call
     // NGRAM_FLAG_SORT: bucket of each token, bucket counts / cursors, processing order
     uint32_t *so_bucket, *so_hist, *so_perm;
+    // ngram_prefetch / ngram_forward_staged: a ring of staged batches in HBM
+    struct Slot {
+        uint32_t *inv;          // [max_tokens * H] row ids into `stage`
+        uint8_t *stage;         // [max_tokens * H][row_bytes] distinct rows
+        float *stage_scale;     // [max_tokens * H] (int8)
+        uint32_t n_seq, T;      // the staged batch (0 tokens: empty slot)
+        uint64_t epoch;         // prefetch call that filled the slot
+    } slot[NGRAM_STAGE_SLOTS];
+    uint64_t prefetch_epoch;
 };
 
 namespace {
@@ -230,6 +242,11 @@ void free_all(ngram_ctx *c) {
             if (e) cudaEventDestroy(e);
         if (c->hp_res[b]) cudaFree(c->hp_res[b]);
         if (c->hp_out[b]) cudaFree(c->hp_out[b]);
+    }
+    for (auto &sl : c->slot) {
+        if (sl.inv) cudaFree(sl.inv);
+        if (sl.stage) cudaFree(sl.stage);
+        if (sl.stage_scale) cudaFree(sl.stage_scale);
     }
     void *bufs[] = {c->hp_tok, c->hp_hist, c->so_bucket, c->so_hist, c->so_perm};
     for (void *p : bufs)
@@ -816,6 +833,65 @@ ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int
         NG_CUDA(cudaStreamWaitEvent(caller, c->hp_d2h[i], 0), "cudaStreamWaitEvent");
     }
     return NGRAM_OK;
+}
+
+ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, const int32_t *history,
+                            uint32_t n_seq, uint32_t T, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (slot >= NGRAM_STAGE_SLOTS)
+        return fail(NGRAM_EINVAL, "slot %u out of range (%u slots)", slot, NGRAM_STAGE_SLOTS);
+    if (c->where == NGRAM_RES_HOST_DMA)
+        return fail(NGRAM_EUNSUPPORTED, "ngram_prefetch reads the table from the GPU: HBM, HOST_UVA or HOST_AUTO");
+    auto &sl = c->slot[slot];
+    sl.n_seq = n_seq;
+    sl.T = T;
+    sl.epoch = ++c->prefetch_epoch;
+    if (N == 0) return NGRAM_OK;
+    NG_CHECK(ensure_dedup_scratch(c));
+    if (!sl.inv) {
+        NG_CUDA(cudaMalloc(&sl.inv, c->dd_cap * 4ull), "staging slot");
+        NG_CUDA(cudaMalloc(&sl.stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging slot");
+        if (c->dtype == NGRAM_INT8_ROWSCALE)
+            NG_CUDA(cudaMalloc(&sl.stage_scale, c->dd_cap * 4ull), "staging slot");
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint32_t M = static_cast<uint32_t>(N) * c->H;
+    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
+    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, sl.inv, c->d_count, s));
+    // each distinct row crosses once; from host memory a few CTAs keep PCIe busy
+    const unsigned grid = (c->where == NGRAM_RES_HBM) ? grid_for(c, M * 32ull, 256)
+                                                      : static_cast<unsigned>(NGRAM_UVA_CTAS);
+    k_compact_rows<<<grid, 256, 0, s>>>(static_cast<const uint8_t *>(c->table_dev), c->row_scale_dev,
+                                        c->d_uniq, c->d_count, c->row_bytes, sl.stage, sl.stage_scale);
+    NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_forward_staged(ngram_ctx *c, uint32_t slot, const uint16_t *residual,
+                                  const float *gate, uint16_t *out, ngram_stream_t stream) {
+    if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
+    if (slot >= NGRAM_STAGE_SLOTS)
+        return fail(NGRAM_EINVAL, "slot %u out of range (%u slots)", slot, NGRAM_STAGE_SLOTS);
+    const auto &sl = c->slot[slot];
+    if (sl.epoch == 0) return fail(NGRAM_EINVAL, "slot %u holds no prefetched batch", slot);
+    const uint64_t N = static_cast<uint64_t>(sl.n_seq) * sl.T;
+    if (N == 0) return NGRAM_OK;
+    if (residual == nullptr || gate == nullptr || out == nullptr)
+        return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
+    if (!aligned16(residual) || !aligned16(gate) || !aligned16(out))
+        return fail(NGRAM_EINVAL, "residual, gate and out must be 16-byte aligned");
+    if (out != residual) {
+        const uint64_t bytes = N * c->d * 2ull;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(out), b = reinterpret_cast<uintptr_t>(residual);
+        if (a < b + bytes && b < a + bytes)
+            return fail(NGRAM_EINVAL, "out overlaps residual without being equal to it");
+    }
+    GatherArgs g = gather_args(c, nullptr, nullptr, sl.T, static_cast<uint32_t>(N), residual, gate, out);
+    g.table = sl.stage;
+    g.row_scale = sl.stage_scale;
+    g.row_ids = sl.inv;
+    return launch_gather(c, g, reinterpret_cast<cudaStream_t>(stream), full_grid(c));
 }
 
 ngram_status ngram_auto_choice(const ngram_ctx *c, uint32_t n_tokens, int *where_out) {

@@ -172,6 +172,29 @@ NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, cons
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
                            const float *gate, uint16_t *out, ngram_stream_t stream);
 
+/* Prefetch: stage the rows a coming batch will read, ahead of its lookup.  The pages
+ * describe prefetching the n-gram vectors of upcoming tokens over PCIe while the GPU
+ * computes ("Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with Heterogeneous Memory
+ * Prefetch", Key point 3).
+ *   ngram_prefetch hashes and dedups the batch on the GPU, then copies each distinct row
+ *   once from the table into HBM staging slot `slot` (0 .. NGRAM_STAGE_SLOTS-1); with a
+ *   host-resident table (HOST_UVA / HOST_AUTO) the copy kernel reads host memory over PCIe
+ *   on 8 CTAs, leaving the other SMs to the work it overlaps.  Asynchronous on `stream`
+ *   (typically a side stream).
+ *   ngram_forward_staged then computes ngram_forward for that batch from HBM staging
+ *   (bit-identical results), on `stream`; the caller orders it after the prefetch
+ *   (e.g. cudaStreamWaitEvent).
+ * The slots and the dedup scratch belong to the context: prefetches on one context must
+ * be ordered with each other, and a slot must not be refilled while a staged forward
+ * still reads it.  Each slot holds max_tokens * H rows (allocated by its first
+ * prefetch).  HOST_DMA residency: NGRAM_EUNSUPPORTED. */
+#define NGRAM_STAGE_SLOTS 2u
+NGRAM_API ngram_status ngram_prefetch(ngram_ctx *ctx, uint32_t slot, const int32_t *tokens,
+                                      const int32_t *history, uint32_t n_seq, uint32_t T,
+                                      ngram_stream_t stream);
+NGRAM_API ngram_status ngram_forward_staged(ngram_ctx *ctx, uint32_t slot, const uint16_t *residual,
+                                            const float *gate, uint16_t *out, ngram_stream_t stream);
+
 /* Bound, in milliseconds, of every host-side wait of the context (default 10,000).  A
  * wait that runs out returns NGRAM_ETIMEOUT; work already enqueued stays enqueued and
  * the context stays usable once the stream drains. */

@@ -145,3 +145,9 @@ def test_sort_flag_combinations_rejected():
             ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, where,
                           ng.ngram_default_hash_params(flags=flags), 16)
         assert ei.value.status == ng.NGRAM_EINVAL
+
+
+def test_prefetch_entry_points_reject_null_context():
+    lib = ng.lib()
+    assert lib.ngram_prefetch(None, 0, None, None, 1, 1, None) == ng.NGRAM_EINVAL
+    assert lib.ngram_forward_staged(None, 0, None, None, None, None) == ng.NGRAM_EINVAL

@@ -239,3 +239,61 @@ def test_host_residency_argument_checks(cuda_device, host_bf16):
     # DMA reads the table with host threads: pageable memory is accepted
     ctx = ng.ngram_init(pageable, 1000, 64, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_DMA, _hp(1000), 8)
     ctx.close()
+
+
+
+# --------------------------------------------------------------------------- prefetch
+def _batch(w, dev, seed):
+    inp, dv = workload_on_device(w, dev, token_seed=seed)
+    return inp, dv
+
+
+@pytest.mark.parametrize("n_seq,T,hist", [(1, 1, True), (64, 1, True), (2, 700, False)])
+def test_prefetch_ring_bitidentical(cuda_device, host_bf16, n_seq, T, hist):
+    """Two batches staged in the two slots (side stream) gather exactly like the plain
+    lookup, from the host-resident table and from the HBM table."""
+    R, d, V = host_bf16.R, host_bf16.d, 151_936
+    w = gen.Workload("pf", R, d, "bf16", V, n_seq, T, history=hist)
+    dev_table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    hbm = ng.ngram_init(dev_table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    batches = [_batch(w, cuda_device, s) for s in (301, 302)]
+    refs = [from_dev_bf16(_forward(hbm, dv)) for _, dv in batches]
+    side = torch.cuda.Stream()
+    for ctx in (host_bf16.ctx(ng.NGRAM_RES_HOST_UVA, V, w.N), hbm):
+        for slot, (_, dv) in enumerate(batches):
+            ng.ngram_prefetch(ctx, slot, dv["tokens"], dv["history"], stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+        for slot, (_, dv) in enumerate(batches):
+            got = ng.ngram_forward_staged(ctx, slot, dv["residual"], dv["gate"])
+            assert np.array_equal(from_dev_bf16(got), refs[slot])
+        # refill slot 0 with batch 1 and read it again
+        ng.ngram_prefetch(ctx, 0, batches[1][1]["tokens"], batches[1][1]["history"])
+        got = ng.ngram_forward_staged(ctx, 0, batches[1][1]["residual"], batches[1][1]["gate"])
+        assert np.array_equal(from_dev_bf16(got), refs[1])
+        assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
+def test_prefetch_int8_and_errors(cuda_device):
+    R, d, V = 5003, 272, 7000
+    w = gen.Workload("pf8", R, d, "int8", V, 3, 50, history=True)
+    inp = gen.make_inputs(w, token_seed=311)
+    table, scale = TABLES.get(R, d, ng.NGRAM_INT8_ROWSCALE, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_INT8_ROWSCALE, ng.NGRAM_RES_HBM, _hp(V), w.N,
+                        row_scale=scale)
+    toks = to_dev_tokens(inp["tokens"], cuda_device)
+    hist = to_dev_tokens(inp["history"], cuda_device)
+    res = to_dev_bf16(inp["residual"], cuda_device).view(w.N, d)
+    gate = torch.from_numpy(inp["gate"]).to(cuda_device)
+    ng.ngram_prefetch(ctx, 1, toks, hist)
+    got = from_dev_bf16(ng.ngram_forward_staged(ctx, 1, res, gate))
+    want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
+                          dtype=oracle.INT8, table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32,
+                          n_threads=N_CPU, vocab_size=V)
+    r = assert_parity(got, want)
+    assert r["exact"] == r["n"]
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_forward_staged(ctx, 0, res, gate)          # slot 0 never filled
+    assert ei.value.status == ng.NGRAM_EINVAL
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_prefetch(ctx, 2, toks, hist)                # out of range
+    assert ei.value.status == ng.NGRAM_EINVAL
