@@ -32,6 +32,9 @@ ACC_F64 = 0
 ACC_F32 = 1
 BF16 = 0
 INT8 = 1
+FP8 = 2      # FP8 E4M3 codes + fp32 row scale
+NVFP4 = 3    # E2M1 codes + E4M3 scale per 16 columns + fp32 global scale
+FP4_GLOBAL_SCALE = float.fromhex("0x1.4fp-9")
 
 DEFAULT_BASE_SEED = 0x6E6772616D5F7631   # ASCII "ngram_v1"
 DEFAULT_PAD_ID = 0x1FFFFF                # 2^21 - 1, outside any vocabulary below 2^21 - 1
@@ -91,6 +94,14 @@ def _load():
                                        ctypes.POINTER(_HashParams), P, P, u32, u32, P, P,
                                        P, u64, ctypes.c_int, ctypes.c_int, P, P, P, P]
         lib.oracle_forward.restype = ctypes.c_int
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_value.restype = ctypes.c_double
+        lib.oracle_fill_fp8.argtypes = [u64, u64, u64, u32, P, P]
+        lib.oracle_fill_fp4.argtypes = [u64, u64, u64, u32, P]
+        lib.oracle_fp4_row_bytes.argtypes = [u32]
+        lib.oracle_fp4_row_bytes.restype = u32
         del i32, i64
         _lib = lib
         return lib
@@ -151,6 +162,33 @@ def fill_int8(seed: int, row0: int, n_rows: int, d: int):
     s = np.zeros(n_rows, dtype=np.float32)
     _load().oracle_fill_int8(seed, row0, n_rows, d, _ptr(q), _ptr(s))
     return q, s
+
+
+def e4m3_value(code: int) -> float:
+    return float(_load().oracle_e4m3_value(code))
+
+
+def e2m1_value(nibble: int) -> float:
+    return float(_load().oracle_e2m1_value(nibble))
+
+
+def fp4_row_bytes(d: int) -> int:
+    return int(_load().oracle_fp4_row_bytes(d))
+
+
+def fill_fp8(seed: int, row0: int, n_rows: int, d: int):
+    """Rows of the synthetic FP8 E4M3 table (uint8 codes) and their fp32 row scales."""
+    q = np.zeros((n_rows, d), dtype=np.uint8)
+    s = np.zeros(n_rows, dtype=np.float32)
+    _load().oracle_fill_fp8(seed, row0, n_rows, d, _ptr(q), _ptr(s))
+    return q, s
+
+
+def fill_fp4(seed: int, row0: int, n_rows: int, d: int) -> np.ndarray:
+    """Rows of the synthetic NVFP4 table as bytes: d/2 code bytes then the block scales."""
+    out = np.zeros((n_rows, fp4_row_bytes(d)), dtype=np.uint8)
+    _load().oracle_fill_fp4(seed, row0, n_rows, d, _ptr(out))
+    return out
 
 
 def rows_bf16(seed: int, rows, d: int) -> np.ndarray:
@@ -223,7 +261,7 @@ def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_see
     if table is None and table_i8 is None and table_seed is None:
         raise ValueError("need a table or a table_seed")
     tb = None if table is None else np.ascontiguousarray(table, dtype=np.uint16)
-    ti = None if table_i8 is None else np.ascontiguousarray(table_i8, dtype=np.int8)
+    ti = None if table_i8 is None else np.ascontiguousarray(table_i8).view(np.int8)
     sc = None if row_scale is None else np.ascontiguousarray(row_scale, dtype=np.float32)
     H = n_bigram + n_trigram
     out = np.zeros((n_sel, d), dtype=np.uint16)

@@ -32,6 +32,9 @@
  *   - table values are synthetic (no trained weights exist): a Philox4x32-10
  *     function of (seed, row, col), see oracle_table_bf16 / oracle_table_int8.
  *
+ * Row formats: bf16; int8 with an fp32 row scale; FP8 E4M3 with an fp32 row scale;
+ * NVFP4 (E2M1 with one E4M3 scale per 16 columns and an fp32 global scale).
+ *
  * Two accumulation modes:
  *   ORACLE_ACC_F64 -- the plain definition.  The 16 products/values are summed in
  *                     double (exact for these operands), gate and add in double, and
@@ -53,6 +56,8 @@
 
 #define ORACLE_BF16 0
 #define ORACLE_INT8 1
+#define ORACLE_FP8 2      /* FP8 E4M3 codes, one fp32 scale per row */
+#define ORACLE_NVFP4 3    /* FP4 E2M1 codes, one E4M3 scale per 16 columns, one fp32 global scale */
 
 /* ------------------------------------------------------------------------------------
  * splitmix64 (Steele, Lea & Flood, "Fast Splittable Pseudorandom Number Generators",
@@ -209,6 +214,112 @@ float oracle_row_scale(uint64_t seed, uint64_t row)
     return 0x1.1bc5f4p-11f * s;
 }
 
+/* ------------------------------------------------------------------------------------
+ * Low-precision element formats (OCP 8-bit floating point and Microscaling formats).
+ *   E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is subnormal
+ *         (m/8 * 2^-6); S.1111.111 is NaN; no infinities.  Largest finite 448.
+ *   E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; exponent 0 is subnormal
+ *         (m * 0.5).  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * ---------------------------------------------------------------------------------- */
+double oracle_e4m3_value(uint8_t code)
+{
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);                  /* m/8 * 2^(1-7) */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+double oracle_e2m1_value(uint8_t nib)
+{
+    int s = (nib >> 3) & 1, e = (nib >> 1) & 3, m = nib & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + m / 2.0, e - 1);
+    return s ? -v : v;
+}
+
+/* Synthetic FP8 rows.  Element (row, col): Philox counter (col/4, row, 4, 0), word
+ * w = x[col % 4]; sign = bit 31, exponent field 4 + bits[3:4] + bits[5:6] (4..10, never
+ * NaN), mantissa bits[0:2].  Row scale: counter (0, row, 5, 0),
+ * s = K * (0.75 + (x0 >> 8) * 2^-25) with K = 0x1.4dp-8 (std of the values ~0.02). */
+uint8_t oracle_table_fp8(uint64_t seed, uint64_t row, uint32_t col)
+{
+    uint32_t key[2], ctr[4], x[4], w, e;
+    seed_key(seed, key);
+    ctr[0] = col >> 2; ctr[1] = (uint32_t)row; ctr[2] = 4u; ctr[3] = 0u;
+    oracle_philox4x32_10(ctr, key, x);
+    w = x[col & 3u];
+    e = 4u + ((w >> 3) & 3u) + ((w >> 5) & 3u);
+    return (uint8_t)(((w >> 31) << 7) | (e << 3) | (w & 7u));
+}
+
+float oracle_row_scale_fp8(uint64_t seed, uint64_t row)
+{
+    uint32_t key[2], ctr[4], x[4];
+    float t, s;
+    seed_key(seed, key);
+    ctr[0] = 0u; ctr[1] = (uint32_t)row; ctr[2] = 5u; ctr[3] = 0u;
+    oracle_philox4x32_10(ctr, key, x);
+    t = (float)(x[0] >> 8) * 0x1p-25f;
+    s = 0.75f + t;
+    return 0x1.4dp-8f * s;
+}
+
+/* Synthetic NVFP4 rows.  Column c's 4-bit code: Philox counter (c/32, row, 6, 0), word
+ * x[(c/8) % 4], nibble c % 8 (bits 4*(c%8)..).  Block b's E4M3 scale (columns 16b ..
+ * 16b+15): counter (b/4, row, 7, 0), word w = x[b % 4]; positive, exponent field
+ * 5 + bits[0:1] + bit[2] (5..9), mantissa bits[3:5].  Global scale 0x1.4fp-9 (std of
+ * the values ~0.02). */
+uint8_t oracle_table_fp4(uint64_t seed, uint64_t row, uint32_t col)
+{
+    uint32_t key[2], ctr[4], x[4];
+    seed_key(seed, key);
+    ctr[0] = col >> 5; ctr[1] = (uint32_t)row; ctr[2] = 6u; ctr[3] = 0u;
+    oracle_philox4x32_10(ctr, key, x);
+    return (uint8_t)((x[(col >> 3) & 3u] >> (4u * (col & 7u))) & 15u);
+}
+
+uint8_t oracle_block_scale_fp4(uint64_t seed, uint64_t row, uint32_t block)
+{
+    uint32_t key[2], ctr[4], x[4], w, e;
+    seed_key(seed, key);
+    ctr[0] = block >> 2; ctr[1] = (uint32_t)row; ctr[2] = 7u; ctr[3] = 0u;
+    oracle_philox4x32_10(ctr, key, x);
+    w = x[block & 3u];
+    e = 5u + (w & 3u) + ((w >> 2) & 1u);
+    return (uint8_t)((e << 3) | ((w >> 3) & 7u));
+}
+
+#define ORACLE_FP4_GLOBAL_SCALE 0x1.4fp-9f
+
+/* Bytes of one NVFP4 row: d/2 code bytes, then d/16 scale bytes padded to 16. */
+uint32_t oracle_fp4_row_bytes(uint32_t d) { return d / 2 + ((d / 16 + 15) / 16) * 16; }
+
+void oracle_fill_fp8(uint64_t seed, uint64_t row0, uint64_t n_rows, uint32_t d,
+                     uint8_t *q_out, float *scale_out)
+{
+    uint64_t r; uint32_t c;
+    for (r = 0; r < n_rows; r++) {
+        for (c = 0; c < d; c++)
+            q_out[r * d + c] = oracle_table_fp8(seed, row0 + r, c);
+        scale_out[r] = oracle_row_scale_fp8(seed, row0 + r);
+    }
+}
+
+void oracle_fill_fp4(uint64_t seed, uint64_t row0, uint64_t n_rows, uint32_t d, uint8_t *out)
+{
+    const uint32_t rb = oracle_fp4_row_bytes(d);
+    uint64_t r; uint32_t c, b;
+    for (r = 0; r < n_rows; r++) {
+        uint8_t *row = out + r * rb;
+        memset(row, 0, rb);
+        for (c = 0; c < d; c++)
+            row[c / 2] |= (uint8_t)(oracle_table_fp4(seed, row0 + r, c) << (4 * (c & 1u)));
+        for (b = 0; b < d / 16; b++)
+            row[d / 2 + b] = oracle_block_scale_fp4(seed, row0 + r, b);
+    }
+}
+
 /* Materialise rows [row0, row0 + n_rows) x d of the synthetic table on the host. */
 void oracle_fill_bf16(uint64_t seed, uint64_t row0, uint64_t n_rows, uint32_t d, uint16_t *out)
 {
@@ -314,12 +425,41 @@ int oracle_indices(const int32_t *tokens, const int32_t *history, uint32_t n_seq
  *   n_threads > 1 splits the token loop across OpenMP threads (per-token work and
  *   arithmetic are unchanged).
  * ---------------------------------------------------------------------------------- */
-/* Element (row, col) of the table: bf16 value v (q = v, s = 1 is not used), or the
- * int8 pair (q, s).  Returns the exact value in double. */
+/* Element (row, col) of the table: bf16 value v (s = 1, unused), or the pair (q, s)
+ * with value q * s (int8: q the integer, s the row scale; fp8: q the E4M3 value, s the
+ * row scale; nvfp4: q the E2M1 value, s = fp32(E4M3 block scale * global scale)).
+ * Returns the exact value q * s in double.  For fp8 / nvfp4 a materialised table is
+ * passed as table_i8 (bytes) and the scales as `scale` (fp8: per row; nvfp4: the global
+ * scale at scale[0], block scales inside the row bytes). */
 static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
                         const float *scale, uint64_t seed, uint64_t row, uint32_t col,
                         uint32_t d, float *v_or_q, float *s_out)
 {
+    if (dtype == ORACLE_FP8) {
+        const uint8_t code = table_i8 ? (uint8_t)table_i8[row * d + col] : oracle_table_fp8(seed, row, col);
+        const float sc = scale ? scale[row] : oracle_row_scale_fp8(seed, row);
+        *v_or_q = (float)oracle_e4m3_value(code);          /* exact */
+        *s_out = sc;
+        return (double)*v_or_q * (double)sc;
+    }
+    if (dtype == ORACLE_NVFP4) {
+        const uint32_t rb = oracle_fp4_row_bytes(d);
+        uint8_t code, bs;
+        float gs, cs;
+        if (table_i8) {
+            const uint8_t *r = (const uint8_t *)table_i8 + row * rb;
+            code = (uint8_t)((r[col / 2] >> (4 * (col & 1u))) & 15u);
+            bs = r[d / 2 + col / 16];
+        } else {
+            code = oracle_table_fp4(seed, row, col);
+            bs = oracle_block_scale_fp4(seed, row, col / 16);
+        }
+        gs = scale ? scale[0] : ORACLE_FP4_GLOBAL_SCALE;
+        cs = (float)oracle_e4m3_value(bs) * gs;             /* rounded to fp32 */
+        *v_or_q = (float)oracle_e2m1_value(code);           /* exact */
+        *s_out = cs;
+        return (double)*v_or_q * (double)cs;
+    }
     if (dtype == ORACLE_BF16) {
         uint16_t b = table_bf16 ? table_bf16[row * d + col] : oracle_table_bf16(seed, row, col);
         float f = oracle_f32_from_bf16(b);
@@ -375,6 +515,7 @@ int oracle_forward(int dtype, const uint16_t *table_bf16, const int8_t *table_i8
                     acc32 = acc32 + v;             /* fp32, head order */
                 else
                     acc32 = fmaf(v, sc, acc32);    /* q * s + acc, one rounding per head */
+                /* (int8, fp8, nvfp4 alike; q exact in fp32 in every case) */
                 mag += fabs(e64);
             }
             if (acc_mode == ORACLE_ACC_F64) {

@@ -424,3 +424,80 @@ def test_int8_fp32_mode_within_tolerance_of_exact():
                                       want_aux=True)
     a, b = _bits_to_f64(o32).reshape(y64.shape), _bits_to_f64(o64).reshape(y64.shape)
     assert np.all(np.abs(a - b) <= _bf16_ulp(b) + 2.0 ** -20 * mag)
+
+
+
+# --------------------------------------------------------------------------- low-precision rows
+def test_e4m3_decode_matches_torch_float8_e4m3fn():
+    want = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_value(c) for c in range(256)])
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and got[0x7E] == 448.0
+
+
+def test_e2m1_decode_matches_the_ocp_value_table():
+    """OCP Microscaling Formats (MX) v1.0, FP4 E2M1: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6
+    for codes 0..7; bit 3 is the sign."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        v = oracle.e2m1_value(c)
+        assert abs(v) == mags[c & 7] and (np.signbit(v) == bool(c & 8))
+
+
+def test_fp8_table_is_never_nan_and_has_its_closed_form_spread():
+    q, s = oracle.fill_fp8(gen.TABLE_SEED, 5, 200, 512)
+    assert not np.any(((q & 0x7F) == 0x7F))                 # no NaN codes
+    e = (q >> 3) & 15
+    assert e.min() >= 4 and e.max() <= 10
+    v = np.array([oracle.e4m3_value(int(c)) for c in q.ravel()[:50000]]) * np.repeat(s, 512)[:50000]
+    assert abs(v.std() / 0.02 - 1) < 0.03 and abs(v.mean()) < 4 * 0.02 / np.sqrt(v.size)
+    K = float.fromhex("0x1.4dp-8")
+    assert np.all(s >= 0.75 * K) and np.all(s < 1.25 * K)
+
+
+def test_fp4_table_layout_and_spread():
+    d = 512
+    rows = oracle.fill_fp4(gen.TABLE_SEED, 7, 100, d)
+    assert rows.shape == (100, d // 2 + d // 16) and oracle.fp4_row_bytes(256) == 144
+    sc = rows[:, d // 2:]
+    e = (sc >> 3) & 15
+    assert e.min() >= 5 and e.max() <= 9 and not np.any(sc & 0x80)
+    codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(100, d)
+    counts = np.bincount(codes.ravel(), minlength=16)
+    assert counts.min() > 0.8 * codes.size / 16                    # uniform over the 16 codes
+    e2 = np.array([oracle.e2m1_value(c) for c in range(16)])
+    bs = np.array([[oracle.e4m3_value(int(b)) for b in r] for r in sc])
+    v = e2[codes] * np.repeat(bs, 16, axis=1) * oracle.FP4_GLOBAL_SCALE
+    assert abs(v.std() / 0.02 - 1) < 0.05
+
+
+@pytest.mark.parametrize("dtype", [oracle.FP8, oracle.NVFP4])
+def test_low_precision_brute_force_and_fp32_mode(dtype):
+    R, d, V = 257, 64, 300
+    toks, res, g = _tiny_case(R=R, d=d, V=V, n_seq=3, T=30)
+    if dtype == oracle.FP8:
+        q, s = oracle.fill_fp8(21, 0, R, d)
+        E = np.array([[oracle.e4m3_value(int(c)) for c in r] for r in q]) * s[:, None].astype(np.float64)
+        tab, sc = q, s
+    else:
+        rows = oracle.fill_fp4(21, 0, R, d)
+        codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(R, d)
+        e2 = np.array([oracle.e2m1_value(c) for c in range(16)])
+        cs = np.array([[np.float32(np.float32(oracle.e4m3_value(int(b))) * np.float32(oracle.FP4_GLOBAL_SCALE))
+                        for b in r[d // 2:d // 2 + d // 16]] for r in rows], dtype=np.float64)
+        E = e2[codes] * np.repeat(cs, 16, axis=1)
+        tab, sc = rows, np.array([oracle.FP4_GLOBAL_SCALE], dtype=np.float32)
+    out, y, mag, idx = oracle.forward(toks, None, res, g, R=R, d=d, dtype=dtype, table_seed=21,
+                                      acc=oracle.ACC_F64, vocab_size=V, want_aux=True)
+    e = _one_hot_sum(idx, E)
+    r = _bits_to_f64(res).reshape(-1, d)
+    assert np.array_equal(y, r + g.astype(np.float64)[None, :] * e)
+    # the materialised table gives the same result as regenerating rows
+    out_m = oracle.forward(toks, None, res, g, R=R, d=d, dtype=dtype, table_i8=tab, row_scale=sc,
+                           acc=oracle.ACC_F64, vocab_size=V)
+    assert np.array_equal(out, out_m)
+    o32 = oracle.forward(toks, None, res, g, R=R, d=d, dtype=dtype, table_seed=21,
+                         acc=oracle.ACC_F32, vocab_size=V)
+    a, b = _bits_to_f64(o32).reshape(y.shape), _bits_to_f64(out).reshape(y.shape)
+    assert np.all(np.abs(a - b) <= _bf16_ulp(b) + 2.0 ** -20 * mag)
