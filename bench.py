@@ -43,7 +43,16 @@ KERNEL_SOURCES = {   # the source files each timed kernel is built from
     "int8": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
              "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
              "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
+    "fp8": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
+            "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
+            "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
+    "nvfp4": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
+              "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
+              "hashed_gram_embedding_ngram_b200/csrc/gather_nvfp4.cuh",
+              "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
 }
+KERNEL_NAME = {"bf16": "k_gather_bf16<16>", "int8": "k_gather_int8<16>",
+               "fp8": "k_gather_fp8<16>", "nvfp4": "k_gather_nvfp4<16>"}
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -51,7 +60,24 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 # --------------------------------------------------------------------------- helpers
 def row_bytes(w) -> int:
+    """Bytes the gather reads per row: bf16 2d; int8 / fp8 d codes + the fp32 row scale;
+    nvfp4 d/2 code bytes + d/16 block-scale bytes (the padding is never read)."""
+    if w.dtype == "bf16":
+        return 2 * w.d
+    if w.dtype == "nvfp4":
+        return w.d // 2 + w.d // 16
+    return w.d + 4
+
+
+def stored_row_bytes(w) -> int:
+    if w.dtype == "nvfp4":
+        return w.d // 2 + -(-(w.d // 16) // 16) * 16
     return 2 * w.d if w.dtype == "bf16" else w.d + 4
+
+
+def oracle_dtype(w) -> int:
+    import oracle
+    return {"bf16": oracle.BF16, "int8": oracle.INT8, "fp8": oracle.FP8, "nvfp4": oracle.NVFP4}[w.dtype]
 
 
 def algorithmic_bytes(w, n_seq=None, T=None) -> int:
@@ -190,7 +216,7 @@ def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0):
     cannot be materialised on the host) on a bounded sample of this workload's tokens."""
     import oracle
     rng = np.random.default_rng(seed)
-    kw = dict(R=w.R, d=w.d, dtype=oracle.BF16 if w.dtype == "bf16" else oracle.INT8,
+    kw = dict(R=w.R, d=w.d, dtype=oracle_dtype(w),
               table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32, n_threads=threads,
               vocab_size=w.vocab)
     probe = rng.choice(w.N, size=min(w.N, 4 * threads), replace=False)
@@ -220,7 +246,7 @@ def run_reference(args, w):
     n_step = int(max(1, min(w.N, per_step_budget / per_tok)))
     rng = np.random.default_rng(7)
     import oracle as orc
-    kw = dict(R=w.R, d=w.d, dtype=orc.BF16 if w.dtype == "bf16" else orc.INT8,
+    kw = dict(R=w.R, d=w.d, dtype=oracle_dtype(w),
               table_seed=gen.TABLE_SEED, acc=orc.ACC_F32, n_threads=threads, vocab_size=w.vocab)
     sels = [np.sort(rng.choice(w.N, size=n_step, replace=False)) for _ in range(steps + warm)]
     for i in range(warm):
@@ -235,7 +261,7 @@ def run_reference(args, w):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": steps, "warmup": warm, "ms_per_step": 1e3 * dt / steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic", "config": config_for(w, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -247,7 +273,7 @@ def run_reference(args, w):
 def config_for(w, args) -> dict:
     return {
         "workload": w.name, "R": w.R, "d": w.d, "table_dtype": w.dtype,
-        "table_gib": round(w.R * row_bytes(w) / 2**30, 2), "n_seq": w.n_seq, "T": w.T,
+        "table_gib": round(w.R * stored_row_bytes(w) / 2**30, 2), "n_seq": w.n_seq, "T": w.T,
         "tokens_per_step_per_gpu": w.N, "heads": "8 bigram + 8 trigram",
         "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
         "accumulate": "fp32, head order", "residency": "hbm", "variant": args.variant,
@@ -281,14 +307,12 @@ def run_ours(args, w):
             dist.barrier()
 
     # ---- table (set-up, untimed): a replica of the whole table on every GPU
-    if w.dtype == "bf16":
-        dtype = ng.NGRAM_BF16
-        table = torch.empty((w.R, w.d), dtype=torch.bfloat16, device=dev)
-        scale = None
-    else:
-        dtype = ng.NGRAM_INT8_ROWSCALE
-        table = torch.empty((w.R, w.d), dtype=torch.int8, device=dev)
-        scale = torch.empty((w.R,), dtype=torch.float32, device=dev)
+    dtype = {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
+             "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[w.dtype]
+    table = torch.empty((w.R, ng.ngram_row_bytes(dtype, w.d)), dtype=torch.uint8, device=dev)
+    scale = None
+    if dtype != ng.NGRAM_BF16:     # per-row scales, or the one NVFP4 global scale
+        scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
     ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
     flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING,
              "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER}[args.variant]
@@ -422,7 +446,7 @@ def run_ours(args, w):
                          "kernel": ("hash + dedup + compact + gather (8 kernels)" if args.variant == "dedup"
                                     else "k_gather_bf16_bulk<16>" if args.variant == "tma"
                                     else ("grouped order (3 kernels) + " if grouped else "")
-                                    + ("k_gather_bf16<16>" if w.dtype == "bf16" else "k_gather_int8<16>")),
+                                    + KERNEL_NAME[w.dtype]),
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -27,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 NGRAM_OK, NGRAM_EINVAL, NGRAM_ENOMEM, NGRAM_ECUDA = 0, 1, 2, 3
 NGRAM_EUNSUPPORTED, NGRAM_ETIMEOUT, NGRAM_EDEVICE = 4, 5, 6
 # ngram_dtype
-NGRAM_BF16, NGRAM_INT8_ROWSCALE = 0, 1
+NGRAM_BF16, NGRAM_INT8_ROWSCALE, NGRAM_FP8_E4M3_ROWSCALE, NGRAM_NVFP4 = 0, 1, 2, 3
 # ngram_residency
 NGRAM_RES_HBM, NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO = 0, 1, 2, 3
 
@@ -97,6 +97,8 @@ _lib.ngram_auto_choice.argtypes = [_P, _u32, ctypes.POINTER(ctypes.c_int)]
 _lib.ngram_auto_choice.restype = _i32
 _lib.ngram_dedup_rows.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
 _lib.ngram_dedup_rows.restype = _i32
+_lib.ngram_row_bytes.argtypes = [_i32, _u32, ctypes.POINTER(_u32)]
+_lib.ngram_row_bytes.restype = _i32
 
 
 def lib() -> ctypes.CDLL:
@@ -169,6 +171,12 @@ class Context:
             self.close()
         except Exception:
             pass
+
+
+def ngram_row_bytes(dtype: int, d: int) -> int:
+    out = ctypes.c_uint32()
+    _check(_lib.ngram_row_bytes(dtype, d, ctypes.byref(out)))
+    return out.value
 
 
 def ngram_init(table: torch.Tensor, R: int, d: int, dtype: int = NGRAM_BF16,

@@ -129,6 +129,21 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     return r;
 }
 
+// 8-byte and 1-byte forms of the same load (the NVFP4 rows: 8 code bytes and one block
+// scale per 16 columns).
+__device__ __forceinline__ uint2 ld_stream_v2(const void *p) {
+    uint2 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0, %1}, [%2];"
+        : "=r"(r.x), "=r"(r.y)
+        : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_stream_u8(const void *p) {
+    uint32_t r;
+    asm("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
 // Packed fp32 pairs (sm_100 add/sub/mul/fma .f32x2): two independent IEEE fp32
 // operations, each rounded to nearest even exactly as the scalar __fadd_rn / __fsub_rn /
 // __fmul_rn / __fmaf_rn, in one instruction.  A packed product whose only use is a packed
@@ -174,6 +189,50 @@ __device__ __forceinline__ float2 bf16x2(uint32_t w) { return make_float2(bf16_l
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Exact FP8 E4M3 and FP4 E2M1 -> fp32 through the sm_100 conversions to f16 pairs: every
+// E4M3 value (448 at most, 2^-9 at least) and every E2M1 value is an f16 value, and
+// f16 -> fp32 is exact.  The conversion puts the lower byte (nibble) of its input in the
+// lower f16, so code k of a word lands in column k.
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h) {
+    float a, b;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+        : "=f"(a), "=f"(b) : "r"(h));
+    return make_float2(a, b);
+}
+
+// Four E4M3 codes (byte k = column k) -> columns (0, 1) and (2, 3).
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float2 &c01, float2 &c23) {
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(h01), "=r"(h23) : "r"(w));
+    c01 = half2_bits_to_float2(h01);
+    c23 = half2_bits_to_float2(h23);
+}
+
+// One E4M3 code (the low byte of b) -> fp32.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+    float f;
+    asm("{\n\t.reg .b16 x, lo, hi;\n\t.reg .b32 h;\n\tcvt.u16.u32 x, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, x;\n\tmov.b32 {lo, hi}, h;\n\tcvt.f32.f16 %0, lo;\n\t}"
+        : "=f"(f) : "r"(b & 0xFFu));
+    return f;
+}
+
+// Eight E2M1 codes (nibble k = column k) -> columns (0, 1), (2, 3), (4, 5), (6, 7).
+__device__ __forceinline__ void e2m1x8_to_float(uint32_t w, float2 c[4]) {
+    uint32_t h0, h1, h2, h3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3) : "r"(w));
+    c[0] = half2_bits_to_float2(h0);
+    c[1] = half2_bits_to_float2(h1);
+    c[2] = half2_bits_to_float2(h2);
+    c[3] = half2_bits_to_float2(h3);
 }
 
 }  // namespace ngram

@@ -1,0 +1,84 @@
+// gather_nvfp4.cuh -- the gather for NVFP4 rows: FP4 E2M1 codes with one E4M3 scale per
+// 16 columns and one fp32 scale for the whole table.
+//
+// The 4-bit table of "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with
+// Heterogeneous Memory Prefetch" (its architecture figure: 51B parameters, ~25.5 GB at
+// FP4; "Qwen3.8-Flash-Next: A 125B MoE for the Local Stack?", section "Hardware math for
+// self-hosting", weighs 4-bit n-gram tables too).  Same operation as k_gather_bf16, with
+// row value  q * cs,  q the E2M1 value of the code and cs = fp32(E4M3 block scale *
+// global scale), summed per head in order with one fused multiply-add per head.
+//
+// Row layout (rb = d/2 + ceil16(d/16) bytes, a multiple of 16 for d % 32 == 0): d/2 code
+// bytes, column 2j in the low nibble of byte j; then d/16 block-scale bytes; then zero
+// padding.  A lane owns 16 columns = one scale block: 8 code bytes and 1 scale byte per
+// head, so a 32-lane strip covers 512 columns as in the 8-bit gather.
+#pragma once
+
+#include "gather_int8.cuh"
+
+namespace ngram {
+
+template <int kH>
+__global__ void __launch_bounds__(256, 2) k_gather_nvfp4(const GatherArgs g) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
+    const uint32_t H = kH ? static_cast<uint32_t>(kH) : g.h.n_heads;
+    const uint32_t nvec = g.d >> 4;                       // scale blocks per row
+    const uint32_t code_bytes = g.d >> 1;
+    const size_t rb = code_bytes + 16u * ((nvec + 15u) >> 4);
+    const uint32_t n_items = g.N * g.groups_per_token;
+    const uint8_t *__restrict__ table = static_cast<const uint8_t *>(g.table);
+    const float gs = __ldg(g.row_scale);                  // the global scale
+
+    for (uint32_t item = warp; item < n_items; item += n_warps) {
+        const uint32_t pos = item / g.groups_per_token;
+        const uint32_t grp = item - pos * g.groups_per_token;
+        const uint32_t tok = g.perm ? __ldg(g.perm + pos) : pos;
+        const uint32_t my_row = warp_head_row(g, tok, lane, H);
+        uint32_t rows[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);
+        const uint32_t s_begin = grp * g.strips_per_item;
+        const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
+        const size_t tok_off = static_cast<size_t>(tok) * g.d;
+        for (uint32_t s = s_begin; s < s_end; ++s) {
+            const uint32_t v = s * 32u + lane;
+            if (v >= nvec) continue;                      // the last strip may be ragged
+            // issue every load of this block before the first multiply-add
+            uint2 e[16];
+            uint32_t bs[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                if (kH || h < static_cast<int>(H)) {
+                    const uint8_t *row = table + static_cast<size_t>(rows[h]) * rb;
+                    e[h] = ld_stream_v2(row + v * 8u);
+                    bs[h] = ld_stream_u8(row + code_bytes + v);
+                }
+            }
+            const uint4 r0 = ld_na_v4(g.residual + tok_off + v * 16u);
+            const uint4 r1 = ld_na_v4(g.residual + tok_off + v * 16u + 8u);
+
+            float2 acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                if (kH || h < static_cast<int>(H)) {
+                    const float cs = __fmul_rn(e4m3_to_float(bs[h]), gs);
+                    const float2 s2 = make_float2(cs, cs);
+                    float2 q[4];
+                    e2m1x8_to_float(e[h].x, q);           // columns 0..7
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[k] = fma2(q[k], s2, acc[k]);
+                    e2m1x8_to_float(e[h].y, q);           // columns 8..15
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[4 + k] = fma2(q[k], s2, acc[4 + k]);
+                }
+            }
+            store_gated16(g, tok_off, v, r0, r1, acc);
+        }
+    }
+}
+
+}  // namespace ngram

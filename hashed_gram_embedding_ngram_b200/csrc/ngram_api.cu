@@ -22,6 +22,7 @@
 #include "fill.cuh"
 #include "gather.cuh"
 #include "gather_int8.cuh"
+#include "gather_nvfp4.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
 #include "order.cuh"
@@ -70,11 +71,12 @@ using namespace ngram;
 struct ngram_ctx {
     const void *table;          // caller's pointer (device, or host for host residency)
     const void *table_dev;      // device-visible alias used by kernels (UVA), or table
-    const float *row_scale;
-    const float *row_scale_dev;
+    const float *row_scale;     // per-row scales (int8, fp8) as passed, else NULL
+    const float *row_scale_dev; // what the gather reads: per-row scales, or the NVFP4
+                                // global scale (d_gscale)
     uint64_t R;
     uint32_t d;
-    uint32_t row_bytes;         // 2d (bf16) or d (int8)
+    uint32_t row_bytes;         // 2d (bf16), d (int8, fp8), d/2 + ceil16(d/16) (nvfp4)
     ngram_dtype dtype;
     ngram_residency where;
     ngram_hash_params hp;
@@ -87,6 +89,7 @@ struct ngram_ctx {
     int bulk_smem_set;
     uint32_t wait_ms;           // bound of every host-side wait
     uint32_t *d_err;            // 4 words
+    float *d_gscale;            // NVFP4: device copy of the global scale
     // dedup scratch, sized for max_tokens (allocated on first use)
     uint32_t dd_cap;            // entries (max_tokens * H)
     uint32_t dd_pcap;           // hash-table slots (power of two >= 2 * dd_cap)
@@ -157,6 +160,32 @@ ngram_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Row formats.  Per-row scales (int8, fp8) travel with the rows through every staging
+// path; the NVFP4 block scales sit inside the row bytes and its global scale stays put.
+bool scale_per_row(ngram_dtype t) { return t == NGRAM_INT8_ROWSCALE || t == NGRAM_FP8_E4M3_ROWSCALE; }
+
+uint32_t row_bytes_of(ngram_dtype t, uint32_t d) {
+    switch (t) {
+        case NGRAM_BF16: return 2u * d;
+        case NGRAM_NVFP4: return d / 2u + 16u * ((d / 16u + 15u) / 16u);
+        default: return d;
+    }
+}
+
+// d and row_scale rules of each format (ngram_init and ngram_fill_synthetic).
+ngram_status check_format(ngram_dtype t, uint32_t d, const float *row_scale) {
+    static const char *const names[] = {"bf16", "int8", "fp8", "nvfp4"};
+    static const uint32_t multiple[] = {8u, 16u, 16u, 32u};
+    if (t < NGRAM_BF16 || t > NGRAM_NVFP4) return fail(NGRAM_EINVAL, "unknown dtype %d", static_cast<int>(t));
+    if (d == 0 || d % multiple[t] != 0)
+        return fail(NGRAM_EINVAL, "%s rows need d %% %u == 0 and d > 0, got %u", names[t], multiple[t], d);
+    if (t == NGRAM_BF16 && row_scale != nullptr) return fail(NGRAM_EINVAL, "bf16 rows take no row_scale");
+    if (t != NGRAM_BF16 && row_scale == nullptr)
+        return fail(NGRAM_EINVAL, "%s rows need row_scale (%s)", names[t],
+                    t == NGRAM_NVFP4 ? "the fp32 global scale" : "one fp32 per row");
+    return NGRAM_OK;
+}
+
 uint32_t ceil_log2(uint64_t x) {
     uint32_t k = 0;
     while ((1ull << k) < x) ++k;
@@ -223,6 +252,7 @@ ngram_status wait_event(const ngram_ctx *c, cudaEvent_t ev, const char *what) {
 }
 
 void free_all(ngram_ctx *c) {
+    if (c->d_gscale) cudaFree(c->d_gscale);
     uint32_t *dev32[] = {c->d_err, c->d_idx, c->d_slot, c->d_pos, c->d_inv, c->d_uniq,
                          c->d_keys, c->d_first, c->d_uid, c->d_bsum, c->d_count};
     for (uint32_t *p : dev32)
@@ -275,7 +305,7 @@ ngram_status ensure_dedup_scratch(ngram_ctx *c) {
 ngram_status ensure_device_stage(ngram_ctx *c) {
     if (c->d_stage) return NGRAM_OK;
     NG_CUDA(cudaMalloc(&c->d_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging");
-    if (c->dtype == NGRAM_INT8_ROWSCALE)
+    if (scale_per_row(c->dtype))
         NG_CUDA(cudaMalloc(&c->d_stage_scale, c->dd_cap * 4ull), "staging");
     return NGRAM_OK;
 }
@@ -285,7 +315,7 @@ ngram_status ensure_host_stage(ngram_ctx *c) {
     NG_CHECK(ensure_device_stage(c));
     NG_CUDA(cudaHostAlloc(&c->h_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes,
                           cudaHostAllocPortable), "pinned staging");
-    if (c->dtype == NGRAM_INT8_ROWSCALE)
+    if (scale_per_row(c->dtype))
         NG_CUDA(cudaHostAlloc(&c->h_stage_scale, c->dd_cap * 4ull, cudaHostAllocPortable),
                 "pinned staging");
     NG_CUDA(cudaHostAlloc(&c->h_uniq, c->dd_cap * 4ull, cudaHostAllocPortable), "pinned staging");
@@ -321,6 +351,13 @@ ngram_status ensure_host_path(ngram_ctx *c) {
 }
 
 // ---------------------------------------------------------------- launch helpers
+// Scales of staged rows: per-row scales are compacted beside the rows; the NVFP4 global
+// scale is read where it is.
+const float *staged_scale_src(const ngram_ctx *c) { return scale_per_row(c->dtype) ? c->row_scale_dev : nullptr; }
+const float *staged_scale(const ngram_ctx *c, const float *stage_scale) {
+    return scale_per_row(c->dtype) ? stage_scale : c->row_scale_dev;
+}
+
 GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t *history,
                        uint32_t T, uint32_t N, const uint16_t *residual, const float *gate,
                        uint16_t *out) {
@@ -340,7 +377,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.N = N;
     g.tok_begin = 0;
     g.d = c->d;
-    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;
+    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;   // 16: 8- and 4-bit rows
     g.n_strips = (c->d / cols_per_lane + 31) / 32;
     g.strips_per_item = g.n_strips;
     g.groups_per_token = 1;
@@ -390,12 +427,20 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
     uint64_t blocks = (items + 7) / 8;
     if (blocks > max_blocks) blocks = max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
-    if (c->dtype == NGRAM_BF16) {
-        if (g.h.n_heads == 16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g);
-        else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
-    } else {
-        if (g.h.n_heads == 16) k_gather_int8<16><<<nb, 256, 0, s>>>(g);
-        else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
+    const bool h16 = g.h.n_heads == 16;
+    switch (c->dtype) {
+        case NGRAM_BF16:
+            if (h16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g); else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_INT8_ROWSCALE:
+            if (h16) k_gather_int8<16><<<nb, 256, 0, s>>>(g); else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_FP8_E4M3_ROWSCALE:
+            if (h16) k_gather_fp8<16><<<nb, 256, 0, s>>>(g); else k_gather_fp8<0><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_NVFP4:
+            if (h16) k_gather_nvfp4<16><<<nb, 256, 0, s>>>(g); else k_gather_nvfp4<0><<<nb, 256, 0, s>>>(g);
+            break;
     }
     NG_CUDA(cudaGetLastError(), "gather kernel launch");
     return NGRAM_OK;
@@ -466,12 +511,12 @@ ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
     NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
     NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
     k_compact_rows<<<grid_for(c, M * 32ull, 256), 256, 0, k.s>>>(
-        static_cast<const uint8_t *>(c->table_dev), c->row_scale_dev, c->d_uniq, c->d_count,
+        static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c), c->d_uniq, c->d_count,
         c->row_bytes, c->d_stage, c->d_stage_scale);
     NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     g.table = c->d_stage;
-    g.row_scale = c->d_stage_scale;
+    g.row_scale = staged_scale(c, c->d_stage_scale);
     g.row_ids = c->d_inv;
     return launch_gather(c, g, k.s, full_grid(c));
 }
@@ -519,7 +564,7 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
     c->stage_in_use = 1;
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     g.table = c->d_stage;
-    g.row_scale = c->d_stage_scale;
+    g.row_scale = staged_scale(c, c->d_stage_scale);
     g.row_ids = c->d_inv;
     return launch_gather(c, g, k.s, full_grid(c));
 }
@@ -638,6 +683,14 @@ ngram_status ngram_host_free(void *p) {
     return NGRAM_OK;
 }
 
+ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *out) {
+    if (out == nullptr) return fail(NGRAM_EINVAL, "out is NULL");
+    const float one = 1.0f;
+    NG_CHECK(check_format(dtype, d, dtype == NGRAM_BF16 ? nullptr : &one));
+    *out = row_bytes_of(dtype, d);
+    return NGRAM_OK;
+}
+
 ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_scale, uint64_t R,
                         uint32_t d, ngram_dtype dtype, ngram_residency where,
                         const ngram_hash_params *hp, uint32_t max_tokens) {
@@ -646,16 +699,7 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (table == nullptr) return fail(NGRAM_EINVAL, "table is NULL");
     if (!aligned16(table)) return fail(NGRAM_EINVAL, "table must be 16-byte aligned");
     if (R == 0 || R > 0xFFFFFFFFull) return fail(NGRAM_EINVAL, "R must be in [1, 2^32 - 1]");
-    if (dtype != NGRAM_BF16 && dtype != NGRAM_INT8_ROWSCALE)
-        return fail(NGRAM_EINVAL, "unknown dtype %d", static_cast<int>(dtype));
-    if (dtype == NGRAM_BF16 && (d == 0 || d % 8 != 0))
-        return fail(NGRAM_EINVAL, "bf16 rows need d %% 8 == 0 and d > 0, got %u", d);
-    if (dtype == NGRAM_INT8_ROWSCALE && (d == 0 || d % 16 != 0))
-        return fail(NGRAM_EINVAL, "int8 rows need d %% 16 == 0 and d > 0, got %u", d);
-    if (dtype == NGRAM_INT8_ROWSCALE && row_scale == nullptr)
-        return fail(NGRAM_EINVAL, "int8 rows need row_scale");
-    if (dtype == NGRAM_BF16 && row_scale != nullptr)
-        return fail(NGRAM_EINVAL, "row_scale is only for int8 rows");
+    NG_CHECK(check_format(dtype, d, row_scale));
     if (where != NGRAM_RES_HBM && where != NGRAM_RES_HOST_UVA && where != NGRAM_RES_HOST_DMA &&
         where != NGRAM_RES_HOST_AUTO)
         return fail(NGRAM_EINVAL, "unknown residency %d", static_cast<int>(where));
@@ -681,11 +725,11 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     memset(c, 0, sizeof(*c));
     c->table = table;
     c->table_dev = table;
-    c->row_scale = row_scale;
-    c->row_scale_dev = row_scale;
+    c->row_scale = scale_per_row(dtype) ? row_scale : nullptr;
+    c->row_scale_dev = c->row_scale;
     c->R = R;
     c->d = d;
-    c->row_bytes = (dtype == NGRAM_BF16) ? 2u * d : d;
+    c->row_bytes = row_bytes_of(dtype, d);
     c->dtype = dtype;
     c->where = where;
     c->hp = p;
@@ -699,14 +743,22 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     ngram_status st = NGRAM_OK;
     cudaError_t e = cudaGetDevice(&c->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
-    if (e == cudaSuccess)
-        e = (dtype == NGRAM_BF16)
-                ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->gather_blocks_per_sm,
-                                                                k_gather_bf16<16>, 256, 0)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->gather_blocks_per_sm,
-                                                                k_gather_int8<16>, 256, 0);
+    if (e == cudaSuccess) {
+        int *bps = &c->gather_blocks_per_sm;
+        switch (dtype) {
+            case NGRAM_BF16: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_bf16<16>, 256, 0); break;
+            case NGRAM_INT8_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_int8<16>, 256, 0); break;
+            case NGRAM_FP8_E4M3_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_fp8<16>, 256, 0); break;
+            case NGRAM_NVFP4: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_nvfp4<16>, 256, 0); break;
+        }
+    }
     if (e == cudaSuccess) e = cudaMalloc(&c->d_err, 4 * sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, 4 * sizeof(uint32_t));
+    if (e == cudaSuccess && dtype == NGRAM_NVFP4) {   // the global scale, from host or device memory
+        e = cudaMalloc(&c->d_gscale, sizeof(float));
+        if (e == cudaSuccess) e = cudaMemcpy(c->d_gscale, row_scale, sizeof(float), cudaMemcpyDefault);
+        c->row_scale_dev = c->d_gscale;
+    }
     if (e != cudaSuccess) st = cuda_fail(e, "ngram_init");
     if (st == NGRAM_OK && where != NGRAM_RES_HBM) {
         cudaPointerAttributes attr;
@@ -721,7 +773,7 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
                 st = fail(NGRAM_EINVAL, "UVA needs pinned, mapped host memory (ngram_host_alloc)");
             else
                 c->table_dev = attr.devicePointer;
-            if (st == NGRAM_OK && row_scale != nullptr) {
+            if (st == NGRAM_OK && c->row_scale != nullptr) {
                 e = cudaPointerGetAttributes(&attr, row_scale);
                 if (e != cudaSuccess || attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr)
                     st = fail(NGRAM_EINVAL, "UVA needs row_scale in pinned, mapped host memory");
@@ -852,7 +904,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     if (!sl.inv) {
         NG_CUDA(cudaMalloc(&sl.inv, c->dd_cap * 4ull), "staging slot");
         NG_CUDA(cudaMalloc(&sl.stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging slot");
-        if (c->dtype == NGRAM_INT8_ROWSCALE)
+        if (scale_per_row(c->dtype))
             NG_CUDA(cudaMalloc(&sl.stage_scale, c->dd_cap * 4ull), "staging slot");
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -862,7 +914,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     // each distinct row crosses once; from host memory a few CTAs keep PCIe busy
     const unsigned grid = (c->where == NGRAM_RES_HBM) ? grid_for(c, M * 32ull, 256)
                                                       : static_cast<unsigned>(NGRAM_UVA_CTAS);
-    k_compact_rows<<<grid, 256, 0, s>>>(static_cast<const uint8_t *>(c->table_dev), c->row_scale_dev,
+    k_compact_rows<<<grid, 256, 0, s>>>(static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c),
                                         c->d_uniq, c->d_count, c->row_bytes, sl.stage, sl.stage_scale);
     NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
     return NGRAM_OK;
@@ -889,7 +941,7 @@ ngram_status ngram_forward_staged(ngram_ctx *c, uint32_t slot, const uint16_t *r
     }
     GatherArgs g = gather_args(c, nullptr, nullptr, sl.T, static_cast<uint32_t>(N), residual, gate, out);
     g.table = sl.stage;
-    g.row_scale = sl.stage_scale;
+    g.row_scale = staged_scale(c, sl.stage_scale);
     g.row_ids = sl.inv;
     return launch_gather(c, g, reinterpret_cast<cudaStream_t>(stream), full_grid(c));
 }
@@ -937,12 +989,7 @@ ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uin
     if (table == nullptr) return fail(NGRAM_EINVAL, "table is NULL");
     if (!aligned16(table)) return fail(NGRAM_EINVAL, "table must be 16-byte aligned");
     if (R == 0 || R > 0xFFFFFFFFull) return fail(NGRAM_EINVAL, "R must be in [1, 2^32 - 1]");
-    if (dtype == NGRAM_BF16 && (d == 0 || d % 8 != 0))
-        return fail(NGRAM_EINVAL, "bf16 rows need d %% 8 == 0 and d > 0, got %u", d);
-    if (dtype == NGRAM_INT8_ROWSCALE && (d == 0 || d % 16 != 0 || row_scale == nullptr))
-        return fail(NGRAM_EINVAL, "int8 rows need d %% 16 == 0 and a row_scale buffer");
-    if (dtype != NGRAM_BF16 && dtype != NGRAM_INT8_ROWSCALE)
-        return fail(NGRAM_EINVAL, "unknown dtype %d", static_cast<int>(dtype));
+    NG_CHECK(check_format(dtype, d, row_scale));
     int dev = 0, sms = 0;
     NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
     NG_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute");
@@ -967,10 +1014,13 @@ ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uin
     if (blocks > R) blocks = R;
     const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == NGRAM_BF16)
-        k_fill_bf16<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<uint16_t *>(dst), R, d, k0, k1);
-    else
-        k_fill_int8<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<int8_t *>(dst), dst_scale, R, d, k0, k1);
+    const unsigned nb = static_cast<unsigned>(blocks);
+    switch (dtype) {
+        case NGRAM_BF16: k_fill_bf16<<<nb, 256, 0, s>>>(static_cast<uint16_t *>(dst), R, d, k0, k1); break;
+        case NGRAM_INT8_ROWSCALE: k_fill_int8<<<nb, 256, 0, s>>>(static_cast<int8_t *>(dst), dst_scale, R, d, k0, k1); break;
+        case NGRAM_FP8_E4M3_ROWSCALE: k_fill_fp8<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, k0, k1); break;
+        case NGRAM_NVFP4: k_fill_fp4<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, k0, k1); break;
+    }
     NG_CUDA(cudaGetLastError(), "k_fill launch");
     return NGRAM_OK;
 }

@@ -64,9 +64,26 @@ typedef enum {
     NGRAM_EDEVICE = 6          /* a kernel flagged bad input (device error word set) */
 } ngram_status;
 
+/* Row formats.  bf16 is the table as the pages size it (20M x 2560, ~95 GiB); the
+ * 8-bit and 4-bit formats are the smaller tables the pages weigh ("Qwen3.8-Flash-Next:
+ * A 51B N-gram Embedding Table with Heterogeneous Memory Prefetch": ~51 GB INT8 in Key
+ * point 3, ~25.5 GB at FP4 in its architecture figure; "Qwen3.8-Flash-Next: A 125B MoE
+ * for the Local Stack?", section "Hardware math for self-hosting": FP8 and 4-bit).  In
+ * every scaled format the value of a code is q * s with q exact in fp32, and the sum over
+ * heads is acc = fma(q, s, acc) in fp32, head order, one rounding per head. */
 typedef enum {
-    NGRAM_BF16 = 0,            /* table [R][d] bf16 */
-    NGRAM_INT8_ROWSCALE = 1    /* table [R][d] int8 + row_scale [R] fp32; value = q * scale */
+    NGRAM_BF16 = 0,            /* table [R][d] bf16; d % 8 == 0 */
+    NGRAM_INT8_ROWSCALE = 1,   /* table [R][d] int8 + row_scale [R] fp32; value = q * scale;
+                                  d % 16 == 0 */
+    NGRAM_FP8_E4M3_ROWSCALE = 2, /* table [R][d] FP8 E4M3 codes (OCP: bias 7, S.1111.111 NaN,
+                                  no infinities) + row_scale [R] fp32; value = e4m3(q) * scale;
+                                  d % 16 == 0 */
+    NGRAM_NVFP4 = 3            /* table [R][rb] bytes, rb = d/2 + ceil16(d/16): d/2 bytes of
+                                  FP4 E2M1 codes (OCP MX: bias 1, magnitudes 0, 0.5, 1, 1.5,
+                                  2, 3, 4, 6; column 2j in the low nibble of byte j), then one
+                                  E4M3 scale byte per 16 columns, then zero padding to rb.
+                                  row_scale points at ONE fp32 global scale gs.  value =
+                                  e2m1(q) * cs, cs = fp32(e4m3(block scale) * gs); d % 32 == 0 */
 } ngram_dtype;
 
 typedef enum {
@@ -128,13 +145,20 @@ NGRAM_API ngram_status ngram_default_hash_params(ngram_hash_params *hp);
 NGRAM_API ngram_status ngram_host_alloc(void **out, uint64_t bytes);
 NGRAM_API ngram_status ngram_host_free(void *p);
 
+/* Bytes of one table row in the dtype's layout (2d bf16; d int8 and fp8;
+ * d/2 + ceil16(d/16) nvfp4), after the same d checks as ngram_init.  Host only, no CUDA
+ * call.  EINVAL for an unknown dtype, a d the dtype does not allow, or out == NULL. */
+NGRAM_API ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *out);
+
 /* Create a lookup context on the current CUDA device.
- *   table      the [R][d] rows (bf16 bits, or int8), 16-byte aligned; not owned, must
+ *   table      the R rows in the dtype's layout (ngram_dtype), 16-byte aligned; not owned, must
  *              outlive the context.  Device memory for NGRAM_RES_HBM; pinned, mapped
  *              host memory (ngram_host_alloc) for HOST_UVA and HOST_AUTO; any host
  *              memory for HOST_DMA (host threads read it).
- *   row_scale  [R] fp32 (int8 only, else NULL), in the same kind of memory; not owned.
- *   R          rows, 1 <= R < 2^32.   d: row width, multiple of 8 (bf16) or 16 (int8).
+ *   row_scale  int8 / fp8: [R] fp32 in the same kind of memory as the table; not owned.
+ *              nvfp4: ONE fp32 (host or device memory), copied by this call.  bf16: NULL.
+ *   R          rows, 1 <= R < 2^32.   d: row width (columns), a multiple of 8 (bf16),
+ *              16 (int8, fp8) or 32 (nvfp4).
  *   where      residency of the table:
  *              HBM       one fused kernel per call;
  *              HOST_UVA  the same kernel reads the rows from host memory over PCIe;
@@ -279,6 +303,15 @@ NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens,
  *   int8: counter (col/4, row, 2, 0), word x[col%4]; q = (sum of its bytes - 510) >> 2;
  *         row_scale[row] = 0x1.1bc5f4p-11 * (0.75 + (x0 >> 8) * 2^-25) with x0 from
  *         counter (0, row, 3, 0), each fp32 step rounded separately.
+ *   fp8:  counter (col/4, row, 4, 0), word w = x[col%4]; code = sign bit 31, exponent
+ *         field 4 + bits[3:4] + bits[5:6] (4..10, never NaN), mantissa bits[0:2];
+ *         row_scale[row] = 0x1.4dp-8 * (0.75 + (x0 >> 8) * 2^-25), x0 from counter
+ *         (0, row, 5, 0), each fp32 step rounded separately.
+ *   nvfp4: code of column c = nibble c%8 of word x[(c/8)%4] of counter (c/32, row, 6, 0)
+ *         (so code bytes 16k..16k+15 are the 16 output bytes of counter k in order);
+ *         scale of block b = word w = x[b%4] of counter (b/4, row, 7, 0): exponent field
+ *         5 + bits[0:1] + bit[2] (5..9), mantissa bits[3:5], positive; padding bytes 0;
+ *         row_scale[0] = 0x1.4fp-9 (the global scale; a buffer of one fp32).
  * Asynchronous on stream. */
 NGRAM_API ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
                                   ngram_dtype dtype, uint64_t seed, ngram_stream_t stream);

@@ -32,7 +32,7 @@ class Workload:
     name: str
     R: int                 # table rows
     d: int                 # row width
-    dtype: str             # "bf16" or "int8"
+    dtype: str             # "bf16", "int8", "fp8" (E4M3 + row scale) or "nvfp4"
     vocab: int
     n_seq: int
     T: int
@@ -69,6 +69,16 @@ WORKLOADS = {
     "profile_int8": Workload("profile_int8", 1_000_000, 2560, "int8", 151_936, 16, 1024, tokens="uniform"),
     # 20M x 2560 int8 + fp32 row scale (47.8 GiB), 65,536 uniform tokens (little reuse)
     "int8_uniform": Workload("int8_uniform", 20_000_000, 2560, "int8", 151_936, 16, 4096, tokens="uniform"),
+    # 20M x 2560 FP8 E4M3 + fp32 row scale (47.8 GiB), one 32,768-token Zipf prefill
+    "fp8_prefill": Workload("fp8_prefill", 20_000_000, 2560, "fp8", 151_936, 1, 32_768),
+    # 20M x 2560 NVFP4, 1,440-byte rows (26.8 GiB), one 32,768-token Zipf prefill
+    "nvfp4_prefill": Workload("nvfp4_prefill", 20_000_000, 2560, "nvfp4", 151_936, 1, 32_768),
+    # the same tables, 65,536 uniform tokens (little reuse)
+    "fp8_uniform": Workload("fp8_uniform", 20_000_000, 2560, "fp8", 151_936, 16, 4096, tokens="uniform"),
+    "nvfp4_uniform": Workload("nvfp4_uniform", 20_000_000, 2560, "nvfp4", 151_936, 16, 4096, tokens="uniform"),
+    # profiling cases: 1M x 2560 fp8 (2.4 GiB) and 2M x 2560 nvfp4 (2.7 GiB), 16 x 1024 uniform
+    "profile_fp8": Workload("profile_fp8", 1_000_000, 2560, "fp8", 151_936, 16, 1024, tokens="uniform"),
+    "profile_nvfp4": Workload("profile_nvfp4", 2_000_000, 2560, "nvfp4", 151_936, 16, 1024, tokens="uniform"),
 }
 
 

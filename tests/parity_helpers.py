@@ -84,9 +84,15 @@ class TableCache:
         if dtype == ng.NGRAM_BF16:
             table = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
             scale = None
-        else:
+        elif dtype == ng.NGRAM_INT8_ROWSCALE:
             table = torch.empty((R, d), dtype=torch.int8, device=dev)
             scale = torch.empty((R,), dtype=torch.float32, device=dev)
+        elif dtype == ng.NGRAM_FP8_E4M3_ROWSCALE:
+            table = torch.empty((R, d), dtype=torch.uint8, device=dev)
+            scale = torch.empty((R,), dtype=torch.float32, device=dev)
+        else:                                   # NVFP4: row bytes, one global scale
+            table = torch.empty((R, ng.ngram_row_bytes(dtype, d)), dtype=torch.uint8, device=dev)
+            scale = torch.empty((1,), dtype=torch.float32, device=dev)
         ng.ngram_fill_synthetic(table, R, d, dtype, seed, row_scale=scale)
         torch.cuda.synchronize()
         self.key, self.table, self.scale = key, table, scale
@@ -99,6 +105,17 @@ class TableCache:
 
 
 TABLES = TableCache()
+
+
+def ng_dtype(name: str) -> int:
+    import hashed_gram_embedding_ngram_b200 as ng
+    return {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
+            "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[name]
+
+
+def oracle_dtype(name: str) -> int:
+    import oracle
+    return {"bf16": oracle.BF16, "int8": oracle.INT8, "fp8": oracle.FP8, "nvfp4": oracle.NVFP4}[name]
 
 
 def workload_on_device(w, dev, token_seed=gen.TOKEN_SEED):

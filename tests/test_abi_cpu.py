@@ -68,6 +68,10 @@ _T = torch.zeros(64, dtype=torch.bfloat16)      # any 16-byte aligned host addre
     (dict(dtype=7), "dtype"),
     (dict(where=9), "residency"),
     (dict(dtype=ng.NGRAM_INT8_ROWSCALE, d=32), "row_scale"),
+    (dict(dtype=ng.NGRAM_FP8_E4M3_ROWSCALE, d=32), "row_scale"),
+    (dict(dtype=ng.NGRAM_FP8_E4M3_ROWSCALE, d=24), "d % 16"),
+    (dict(dtype=ng.NGRAM_NVFP4, d=48), "d % 32"),
+    (dict(dtype=ng.NGRAM_NVFP4, d=64), "global scale"),
     (dict(d=264, max_tokens=2**31), "too large"),
 ])
 def test_init_rejects_bad_arguments_before_cuda(kw, msg):
@@ -80,6 +84,27 @@ def test_init_rejects_bad_arguments_before_cuda(kw, msg):
                       args["max_tokens"])
     assert ei.value.status == ng.NGRAM_EINVAL
     assert msg in str(ei.value)
+
+
+def test_row_bytes_of_every_format():
+    assert ng.ngram_row_bytes(ng.NGRAM_BF16, 2560) == 5120
+    assert ng.ngram_row_bytes(ng.NGRAM_INT8_ROWSCALE, 2560) == 2560
+    assert ng.ngram_row_bytes(ng.NGRAM_FP8_E4M3_ROWSCALE, 2560) == 2560
+    # nvfp4: d/2 code bytes + d/16 scale bytes padded to 16 (always a multiple of 16)
+    for d in (32, 96, 256, 2560, 2592, 4096):
+        rb = ng.ngram_row_bytes(ng.NGRAM_NVFP4, d)
+        assert rb == d // 2 + -(-(d // 16) // 16) * 16 and rb % 16 == 0
+    assert ng.ngram_row_bytes(ng.NGRAM_NVFP4, 2560) == 1440
+    for dt, d in ((ng.NGRAM_NVFP4, 16), (ng.NGRAM_FP8_E4M3_ROWSCALE, 8), (ng.NGRAM_BF16, 4), (9, 64)):
+        with pytest.raises(ng.NgramError):
+            ng.ngram_row_bytes(dt, d)
+
+
+def test_bf16_init_rejects_a_row_scale():
+    s = torch.zeros(4, dtype=torch.float32)
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, None, 16, row_scale=s)
+    assert "no row_scale" in str(ei.value)
 
 
 def test_init_rejects_null_and_misaligned_table():
@@ -107,6 +132,10 @@ def test_fill_rejects_bad_arguments():
         ng.ngram_fill_synthetic(_T, 10, 12, stream=0)
     with pytest.raises(ng.NgramError):
         ng.ngram_fill_synthetic(_T, 10, 32, ng.NGRAM_INT8_ROWSCALE, stream=0)   # no row_scale
+    with pytest.raises(ng.NgramError):
+        ng.ngram_fill_synthetic(_T, 10, 32, ng.NGRAM_NVFP4, stream=0)           # no global scale
+    with pytest.raises(ng.NgramError):
+        ng.ngram_fill_synthetic(_T, 10, 48, ng.NGRAM_NVFP4, row_scale=_T, stream=0)
 
 
 def test_null_context_is_rejected():

@@ -14,7 +14,7 @@ import torch
 import ngram_inputs as gen
 import oracle
 import hashed_gram_embedding_ngram_b200 as ng
-from parity_helpers import (N_CPU, TABLES, assert_parity, from_dev_bf16, parity_report,
+from parity_helpers import (N_CPU, TABLES, assert_parity, from_dev_bf16, ng_dtype, oracle_dtype, parity_report,
                             sample_tokens, to_dev_bf16, to_dev_tokens, workload_on_device)
 
 pytestmark = pytest.mark.gpu
@@ -28,7 +28,7 @@ def _hp(vocab, nb=8, nt=8, **kw):
 
 def _oracle(w, inp, sel=None, acc=oracle.ACC_F32, want_aux=False, **kw):
     return oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"],
-                          R=w.R, d=w.d, dtype=oracle.BF16 if w.dtype == "bf16" else oracle.INT8,
+                          R=w.R, d=w.d, dtype=oracle_dtype(w.dtype),
                           table_seed=gen.TABLE_SEED, sel=sel, acc=acc, n_threads=N_CPU,
                           vocab_size=w.vocab, want_aux=want_aux, **kw)
 
@@ -39,7 +39,7 @@ def _run(w, dev, inp_dev, ctx, out=None):
 
 
 def _ctx_for(w, dev, max_tokens=None):
-    dtype = ng.NGRAM_BF16 if w.dtype == "bf16" else ng.NGRAM_INT8_ROWSCALE
+    dtype = ng_dtype(w.dtype)
     table, scale = TABLES.get(w.R, w.d, dtype, gen.TABLE_SEED, dev)
     return ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, _hp(w.vocab),
                          max_tokens or w.N, row_scale=scale)
@@ -413,7 +413,7 @@ def test_sort_flag_is_bit_identical(cuda_device, name):
     the default (grouped from NGRAM_SORT_MIN_TOKENS tokens) agrees with both."""
     w = W[name]
     inp, dv = workload_on_device(w, cuda_device)
-    dtype = ng.NGRAM_BF16 if w.dtype == "bf16" else ng.NGRAM_INT8_ROWSCALE
+    dtype = ng_dtype(w.dtype)
     table, scale = TABLES.get(w.R, w.d, dtype, gen.TABLE_SEED, cuda_device)
     ctxs = [ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, _hp(w.vocab, flags=f), w.N,
                           row_scale=scale)
