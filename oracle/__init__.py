@@ -91,9 +91,16 @@ def _load():
         lib.oracle_indices.argtypes = [P, P, u32, u32, u64, ctypes.POINTER(_HashParams), P]
         lib.oracle_indices.restype = ctypes.c_int
         lib.oracle_forward.argtypes = [ctypes.c_int, P, P, P, u64, u64, u32,
-                                       ctypes.POINTER(_HashParams), P, P, u32, u32, P, P,
+                                       ctypes.POINTER(_HashParams), P, P, u32, u32, P, P, P,
                                        P, u64, ctypes.c_int, ctypes.c_int, P, P, P, P]
         lib.oracle_forward.restype = ctypes.c_int
+        lib.oracle_backward_rows.argtypes = [u64, u32, ctypes.POINTER(_HashParams), P, P, u32, u32,
+                                             P, P, P, P, u64, ctypes.c_int, ctypes.c_int, P, P, P]
+        lib.oracle_backward_rows.restype = ctypes.c_int64
+        lib.oracle_backward_gate.argtypes = [ctypes.c_int, P, P, P, u64, u64, u32,
+                                             ctypes.POINTER(_HashParams), P, P, u32, u32, P,
+                                             ctypes.c_int, P, u64, ctypes.c_int, ctypes.c_int, P, P]
+        lib.oracle_backward_gate.restype = ctypes.c_int
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
@@ -240,10 +247,11 @@ def unique_rows(idx):
 def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_seed=None,
             table=None, table_i8=None, row_scale=None, sel=None, acc=ACC_F32, n_threads=1,
             base_seed=DEFAULT_BASE_SEED, n_bigram=8, n_trigram=8, pad_id=DEFAULT_PAD_ID,
-            vocab_size=DEFAULT_PAD_ID, want_aux=False):
+            vocab_size=DEFAULT_PAD_ID, want_aux=False, gate_tok=None):
     """Gated gather-sum for the selected tokens.
 
-    residual_bits: [N][d] uint16 (bf16 bit patterns); gate: [d] float32.
+    residual_bits: [N][d] uint16 (bf16 bit patterns); gate: [d] float32, or (gate_tok)
+    a per-token gate [N][d] uint16 (bf16 bit patterns), in which case gate is unused.
     Rows come from ``table`` (uint16 [R][d]) / ``table_i8`` + ``row_scale`` if given,
     otherwise they are regenerated from ``table_seed``.
     Returns out bits [n_sel][d] uint16, and with want_aux also (y, mag, idx).
@@ -255,7 +263,9 @@ def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_see
     N = n_seq * T
     hist = None if history is None else np.ascontiguousarray(history, dtype=np.int32)
     res = np.ascontiguousarray(residual_bits, dtype=np.uint16).reshape(N, d)
-    g = np.ascontiguousarray(gate, dtype=np.float32).reshape(d)
+    g = None if gate is None else np.ascontiguousarray(gate, dtype=np.float32).reshape(d)
+    if g is None and gate_tok is None:
+        raise ValueError("need gate or gate_tok")
     sel_a = None if sel is None else np.ascontiguousarray(sel, dtype=np.int64).ravel()
     n_sel = N if sel_a is None else sel_a.size
     if table is None and table_i8 is None and table_seed is None:
@@ -263,6 +273,7 @@ def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_see
     tb = None if table is None else np.ascontiguousarray(table, dtype=np.uint16)
     ti = None if table_i8 is None else np.ascontiguousarray(table_i8).view(np.int8)
     sc = None if row_scale is None else np.ascontiguousarray(row_scale, dtype=np.float32)
+    gt = None if gate_tok is None else np.ascontiguousarray(gate_tok, dtype=np.uint16).reshape(N, d)
     H = n_bigram + n_trigram
     out = np.zeros((n_sel, d), dtype=np.uint16)
     y = np.zeros((n_sel, d), dtype=np.float64) if want_aux else None
@@ -271,7 +282,7 @@ def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_see
     hp = _hp(base_seed, n_bigram, n_trigram, pad_id, vocab_size)
     rc = _load().oracle_forward(dtype, _ptr(tb), _ptr(ti), _ptr(sc),
                                 (table_seed or 0) & (2**64 - 1), R, d, ctypes.byref(hp),
-                                _ptr(tok), _ptr(hist), n_seq, T, _ptr(res), _ptr(g),
+                                _ptr(tok), _ptr(hist), n_seq, T, _ptr(res), _ptr(g), _ptr(gt),
                                 _ptr(sel_a), n_sel, acc, n_threads,
                                 _ptr(out), _ptr(y), _ptr(mag), _ptr(idx))
     if rc != 0:
@@ -279,3 +290,81 @@ def forward(tokens, history, residual_bits, gate, *, R, d, dtype=BF16, table_see
     if want_aux:
         return out, y, mag, idx
     return out
+
+
+def backward_rows(tokens, history, dy_bits, gate, *, R, d, gate_tok=None, sel_u=None,
+                  acc=ACC_F32, n_threads=1, base_seed=DEFAULT_BASE_SEED, n_bigram=8,
+                  n_trigram=8, pad_id=DEFAULT_PAD_ID, vocab_size=DEFAULT_PAD_ID, want_mag=False):
+    """Gradient with respect to the table rows the batch read.
+
+    dy_bits: [N][d] uint16 (bf16 bits of dL/dout); gate: [d] float32, or gate_tok [N][d]
+    uint16.  Returns (uniq [U] uint32 in order of first occurrence, grad [n_sel][d] fp64
+    for the positions sel_u of that list (all U if None)[, mag])."""
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    if tok.ndim == 1:
+        tok = tok[None, :]
+    n_seq, T = tok.shape
+    N = n_seq * T
+    H = n_bigram + n_trigram
+    hist = None if history is None else np.ascontiguousarray(history, dtype=np.int32)
+    dyb = np.ascontiguousarray(dy_bits, dtype=np.uint16).reshape(N, d)
+    g = None if gate is None else np.ascontiguousarray(gate, dtype=np.float32).reshape(d)
+    gt = None if gate_tok is None else np.ascontiguousarray(gate_tok, dtype=np.uint16).reshape(N, d)
+    if g is None and gt is None:
+        raise ValueError("need gate or gate_tok")
+    uniq = np.zeros(max(1, N * H), dtype=np.uint32)
+    if sel_u is None:
+        # U is not known before the call: size for the largest possible U
+        n_sel, sel_a = N * H, None
+    else:
+        sel_a = np.ascontiguousarray(sel_u, dtype=np.int64).ravel()
+        n_sel = sel_a.size
+    grad = np.zeros((n_sel, d), dtype=np.float64)
+    mag = np.zeros((n_sel, d), dtype=np.float64) if want_mag else None
+    hp = _hp(base_seed, n_bigram, n_trigram, pad_id, vocab_size)
+    U = _load().oracle_backward_rows(R, d, ctypes.byref(hp), _ptr(tok), _ptr(hist), n_seq, T,
+                                     _ptr(dyb), _ptr(g), _ptr(gt), _ptr(sel_a), n_sel, acc,
+                                     n_threads, _ptr(uniq), _ptr(grad), _ptr(mag))
+    if U < 0:
+        raise ValueError("oracle_backward_rows: bad arguments")
+    if sel_u is None:
+        grad = grad[:U]
+        mag = None if mag is None else mag[:U]
+    uniq = uniq[:U]
+    return (uniq, grad, mag) if want_mag else (uniq, grad)
+
+
+def backward_gate(tokens, history, dy_bits, *, R, d, dtype=BF16, table_seed=None, table=None,
+                  table_i8=None, row_scale=None, per_token=False, sel=None, acc=ACC_F32,
+                  n_threads=1, base_seed=DEFAULT_BASE_SEED, n_bigram=8, n_trigram=8,
+                  pad_id=DEFAULT_PAD_ID, vocab_size=DEFAULT_PAD_ID, want_mag=False):
+    """Gradient with respect to the gate: [d] (shared gate, every token summed) or
+    [n_sel][d] (per-token gate, the tokens in sel, all if None); fp64 values."""
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    if tok.ndim == 1:
+        tok = tok[None, :]
+    n_seq, T = tok.shape
+    N = n_seq * T
+    hist = None if history is None else np.ascontiguousarray(history, dtype=np.int32)
+    dyb = np.ascontiguousarray(dy_bits, dtype=np.uint16).reshape(N, d)
+    if table is None and table_i8 is None and table_seed is None:
+        raise ValueError("need a table or a table_seed")
+    tb = None if table is None else np.ascontiguousarray(table, dtype=np.uint16)
+    ti = None if table_i8 is None else np.ascontiguousarray(table_i8).view(np.int8)
+    sc = None if row_scale is None else np.ascontiguousarray(row_scale, dtype=np.float32)
+    sel_a = None if (sel is None or not per_token) else np.ascontiguousarray(sel, dtype=np.int64).ravel()
+    rows = (N if sel_a is None else sel_a.size) if per_token else 1
+    out = np.zeros((rows, d), dtype=np.float64)
+    mag = np.zeros((rows, d), dtype=np.float64) if want_mag else None
+    hp = _hp(base_seed, n_bigram, n_trigram, pad_id, vocab_size)
+    rc = _load().oracle_backward_gate(dtype, _ptr(tb), _ptr(ti), _ptr(sc),
+                                      (table_seed or 0) & (2**64 - 1), R, d, ctypes.byref(hp),
+                                      _ptr(tok), _ptr(hist), n_seq, T, _ptr(dyb), int(per_token),
+                                      _ptr(sel_a), 0 if sel_a is None else sel_a.size, acc,
+                                      n_threads, _ptr(out), _ptr(mag))
+    if rc != 0:
+        raise ValueError("oracle_backward_gate: bad arguments")
+    if not per_token:
+        out = out[0]
+        mag = None if mag is None else mag[0]
+    return (out, mag) if want_mag else out

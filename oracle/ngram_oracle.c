@@ -50,6 +50,7 @@
 #include <stddef.h>
 #include <string.h>
 #include <math.h>
+#include <stdlib.h>
 
 #define ORACLE_ACC_F64 0
 #define ORACLE_ACC_F32 1
@@ -475,11 +476,42 @@ static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *tab
     }
 }
 
+/* The head sum of one column of one token (rows idx[0..H-1]):
+ *   acc64 the exact sum (fp64; exact for these operands),
+ *   acc32 the fp32 sum in head order: bf16 rows acc = acc + v; scaled rows
+ *         acc = fmaf(q, s, acc), one rounding per head (int8, fp8, nvfp4 alike; q exact
+ *         in fp32 in every case),
+ *   mag   sum_h |E_h| (error-bound scale). */
+static void head_sum(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
+                     const float *row_scale, uint64_t table_seed, const uint32_t *idx,
+                     uint32_t H, uint32_t c, uint32_t d, float *acc32, double *acc64, double *mag)
+{
+    uint32_t h;
+    float a32 = 0.0f;
+    double a64 = 0.0, m = 0.0;
+    for (h = 0; h < H; h++) {
+        float v, sc;
+        double e64 = row_value(dtype, table_bf16, table_i8, row_scale, table_seed, idx[h], c, d,
+                               &v, &sc);
+        a64 += e64;
+        if (dtype == ORACLE_BF16)
+            a32 = a32 + v;
+        else
+            a32 = fmaf(v, sc, a32);
+        m += fabs(e64);
+    }
+    *acc32 = a32;
+    *acc64 = a64;
+    *mag = m;
+}
+
+/* gate_tok: NULL for the shared gate [d] fp32; else the per-token gate [N][d] bf16 bits
+ * (gate is then unused): g = fp32(gate_tok[flat][c]), the same arithmetic otherwise. */
 int oracle_forward(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
                    const float *row_scale, uint64_t table_seed, uint64_t R, uint32_t d,
                    const oracle_hash_params *hp,
                    const int32_t *tokens, const int32_t *history, uint32_t n_seq, uint32_t T,
-                   const uint16_t *residual, const float *gate,
+                   const uint16_t *residual, const float *gate, const uint16_t *gate_tok,
                    const int64_t *sel, uint64_t n_sel, int acc_mode, int n_threads,
                    uint16_t *out, double *y_out, double *mag_out, uint32_t *idx_out)
 {
@@ -502,22 +534,12 @@ int oracle_forward(int dtype, const uint16_t *table_bf16, const int8_t *table_i8
         if (idx_out)
             for (h = 0; h < H; h++) idx_out[(size_t)i * H + h] = idx[h];
         for (c = 0; c < d; c++) {
-            double acc64 = 0.0, mag = 0.0, y64;
-            float acc32 = 0.0f;
+            double acc64, mag, y64;
+            float acc32;
             float r32 = oracle_f32_from_bf16(residual[flat * d + c]);
-            float g32 = gate[c];
-            for (h = 0; h < H; h++) {
-                float v, sc;
-                double e64 = row_value(dtype, table_bf16, table_i8, row_scale, table_seed,
-                                       idx[h], c, d, &v, &sc);
-                acc64 += e64;
-                if (dtype == ORACLE_BF16)
-                    acc32 = acc32 + v;             /* fp32, head order */
-                else
-                    acc32 = fmaf(v, sc, acc32);    /* q * s + acc, one rounding per head */
-                /* (int8, fp8, nvfp4 alike; q exact in fp32 in every case) */
-                mag += fabs(e64);
-            }
+            float g32 = gate_tok ? oracle_f32_from_bf16(gate_tok[flat * d + c]) : gate[c];
+            head_sum(dtype, table_bf16, table_i8, row_scale, table_seed, idx, H, c, d,
+                     &acc32, &acc64, &mag);
             if (acc_mode == ORACLE_ACC_F64) {
                 y64 = (double)r32 + (double)g32 * acc64;
                 out[(size_t)i * d + c] = oracle_bf16_from_f64(y64);
@@ -530,6 +552,179 @@ int oracle_forward(int dtype, const uint16_t *table_bf16, const int8_t *table_i8
             if (y_out) y_out[(size_t)i * d + c] = y64;
             if (mag_out) mag_out[(size_t)i * d + c] = fabs((double)r32) + fabs((double)g32) * mag;
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Backward of out = residual + g (elementwise) sum_h E[idx_h], with dy = dL/dout given
+ * as bf16 [N][d] (the gradient with respect to the residual is dy itself).
+ * ---------------------------------------------------------------------------------- */
+
+/* Gradient with respect to the table: only the rows the batch read have one.  The
+ * occurrences are i = flat * H + h in ascending order; row idx[i] receives the
+ * contribution of token flat = i / H once per occurrence (a row read by two heads of
+ * one token receives it twice).  The distinct rows are listed in order of first
+ * occurrence (uniq_out, U entries; the same list as the dedup step).  For the rows
+ * u in sel_u (ascending positions in that list; NULL = all U rows):
+ *   shared gate [d]:        grad[u] = g (elementwise) sum_i dy[flat(i)]
+ *   per-token gate [N][d]:  grad[u] = sum_i g[flat(i)] (elementwise) dy[flat(i)]
+ *   ACC_F64: fp64 (products of bf16 and fp32 values are exact in fp64; sums in
+ *            ascending i);
+ *   ACC_F32: shared: S = fp32 sum in ascending i (acc = acc + dy, from 0), then
+ *            grad = fp32(g * S); per-token: acc = fmaf(g_t, dy_t, acc) in ascending i.
+ * grad_out [n_sel][d] double; mag_out [n_sel][d] (sum_i |g dy|) or NULL.
+ * Returns U, or -1 on bad arguments. */
+int64_t oracle_backward_rows(uint64_t R, uint32_t d, const oracle_hash_params *hp,
+                             const int32_t *tokens, const int32_t *history, uint32_t n_seq,
+                             uint32_t T, const uint16_t *dy, const float *gate,
+                             const uint16_t *gate_tok, const int64_t *sel_u, uint64_t n_sel,
+                             int acc_mode, int n_threads, uint32_t *uniq_out, double *grad_out,
+                             double *mag_out)
+{
+    const uint32_t H = hp->n_bigram_heads + hp->n_trigram_heads;
+    const uint64_t N = (uint64_t)n_seq * T, M = N * H;
+    uint32_t *idx, *u_of, *keys, *vals, *start, *occ;
+    uint64_t P = 16, i, U = 0;
+    int64_t k;
+    if (H == 0 || H > 64 || R == 0 || d == 0) return -1;
+    if (M == 0) return 0;
+    idx = malloc(M * sizeof(uint32_t));
+    u_of = malloc(M * sizeof(uint32_t));
+    while (P < 2 * M) P <<= 1;
+    keys = malloc(P * sizeof(uint32_t));
+    vals = malloc(P * sizeof(uint32_t));
+    start = calloc(M + 1, sizeof(uint32_t));
+    occ = malloc(M * sizeof(uint32_t));
+    if (!idx || !u_of || !keys || !vals || !start || !occ) {
+        free(idx); free(u_of); free(keys); free(vals); free(start); free(occ);
+        return -1;
+    }
+    oracle_indices(tokens, history, n_seq, T, R, hp, idx);
+    /* first-occurrence numbering through a plain open-addressing map row -> u */
+    for (i = 0; i < P; i++) keys[i] = 0xFFFFFFFFu;
+    for (i = 0; i < M; i++) {
+        uint64_t slot = ((uint64_t)idx[i] * 0x9E3779B97F4A7C15ull) & (P - 1);
+        while (keys[slot] != 0xFFFFFFFFu && keys[slot] != idx[i]) slot = (slot + 1) & (P - 1);
+        if (keys[slot] == 0xFFFFFFFFu) {
+            keys[slot] = idx[i];
+            vals[slot] = (uint32_t)U;
+            uniq_out[U++] = idx[i];
+        }
+        u_of[i] = vals[slot];
+    }
+    /* the occurrences of each u in ascending i (counting sort, stable by construction) */
+    for (i = 0; i < M; i++) start[u_of[i] + 1]++;
+    for (i = 0; i < U; i++) start[i + 1] += start[i];
+    {
+        uint32_t *fill = malloc(U * sizeof(uint32_t));
+        if (!fill) { free(idx); free(u_of); free(keys); free(vals); free(start); free(occ); return -1; }
+        memcpy(fill, start, U * sizeof(uint32_t));
+        for (i = 0; i < M; i++) occ[fill[u_of[i]]++] = (uint32_t)i;
+        free(fill);
+    }
+    if (sel_u == NULL) n_sel = U;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (k = 0; k < (int64_t)n_sel; k++) {
+        const uint64_t u = sel_u ? (uint64_t)sel_u[k] : (uint64_t)k;
+        uint32_t c, j;
+        if (u >= U) continue;
+        for (c = 0; c < d; c++) {
+            float acc32 = 0.0f;
+            double acc64 = 0.0, mag = 0.0;
+            for (j = start[u]; j < start[u + 1]; j++) {
+                const uint64_t flat = occ[j] / H;
+                const float dy32 = oracle_f32_from_bf16(dy[flat * d + c]);
+                const float g32 = gate_tok ? oracle_f32_from_bf16(gate_tok[flat * d + c]) : gate[c];
+                if (gate_tok) {
+                    acc32 = fmaf(g32, dy32, acc32);
+                    acc64 += (double)g32 * (double)dy32;
+                } else {
+                    acc32 = acc32 + dy32;
+                    acc64 += (double)dy32;
+                }
+                mag += fabs((double)g32 * (double)dy32);
+            }
+            if (!gate_tok) {
+                acc32 = gate[c] * acc32;
+                acc64 = (double)gate[c] * acc64;
+            }
+            grad_out[(size_t)k * d + c] = (acc_mode == ORACLE_ACC_F64) ? acc64 : (double)acc32;
+            if (mag_out) mag_out[(size_t)k * d + c] = mag;
+        }
+    }
+    free(idx); free(u_of); free(keys); free(vals); free(start); free(occ);
+    return (int64_t)U;
+}
+
+/* Gradient with respect to the gate; e[t] = the head sum of token t (head_sum).
+ *   shared gate:    dg[c] = sum over all N tokens of dy[t][c] * e[t][c]     (out [d])
+ *   per-token gate: dg[t][c] = dy[t][c] * e[t][c] for the tokens in sel      (out [n_sel][d])
+ *   ACC_F64: e exact; products and the sum in fp64.
+ *   ACC_F32: e = the fp32 head-order sum (as in forward); p = dy * e is exact in fp64;
+ *            shared: the fp64 sum in ascending t, rounded once to fp32; per-token: p
+ *            rounded to fp32.
+ * mag_out (same shape, or NULL): |dy| * sum_h |E_h| (summed over t for the shared gate).
+ * The shared gate sums every token (sel is ignored). */
+int oracle_backward_gate(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
+                         const float *row_scale, uint64_t table_seed, uint64_t R, uint32_t d,
+                         const oracle_hash_params *hp, const int32_t *tokens,
+                         const int32_t *history, uint32_t n_seq, uint32_t T, const uint16_t *dy,
+                         int per_token, const int64_t *sel, uint64_t n_sel, int acc_mode,
+                         int n_threads, double *dg_out, double *mag_out)
+{
+    uint64_t seeds[64];
+    const uint32_t H = hp->n_bigram_heads + hp->n_trigram_heads;
+    const uint64_t N = (uint64_t)n_seq * T;
+    double *terms = NULL, *mags = NULL;
+    int64_t i;
+    if (H == 0 || H > 64 || R == 0 || d == 0) return -1;
+    if (!per_token || sel == NULL) n_sel = N;
+    if (!per_token) {
+        /* every token's terms first (in parallel), then one sum per column in ascending t */
+        terms = malloc(N * d * sizeof(double));
+        mags = malloc(N * d * sizeof(double));
+        if (N > 0 && (!terms || !mags)) { free(terms); free(mags); return -1; }
+    }
+    oracle_head_seeds(hp->base_seed, H, seeds);
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (i = 0; i < (int64_t)n_sel; i++) {
+        const uint64_t flat = (per_token && sel) ? (uint64_t)sel[i] : (uint64_t)i;
+        const uint32_t s = (uint32_t)(flat / T), t = (uint32_t)(flat % T);
+        uint32_t w0, w1, w2, idx[64], c;
+        if (flat >= N) continue;
+        context_of(tokens, history, T, s, t, hp, &w0, &w1, &w2);
+        token_indices(w0, w1, w2, seeds, hp, R, idx);
+        for (c = 0; c < d; c++) {
+            float acc32;
+            double acc64, mag, p;
+            const double dy64 = (double)oracle_f32_from_bf16(dy[flat * d + c]);
+            head_sum(dtype, table_bf16, table_i8, row_scale, table_seed, idx, H, c, d,
+                     &acc32, &acc64, &mag);
+            p = dy64 * ((acc_mode == ORACLE_ACC_F64) ? acc64 : (double)acc32);
+            if (per_token) {
+                dg_out[(size_t)i * d + c] = (acc_mode == ORACLE_ACC_F64) ? p : (double)(float)p;
+                if (mag_out) mag_out[(size_t)i * d + c] = fabs(dy64) * mag;
+            } else {
+                terms[flat * d + c] = p;
+                mags[flat * d + c] = fabs(dy64) * mag;
+            }
+        }
+    }
+    if (!per_token) {
+        uint32_t c;
+        uint64_t t;
+        for (c = 0; c < d; c++) {
+            double sum = 0.0, m = 0.0;
+            for (t = 0; t < N; t++) {
+                sum += terms[t * d + c];
+                m += mags[t * d + c];
+            }
+            dg_out[c] = (acc_mode == ORACLE_ACC_F64) ? sum : (double)(float)sum;
+            if (mag_out) mag_out[c] = m;
+        }
+        free(terms);
+        free(mags);
     }
     return 0;
 }

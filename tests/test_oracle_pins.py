@@ -501,3 +501,112 @@ def test_low_precision_brute_force_and_fp32_mode(dtype):
                          acc=oracle.ACC_F32, vocab_size=V)
     a, b = _bits_to_f64(o32).reshape(y.shape), _bits_to_f64(out).reshape(y.shape)
     assert np.all(np.abs(a - b) <= _bf16_ulp(b) + 2.0 ** -20 * mag)
+
+
+# --------------------------------------------------------------------------- per-token gate, backward
+def _bf16_bits(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _autograd_case(seed, gate_tok, R=61, d=16, V=40, n_seq=2, T=13, nb=5, nt=3):
+    """Small batch with a bf16 table: fp64 autograd of L = sum(dy * out) with
+    out = r + g * (A E) (A the occurrence counts of the hashed rows)."""
+    toks, res, g = _tiny_case(seed=seed, n_seq=n_seq, T=T, V=V, R=R, d=d, nb=nb, nt=nt)
+    N = n_seq * T
+    rng = np.random.default_rng(seed + 9)
+    dy = _bf16_bits(rng.normal(0, 1.0, (N, d)))
+    gt = _bf16_bits(rng.normal(0, 1.0, (N, d))) if gate_tok else None
+    Eb = oracle.fill_bf16(77, 0, R, d)
+    idx = oracle.indices(toks, None, R=R, n_bigram=nb, n_trigram=nt, vocab_size=V).reshape(N, nb + nt)
+    E = torch.tensor(_bits_to_f64(Eb).reshape(R, d), requires_grad=True)
+    G = torch.tensor(_bits_to_f64(gt).reshape(N, d) if gate_tok else g.astype(np.float64),
+                     requires_grad=True)
+    e = torch.nn.functional.embedding_bag(torch.from_numpy(idx.astype(np.int64)), E, mode="sum")
+    out = torch.tensor(_bits_to_f64(res).reshape(N, d)) + G * e
+    (torch.tensor(_bits_to_f64(dy).reshape(N, d)) * out).sum().backward()
+    return dict(toks=toks, res=res, g=g, dy=dy, gt=gt, Eb=Eb, idx=idx, R=R, d=d, V=V, nb=nb, nt=nt,
+                dE=E.grad.numpy(), dG=G.grad.numpy())
+
+
+@pytest.mark.parametrize("gate_tok", [False, True])
+def test_backward_rows_matches_autograd(gate_tok):
+    c = _autograd_case(11, gate_tok)
+    kw = dict(R=c["R"], d=c["d"], gate_tok=c["gt"], n_bigram=c["nb"], n_trigram=c["nt"], vocab_size=c["V"])
+    uniq, grad = oracle.backward_rows(c["toks"], None, c["dy"], c["g"], acc=oracle.ACC_F64, **kw)
+    # the distinct rows in order of first occurrence (flat token-major, head-minor order)
+    first = {}
+    for r in c["idx"].ravel():
+        first.setdefault(int(r), len(first))
+    assert list(uniq) == list(first)
+    assert np.allclose(grad, c["dE"][uniq], rtol=1e-12, atol=1e-12)
+    others = np.setdiff1d(np.arange(c["R"]), uniq)
+    assert np.all(c["dE"][others] == 0.0)
+    # fp32 mode: within the sequential-sum bound of the exact one
+    u32, g32, mag = oracle.backward_rows(c["toks"], None, c["dy"], c["g"], acc=oracle.ACC_F32,
+                                         want_mag=True, **kw)
+    count = np.bincount(np.searchsorted(np.sort(uniq), c["idx"].ravel()), minlength=len(uniq))
+    n_terms = count[np.argsort(np.argsort(uniq))][:, None]
+    assert np.array_equal(u32, uniq)
+    assert np.all(np.abs(g32 - grad) <= (n_terms + 1) * 2.0 ** -24 * mag + 1e-300)
+    # a selection of rows gives those rows
+    sel = np.array([len(uniq) - 1, 0, 3])
+    _, gs = oracle.backward_rows(c["toks"], None, c["dy"], c["g"], acc=oracle.ACC_F32, sel_u=sel, **kw)
+    assert np.array_equal(gs, g32[sel])
+
+
+def test_backward_rows_closed_form_single_row():
+    """R = 1: every occurrence hits row 0, so grad = g * H * sum_t dy[t]; with dy small
+    multiples of 2^-4 every fp32 sum is exact and the fp32 mode equals it exactly."""
+    n_seq, T, d, V = 2, 9, 8, 30
+    rng = np.random.default_rng(5)
+    toks = rng.integers(0, V, (n_seq, T)).astype(np.int32)
+    dyv = rng.integers(-8, 9, (n_seq * T, d)) / 16.0
+    g = np.array([0.5, -1.0, 3.0, 0.25, 1.0, -2.0, 0.125, 7.0], dtype=np.float32)
+    uniq, grad = oracle.backward_rows(toks, None, _bf16_bits(dyv), g, R=1, d=d, vocab_size=V)
+    assert list(uniq) == [0]
+    assert np.array_equal(grad[0], g.astype(np.float64) * 16 * dyv.sum(0))
+
+
+@pytest.mark.parametrize("gate_tok", [False, True])
+def test_backward_gate_matches_autograd(gate_tok):
+    c = _autograd_case(12, gate_tok)
+    kw = dict(R=c["R"], d=c["d"], dtype=oracle.BF16, table=c["Eb"].reshape(c["R"], c["d"]),
+              per_token=gate_tok, n_bigram=c["nb"], n_trigram=c["nt"], vocab_size=c["V"])
+    dg = oracle.backward_gate(c["toks"], None, c["dy"], acc=oracle.ACC_F64, **kw)
+    assert np.allclose(dg, c["dG"], rtol=1e-12, atol=1e-15)
+    dg32, mag = oracle.backward_gate(c["toks"], None, c["dy"], acc=oracle.ACC_F32, want_mag=True, **kw)
+    # fp32 head sum (16 roundings) and one rounding of the product / of the fp64 sum
+    H = c["nb"] + c["nt"]
+    assert np.all(np.abs(dg32 - dg) <= (H + 2) * 2.0 ** -24 * mag + 2.0 ** -24 * np.abs(dg))
+    if gate_tok:
+        sel = np.array([5, 0, 20])
+        part = oracle.backward_gate(c["toks"], None, c["dy"], acc=oracle.ACC_F32, sel=sel, **kw)
+        assert np.array_equal(part, dg32[sel])
+
+
+def test_backward_gate_shared_is_the_sum_of_per_token():
+    c = _autograd_case(13, False)
+    kw = dict(R=c["R"], d=c["d"], dtype=oracle.BF16, table=c["Eb"].reshape(c["R"], c["d"]),
+              n_bigram=c["nb"], n_trigram=c["nt"], vocab_size=c["V"], acc=oracle.ACC_F64)
+    shared = oracle.backward_gate(c["toks"], None, c["dy"], per_token=False, **kw)
+    per_tok = oracle.backward_gate(c["toks"], None, c["dy"], per_token=True, **kw)
+    assert np.allclose(shared, per_tok.sum(0), rtol=1e-13, atol=1e-15)
+
+
+def test_forward_per_token_gate():
+    """A per-token gate whose rows all equal bf16(g) gives the shared-gate result with
+    that gate bit for bit; a general one matches r + G * (A E) in fp64."""
+    R, d, V = 97, 24, 50
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    N = toks.size
+    gb = _bf16_bits(g)
+    kw = dict(R=R, d=d, table_seed=3, vocab_size=V)
+    a = oracle.forward(toks, None, res, _bits_to_f64(gb).astype(np.float32), **kw)
+    b = oracle.forward(toks, None, res, None, gate_tok=np.tile(gb, (N, 1)), **kw)
+    assert np.array_equal(a, b)
+    G = _bf16_bits(np.random.default_rng(3).normal(0, 1, (N, d)))
+    _, y, _, idx = oracle.forward(toks, None, res, None, gate_tok=G, acc=oracle.ACC_F64,
+                                  want_aux=True, **kw)
+    E = _bits_to_f64(oracle.fill_bf16(3, 0, R, d)).reshape(R, d)
+    want = _bits_to_f64(res).reshape(N, d) + _bits_to_f64(G).reshape(N, d) * _one_hot_sum(idx, E)
+    assert np.array_equal(y, want)
