@@ -35,6 +35,7 @@ NGRAM_FLAG_DEDUP = 0x1
 NGRAM_FLAG_TMA_STAGING = 0x2
 NGRAM_FLAG_SORT = 0x4
 NGRAM_FLAG_BATCH_ORDER = 0x8
+NGRAM_FLAG_TOKEN_GATE = 0x10
 NGRAM_SORT_MIN_TOKENS = 16384
 NGRAM_STAGE_SLOTS = 2
 
@@ -99,6 +100,10 @@ _lib.ngram_dedup_rows.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P]
 _lib.ngram_dedup_rows.restype = _i32
 _lib.ngram_row_bytes.argtypes = [_i32, _u32, ctypes.POINTER(_u32)]
 _lib.ngram_row_bytes.restype = _i32
+_lib.ngram_backward_rows.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P, _P, _P]
+_lib.ngram_backward_rows.restype = _i32
+_lib.ngram_backward_gate.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P]
+_lib.ngram_backward_gate.restype = _i32
 
 
 def lib() -> ctypes.CDLL:
@@ -190,6 +195,22 @@ def ngram_init(table: torch.Tensor, R: int, d: int, dtype: int = NGRAM_BF16,
     return Context(handle.value, table, row_scale, R, d, dtype, where, hp, max_tokens)
 
 
+def _token_gate(ctx: Context) -> bool:
+    return bool(ctx.hp.flags & NGRAM_FLAG_TOKEN_GATE)
+
+
+def _check_gate(ctx: Context, gate: torch.Tensor, N: int, dev) -> None:
+    """fp32 [d], or bf16 [N][d] for a context made with NGRAM_FLAG_TOKEN_GATE."""
+    if _token_gate(ctx):
+        _need(gate, "gate", torch.bfloat16, dev)
+        if gate.numel() != N * ctx.d:
+            raise ValueError("a per-token gate must hold N * d = %d elements" % (N * ctx.d))
+    else:
+        _need(gate, "gate", torch.float32, dev)
+        if gate.numel() != ctx.d:
+            raise ValueError("gate must hold d = %d elements" % ctx.d)
+
+
 def ngram_forward(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor,
                   gate: torch.Tensor, out: torch.Tensor | None = None,
                   history: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -203,9 +224,7 @@ def ngram_forward(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor,
     _need(residual, "residual", torch.bfloat16, dev)
     if residual.numel() != N * ctx.d:
         raise ValueError("residual must hold N * d = %d elements" % (N * ctx.d))
-    _need(gate, "gate", torch.float32, dev)
-    if gate.numel() != ctx.d:
-        raise ValueError("gate must hold d = %d elements" % ctx.d)
+    _check_gate(ctx, gate, N, dev)
     if history is not None:
         _need(history, "history", torch.int32, dev, ndim=2)
         if tuple(history.shape) != (n_seq, 2):
@@ -372,10 +391,66 @@ def ngram_forward_staged(ctx: Context, slot: int, residual: torch.Tensor, gate: 
                          out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """ngram_forward for the batch staged in `slot`, gathering from HBM staging."""
     _need(residual, "residual", torch.bfloat16)
-    _need(gate, "gate", torch.float32, residual.device)
+    _check_gate(ctx, gate, residual.numel() // ctx.d, residual.device)
     if out is None:
         out = torch.empty_like(residual)
     _need(out, "out", torch.bfloat16, residual.device)
     _check(_lib.ngram_forward_staged(ctx.handle, slot, _ptr(residual), _ptr(gate), _ptr(out),
                                      _stream(stream)))
+    return out
+
+
+def ngram_backward_rows(ctx: Context, tokens: torch.Tensor, grad_out: torch.Tensor,
+                        gate: torch.Tensor, history: torch.Tensor | None = None,
+                        uniq_out: torch.Tensor | None = None, count_out: torch.Tensor | None = None,
+                        grad_rows: torch.Tensor | None = None, stream=None):
+    """Gradient with respect to the table rows the batch read.  Returns (uniq int32 [N*H],
+    count int32 [1], grad_rows fp32 [N*H][d]); the first count entries / rows are valid."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    dev = tokens.device
+    n_seq, T = tokens.shape
+    N = n_seq * T
+    M = N * ctx.n_heads
+    _need(grad_out, "grad_out", torch.bfloat16, dev)
+    if grad_out.numel() != N * ctx.d:
+        raise ValueError("grad_out must hold N * d elements")
+    _check_gate(ctx, gate, N, dev)
+    if history is not None:
+        _need(history, "history", torch.int32, dev, ndim=2)
+    if uniq_out is None:
+        uniq_out = torch.empty(max(1, M), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty(1, dtype=torch.int32, device=dev)
+    if grad_rows is None:
+        grad_rows = torch.empty((max(1, M), ctx.d), dtype=torch.float32, device=dev)
+    _need(grad_rows, "grad_rows", torch.float32, dev)
+    if grad_rows.numel() < M * ctx.d:
+        raise ValueError("grad_rows must hold N * H * d elements")
+    _check(_lib.ngram_backward_rows(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                                    _ptr(grad_out), _ptr(gate), _ptr(uniq_out), _ptr(count_out),
+                                    _ptr(grad_rows), _stream(stream)))
+    return uniq_out, count_out, grad_rows
+
+
+def ngram_backward_gate(ctx: Context, tokens: torch.Tensor, grad_out: torch.Tensor,
+                        history: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """Gradient with respect to the gate: fp32 [d], or fp32 [N][d] for a per-token gate."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    dev = tokens.device
+    n_seq, T = tokens.shape
+    N = n_seq * T
+    _need(grad_out, "grad_out", torch.bfloat16, dev)
+    if grad_out.numel() != N * ctx.d:
+        raise ValueError("grad_out must hold N * d elements")
+    if history is not None:
+        _need(history, "history", torch.int32, dev, ndim=2)
+    shape = (N, ctx.d) if _token_gate(ctx) else (ctx.d,)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    if out.numel() != (N * ctx.d if _token_gate(ctx) else ctx.d):
+        raise ValueError("out must hold %s elements" % (shape,))
+    _check(_lib.ngram_backward_gate(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
+                                    _ptr(grad_out), _ptr(out), _stream(stream)))
     return out

@@ -31,7 +31,8 @@ struct GatherArgs {
     const int32_t *tokens;      // [n_seq][T]
     const int32_t *history;     // [n_seq][2] or null
     const uint16_t *residual;   // [N][d] bf16 bits
-    const float *gate;          // [d]
+    const float *gate;          // [d], shared by every token
+    const uint16_t *gate_tok;   // [N][d] bf16 bits, a gate per token (replaces gate), or null
     uint16_t *out;              // [N][d] bf16 bits (may alias residual)
     const uint32_t *row_ids;    // [N][H] precomputed row ids into `table`, or null (hash)
     const uint32_t *perm;       // [N] processing order of the tokens, or null (batch order)
@@ -75,11 +76,33 @@ __device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t 
     return row;
 }
 
+// The gate of columns 8v .. 8v+7 of one token: the shared fp32 gate, or (kTokGate) the
+// token's bf16 gate (exact in fp32).
+template <bool kTokGate>
+__device__ __forceinline__ void load_gate8(const GatherArgs &g, size_t tok_off, uint32_t v, float gv[8]) {
+    if (kTokGate) {
+        const uint4 w = ld_na_v4(g.gate_tok + tok_off + v * 8u);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            gv[2 * p] = bf16_lo(ww[p]);
+            gv[2 * p + 1] = bf16_hi(ww[p]);
+        }
+    } else {
+        const float4 ga = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v);
+        const float4 gb = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v + 1u);
+        gv[0] = ga.x; gv[1] = ga.y; gv[2] = ga.z; gv[3] = ga.w;
+        gv[4] = gb.x; gv[5] = gb.y; gv[6] = gb.z; gv[7] = gb.w;
+    }
+}
+
 #ifndef NGRAM_LDG_MIN_BLOCKS          // resident CTAs per SM the register budget targets
 #define NGRAM_LDG_MIN_BLOCKS 2
 #endif
 
-template <int kH>   // compile-time head count (16), or 0: runtime g.h.n_heads <= 16
+// kH: compile-time head count (16), or 0: runtime g.h.n_heads <= 16.  kTokGate: the gate
+// is g.gate_tok (per token) instead of g.gate.
+template <int kH, bool kTokGate = false>
 __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const GatherArgs g) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -111,8 +134,8 @@ __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const
                 if (kH || h < static_cast<int>(H))
                     e[h] = ld_stream_v4(table + static_cast<size_t>(rows[h]) * g.d + v * 8u);
             const uint4 r = ld_na_v4(g.residual + tok_off + v * 8u);
-            const float4 ga = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v);
-            const float4 gb = __ldg(reinterpret_cast<const float4 *>(g.gate) + 2u * v + 1u);
+            float gv[8];
+            load_gate8<kTokGate>(g, tok_off, v, gv);
 
             // acc[p] holds columns (2p, 2p+1): packed pair adds round each lane exactly as
             // the scalar head-order sum
@@ -129,7 +152,6 @@ __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const
                 }
             }
             // y = r + (g * acc): the product is rounded on its own (scalar, never fused)
-            const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
             const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
             uint32_t o[4];
 #pragma unroll

@@ -38,12 +38,12 @@ struct E4m3Codes {
 
 // y = r + (g * acc) for columns 16v .. 16v+15 of one token (residual words r0, r1 loaded
 // before the sum); the product is rounded on its own (scalar, never fused).
+template <bool kTokGate>
 __device__ __forceinline__ void store_gated16(const GatherArgs &g, size_t tok_off, uint32_t v,
                                               const uint4 &r0, const uint4 &r1, const float2 acc[8]) {
-    const float4 *gp = reinterpret_cast<const float4 *>(g.gate) + 4u * v;
-    const float4 g0 = __ldg(gp), g1 = __ldg(gp + 1), g2 = __ldg(gp + 2), g3 = __ldg(gp + 3);
-    const float gv[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w,
-                          g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
+    float gv[16];
+    load_gate8<kTokGate>(g, tok_off, 2u * v, gv);
+    load_gate8<kTokGate>(g, tok_off, 2u * v + 1u, gv + 8);
     const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
     uint32_t o[8];
 #pragma unroll
@@ -62,7 +62,7 @@ __device__ __forceinline__ void store_gated16(const GatherArgs &g, size_t tok_of
 // by the hashing lanes and broadcast with the row indices.  Sum per head in order with
 // one fused multiply-add per head, acc = fma(q, s, acc) (one rounding per head), then
 // the same bf16 epilogue as the bf16 rows.
-template <int kH, class Codes>
+template <int kH, class Codes, bool kTokGate>
 __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -121,19 +121,19 @@ __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
                     }
                 }
             }
-            store_gated16(g, tok_off, v, r0, r1, acc);
+            store_gated16<kTokGate>(g, tok_off, v, r0, r1, acc);
         }
     }
 }
 
-template <int kH>
+template <int kH, bool kTokGate = false>
 __global__ void __launch_bounds__(256, 2) k_gather_int8(const GatherArgs g) {
-    gather_rowscale<kH, Int8Codes>(g);
+    gather_rowscale<kH, Int8Codes, kTokGate>(g);
 }
 
-template <int kH>
+template <int kH, bool kTokGate = false>
 __global__ void __launch_bounds__(256, 2) k_gather_fp8(const GatherArgs g) {
-    gather_rowscale<kH, E4m3Codes>(g);
+    gather_rowscale<kH, E4m3Codes, kTokGate>(g);
 }
 
 }  // namespace ngram

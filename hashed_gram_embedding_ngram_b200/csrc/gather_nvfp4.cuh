@@ -18,8 +18,12 @@
 
 namespace ngram {
 
-template <int kH>
-__global__ void __launch_bounds__(256, 2) k_gather_nvfp4(const GatherArgs g) {
+#ifndef NGRAM_NVFP4_MIN_BLOCKS        // resident CTAs per SM the register budget targets
+#define NGRAM_NVFP4_MIN_BLOCKS 2
+#endif
+
+template <int kH, bool kTokGate = false>
+__global__ void __launch_bounds__(256, NGRAM_NVFP4_MIN_BLOCKS) k_gather_nvfp4(const GatherArgs g) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(256, 2) k_gather_nvfp4(const GatherArgs g) {
                     for (int k = 0; k < 4; ++k) acc[4 + k] = fma2(q[k], s2, acc[4 + k]);
                 }
             }
-            store_gated16(g, tok_off, v, r0, r1, acc);
+            store_gated16<kTokGate>(g, tok_off, v, r0, r1, acc);
         }
     }
 }

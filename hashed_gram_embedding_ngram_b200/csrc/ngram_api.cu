@@ -23,11 +23,21 @@
 #include "gather.cuh"
 #include "gather_int8.cuh"
 #include "gather_nvfp4.cuh"
+#include "gather_c8.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
 #include "order.cuh"
+#include "sort.cuh"
+#include "backward.cuh"
 
 using namespace ngram;
+
+// Row formats (bit t = ngram_dtype t) whose gather runs k_gather_c8 (8 columns per lane)
+// instead of the format's 16-column kernel.
+#ifndef NGRAM_C8_FORMATS
+#define NGRAM_C8_FORMATS 0u
+#endif
+static bool use_c8(ngram_dtype t) { return t != NGRAM_BF16 && ((NGRAM_C8_FORMATS >> t) & 1u); }
 
 // Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
 //   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
@@ -116,6 +126,10 @@ struct ngram_ctx {
     cudaEvent_t hp_d2h[NGRAM_HOST_BUFFERS];   // end of each stream's part of the last call
     // NGRAM_FLAG_SORT: bucket of each token, bucket counts / cursors, processing order
     uint32_t *so_bucket, *so_hist, *so_perm;
+    // backward: radix-sort buffers (keys, values, twice), digit counts, scan totals,
+    // segment starts; the shared-gate gradient's fp64 partials
+    uint32_t *bw_k[2], *bw_v[2], *bw_hist, *bw_tot, *bw_seg, *bw_word;
+    double *bw_part;
     // ngram_prefetch / ngram_forward_staged: a ring of staged batches in HBM
     struct Slot {
         uint32_t *inv;          // [max_tokens * H] row ids into `stage`
@@ -278,7 +292,9 @@ void free_all(ngram_ctx *c) {
         if (sl.stage) cudaFree(sl.stage);
         if (sl.stage_scale) cudaFree(sl.stage_scale);
     }
-    void *bufs[] = {c->hp_tok, c->hp_hist, c->so_bucket, c->so_hist, c->so_perm};
+    void *bufs[] = {c->hp_tok, c->hp_hist, c->so_bucket, c->so_hist, c->so_perm, c->bw_k[0],
+                    c->bw_k[1], c->bw_v[0], c->bw_v[1], c->bw_hist, c->bw_tot, c->bw_seg,
+                    c->bw_word, c->bw_part};
     for (void *p : bufs)
         if (p) cudaFree(p);
     for (cudaStream_t s : c->hp_s)
@@ -359,7 +375,7 @@ const float *staged_scale(const ngram_ctx *c, const float *stage_scale) {
 }
 
 GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t *history,
-                       uint32_t T, uint32_t N, const uint16_t *residual, const float *gate,
+                       uint32_t T, uint32_t N, const uint16_t *residual, const void *gate,
                        uint16_t *out) {
     GatherArgs g;
     g.h = hash_args(c);
@@ -368,7 +384,9 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.tokens = tokens;
     g.history = history;
     g.residual = residual;
-    g.gate = gate;
+    const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
+    g.gate = tok_gate ? nullptr : static_cast<const float *>(gate);
+    g.gate_tok = tok_gate ? static_cast<const uint16_t *>(gate) : nullptr;
     g.out = out;
     g.row_ids = nullptr;
     g.perm = nullptr;
@@ -377,7 +395,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.N = N;
     g.tok_begin = 0;
     g.d = c->d;
-    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;   // 16: 8- and 4-bit rows
+    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16 || use_c8(c->dtype)) ? 8u : 16u;
     g.n_strips = (c->d / cols_per_lane + 31) / 32;
     g.strips_per_item = g.n_strips;
     g.groups_per_token = 1;
@@ -417,7 +435,41 @@ ngram_status launch_bulk(ngram_ctx *c, GatherArgs &g, cudaStream_t s) {
     return NGRAM_OK;
 }
 
-// The register gather (bf16 or int8); max_blocks bounds the persistent grid.
+template <class Rows, bool kTok>
+void launch_c8(const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
+    if (g.h.n_heads == 16) k_gather_c8<16, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
+    else k_gather_c8<0, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
+}
+
+template <bool kTok>
+void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
+    const bool h16 = g.h.n_heads == 16;
+    if (use_c8(t)) {
+        switch (t) {
+            case NGRAM_INT8_ROWSCALE: launch_c8<Rows8bit<Int8Codes>, kTok>(g, nb, s, rb); break;
+            case NGRAM_FP8_E4M3_ROWSCALE: launch_c8<Rows8bit<E4m3Codes>, kTok>(g, nb, s, rb); break;
+            case NGRAM_NVFP4: launch_c8<RowsNvfp4, kTok>(g, nb, s, rb); break;
+            default: break;
+        }
+        return;
+    }
+    switch (t) {
+        case NGRAM_BF16:
+            if (h16) k_gather_bf16<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_bf16<0, kTok><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_INT8_ROWSCALE:
+            if (h16) k_gather_int8<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_int8<0, kTok><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_FP8_E4M3_ROWSCALE:
+            if (h16) k_gather_fp8<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_fp8<0, kTok><<<nb, 256, 0, s>>>(g);
+            break;
+        case NGRAM_NVFP4:
+            if (h16) k_gather_nvfp4<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_nvfp4<0, kTok><<<nb, 256, 0, s>>>(g);
+            break;
+    }
+}
+
+// The register gather (every row format); max_blocks bounds the persistent grid.
 ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t max_blocks) {
     const uint64_t resident_warps = max_blocks * 8u;
     g.strips_per_item = (NGRAM_SPI_ALWAYS_ONE ||
@@ -427,21 +479,8 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
     uint64_t blocks = (items + 7) / 8;
     if (blocks > max_blocks) blocks = max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
-    const bool h16 = g.h.n_heads == 16;
-    switch (c->dtype) {
-        case NGRAM_BF16:
-            if (h16) k_gather_bf16<16><<<nb, 256, 0, s>>>(g); else k_gather_bf16<0><<<nb, 256, 0, s>>>(g);
-            break;
-        case NGRAM_INT8_ROWSCALE:
-            if (h16) k_gather_int8<16><<<nb, 256, 0, s>>>(g); else k_gather_int8<0><<<nb, 256, 0, s>>>(g);
-            break;
-        case NGRAM_FP8_E4M3_ROWSCALE:
-            if (h16) k_gather_fp8<16><<<nb, 256, 0, s>>>(g); else k_gather_fp8<0><<<nb, 256, 0, s>>>(g);
-            break;
-        case NGRAM_NVFP4:
-            if (h16) k_gather_nvfp4<16><<<nb, 256, 0, s>>>(g); else k_gather_nvfp4<0><<<nb, 256, 0, s>>>(g);
-            break;
-    }
+    if (g.gate_tok != nullptr) launch_gather_kernel<true>(c->dtype, g, nb, s, c->row_bytes);
+    else launch_gather_kernel<false>(c->dtype, g, nb, s, c->row_bytes);
     NG_CUDA(cudaGetLastError(), "gather kernel launch");
     return NGRAM_OK;
 }
@@ -486,7 +525,7 @@ struct Call {
     const int32_t *tokens, *history;
     uint32_t T, N;
     const uint16_t *residual;
-    const float *gate;
+    const void *gate;
     uint16_t *out;
     cudaStream_t s;
 };
@@ -719,6 +758,8 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if ((p.flags & NGRAM_FLAG_SORT) &&
         (p.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_BATCH_ORDER)))
         return fail(NGRAM_EINVAL, "NGRAM_FLAG_SORT does not combine with DEDUP, TMA_STAGING or BATCH_ORDER");
+    if ((p.flags & NGRAM_FLAG_TOKEN_GATE) && (p.flags & NGRAM_FLAG_TMA_STAGING))
+        return fail(NGRAM_EINVAL, "NGRAM_FLAG_TOKEN_GATE does not combine with TMA_STAGING");
 
     // ---- CUDA from here on
     ngram_ctx *c = new ngram_ctx();
@@ -745,7 +786,14 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess) {
         int *bps = &c->gather_blocks_per_sm;
-        switch (dtype) {
+        if (use_c8(dtype)) {
+            if (dtype == NGRAM_NVFP4)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, RowsNvfp4, false>, 256, 0);
+            else if (dtype == NGRAM_FP8_E4M3_ROWSCALE)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, Rows8bit<E4m3Codes>, false>, 256, 0);
+            else
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, Rows8bit<Int8Codes>, false>, 256, 0);
+        } else switch (dtype) {
             case NGRAM_BF16: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_bf16<16>, 256, 0); break;
             case NGRAM_INT8_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_int8<16>, 256, 0); break;
             case NGRAM_FP8_E4M3_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_fp8<16>, 256, 0); break;
@@ -800,7 +848,7 @@ ngram_status ngram_set_wait_timeout(ngram_ctx *c, uint32_t ms) {
 }
 
 ngram_status ngram_forward(ngram_ctx *c, const int32_t *tokens, const int32_t *history,
-                           uint32_t n_seq, uint32_t T, const uint16_t *residual, const float *gate,
+                           uint32_t n_seq, uint32_t T, const uint16_t *residual, const void *gate,
                            uint16_t *out, ngram_stream_t stream) {
     uint64_t N = 0;
     NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
@@ -838,7 +886,8 @@ ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int
     if (residual_h == nullptr || gate == nullptr || out_h == nullptr)
         return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
     if (!aligned16(gate)) return fail(NGRAM_EINVAL, "gate must be 16-byte aligned");
-    if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT)) ||  // chunks keep batch order
+    if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT |
+                        NGRAM_FLAG_TOKEN_GATE)) ||  // chunks keep batch order
         (c->where != NGRAM_RES_HBM && c->where != NGRAM_RES_HOST_UVA))
         return fail(NGRAM_EUNSUPPORTED,
                     "ngram_forward_host pipelines the fused gather: HBM or HOST_UVA residency, no flags");
@@ -921,7 +970,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
 }
 
 ngram_status ngram_forward_staged(ngram_ctx *c, uint32_t slot, const uint16_t *residual,
-                                  const float *gate, uint16_t *out, ngram_stream_t stream) {
+                                  const void *gate, uint16_t *out, ngram_stream_t stream) {
     if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
     if (slot >= NGRAM_STAGE_SLOTS)
         return fail(NGRAM_EINVAL, "slot %u out of range (%u slots)", slot, NGRAM_STAGE_SLOTS);
@@ -1022,6 +1071,150 @@ ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uin
         case NGRAM_NVFP4: k_fill_fp4<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, k0, k1); break;
     }
     NG_CUDA(cudaGetLastError(), "k_fill launch");
+    return NGRAM_OK;
+}
+
+// ---------------------------------------------------------------- backward
+}  // extern "C"
+
+namespace {
+
+ngram_status ensure_backward_sort(ngram_ctx *c) {
+    if (c->bw_k[0]) return NGRAM_OK;
+    const uint64_t M = c->dd_cap;
+    const uint64_t n_tiles = (M + kSortTile - 1) / kSortTile;
+    const uint64_t L = kSortRadix * n_tiles;
+    const uint64_t nb = (L + kScanChunk - 1) / kScanChunk;
+    for (int b = 0; b < 2; ++b) {
+        NG_CUDA(cudaMalloc(&c->bw_k[b], M * 4), "backward scratch");
+        NG_CUDA(cudaMalloc(&c->bw_v[b], M * 4), "backward scratch");
+    }
+    NG_CUDA(cudaMalloc(&c->bw_hist, L * 4), "backward scratch");
+    NG_CUDA(cudaMalloc(&c->bw_tot, nb * 4), "backward scratch");
+    NG_CUDA(cudaMalloc(&c->bw_seg, (M + 1) * 4), "backward scratch");
+    NG_CUDA(cudaMalloc(&c->bw_word, 4), "backward scratch");
+    return NGRAM_OK;
+}
+
+// Exclusive scan of a[0..n) in place.
+ngram_status scan_exclusive(ngram_ctx *c, uint32_t *a, uint32_t n, cudaStream_t s) {
+    const uint32_t nb = (n + kScanChunk - 1) / kScanChunk;
+    k_scan_local<<<nb, 256, 0, s>>>(a, n, a, c->bw_tot);
+    k_dedup_scan_blocks<<<1, 1024, 0, s>>>(c->bw_tot, nb, c->bw_word);
+    k_scan_add<<<(n + 255) / 256, 256, 0, s>>>(a, n, c->bw_tot);
+    NG_CUDA(cudaGetLastError(), "scan launch");
+    return NGRAM_OK;
+}
+
+// Stable sort of the M occurrences by key (their row's position u < M); the values are
+// the occurrences' tokens (p / H).  Returns the sorted keys and values.
+ngram_status sort_occurrences(ngram_ctx *c, const uint32_t *keys, uint32_t M, cudaStream_t s,
+                              const uint32_t **skeys, const uint32_t **svals) {
+    const uint32_t bits = std::max<uint32_t>(1u, ceil_log2(M));
+    const uint32_t passes = (bits + 7) / 8;
+    const uint32_t n_tiles = (M + kSortTile - 1) / kSortTile;
+    const unsigned grid = static_cast<unsigned>(std::min<uint64_t>(n_tiles, static_cast<uint64_t>(c->num_sms) * 8));
+    const uint32_t *kin = keys, *vin = nullptr;
+    for (uint32_t pass = 0; pass < passes; ++pass) {
+        const uint32_t shift = 8 * pass;
+        k_radix_hist<<<grid, 256, 0, s>>>(kin, M, shift, n_tiles, c->bw_hist);
+        NG_CHECK(scan_exclusive(c, c->bw_hist, kSortRadix * n_tiles, s));
+        const int o = static_cast<int>(pass & 1u);
+        k_radix_scatter<<<grid, 256, 0, s>>>(kin, vin, c->H, M, shift, n_tiles, c->bw_hist,
+                                             c->bw_k[o], c->bw_v[o]);
+        NG_CUDA(cudaGetLastError(), "radix sort launch");
+        kin = c->bw_k[o];
+        vin = c->bw_v[o];
+    }
+    *skeys = kin;
+    *svals = vin;
+    return NGRAM_OK;
+}
+
+template <class Rows, bool kTok>
+void launch_gate_grad_fmt(const GatherArgs &g, unsigned grid, cudaStream_t s, const uint16_t *dy,
+                          float *dg, double *part, uint32_t rb) {
+    if (g.h.n_heads == 16) k_gate_grad<16, Rows, kTok><<<grid, 256, 0, s>>>(g, dy, dg, part, rb);
+    else k_gate_grad<0, Rows, kTok><<<grid, 256, 0, s>>>(g, dy, dg, part, rb);
+}
+
+template <bool kTok>
+void launch_gate_grad(ngram_dtype t, const GatherArgs &g, unsigned grid, cudaStream_t s,
+                      const uint16_t *dy, float *dg, double *part, uint32_t rb) {
+    switch (t) {
+        case NGRAM_BF16: launch_gate_grad_fmt<RowsBf16, kTok>(g, grid, s, dy, dg, part, rb); break;
+        case NGRAM_INT8_ROWSCALE: launch_gate_grad_fmt<Rows8bit<Int8Codes>, kTok>(g, grid, s, dy, dg, part, rb); break;
+        case NGRAM_FP8_E4M3_ROWSCALE: launch_gate_grad_fmt<Rows8bit<E4m3Codes>, kTok>(g, grid, s, dy, dg, part, rb); break;
+        case NGRAM_NVFP4: launch_gate_grad_fmt<RowsNvfp4, kTok>(g, grid, s, dy, dg, part, rb); break;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+ngram_status ngram_backward_rows(ngram_ctx *c, const int32_t *tokens, const int32_t *history,
+                                 uint32_t n_seq, uint32_t T, const uint16_t *grad_out,
+                                 const void *gate, uint32_t *uniq_out, uint32_t *count_out,
+                                 float *grad_rows, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (count_out == nullptr) return fail(NGRAM_EINVAL, "count_out is NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        NG_CUDA(cudaMemsetAsync(count_out, 0, 4, s), "cudaMemsetAsync");
+        return NGRAM_OK;
+    }
+    if (grad_out == nullptr || gate == nullptr || uniq_out == nullptr || grad_rows == nullptr)
+        return fail(NGRAM_EINVAL, "grad_out, gate, uniq_out and grad_rows must be non-NULL");
+    if (!aligned16(grad_out) || !aligned16(gate) || !aligned16(grad_rows))
+        return fail(NGRAM_EINVAL, "grad_out, gate and grad_rows must be 16-byte aligned");
+    NG_CHECK(ensure_dedup_scratch(c));
+    NG_CHECK(ensure_backward_sort(c));
+    const uint32_t M = static_cast<uint32_t>(N) * c->H;
+    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
+    NG_CHECK(launch_dedup(c, c->d_idx, M, uniq_out, c->d_inv, count_out, s));
+    const uint32_t *skeys = nullptr, *stok = nullptr;
+    NG_CHECK(sort_occurrences(c, c->d_inv, M, s, &skeys, &stok));
+    k_seg_starts<<<grid_for(c, M, 256), 256, 0, s>>>(skeys, M, c->bw_seg);
+    const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
+    k_rows_grad<<<static_cast<unsigned>(c->num_sms) * 8u, 256, 0, s>>>(
+        count_out, c->bw_seg, stok, grad_out, tok_gate ? nullptr : static_cast<const float *>(gate),
+        tok_gate ? static_cast<const uint16_t *>(gate) : nullptr, c->d, grad_rows);
+    NG_CUDA(cudaGetLastError(), "k_rows_grad launch");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int32_t *history,
+                                 uint32_t n_seq, uint32_t T, const uint16_t *grad_out,
+                                 float *grad_gate, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (grad_gate == nullptr) return fail(NGRAM_EINVAL, "grad_gate is NULL");
+    if (!aligned16(grad_gate)) return fail(NGRAM_EINVAL, "grad_gate must be 16-byte aligned");
+    if (c->where == NGRAM_RES_HOST_DMA)
+        return fail(NGRAM_EUNSUPPORTED, "ngram_backward_gate reads the table from the GPU: HBM, HOST_UVA or HOST_AUTO");
+    const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (!tok_gate) NG_CUDA(cudaMemsetAsync(grad_gate, 0, c->d * 4ull, s), "cudaMemsetAsync");
+        return NGRAM_OK;
+    }
+    if (grad_out == nullptr) return fail(NGRAM_EINVAL, "grad_out is NULL");
+    if (!aligned16(grad_out)) return fail(NGRAM_EINVAL, "grad_out must be 16-byte aligned");
+    const GatherArgs g = gather_args(c, tokens, history, T, static_cast<uint32_t>(N), nullptr, nullptr, nullptr);
+    const unsigned grid = static_cast<unsigned>(c->num_sms) * 2u;
+    if (tok_gate) {
+        launch_gate_grad<true>(c->dtype, g, grid, s, grad_out, grad_gate, nullptr, c->row_bytes);
+    } else {
+        if (!c->bw_part)
+            NG_CUDA(cudaMalloc(&c->bw_part, ((c->max_tokens + kGateChunk - 1) / kGateChunk) * 8ull * c->d),
+                    "backward scratch");
+        const uint32_t n_chunks = static_cast<uint32_t>((N + kGateChunk - 1) / kGateChunk);
+        launch_gate_grad<false>(c->dtype, g, grid, s, grad_out, nullptr, c->bw_part, c->row_bytes);
+        k_gate_reduce<<<(c->d + 255) / 256, 256, 0, s>>>(c->bw_part, n_chunks, c->d, grad_gate);
+    }
+    NG_CUDA(cudaGetLastError(), "k_gate_grad launch");
     return NGRAM_OK;
 }
 

@@ -114,8 +114,15 @@ typedef enum {
 #define NGRAM_FLAG_SORT 0x4u
 #define NGRAM_FLAG_BATCH_ORDER 0x8u
 #define NGRAM_SORT_MIN_TOKENS 16384u
+/* A gate per token: the `gate` argument of ngram_forward, ngram_forward_staged and the
+ * backward calls is bf16 [N][d] (16-byte aligned, token-major like residual) instead of
+ * fp32 [d] -- the output of a gating network computed from the hidden state
+ * ("Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with Heterogeneous Memory
+ * Prefetch", Summary).  y = fp32(residual) + fp32(gate[t][c]) * sum, rounded as with the
+ * shared gate.  Not with TMA_STAGING (EINVAL) nor ngram_forward_host (EUNSUPPORTED). */
+#define NGRAM_FLAG_TOKEN_GATE 0x10u
 #define NGRAM_FLAGS_KNOWN (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT | \
-                           NGRAM_FLAG_BATCH_ORDER)
+                           NGRAM_FLAG_BATCH_ORDER | NGRAM_FLAG_TOKEN_GATE)
 
 #define NGRAM_MAX_HEADS 16u
 #define NGRAM_TOKEN_BITS 21u
@@ -186,7 +193,8 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  *   tokens    device int32 [n_seq][T] (row-major).
  *   history   device int32 [n_seq][2] = {w_-2, w_-1} per sequence, or NULL (PAD).
  *   residual  device bf16 [N][d], 16-byte aligned.
- *   gate      device fp32 [d], 16-byte aligned (the static gate W_g).
+ *   gate      device fp32 [d], 16-byte aligned (the static gate W_g); with
+ *             NGRAM_FLAG_TOKEN_GATE device bf16 [N][d] (one gate per token).
  *   out       device bf16 [N][d], 16-byte aligned; may equal residual (in place),
  *             must not otherwise overlap it.
  * One kernel launch on stream; N == 0 launches nothing.  EINVAL if N > max_tokens,
@@ -194,7 +202,7 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  * ngram_get_device_error. */
 NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
-                           const float *gate, uint16_t *out, ngram_stream_t stream);
+                           const void *gate, uint16_t *out, ngram_stream_t stream);
 
 /* Prefetch: stage the rows a coming batch will read, ahead of its lookup.  The pages
  * describe prefetching the n-gram vectors of upcoming tokens over PCIe while the GPU
@@ -217,7 +225,42 @@ NGRAM_API ngram_status ngram_prefetch(ngram_ctx *ctx, uint32_t slot, const int32
                                       const int32_t *history, uint32_t n_seq, uint32_t T,
                                       ngram_stream_t stream);
 NGRAM_API ngram_status ngram_forward_staged(ngram_ctx *ctx, uint32_t slot, const uint16_t *residual,
-                                            const float *gate, uint16_t *out, ngram_stream_t stream);
+                                            const void *gate, uint16_t *out, ngram_stream_t stream);
+
+/* Backward of out = residual + gate * sum_h E[idx_h(t)], given grad_out = dL/dout (device
+ * bf16 [N][d], 16-byte aligned).  The gradient with respect to residual is grad_out itself.
+ *
+ * ngram_backward_rows: the gradient with respect to the table, which only the rows the
+ * batch read have.  uniq_out (device uint32 [N*H]) receives the distinct rows in order of
+ * first occurrence (the list ngram_dedup_rows gives), count_out (device uint32 [1]) their
+ * number U, and grad_rows (device fp32 [N*H][d], 16-byte aligned; rows 0..U-1 written)
+ * row u's gradient: over the occurrences i = t * H + h of uniq_out[u] in ascending order,
+ *   shared gate:    grad = fp32(gate * S),  S = the fp32 sum of grad_out[t] in that order;
+ *   per-token gate: grad = the chain acc = fma(gate[t], grad_out[t], acc) in that order.
+ * A row read by several heads of one token counts once per head.  The order is fixed by a
+ * stable radix sort of the occurrences (no floating-point atomics), so the result is the
+ * same bit for bit on every run.  Scratch (about 20 bytes per max_tokens * H entry) is
+ * allocated by the first call.  The table itself is not read.
+ *
+ * ngram_backward_gate: the gradient with respect to the gate (recomputes the head sums
+ * e[t] exactly as ngram_forward does; HBM, HOST_UVA or HOST_AUTO residency, else
+ * NGRAM_EUNSUPPORTED):
+ *   shared gate:    grad_gate device fp32 [d] = fp32 of the sum over every token of
+ *                   grad_out[t] * e[t]: each product exact in fp64, summed in fp64 over
+ *                   fixed chunks of 16 tokens and then over the chunks in order (same
+ *                   result on every run and any GPU size); scratch N/16 * d fp64;
+ *   per-token gate: grad_gate device fp32 [N][d] = fp32(grad_out[t] * e[t]).
+ * Both are asynchronous on stream; N == 0: count_out set to 0 / grad_gate zeroed
+ * (shared) or untouched (per-token).  EINVAL as for ngram_forward. */
+NGRAM_API ngram_status ngram_backward_rows(ngram_ctx *ctx, const int32_t *tokens,
+                                           const int32_t *history, uint32_t n_seq, uint32_t T,
+                                           const uint16_t *grad_out, const void *gate,
+                                           uint32_t *uniq_out, uint32_t *count_out,
+                                           float *grad_rows, ngram_stream_t stream);
+NGRAM_API ngram_status ngram_backward_gate(ngram_ctx *ctx, const int32_t *tokens,
+                                           const int32_t *history, uint32_t n_seq, uint32_t T,
+                                           const uint16_t *grad_out, float *grad_gate,
+                                           ngram_stream_t stream);
 
 /* Bound, in milliseconds, of every host-side wait of the context (default 10,000).  A
  * wait that runs out returns NGRAM_ETIMEOUT; work already enqueued stays enqueued and
@@ -279,7 +322,8 @@ NGRAM_API ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, uin
  *   but its copies do not overlap.
  * Ordering: starts after the work already on `stream`; `stream` waits for the last
  * output chunk, so synchronising `stream` means out_h is complete.  Host buffers must
- * stay valid until then.  HBM or HOST_UVA residency without flags, else
+ * stay valid until then.  HBM or HOST_UVA residency without flags (BATCH_ORDER aside),
+ * else
  * NGRAM_EUNSUPPORTED.  The device copies of the inputs (max_tokens tokens, two chunks
  * of residual and output) are allocated by the first call. */
 NGRAM_API ngram_status ngram_forward_host(ngram_ctx *ctx, const int32_t *tokens_h,

@@ -72,6 +72,7 @@ _T = torch.zeros(64, dtype=torch.bfloat16)      # any 16-byte aligned host addre
     (dict(dtype=ng.NGRAM_FP8_E4M3_ROWSCALE, d=24), "d % 16"),
     (dict(dtype=ng.NGRAM_NVFP4, d=48), "d % 32"),
     (dict(dtype=ng.NGRAM_NVFP4, d=64), "global scale"),
+    (dict(hp=dict(flags=0x12)), "TOKEN_GATE"),
     (dict(d=264, max_tokens=2**31), "too large"),
 ])
 def test_init_rejects_bad_arguments_before_cuda(kw, msg):
@@ -136,6 +137,12 @@ def test_fill_rejects_bad_arguments():
         ng.ngram_fill_synthetic(_T, 10, 32, ng.NGRAM_NVFP4, stream=0)           # no global scale
     with pytest.raises(ng.NgramError):
         ng.ngram_fill_synthetic(_T, 10, 48, ng.NGRAM_NVFP4, row_scale=_T, stream=0)
+
+
+def test_backward_entry_points_reject_a_null_context():
+    lib = ng.lib()
+    assert lib.ngram_backward_rows(None, None, None, 1, 1, None, None, None, None, None, None) == ng.NGRAM_EINVAL
+    assert lib.ngram_backward_gate(None, None, None, 1, 1, None, None, None) == ng.NGRAM_EINVAL
 
 
 def test_null_context_is_rejected():
