@@ -683,6 +683,207 @@ def run_host(args):
     ht.close()
 
 
+def run_shard(args, w):
+    """Column-sharded table (--variant shard): rank r of P holds columns [r d/P, (r+1) d/P)
+    of every row; each step, every rank runs ngram_forward_shard on the whole batch, which
+    stores its columns into every rank's output buffer through CUDA IPC mappings (the
+    fused all-gather), between two one-element NCCL all-reduces that order the ranks.  The
+    whole job computes one N-token batch per step (strong scaling).  With one GPU the one
+    shard is the whole table and no collective runs."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_ngram_b200 as ng
+    from hashed_gram_embedding_ngram_b200 import shard
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    dtype = {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
+             "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[w.dtype]
+    col0, d = shard.shard_columns(w.d, world, rank, dtype)
+    table = torch.empty((w.R, ng.ngram_row_bytes(dtype, d)), dtype=torch.uint8, device=dev)
+    scale = None
+    if dtype != ng.NGRAM_BF16:
+        scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
+    ng.ngram_fill_synthetic_cols(table, w.R, d, col0, dtype, gen.TABLE_SEED, row_scale=scale)
+    ctx = ng.ngram_init(table, w.R, d, dtype, ng.NGRAM_RES_HBM,
+                        ng.ngram_default_hash_params(vocab_size=w.vocab), w.N, row_scale=scale)
+    toks = [torch.from_numpy(gen.tokens_for(w, gen.TOKEN_SEED + b)).to(dev) for b in range(args.batches)]
+    hists = [None if not w.history else torch.from_numpy(gen.history_for(w, gen.HISTORY_SEED + b)).to(dev)
+             for b in range(args.batches)]
+    res_cpu = torch.from_numpy(gen.residual_bf16_bits(w.N, w.d).view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
+    residual = res_cpu.to(dev)
+    gate = torch.from_numpy(gen.gate_f32(w.d)).to(dev)
+    if world > 1:
+        peers = shard.PeerOutputs(w.N, w.d, device=dev)
+        outs = peers.ptrs
+        out = peers.out
+    else:
+        peers = None
+        out = torch.empty_like(residual)
+        outs = [out]
+    stream = torch.cuda.current_stream()
+
+    def order():
+        if world > 1:
+            shard.complete()
+
+    def step(i):
+        b = i % args.batches
+        order()
+        ng.ngram_forward_shard(ctx, toks[b], residual, gate, outs, w.d, col0, history=hists[b],
+                               stream=stream)
+        order()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id_for(dev)) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(K):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+    # end to end: tokens and residual from pinned host memory, the output back
+    tok_h = [t.cpu().pin_memory() for t in toks]
+    res_h, out_h = res_cpu.pin_memory(), torch.empty_like(res_cpu).pin_memory()
+    E = max(1, args.e2e_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(E):
+        b = i % args.batches
+        toks[b].copy_(tok_h[b], non_blocking=True)
+        residual.copy_(res_h, non_blocking=True)
+        step(i)
+        out_h.copy_(out[:w.N], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+    if rank == 0:
+        grouped = w.N >= ng.NGRAM_SORT_MIN_TOKENS
+        line = {
+            "metric": METRIC, "value": w.N * K / (elapsed_ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": dict(config_for(w, args), parallelism="column shard x%d, fused all-gather over "
+                                                            "peer memory" % world, shard_columns=d),
+            "e2e": {"value": w.N * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": w.N * 4 + w.N * w.d * 2,
+                    "d2h_bytes_per_step": w.N * w.d * 2, "steps": E},
+            "clocks": clk.summary(),
+            "gpu_launches": K * (4 if grouped else 1),
+        }
+        print(json.dumps(line), flush=True)
+    if peers is not None:
+        dist.barrier()
+        peers.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_backward(args, w):
+    """The backward pass of the lookup, timed like the forward: one step = the table
+    gradient (ngram_backward_rows) + the shared-gate gradient (ngram_backward_gate) of one
+    batch, on one GPU.  CUDA events around each call give the per-kernel-group times."""
+    import torch
+
+    import hashed_gram_embedding_ngram_b200 as ng
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    dtype = {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
+             "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[w.dtype]
+    table = torch.empty((w.R, ng.ngram_row_bytes(dtype, w.d)), dtype=torch.uint8, device=dev)
+    scale = None
+    if dtype != ng.NGRAM_BF16:
+        scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
+    ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
+    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM,
+                        ng.ngram_default_hash_params(vocab_size=w.vocab), w.N, row_scale=scale)
+    N, d, H = w.N, w.d, HEADS
+    toks = [torch.from_numpy(gen.tokens_for(w, gen.TOKEN_SEED + b)).to(dev) for b in range(args.batches)]
+    hists = [None if not w.history else torch.from_numpy(gen.history_for(w, gen.HISTORY_SEED + b)).to(dev)
+             for b in range(args.batches)]
+    rng = np.random.default_rng(11)
+    dy = torch.from_numpy(rng.standard_normal((N, d), dtype=np.float32)).to(torch.bfloat16).to(dev)
+    gate = torch.from_numpy(gen.gate_f32(d)).to(dev)
+    uniq = torch.empty(N * H, dtype=torch.int32, device=dev)
+    count = torch.empty(1, dtype=torch.int32, device=dev)
+    grad_rows = torch.empty((N * H, d), dtype=torch.float32, device=dev)
+    grad_gate = torch.empty(d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def rows(i):
+        b = i % args.batches
+        ng.ngram_backward_rows(ctx, toks[b], dy, gate, history=hists[b], uniq_out=uniq,
+                               count_out=count, grad_rows=grad_rows, stream=stream)
+
+    def gate_grad(i):
+        b = i % args.batches
+        ng.ngram_backward_gate(ctx, toks[b], dy, history=hists[b], out=grad_gate, stream=stream)
+
+    for i in range(args.warmup):
+        rows(i)
+        gate_grad(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    Us = []
+    with ClockSampler(gpu_id_for(dev)) as clk:
+        torch.cuda.synchronize()
+        for i in range(K):
+            ev[i][0].record(stream)
+            rows(i)
+            ev[i][1].record(stream)
+            gate_grad(i)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    for b in range(args.batches):          # distinct rows of each batch (outside the timing)
+        rows(b)
+        Us.append(int(count.item()))
+    rows_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
+    gate_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
+    step_ms = statistics.fmean(e[0].elapsed_time(e[2]) for e in ev)
+    U = statistics.fmean(Us)
+    peaks = measured_peaks()
+    # algorithmic bytes: table gradient = dy read once + one fp32 row per distinct row
+    # written; gate gradient = the forward's row reads + dy read (+ fp64 partials)
+    rows_bytes = N * 2 * d + U * 4 * d + 4 * d
+    gate_bytes = N * (HEADS * row_bytes(w) + 2 * d + 4) + 2 * 8 * d * ((N + 15) // 16) + 4 * d
+    line = {
+        "metric": "n-gram embed backward tokens/s (table + gate gradients), 1 B200",
+        "value": N / (step_ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(config_for(w, args), mode="backward", distinct_rows_per_batch=U),
+        "backward_rows": {"ms": rows_ms, "algorithmic_bytes": rows_bytes,
+                          "achieved_gbs": rows_bytes / rows_ms / 1e6,
+                          "frac": rows_bytes / rows_ms / 1e6 / peaks["hbm_gbs"],
+                          "kernels": "hash, dedup (5), radix sort (%d passes x 5), segments, k_rows_grad"
+                                     % ((max(1, (N * H - 1).bit_length()) + 7) // 8)},
+        "backward_gate": {"ms": gate_ms, "algorithmic_bytes": gate_bytes,
+                          "achieved_gbs": gate_bytes / gate_ms / 1e6,
+                          "frac": gate_bytes / gate_ms / 1e6 / peaks["hbm_gbs"],
+                          "kernels": "k_gate_grad + k_gate_reduce"},
+        "peak": {"hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"]},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -698,13 +899,16 @@ def main():
     ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
                     help="eager launches, or 100-step CUDA graphs (auto: graph for N <= 1024)")
     ap.add_argument("--variant", default="default",
-                    choices=["default", "dedup", "tma", "sort", "batch_order"],
+                    choices=["default", "dedup", "tma", "sort", "batch_order", "shard"],
                     help="HBM path: library default (grouped order from 16,384 tokens), dedup + "
-                         "staged gather, TMA staging, always grouped, always batch order")
+                         "staged gather, TMA staging, always grouped, always batch order; shard: "
+                         "the table split by columns over the ranks (strong scaling)")
     ap.add_argument("--host-workloads", default="host_decode_1,host_decode_16,host_decode_64,"
                                                 "host_decode_256,host_prefill")
     ap.add_argument("--host-steps", type=int, default=200)
     ap.add_argument("--host-rows", type=int, default=0, help="override R for the host table")
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward"],
+                    help="forward: the lookup (the benchmark); backward: table + gate gradients")
     args = ap.parse_args()
     w = gen.WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
@@ -714,6 +918,13 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w)
+        return
+    if args.mode == "backward":
+        if rank == 0:
+            run_backward(args, w)
+        return
+    if args.variant == "shard":
+        run_shard(args, w)
         return
     run_ours(args, w)
 

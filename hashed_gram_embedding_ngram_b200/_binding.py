@@ -104,6 +104,20 @@ _lib.ngram_backward_rows.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P, _P, _P,
 _lib.ngram_backward_rows.restype = _i32
 _lib.ngram_backward_gate.argtypes = [_P, _P, _P, _u32, _u32, _P, _P, _P]
 _lib.ngram_backward_gate.restype = _i32
+_lib.ngram_fill_synthetic_cols.argtypes = [_P, _P, _u64, _u32, _u32, _i32, _u64, _P]
+_lib.ngram_fill_synthetic_cols.restype = _i32
+_lib.ngram_forward_shard.argtypes = [_P, _P, _P, _u32, _u32, _u32, _u32, _P, _P, _P, _u32, _P]
+_lib.ngram_forward_shard.restype = _i32
+_lib.ngram_device_alloc.argtypes = [ctypes.POINTER(_P), _u64]
+_lib.ngram_device_alloc.restype = _i32
+_lib.ngram_device_free.argtypes = [_P]
+_lib.ngram_device_free.restype = _i32
+_lib.ngram_ipc_get_handle.argtypes = [_P, ctypes.c_char_p]
+_lib.ngram_ipc_get_handle.restype = _i32
+_lib.ngram_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(_P)]
+_lib.ngram_ipc_open.restype = _i32
+_lib.ngram_ipc_close.argtypes = [_P]
+_lib.ngram_ipc_close.restype = _i32
 
 
 def lib() -> ctypes.CDLL:
@@ -454,3 +468,80 @@ def ngram_backward_gate(ctx: Context, tokens: torch.Tensor, grad_out: torch.Tens
     _check(_lib.ngram_backward_gate(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T,
                                     _ptr(grad_out), _ptr(out), _stream(stream)))
     return out
+
+
+def ngram_fill_synthetic_cols(table: torch.Tensor, R: int, d: int, col0: int, dtype: int = NGRAM_BF16,
+                              seed: int = 0, row_scale: torch.Tensor | None = None, stream=None) -> None:
+    """Columns [col0, col0 + d) of the synthetic table (a column shard)."""
+    _check(_lib.ngram_fill_synthetic_cols(_ptr(table), _ptr(row_scale), R, d, col0, dtype,
+                                          seed & (2**64 - 1), _stream(stream)))
+
+
+def _addr(x) -> int:
+    return x.data_ptr() if isinstance(x, torch.Tensor) else int(x)
+
+
+def ngram_forward_shard(ctx: Context, tokens: torch.Tensor, residual: torch.Tensor, gate: torch.Tensor,
+                        outs, d_full: int, col0: int, history: torch.Tensor | None = None,
+                        stream=None) -> None:
+    """This rank's columns [col0, col0 + ctx.d) of the lookup, stored into every buffer of
+    `outs` (tensors or device addresses of bf16 [N][d_full]: this rank's output and the
+    peers' mapped ones).  residual bf16 [N][d_full]; gate fp32 [d_full] (or bf16
+    [N][d_full] with NGRAM_FLAG_TOKEN_GATE)."""
+    _need(tokens, "tokens", torch.int32, ndim=2)
+    dev = tokens.device
+    n_seq, T = tokens.shape
+    N = n_seq * T
+    _need(residual, "residual", torch.bfloat16, dev)
+    if residual.numel() != N * d_full:
+        raise ValueError("residual must hold N * d_full elements")
+    if _token_gate(ctx):
+        _need(gate, "gate", torch.bfloat16, dev)
+        if gate.numel() != N * d_full:
+            raise ValueError("a per-token gate must hold N * d_full elements")
+    else:
+        _need(gate, "gate", torch.float32, dev)
+        if gate.numel() != d_full:
+            raise ValueError("gate must hold d_full elements")
+    if history is not None:
+        _need(history, "history", torch.int32, dev, ndim=2)
+    ptrs = (_P * 8)()
+    outs = list(outs)
+    if not 1 <= len(outs) <= 8:
+        raise ValueError("1 to 8 output buffers")
+    for i, o in enumerate(outs):
+        if isinstance(o, torch.Tensor):
+            _need(o, "outs[%d]" % i, torch.bfloat16)
+            if o.numel() < N * d_full:
+                raise ValueError("outs[%d] must hold N * d_full elements" % i)
+        ptrs[i] = _addr(o)
+    _check(_lib.ngram_forward_shard(ctx.handle, _ptr(tokens), _ptr(history), n_seq, T, d_full, col0,
+                                    _ptr(residual), _ptr(gate), ptrs, len(outs), _stream(stream)))
+
+
+def ngram_device_alloc(nbytes: int) -> int:
+    p = _P()
+    _check(_lib.ngram_device_alloc(ctypes.byref(p), nbytes))
+    return p.value
+
+
+def ngram_device_free(ptr: int) -> None:
+    _check(_lib.ngram_device_free(ptr))
+
+
+def ngram_ipc_get_handle(ptr: int) -> bytes:
+    buf = ctypes.create_string_buffer(64)
+    _check(_lib.ngram_ipc_get_handle(ptr, buf))
+    return buf.raw
+
+
+def ngram_ipc_open(handle: bytes) -> int:
+    if len(handle) != 64:
+        raise ValueError("an IPC handle is 64 bytes")
+    p = _P()
+    _check(_lib.ngram_ipc_open(handle, ctypes.byref(p)))
+    return p.value
+
+
+def ngram_ipc_close(ptr: int) -> None:
+    _check(_lib.ngram_ipc_close(ptr))

@@ -29,10 +29,14 @@ __device__ __forceinline__ int32_t synth_int8_value(uint32_t w) {
     return (sum - 510) >> 2;
 }
 
+// Every fill writes columns col0 .. col0 + d - 1 of the synthetic table (col0 = 0: the
+// whole table; else a column shard of a wider one), the values of those columns being the
+// same whatever the table's full width.
+//
 // One CTA per row (grid-stride over rows); each thread writes 8 columns (16 bytes)
 // per step, from four Philox calls with counters (col/2, row, 1, 0).
 __global__ void __launch_bounds__(256) k_fill_bf16(uint16_t *__restrict__ table, uint64_t R,
-                                                   uint32_t d, uint32_t k0, uint32_t k1) {
+                                                   uint32_t d, uint32_t col0, uint32_t k0, uint32_t k1) {
     const uint32_t nvec = d >> 3;
     for (uint64_t row = blockIdx.x; row < R; row += gridDim.x) {
         uint4 *dst = reinterpret_cast<uint4 *>(table + row * d);
@@ -41,7 +45,7 @@ __global__ void __launch_bounds__(256) k_fill_bf16(uint16_t *__restrict__ table,
 #pragma unroll
             for (int p = 0; p < 4; ++p) {                // column pair 4v+p: cols 8v+2p, +1
                 const uint4 x = philox4x32_10(
-                    make_uint4(4u * v + p, static_cast<uint32_t>(row), 1u, 0u), k0, k1);
+                    make_uint4((col0 >> 1) + 4u * v + p, static_cast<uint32_t>(row), 1u, 0u), k0, k1);
                 words[p] = pack_bf16x2(synth_bf16_value(x.x, x.y), synth_bf16_value(x.z, x.w));
             }
             dst[v] = make_uint4(words[0], words[1], words[2], words[3]);
@@ -54,7 +58,7 @@ __global__ void __launch_bounds__(256) k_fill_bf16(uint16_t *__restrict__ table,
 // (0, row, 3, 0)).
 __global__ void __launch_bounds__(256) k_fill_int8(int8_t *__restrict__ table,
                                                    float *__restrict__ row_scale, uint64_t R,
-                                                   uint32_t d, uint32_t k0, uint32_t k1) {
+                                                   uint32_t d, uint32_t col0, uint32_t k0, uint32_t k1) {
     const uint32_t nvec = d >> 4;
     for (uint64_t row = blockIdx.x; row < R; row += gridDim.x) {
         uint4 *dst = reinterpret_cast<uint4 *>(table + row * d);
@@ -63,7 +67,7 @@ __global__ void __launch_bounds__(256) k_fill_int8(int8_t *__restrict__ table,
 #pragma unroll
             for (int p = 0; p < 4; ++p) {                // columns 16v+4p .. 16v+4p+3
                 const uint4 x = philox4x32_10(
-                    make_uint4(4u * v + p, static_cast<uint32_t>(row), 2u, 0u), k0, k1);
+                    make_uint4((col0 >> 2) + 4u * v + p, static_cast<uint32_t>(row), 2u, 0u), k0, k1);
                 const uint32_t q0 = synth_int8_value(x.x) & 0xFFu;
                 const uint32_t q1 = synth_int8_value(x.y) & 0xFFu;
                 const uint32_t q2 = synth_int8_value(x.z) & 0xFFu;
@@ -99,7 +103,7 @@ __device__ __forceinline__ uint32_t synth_fp4_block_scale(uint32_t w) {
 // row scale from counter (0, row, 5, 0).
 __global__ void __launch_bounds__(256) k_fill_fp8(uint8_t *__restrict__ table,
                                                   float *__restrict__ row_scale, uint64_t R,
-                                                  uint32_t d, uint32_t k0, uint32_t k1) {
+                                                  uint32_t d, uint32_t col0, uint32_t k0, uint32_t k1) {
     const uint32_t nvec = d >> 4;
     for (uint64_t row = blockIdx.x; row < R; row += gridDim.x) {
         uint4 *dst = reinterpret_cast<uint4 *>(table + row * d);
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(256) k_fill_fp8(uint8_t *__restrict__ table,
 #pragma unroll
             for (int p = 0; p < 4; ++p) {                // columns 16v+4p .. 16v+4p+3
                 const uint4 x = philox4x32_10(
-                    make_uint4(4u * v + p, static_cast<uint32_t>(row), 4u, 0u), k0, k1);
+                    make_uint4((col0 >> 2) + 4u * v + p, static_cast<uint32_t>(row), 4u, 0u), k0, k1);
                 words[p] = synth_e4m3(x.x) | (synth_e4m3(x.y) << 8) | (synth_e4m3(x.z) << 16) |
                            (synth_e4m3(x.w) << 24);
             }
@@ -126,10 +130,12 @@ __global__ void __launch_bounds__(256) k_fill_fp8(uint8_t *__restrict__ table,
 // nibble of byte j), then one E4M3 scale byte per 16 columns, zero-padded to 16 bytes.
 // Codes of columns 32k .. 32k+31 are the 16 bytes of Philox (k, row, 6, 0) in order (nibble
 // c%8 of word (c/8)%4 is column c); the scale of block b comes from word b%4 of Philox
-// (b/4, row, 7, 0).  The global scale is written to gscale[0] by the first CTA.
+// (b/4, row, 7, 0).  The global scale is written to gscale[0] by the first CTA.  With a
+// column offset col0 (a multiple of 32), code vector v is counter col0/32 + v and local
+// block b is global block col0/16 + b.
 __global__ void __launch_bounds__(256) k_fill_fp4(uint8_t *__restrict__ table,
                                                   float *__restrict__ gscale, uint64_t R,
-                                                  uint32_t d, uint32_t k0, uint32_t k1) {
+                                                  uint32_t d, uint32_t col0, uint32_t k0, uint32_t k1) {
     const uint32_t n_blocks = d >> 4;
     const uint32_t code_vec = d >> 5;
     const uint32_t scale_vec = (n_blocks + 15u) >> 4;
@@ -139,22 +145,27 @@ __global__ void __launch_bounds__(256) k_fill_fp4(uint8_t *__restrict__ table,
         uint4 *dst = reinterpret_cast<uint4 *>(table + row * rb);
         for (uint32_t v = threadIdx.x; v < code_vec + scale_vec; v += blockDim.x) {
             if (v < code_vec) {
-                dst[v] = philox4x32_10(make_uint4(v, static_cast<uint32_t>(row), 6u, 0u), k0, k1);
+                dst[v] = philox4x32_10(make_uint4((col0 >> 5) + v, static_cast<uint32_t>(row), 6u, 0u),
+                                       k0, k1);
                 continue;
             }
-            const uint32_t sv = v - code_vec;            // blocks 16sv .. 16sv+15
-            uint32_t words[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {                // blocks 16sv+4p .. 16sv+4p+3
-                const uint32_t b0 = 16u * sv + 4u * p;
-                const uint4 x = philox4x32_10(
-                    make_uint4(b0 >> 2, static_cast<uint32_t>(row), 7u, 0u), k0, k1);
-                const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-                uint32_t w = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (b0 + j < n_blocks) w |= synth_fp4_block_scale(xs[j]) << (8 * j);
-                words[p] = w;
+            const uint32_t sv = v - code_vec;            // local blocks 16sv .. 16sv+15
+            uint32_t words[4] = {0u, 0u, 0u, 0u};
+            uint32_t ctr = 0xFFFFFFFFu;
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            for (uint32_t j = 0; j < 16u && 16u * sv + j < n_blocks; ++j) {
+                const uint32_t B = (col0 >> 4) + 16u * sv + j;   // global block
+                if ((B >> 2) != ctr) {
+                    ctr = B >> 2;
+                    x = philox4x32_10(make_uint4(ctr, static_cast<uint32_t>(row), 7u, 0u), k0, k1);
+                }
+                const uint32_t k = B & 3u;
+                const uint32_t w = k == 0u ? x.x : k == 1u ? x.y : k == 2u ? x.z : x.w;
+                const uint32_t byte = synth_fp4_block_scale(w) << (8u * (j & 3u));
+                if (j < 4u) words[0] |= byte;
+                else if (j < 8u) words[1] |= byte;
+                else if (j < 12u) words[2] |= byte;
+                else words[3] |= byte;
             }
             dst[v] = make_uint4(words[0], words[1], words[2], words[3]);
         }

@@ -45,6 +45,12 @@ struct GatherArgs {
     uint32_t n_strips;          // strips of 32 column vectors per token
     uint32_t strips_per_item;
     uint32_t groups_per_token;  // ceil(n_strips / strips_per_item)
+    // column-sharded table (k_gather_c8<.., kShard = true> only): residual, gate_tok and
+    // every outs[p] are rows of ld elements, already offset to this shard's first column;
+    // the shard's columns of each token are stored to all n_outs buffers
+    uint32_t ld;
+    uint32_t n_outs;
+    uint16_t *outs[8];
 };
 
 // 16-byte load through L2 without L1 allocation; coherent (the residual may be the

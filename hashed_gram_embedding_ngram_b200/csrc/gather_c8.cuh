@@ -7,6 +7,14 @@
 // 8- and 4-bit formats hold, so a CTA needs fewer registers and more CTAs fit on an SM;
 // which of the two layouts is faster for a format is a measured choice (the build switch
 // NGRAM_C8_FORMATS, bit t for ngram_dtype t).
+//
+// kShard: the table holds a column shard (columns col0 .. col0 + d - 1 of a wider table, as
+// the per-rank shards of the SGLang TP4 setup on "Qwen Brought Back N-Grams. All 51 Billion
+// Parameters of Them.", section "Which is why the offload matters more than the parameter
+// count").  The residual and the outputs are full rows of g.ld elements; the kernel
+// computes the shard's columns and stores them into every buffer of g.outs -- this GPU's
+// output and, through peer mappings, the other ranks' -- so the gather and the all-gather
+// of the output are one kernel.
 #pragma once
 
 #include "rows.cuh"
@@ -17,7 +25,7 @@ namespace ngram {
 #define NGRAM_C8_MIN_BLOCKS 3
 #endif
 
-template <int kH, class Rows, bool kTokGate>
+template <int kH, class Rows, bool kTokGate, bool kShard = false>
 __global__ void __launch_bounds__(256, NGRAM_C8_MIN_BLOCKS) k_gather_c8(const GatherArgs g,
                                                                         uint32_t row_bytes) {
     const uint32_t lane = threadIdx.x & 31u;
@@ -40,7 +48,7 @@ __global__ void __launch_bounds__(256, NGRAM_C8_MIN_BLOCKS) k_gather_c8(const Ga
         for (int h = 0; h < 16; ++h) rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);
         const uint32_t s_begin = grp * g.strips_per_item;
         const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
-        const size_t tok_off = static_cast<size_t>(tok) * g.d;
+        const size_t tok_off = static_cast<size_t>(tok) * (kShard ? g.ld : g.d);
         for (uint32_t s = s_begin; s < s_end; ++s) {
             const uint32_t v = s * 32u + lane;
             const bool active = v < nvec;
@@ -74,7 +82,13 @@ __global__ void __launch_bounds__(256, NGRAM_C8_MIN_BLOCKS) k_gather_c8(const Ga
                 const float y1 = __fadd_rn(bf16_hi(rw[p]), __fmul_rn(gv[2 * p + 1], acc[p].y));
                 o[p] = pack_bf16x2(y0, y1);
             }
-            *reinterpret_cast<uint4 *>(g.out + tok_off + v * 8u) = make_uint4(o[0], o[1], o[2], o[3]);
+            const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+            if (kShard) {
+                for (uint32_t p = 0; p < g.n_outs; ++p)
+                    *reinterpret_cast<uint4 *>(g.outs[p] + tok_off + v * 8u) = ov;
+            } else {
+                *reinterpret_cast<uint4 *>(g.out + tok_off + v * 8u) = ov;
+            }
         }
     }
 }

@@ -399,6 +399,9 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.n_strips = (c->d / cols_per_lane + 31) / 32;
     g.strips_per_item = g.n_strips;
     g.groups_per_token = 1;
+    g.ld = c->d;
+    g.n_outs = 0;
+    for (uint16_t *&o : g.outs) o = nullptr;
     return g;
 }
 
@@ -439,6 +442,22 @@ template <class Rows, bool kTok>
 void launch_c8(const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
     if (g.h.n_heads == 16) k_gather_c8<16, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
     else k_gather_c8<0, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
+}
+
+template <class Rows, bool kTok>
+void launch_c8_shard(const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
+    if (g.h.n_heads == 16) k_gather_c8<16, Rows, kTok, true><<<nb, 256, 0, s>>>(g, rb);
+    else k_gather_c8<0, Rows, kTok, true><<<nb, 256, 0, s>>>(g, rb);
+}
+
+template <bool kTok>
+void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
+    switch (t) {
+        case NGRAM_BF16: launch_c8_shard<RowsBf16, kTok>(g, nb, s, rb); break;
+        case NGRAM_INT8_ROWSCALE: launch_c8_shard<Rows8bit<Int8Codes>, kTok>(g, nb, s, rb); break;
+        case NGRAM_FP8_E4M3_ROWSCALE: launch_c8_shard<Rows8bit<E4m3Codes>, kTok>(g, nb, s, rb); break;
+        case NGRAM_NVFP4: launch_c8_shard<RowsNvfp4, kTok>(g, nb, s, rb); break;
+    }
 }
 
 template <bool kTok>
@@ -623,7 +642,8 @@ bool grouped_order(const ngram_ctx *c, uint32_t N) {
 // Grouped order: tokens grouped by bigram context (counting sort on a 13-bit hash),
 // then the fused gather walks them in that order.  Same outputs; repeated rows run back
 // to back so L2 serves the repeats.
-ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
+// Grouped order of a batch's tokens into c->so_perm (3 kernels and a memset).
+ngram_status order_tokens(ngram_ctx *c, const Call &k) {
     if (!c->so_perm) {
         NG_CUDA(cudaMalloc(&c->so_bucket, c->max_tokens * 4ull), "order scratch");
         NG_CUDA(cudaMalloc(&c->so_hist, kOrderBuckets * 4ull), "order scratch");
@@ -636,6 +656,11 @@ ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
     k_order_scan<<<1, 1024, 0, k.s>>>(c->so_hist);
     k_order_scatter<<<gn, 256, 0, k.s>>>(c->so_bucket, k.N, c->so_hist, c->so_perm);
     NG_CUDA(cudaGetLastError(), "order launch");
+    return NGRAM_OK;
+}
+
+ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
+    NG_CHECK(order_tokens(c, k));
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     g.perm = c->so_perm;
     return launch_gather(c, g, k.s, max_blocks);
@@ -1035,10 +1060,17 @@ ngram_status ngram_dedup_rows(ngram_ctx *c, const int32_t *tokens, const int32_t
 
 ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
                                   ngram_dtype dtype, uint64_t seed, ngram_stream_t stream) {
+    return ngram_fill_synthetic_cols(table, row_scale, R, d, 0, dtype, seed, stream);
+}
+
+ngram_status ngram_fill_synthetic_cols(void *table, float *row_scale, uint64_t R, uint32_t d,
+                                       uint32_t col0, ngram_dtype dtype, uint64_t seed,
+                                       ngram_stream_t stream) {
     if (table == nullptr) return fail(NGRAM_EINVAL, "table is NULL");
     if (!aligned16(table)) return fail(NGRAM_EINVAL, "table must be 16-byte aligned");
     if (R == 0 || R > 0xFFFFFFFFull) return fail(NGRAM_EINVAL, "R must be in [1, 2^32 - 1]");
     NG_CHECK(check_format(dtype, d, row_scale));
+    NG_CHECK(check_format(dtype, col0 + d, row_scale));     // col0: a multiple of the d rule
     int dev = 0, sms = 0;
     NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
     NG_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute");
@@ -1065,12 +1097,105 @@ ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uin
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned nb = static_cast<unsigned>(blocks);
     switch (dtype) {
-        case NGRAM_BF16: k_fill_bf16<<<nb, 256, 0, s>>>(static_cast<uint16_t *>(dst), R, d, k0, k1); break;
-        case NGRAM_INT8_ROWSCALE: k_fill_int8<<<nb, 256, 0, s>>>(static_cast<int8_t *>(dst), dst_scale, R, d, k0, k1); break;
-        case NGRAM_FP8_E4M3_ROWSCALE: k_fill_fp8<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, k0, k1); break;
-        case NGRAM_NVFP4: k_fill_fp4<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, k0, k1); break;
+        case NGRAM_BF16: k_fill_bf16<<<nb, 256, 0, s>>>(static_cast<uint16_t *>(dst), R, d, col0, k0, k1); break;
+        case NGRAM_INT8_ROWSCALE: k_fill_int8<<<nb, 256, 0, s>>>(static_cast<int8_t *>(dst), dst_scale, R, d, col0, k0, k1); break;
+        case NGRAM_FP8_E4M3_ROWSCALE: k_fill_fp8<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, col0, k0, k1); break;
+        case NGRAM_NVFP4: k_fill_fp4<<<nb, 256, 0, s>>>(static_cast<uint8_t *>(dst), dst_scale, R, d, col0, k0, k1); break;
     }
     NG_CUDA(cudaGetLastError(), "k_fill launch");
+    return NGRAM_OK;
+}
+
+// ---------------------------------------------------------------- column-sharded table
+ngram_status ngram_forward_shard(ngram_ctx *c, const int32_t *tokens, const int32_t *history,
+                                 uint32_t n_seq, uint32_t T, uint32_t d_full, uint32_t col0,
+                                 const uint16_t *residual, const void *gate, uint16_t *const *outs,
+                                 uint32_t n_outs, ngram_stream_t stream) {
+    uint64_t N = 0;
+    NG_CHECK(check_batch(c, tokens, n_seq, T, &N));
+    if (c->where != NGRAM_RES_HBM)
+        return fail(NGRAM_EUNSUPPORTED, "ngram_forward_shard: HBM residency only");
+    if (c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING))
+        return fail(NGRAM_EUNSUPPORTED, "ngram_forward_shard: no DEDUP or TMA_STAGING");
+    if (static_cast<uint64_t>(col0) + c->d > d_full)
+        return fail(NGRAM_EINVAL, "shard columns [%u, %u) exceed d_full %u", col0, col0 + c->d, d_full);
+    if (col0 % 8 != 0 || d_full % 8 != 0)
+        return fail(NGRAM_EINVAL, "col0 and d_full must be multiples of 8");
+    if (n_outs == 0 || n_outs > 8 || outs == nullptr)
+        return fail(NGRAM_EINVAL, "n_outs must be in [1, 8] with outs non-NULL");
+    if (N == 0) return NGRAM_OK;
+    if (residual == nullptr || gate == nullptr) return fail(NGRAM_EINVAL, "residual and gate must be non-NULL");
+    if (!aligned16(residual) || !aligned16(gate)) return fail(NGRAM_EINVAL, "residual and gate must be 16-byte aligned");
+    for (uint32_t p = 0; p < n_outs; ++p)
+        if (outs[p] == nullptr || !aligned16(outs[p])) return fail(NGRAM_EINVAL, "outs[%u] NULL or misaligned", p);
+    const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
+    const Call k{tokens, history, T, static_cast<uint32_t>(N), residual, gate, nullptr,
+                 reinterpret_cast<cudaStream_t>(stream)};
+    GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, residual + col0,
+                               tok_gate ? static_cast<const void *>(static_cast<const uint16_t *>(gate) + col0)
+                                        : static_cast<const void *>(static_cast<const float *>(gate) + col0),
+                               nullptr);
+    // 8 columns per lane for every format
+    g.n_strips = (c->d / 8 + 31) / 32;
+    g.strips_per_item = 1;
+    g.groups_per_token = g.n_strips;
+    g.ld = d_full;
+    g.n_outs = n_outs;
+    for (uint32_t p = 0; p < n_outs; ++p) g.outs[p] = outs[p] + col0;
+    if (grouped_order(c, k.N)) {
+        NG_CHECK(order_tokens(c, k));
+        g.perm = c->so_perm;
+    }
+    const uint64_t items = static_cast<uint64_t>(g.N) * g.groups_per_token;
+    uint64_t blocks = (items + 7) / 8;
+    const uint64_t cap = static_cast<uint64_t>(c->num_sms) * NGRAM_C8_MIN_BLOCKS;
+    if (blocks > cap) blocks = cap;
+    const unsigned nb = static_cast<unsigned>(blocks);
+    if (tok_gate) launch_shard<true>(c->dtype, g, nb, k.s, c->row_bytes);
+    else launch_shard<false>(c->dtype, g, nb, k.s, c->row_bytes);
+    NG_CUDA(cudaGetLastError(), "k_gather_c8 (shard) launch");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_device_alloc(void **out, uint64_t bytes) {
+    if (out == nullptr) return fail(NGRAM_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (bytes == 0) return fail(NGRAM_EINVAL, "bytes must be > 0");
+    const cudaError_t e = cudaMalloc(out, bytes);
+    if (e != cudaSuccess) {
+        *out = nullptr;
+        return cuda_fail(e, "cudaMalloc");
+    }
+    return NGRAM_OK;
+}
+
+ngram_status ngram_device_free(void *p) {
+    if (p == nullptr) return NGRAM_OK;
+    NG_CUDA(cudaFree(p), "cudaFree");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_ipc_get_handle(const void *dev_ptr, uint8_t handle[64]) {
+    if (dev_ptr == nullptr || handle == nullptr) return fail(NGRAM_EINVAL, "dev_ptr and handle must be non-NULL");
+    cudaIpcMemHandle_t h;
+    NG_CUDA(cudaIpcGetMemHandle(&h, const_cast<void *>(dev_ptr)), "cudaIpcGetMemHandle");
+    static_assert(sizeof(h) == 64, "cudaIpcMemHandle_t is 64 bytes");
+    memcpy(handle, &h, 64);
+    return NGRAM_OK;
+}
+
+ngram_status ngram_ipc_open(const uint8_t handle[64], void **dev_ptr) {
+    if (dev_ptr == nullptr || handle == nullptr) return fail(NGRAM_EINVAL, "dev_ptr and handle must be non-NULL");
+    *dev_ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, 64);
+    NG_CUDA(cudaIpcOpenMemHandle(dev_ptr, h, cudaIpcMemLazyEnablePeerAccess), "cudaIpcOpenMemHandle");
+    return NGRAM_OK;
+}
+
+ngram_status ngram_ipc_close(void *dev_ptr) {
+    if (dev_ptr == nullptr) return fail(NGRAM_EINVAL, "dev_ptr is NULL");
+    NG_CUDA(cudaIpcCloseMemHandle(dev_ptr), "cudaIpcCloseMemHandle");
     return NGRAM_OK;
 }
 

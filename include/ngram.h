@@ -360,6 +360,47 @@ NGRAM_API ngram_status ngram_hash_indices(ngram_ctx *ctx, const int32_t *tokens,
 NGRAM_API ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
                                   ngram_dtype dtype, uint64_t seed, ngram_stream_t stream);
 
+/* ngram_fill_synthetic for columns [col0, col0 + d) of the synthetic table: a column shard
+ * (the values of a column do not depend on the table's full width).  col0 must be a
+ * multiple of the format's d rule (8 bf16, 16 int8 / fp8, 32 nvfp4); the shard's rows use
+ * the format's layout for width d; int8 / fp8 row scales are the full table's. */
+NGRAM_API ngram_status ngram_fill_synthetic_cols(void *table, float *row_scale, uint64_t R,
+                                                 uint32_t d, uint32_t col0, ngram_dtype dtype,
+                                                 uint64_t seed, ngram_stream_t stream);
+
+/* Column-sharded table.  The pages' serving stack keeps "each rank's shard" of the table per
+ * GPU at TP4 ("Qwen Brought Back N-Grams. All 51 Billion Parameters of Them.", section
+ * "Which is why the offload matters more than the parameter count"; the shard axis is not
+ * given).  Here rank r of P holds columns [col0, col0 + d) of every row (a context made over
+ * its [R][d] shard, e.g. filled with ngram_fill_synthetic_cols), and every rank holds the
+ * full-width residual (tensor-parallel activations).  ngram_forward_shard computes the
+ * shard's columns of out = residual + gate * sum_h E[idx_h] for all N tokens and stores them
+ * into each of the n_outs output buffers -- this rank's and, through peer mappings
+ * (ngram_ipc_open), the other ranks' -- so the lookup and the all-gather of its output are
+ * one kernel over NVLink.
+ *   residual  device bf16 [N][d_full]; gate fp32 [d_full] (or bf16 [N][d_full] with
+ *             NGRAM_FLAG_TOKEN_GATE); outs[p] device-accessible bf16 [N][d_full];
+ *   d_full, col0 multiples of 8; col0 + d <= d_full; 1 <= n_outs <= 8.
+ * Columns outside the shard are not touched.  The results are bit-identical to
+ * ngram_forward over the full table.  The caller orders the ranks' calls before any read of
+ * the outputs (e.g. a one-element NCCL all-reduce on the same stream after this call).  HBM
+ * residency, no DEDUP / TMA_STAGING (else NGRAM_EUNSUPPORTED). */
+NGRAM_API ngram_status ngram_forward_shard(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
+                                           uint32_t n_seq, uint32_t T, uint32_t d_full, uint32_t col0,
+                                           const uint16_t *residual, const void *gate,
+                                           uint16_t *const *outs, uint32_t n_outs,
+                                           ngram_stream_t stream);
+
+/* CUDA IPC of a device buffer between the processes of one node, for ngram_forward_shard's
+ * peer outputs: ngram_ipc_get_handle writes the 64-byte handle of the allocation that
+ * starts at dev_ptr (cudaMalloc memory, not a sub-allocation); ngram_ipc_open maps another
+ * process's handle into this one (peer access enabled); ngram_ipc_close unmaps it. */
+NGRAM_API ngram_status ngram_device_alloc(void **out, uint64_t bytes);   /* cudaMalloc */
+NGRAM_API ngram_status ngram_device_free(void *p);                        /* cudaFree; NULL ok */
+NGRAM_API ngram_status ngram_ipc_get_handle(const void *dev_ptr, uint8_t handle[64]);
+NGRAM_API ngram_status ngram_ipc_open(const uint8_t handle[64], void **dev_ptr);
+NGRAM_API ngram_status ngram_ipc_close(void *dev_ptr);
+
 /* Synchronise the context's device, read and optionally clear its error word.
  * info (may be NULL) receives {code, flat position, bad id, 0}.  Code 1: a token id was
  * out of range (a position with bit 31 set names history entry (position & 0x7FFFFFFF)
