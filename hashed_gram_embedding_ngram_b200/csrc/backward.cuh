@@ -12,8 +12,9 @@
 //     result, are the same on every run; no floating-point atomics.
 //   * gate: shared gate [d]: dg = sum over tokens of dy * e, with e the forward's fp32 head
 //     sum recomputed here; each product dy * e is exact in fp64 and the sum runs in fp64
-//     over fixed chunks of kGateChunk tokens (per (chunk, column) partials), then over the
-//     chunks in order, rounded once to fp32 -- deterministic for any grid size.
+//     over fixed chunks of kGateChunk tokens (per (chunk, column) partials), then over
+//     groups of kGateGroup chunks and over the groups, each in order, rounded once to fp32
+//     -- a fixed order, so the same result for any grid size.
 //     Per-token gate [N][d]: dg[t] = fp32(dy[t] * e[t]).
 //   * residual: dL/dresidual = dy; nothing to compute.
 //
@@ -108,13 +109,31 @@ __global__ void __launch_bounds__(256, 2) k_gate_grad(const GatherArgs g, const 
     }
 }
 
-// dg[c] = fp32(sum over chunks, in order, of partial[chunk][c]).
-__global__ void __launch_bounds__(256) k_gate_reduce(const double *__restrict__ partial, uint32_t n_chunks,
+// Shared-gate gradient from the [n_chunks][d] fp64 partials, in a fixed two-level order:
+// k_gate_reduce_groups sums each group of kGateGroup consecutive chunks in order into
+// group[g][d]; k_gate_reduce sums the groups in order and rounds once to fp32.  The order
+// depends only on N, so the result is the same on every run.
+constexpr uint32_t kGateGroup = 32;
+
+__global__ void __launch_bounds__(256) k_gate_reduce_groups(const double *__restrict__ partial,
+                                                            uint32_t n_chunks, uint32_t d,
+                                                            double *__restrict__ group) {
+    const uint32_t c = blockIdx.x * blockDim.x + threadIdx.x;
+    const uint32_t gi = blockIdx.y;
+    if (c >= d) return;
+    const uint32_t ch_end = min(n_chunks, (gi + 1u) * kGateGroup);
+    double s = 0.0;
+    for (uint32_t ch = gi * kGateGroup; ch < ch_end; ++ch)
+        s = __dadd_rn(s, partial[static_cast<size_t>(ch) * d + c]);
+    group[static_cast<size_t>(gi) * d + c] = s;
+}
+
+__global__ void __launch_bounds__(256) k_gate_reduce(const double *__restrict__ group, uint32_t n_groups,
                                                      uint32_t d, float *__restrict__ dg) {
     const uint32_t c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= d) return;
     double s = 0.0;
-    for (uint32_t ch = 0; ch < n_chunks; ++ch) s = __dadd_rn(s, partial[static_cast<size_t>(ch) * d + c]);
+    for (uint32_t gi = 0; gi < n_groups; ++gi) s = __dadd_rn(s, group[static_cast<size_t>(gi) * d + c]);
     dg[c] = __double2float_rn(s);
 }
 
@@ -129,10 +148,15 @@ __global__ void __launch_bounds__(256) k_seg_starts(const uint32_t *__restrict__
     }
 }
 
-// One warp per (distinct row u, strip of 256 columns); a lane owns 8 columns.  The row's
-// occurrences occ_tok[seg[u] .. seg[u+1]) (token of each, ascending) are read in groups
-// of 4 loads in flight and summed in order.
-__global__ void __launch_bounds__(256) k_rows_grad(const uint32_t *__restrict__ count,
+// One warp per (chunk of 32 consecutive distinct rows u0 .. u0+31, strip of 256 columns);
+// a lane owns 8 columns.  Lane i loads seg[u0 + i], so the occurrence range of every row of
+// the chunk is known at once; the chunk's occurrences [P0, P1) -- each row's own in
+// ascending order, rows one after the other -- are walked in batches of 8: the 8 dy
+// loads are issued first (the tokens come from one coalesced load of occ_tok; a token's
+// heads usually open consecutive rows, so L1 serves the repeats), then added in order,
+// and a row's gradient is stored as soon as its last occurrence is in.
+template <bool kTokGate>
+__global__ void __launch_bounds__(256, 2) k_rows_grad(const uint32_t *__restrict__ count,
                                                    const uint32_t *__restrict__ seg,
                                                    const uint32_t *__restrict__ occ_tok,
                                                    const uint16_t *__restrict__ dy,
@@ -145,57 +169,81 @@ __global__ void __launch_bounds__(256) k_rows_grad(const uint32_t *__restrict__ 
     const uint32_t nvec = d >> 3;
     const uint32_t n_strips = (nvec + 31u) >> 5;
     const uint32_t U = *count;
-    const uint32_t n_items = U * n_strips;
+    const uint32_t n_items = ((U + 31u) >> 5) * n_strips;
     for (uint32_t item = warp; item < n_items; item += n_warps) {
-        const uint32_t u = item / n_strips;
-        const uint32_t v = (item - u * n_strips) * 32u + lane;
-        if (v >= nvec) continue;
-        const uint32_t j0 = __ldg(seg + u), j1 = __ldg(seg + u + 1);
+        const uint32_t ch = item / n_strips;
+        const uint32_t v = (item - ch * n_strips) * 32u + lane;
+        const bool active = v < nvec;
+        const uint32_t u0 = ch * 32u;
+        const uint32_t nu = min(32u, U - u0);
+        const uint32_t P1 = __ldg(seg + u0 + nu);                     // end of the chunk's last row
+        const uint32_t my_seg = lane < nu ? __ldg(seg + u0 + lane) : P1;
+        const uint32_t P0 = __shfl_sync(0xFFFFFFFFu, my_seg, 0);
+        float gv[8];
+        if (!kTokGate && active) {
+            const float4 ga = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v);
+            const float4 gb = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v + 1u);
+            gv[0] = ga.x; gv[1] = ga.y; gv[2] = ga.z; gv[3] = ga.w;
+            gv[4] = gb.x; gv[5] = gb.y; gv[6] = gb.z; gv[7] = gb.w;
+        }
+        uint32_t r = 0;                                              // current row of the chunk
+        uint32_t next_end = __shfl_sync(0xFFFFFFFFu, my_seg, 1);      // first position after it
+        if (nu == 1) next_end = P1;
         float acc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
-        for (uint32_t j = j0; j < j1; j += 4) {
-            const uint32_t nq = min(4u, j1 - j);
-            uint4 w[4], gw[4];
+        for (uint32_t p0 = P0; p0 < P1; p0 += 32u) {
+            const uint32_t nb = min(32u, P1 - p0);
+            const uint32_t my_tok = lane < nb ? __ldg(occ_tok + p0 + lane) : 0u;
+            for (uint32_t j0 = 0; j0 < nb; j0 += 8u) {
+                uint4 w[8], gw[8];
 #pragma unroll
-            for (uint32_t q = 0; q < 4; ++q) {
-                if (q < nq) {
-                    const size_t off = static_cast<size_t>(__ldg(occ_tok + j + q)) * d + v * 8u;
-                    w[q] = ld_na_v4(dy + off);
-                    if (gate_tok) gw[q] = ld_na_v4(gate_tok + off);
+                for (uint32_t q = 0; q < 8; ++q) {
+                    const uint32_t tok = __shfl_sync(0xFFFFFFFFu, my_tok, (j0 + q) & 31u);
+                    if (j0 + q < nb && active) {
+                        const size_t off = static_cast<size_t>(tok) * d + v * 8u;
+                        w[q] = __ldg(reinterpret_cast<const uint4 *>(dy + off));
+                        if (kTokGate) gw[q] = __ldg(reinterpret_cast<const uint4 *>(gate_tok + off));
+                    }
                 }
-            }
 #pragma unroll
-            for (uint32_t q = 0; q < 4; ++q) {
-                if (q < nq) {
-                    const uint32_t ww[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
-                    if (gate_tok) {
-                        const uint32_t gg[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
+                for (uint32_t q = 0; q < 8; ++q) {
+                    if (j0 + q >= nb) break;                          // warp-uniform
+                    if (active) {
+                        const uint32_t ww[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+                        if (kTokGate) {
+                            const uint32_t gg[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            acc[2 * p] = __fmaf_rn(bf16_lo(gg[p]), bf16_lo(ww[p]), acc[2 * p]);
-                            acc[2 * p + 1] = __fmaf_rn(bf16_hi(gg[p]), bf16_hi(ww[p]), acc[2 * p + 1]);
+                            for (int p = 0; p < 4; ++p) {
+                                acc[2 * p] = __fmaf_rn(bf16_lo(gg[p]), bf16_lo(ww[p]), acc[2 * p]);
+                                acc[2 * p + 1] = __fmaf_rn(bf16_hi(gg[p]), bf16_hi(ww[p]), acc[2 * p + 1]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) {
+                                acc[2 * p] = __fadd_rn(acc[2 * p], bf16_lo(ww[p]));
+                                acc[2 * p + 1] = __fadd_rn(acc[2 * p + 1], bf16_hi(ww[p]));
+                            }
                         }
-                    } else {
+                    }
+                    if (p0 + j0 + q + 1u == next_end) {                // row u0 + r is complete
+                        if (active) {
+                            float o[8];
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            acc[2 * p] = __fadd_rn(acc[2 * p], bf16_lo(ww[p]));
-                            acc[2 * p + 1] = __fadd_rn(acc[2 * p + 1], bf16_hi(ww[p]));
+                            for (int k = 0; k < 8; ++k) o[k] = kTokGate ? acc[k] : __fmul_rn(gv[k], acc[k]);
+                            float4 *dst = reinterpret_cast<float4 *>(grad + static_cast<size_t>(u0 + r) * d + v * 8u);
+                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
                         }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+                        ++r;
+                        const uint32_t e = __shfl_sync(0xFFFFFFFFu, my_seg, (r + 1u) & 31u);
+                        next_end = (r + 1u < nu) ? e : P1;
                     }
                 }
             }
         }
-        if (!gate_tok) {
-            const float4 ga = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v);
-            const float4 gb = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v + 1u);
-            const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-#pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = __fmul_rn(gv[k], acc[k]);
-        }
-        float4 *dst = reinterpret_cast<float4 *>(grad + static_cast<size_t>(u) * d + v * 8u);
-        dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 

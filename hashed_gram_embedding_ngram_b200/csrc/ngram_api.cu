@@ -24,6 +24,8 @@
 #include "gather_int8.cuh"
 #include "gather_nvfp4.cuh"
 #include "gather_c8.cuh"
+#include "gather_staged.cuh"
+#include "gather_async.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
 #include "order.cuh"
@@ -39,6 +41,13 @@ using namespace ngram;
 #endif
 static bool use_c8(ngram_dtype t) { return t != NGRAM_BF16 && ((NGRAM_C8_FORMATS >> t) & 1u); }
 
+// NVFP4 rows gathered by k_gather_nvfp4_async (cp.async double buffer per warp) instead
+// of the register gather k_gather_nvfp4.
+#ifndef NGRAM_NVFP4_ASYNC
+#define NGRAM_NVFP4_ASYNC 0
+#endif
+static constexpr uint32_t kAsyncSmem = kAsyncWarps * kAsyncWarpBytes;
+
 // Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
 //   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
 //     strips of a token run on 10 warps at once (455 us) instead of one warp walking
@@ -53,6 +62,12 @@ static bool use_c8(ngram_dtype t) { return t != NGRAM_BF16 && ((NGRAM_C8_FORMATS
 #endif
 #ifndef NGRAM_BULK_SMEM_BYTES           // shared memory per CTA for the stage ring
 #define NGRAM_BULK_SMEM_BYTES (100 * 1024)
+#endif
+#ifndef NGRAM_STAGED_SMEM_BYTES         // shared memory per CTA of the staged 8- and 4-bit gathers
+#define NGRAM_STAGED_SMEM_BYTES (200 * 1024)
+#endif
+#ifndef NGRAM_STAGED_CTAS_PER_SM
+#define NGRAM_STAGED_CTAS_PER_SM 1
 #endif
 #ifndef NGRAM_BULK_CTAS_PER_SM
 #define NGRAM_BULK_CTAS_PER_SM 2
@@ -97,6 +112,8 @@ struct ngram_ctx {
     int num_sms;
     int gather_blocks_per_sm;
     int bulk_smem_set;
+    int staged_smem_set;
+    int async_smem_set;
     uint32_t wait_ms;           // bound of every host-side wait
     uint32_t *d_err;            // 4 words
     float *d_gscale;            // NVFP4: device copy of the global scale
@@ -463,6 +480,11 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 template <bool kTok>
 void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
     const bool h16 = g.h.n_heads == 16;
+    if (NGRAM_NVFP4_ASYNC && t == NGRAM_NVFP4) {
+        if (h16) k_gather_nvfp4_async<16, kTok><<<nb, 256, kAsyncSmem, s>>>(g);
+        else k_gather_nvfp4_async<0, kTok><<<nb, 256, kAsyncSmem, s>>>(g);
+        return;
+    }
     if (use_c8(t)) {
         switch (t) {
             case NGRAM_INT8_ROWSCALE: launch_c8<Rows8bit<Int8Codes>, kTok>(g, nb, s, rb); break;
@@ -488,8 +510,51 @@ void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaS
     }
 }
 
+// The TMA-staged gather of the 8- and 4-bit formats: whole rows through a shared-memory
+// ring, one token per item (gather_staged.cuh).
+template <class Rows>
+ngram_status launch_staged_fmt(ngram_ctx *c, const GatherArgs &g, const StagedPlan &p, unsigned grid,
+                               uint32_t smem, cudaStream_t s) {
+    if (!c->staged_smem_set) {
+        NG_CUDA(cudaFuncSetAttribute(k_gather_staged<16, Rows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     NGRAM_STAGED_SMEM_BYTES), "cudaFuncSetAttribute (staged gather)");
+        NG_CUDA(cudaFuncSetAttribute(k_gather_staged<0, Rows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     NGRAM_STAGED_SMEM_BYTES), "cudaFuncSetAttribute (staged gather)");
+        c->staged_smem_set = 1;
+    }
+    if (g.h.n_heads == 16) k_gather_staged<16, Rows><<<grid, 352, smem, s>>>(g, p);
+    else k_gather_staged<0, Rows><<<grid, 352, smem, s>>>(g, p);
+    NG_CUDA(cudaGetLastError(), "k_gather_staged launch");
+    return NGRAM_OK;
+}
+
+ngram_status launch_staged(ngram_ctx *c, const GatherArgs &g, cudaStream_t s) {
+    StagedPlan p;
+    p.row_bytes = c->row_bytes;
+    p.res_off = 16u * c->row_bytes;
+    p.scale_off = p.res_off + 2u * c->d;
+    p.stage_bytes = (p.scale_off + 64u + 127u) & ~127u;
+    uint32_t stages = (NGRAM_STAGED_SMEM_BYTES - 128u) / p.stage_bytes;
+    if (stages > kBulkMaxStages) stages = kBulkMaxStages;
+    if (stages < 2) return fail(NGRAM_EUNSUPPORTED, "staged gather: stage of %u bytes too large", p.stage_bytes);
+    p.stages = stages;
+    const uint32_t smem = stages * p.stage_bytes + 128u;
+    uint64_t grid = static_cast<uint64_t>(c->num_sms) * NGRAM_STAGED_CTAS_PER_SM;
+    if (grid > g.N) grid = g.N;
+    const unsigned nb = static_cast<unsigned>(grid);
+    switch (c->dtype) {
+        case NGRAM_INT8_ROWSCALE: return launch_staged_fmt<Rows8bit<Int8Codes>>(c, g, p, nb, smem, s);
+        case NGRAM_FP8_E4M3_ROWSCALE: return launch_staged_fmt<Rows8bit<E4m3Codes>>(c, g, p, nb, smem, s);
+        case NGRAM_NVFP4: return launch_staged_fmt<RowsNvfp4>(c, g, p, nb, smem, s);
+        default: return fail(NGRAM_EUNSUPPORTED, "staged gather: bf16 uses the chunked TMA gather");
+    }
+}
+
 // The register gather (every row format); max_blocks bounds the persistent grid.
 ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t max_blocks) {
+    if ((c->hp.flags & NGRAM_FLAG_TMA_STAGING) && c->dtype != NGRAM_BF16 && c->where == NGRAM_RES_HBM &&
+        g.row_ids == nullptr && g.gate_tok == nullptr && g.tok_begin == 0)
+        return launch_staged(c, g, s);
     const uint64_t resident_warps = max_blocks * 8u;
     g.strips_per_item = (NGRAM_SPI_ALWAYS_ONE ||
                          static_cast<uint64_t>(g.N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
@@ -635,7 +700,8 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
 bool grouped_order(const ngram_ctx *c, uint32_t N) {
     const uint32_t f = c->hp.flags;
     if (f & NGRAM_FLAG_SORT) return true;
-    if (f & (NGRAM_FLAG_BATCH_ORDER | NGRAM_FLAG_TMA_STAGING)) return false;
+    if (f & NGRAM_FLAG_BATCH_ORDER) return false;
+    if ((f & NGRAM_FLAG_TMA_STAGING) && c->dtype == NGRAM_BF16) return false;
     return N >= NGRAM_SORT_MIN_TOKENS;
 }
 
@@ -811,7 +877,17 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess) {
         int *bps = &c->gather_blocks_per_sm;
-        if (use_c8(dtype)) {
+        if (NGRAM_NVFP4_ASYNC && dtype == NGRAM_NVFP4) {
+            const void *fns[] = {reinterpret_cast<const void *>(k_gather_nvfp4_async<16, false>),
+                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<0, false>),
+                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<16, true>),
+                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<0, true>)};
+            for (const void *f : fns)
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kAsyncSmem);
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_nvfp4_async<16, false>, 256, kAsyncSmem);
+        } else if (use_c8(dtype)) {
             if (dtype == NGRAM_NVFP4)
                 e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, RowsNvfp4, false>, 256, 0);
             else if (dtype == NGRAM_FP8_E4M3_ROWSCALE)
@@ -1303,9 +1379,16 @@ ngram_status ngram_backward_rows(ngram_ctx *c, const int32_t *tokens, const int3
     NG_CHECK(sort_occurrences(c, c->d_inv, M, s, &skeys, &stok));
     k_seg_starts<<<grid_for(c, M, 256), 256, 0, s>>>(skeys, M, c->bw_seg);
     const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
-    k_rows_grad<<<static_cast<unsigned>(c->num_sms) * 8u, 256, 0, s>>>(
-        count_out, c->bw_seg, stok, grad_out, tok_gate ? nullptr : static_cast<const float *>(gate),
-        tok_gate ? static_cast<const uint16_t *>(gate) : nullptr, c->d, grad_rows);
+    int per_sm = 0;
+    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, tok_gate ? k_rows_grad<true> : k_rows_grad<false>, 256, 0), "occupancy");
+    const unsigned grid = static_cast<unsigned>(c->num_sms) * static_cast<unsigned>(std::max(1, per_sm));
+    if (tok_gate)
+        k_rows_grad<true><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out, nullptr,
+                                               static_cast<const uint16_t *>(gate), c->d, grad_rows);
+    else
+        k_rows_grad<false><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out,
+                                                static_cast<const float *>(gate), nullptr, c->d, grad_rows);
     NG_CUDA(cudaGetLastError(), "k_rows_grad launch");
     return NGRAM_OK;
 }
@@ -1332,12 +1415,16 @@ ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int3
     if (tok_gate) {
         launch_gate_grad<true>(c->dtype, g, grid, s, grad_out, grad_gate, nullptr, c->row_bytes);
     } else {
-        if (!c->bw_part)
-            NG_CUDA(cudaMalloc(&c->bw_part, ((c->max_tokens + kGateChunk - 1) / kGateChunk) * 8ull * c->d),
-                    "backward scratch");
+        const uint64_t max_chunks = (c->max_tokens + kGateChunk - 1) / kGateChunk;
+        const uint64_t max_groups = (max_chunks + kGateGroup - 1) / kGateGroup;
+        if (!c->bw_part)      // chunk partials, then group partials
+            NG_CUDA(cudaMalloc(&c->bw_part, (max_chunks + max_groups) * 8ull * c->d), "backward scratch");
         const uint32_t n_chunks = static_cast<uint32_t>((N + kGateChunk - 1) / kGateChunk);
+        const uint32_t n_groups = (n_chunks + kGateGroup - 1) / kGateGroup;
+        double *groups = c->bw_part + max_chunks * c->d;
         launch_gate_grad<false>(c->dtype, g, grid, s, grad_out, nullptr, c->bw_part, c->row_bytes);
-        k_gate_reduce<<<(c->d + 255) / 256, 256, 0, s>>>(c->bw_part, n_chunks, c->d, grad_gate);
+        k_gate_reduce_groups<<<dim3((c->d + 255) / 256, n_groups), 256, 0, s>>>(c->bw_part, n_chunks, c->d, groups);
+        k_gate_reduce<<<(c->d + 255) / 256, 256, 0, s>>>(groups, n_groups, c->d, grad_gate);
     }
     NG_CUDA(cudaGetLastError(), "k_gate_grad launch");
     return NGRAM_OK;

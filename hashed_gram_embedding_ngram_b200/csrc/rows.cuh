@@ -28,6 +28,9 @@ struct RowsBf16 {
     static __device__ __forceinline__ Frag load(const uint8_t *row, uint32_t v, uint32_t /*d*/) {
         return ld_stream_v4(row + v * 16u);
     }
+    static __device__ __forceinline__ Frag load_smem(const uint8_t *row, uint32_t v, uint32_t) {
+        return *reinterpret_cast<const uint4 *>(row + v * 16u);
+    }
     static __device__ __forceinline__ void add(float2 (&acc)[4], const Frag &f, float, float) {
         acc[0] = add2(acc[0], bf16x2(f.x));
         acc[1] = add2(acc[1], bf16x2(f.y));
@@ -42,6 +45,9 @@ struct Rows8bit {                       // int8 / FP8 E4M3 codes with a per-row 
     typedef uint2 Frag;
     static __device__ __forceinline__ Frag load(const uint8_t *row, uint32_t v, uint32_t) {
         return ld_stream_v2(row + v * 8u);
+    }
+    static __device__ __forceinline__ Frag load_smem(const uint8_t *row, uint32_t v, uint32_t) {
+        return *reinterpret_cast<const uint2 *>(row + v * 8u);
     }
     static __device__ __forceinline__ void add(float2 (&acc)[4], const Frag &f, float s, float) {
         const float2 s2 = make_float2(s, s);
@@ -62,6 +68,9 @@ struct RowsNvfp4 {                      // E2M1 codes, E4M3 block scale, global 
     };
     static __device__ __forceinline__ Frag load(const uint8_t *row, uint32_t v, uint32_t d) {
         return Frag{ld_stream_u32(row + v * 4u), ld_stream_u8(row + (d >> 1) + (v >> 1))};
+    }
+    static __device__ __forceinline__ Frag load_smem(const uint8_t *row, uint32_t v, uint32_t d) {
+        return Frag{*reinterpret_cast<const uint32_t *>(row + v * 4u), row[(d >> 1) + (v >> 1)]};
     }
     static __device__ __forceinline__ void add(float2 (&acc)[4], const Frag &f, float, float gs) {
         const float cs = __fmul_rn(e4m3_to_float(f.bs), gs);

@@ -191,6 +191,27 @@ def test_nvfp4_global_scale_from_host_memory_and_other_values(cuda_device):
 
 
 # --------------------------------------------------------------------------- modes and flags
+@pytest.mark.parametrize("fmt", ["int8", "fp8", "nvfp4"])
+@pytest.mark.parametrize("n_seq,T,hist", [(3, 200, True), (1, 20_000, False)])
+def test_tma_staged_gather_bitidentical(cuda_device, fmt, n_seq, T, hist):
+    """NGRAM_FLAG_TMA_STAGING (whole rows staged in shared memory by cp.async.bulk) gives
+    the register gather's bits, in batch order and in grouped order (20,000 tokens)."""
+    R, d, V = 400_000, 2560, 151_936
+    w = gen.Workload(fmt + "_tma", R, d, fmt, V, n_seq, T, history=hist)
+    inp, dv = workload_on_device(w, cuda_device, token_seed=65)
+    dt = ng_dtype(fmt)
+    table, scale = TABLES.get(R, d, dt, gen.TABLE_SEED, cuda_device)
+    ref = from_dev_bf16(_fwd(ng.ngram_init(table, R, d, dt, ng.NGRAM_RES_HBM, _hp(V), w.N, row_scale=scale), dv))
+    c = ng.ngram_init(table, R, d, dt, ng.NGRAM_RES_HBM, _hp(V, flags=ng.NGRAM_FLAG_TMA_STAGING), w.N,
+                      row_scale=scale)
+    for _ in range(2):
+        assert np.array_equal(from_dev_bf16(_fwd(c, dv)), ref)
+    assert ng.ngram_get_device_error(c)[0] == ng.NGRAM_OK
+    sel = sample_tokens(w, 64, seed=4)
+    r = assert_parity(ref.reshape(w.N, d)[sel], _oracle(w, inp, sel=sel))
+    assert r["exact"] == r["n"]
+
+
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
 def test_flags_and_staging_bitidentical(cuda_device, fmt):
     """Dedup staging, grouped order, batch order and prefetch + staged gather give the
