@@ -148,95 +148,140 @@ __global__ void __launch_bounds__(256) k_seg_starts(const uint32_t *__restrict__
     }
 }
 
-// One warp per (chunk of 32 consecutive distinct rows u0 .. u0+31, strip of 256 columns);
-// a lane owns 8 columns.  Lane i loads seg[u0 + i], so the occurrence range of every row of
-// the chunk is known at once; the chunk's occurrences [P0, P1) -- each row's own in
-// ascending order, rows one after the other -- are walked in batches of 8: the 8 dy
-// loads are issued first (the tokens come from one coalesced load of occ_tok; a token's
-// heads usually open consecutive rows, so L1 serves the repeats), then added in order,
-// and a row's gradient is stored as soon as its last occurrence is in.
-template <bool kTokGate>
+// One warp per (chunk of 32 consecutive distinct rows u0 .. u0+31, group of kStrips strips
+// of 256 columns).  In each strip a lane owns columns 4l .. 4l+3 and 128+4l .. 128+4l+3,
+// so each of its two float4 stores is part of a contiguous 512-byte warp store (whole
+// sectors), and dy comes in two 8-byte loads.  Lane i loads seg[u0 + i], so the occurrence
+// range of every row of the chunk is known at once; the chunk's occurrences [P0, P1) --
+// each row's own in ascending order, rows one after the other -- are walked in batches of
+// kBatch: the batch's loads are issued first (the tokens come from one coalesced load of
+// occ_tok; a token's heads usually open consecutive rows, so L1 serves the repeats), then
+// added in order, and a row's gradient is stored as soon as its last occurrence is in.
+// Warps take items from an atomic counter (*next_item, zeroed before the launch): chunks
+// holding the most frequent rows come first (frequent contexts appear early in a batch),
+// and no warp is left with a long tail.
+#ifndef NGRAM_ROWS_GRAD_STRIPS
+#define NGRAM_ROWS_GRAD_STRIPS 1
+#endif
+
+template <bool kTokGate, int kStrips>
 __global__ void __launch_bounds__(256, 2) k_rows_grad(const uint32_t *__restrict__ count,
-                                                   const uint32_t *__restrict__ seg,
-                                                   const uint32_t *__restrict__ occ_tok,
-                                                   const uint16_t *__restrict__ dy,
-                                                   const float *__restrict__ gate,
-                                                   const uint16_t *__restrict__ gate_tok,
-                                                   uint32_t d, float *__restrict__ grad) {
+                                                      const uint32_t *__restrict__ seg,
+                                                      const uint32_t *__restrict__ occ_tok,
+                                                      const uint16_t *__restrict__ dy,
+                                                      const float *__restrict__ gate,
+                                                      const uint16_t *__restrict__ gate_tok,
+                                                      uint32_t d, float *__restrict__ grad,
+                                                      uint32_t *next_item) {
+    constexpr uint32_t kBatch = (kTokGate ? 8u : 16u) / kStrips;   // 16 (8) fragments in flight
     const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
-    const uint32_t nvec = d >> 3;
-    const uint32_t n_strips = (nvec + 31u) >> 5;
+    const uint32_t n_strips = ((d >> 3) + 31u) >> 5;
+    const uint32_t n_groups = (n_strips + kStrips - 1u) / kStrips;
     const uint32_t U = *count;
-    const uint32_t n_items = ((U + 31u) >> 5) * n_strips;
-    for (uint32_t item = warp; item < n_items; item += n_warps) {
-        const uint32_t ch = item / n_strips;
-        const uint32_t v = (item - ch * n_strips) * 32u + lane;
-        const bool active = v < nvec;
+    const uint32_t n_items = ((U + 31u) >> 5) * n_groups;
+    for (;;) {
+        uint32_t item = 0;
+        if (lane == 0) item = atomicAdd(next_item, 1u);
+        item = __shfl_sync(0xFFFFFFFFu, item, 0);
+        if (item >= n_items) break;
+        const uint32_t ch = item / n_groups;
+        const uint32_t grp = item - ch * n_groups;
+        uint32_t c0[kStrips];                 // first column of the lane's first quad in each strip
+        bool act[kStrips][2];                 // quad h (columns c0 + 128h ..) inside the row
+#pragma unroll
+        for (int k = 0; k < kStrips; ++k) {
+            c0[k] = (grp * kStrips + k) * 256u + lane * 4u;
+            act[k][0] = c0[k] < d;            // d % 8 == 0: a quad is wholly in or out
+            act[k][1] = c0[k] + 128u < d;
+        }
         const uint32_t u0 = ch * 32u;
         const uint32_t nu = min(32u, U - u0);
         const uint32_t P1 = __ldg(seg + u0 + nu);                     // end of the chunk's last row
         const uint32_t my_seg = lane < nu ? __ldg(seg + u0 + lane) : P1;
         const uint32_t P0 = __shfl_sync(0xFFFFFFFFu, my_seg, 0);
-        float gv[8];
-        if (!kTokGate && active) {
-            const float4 ga = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v);
-            const float4 gb = __ldg(reinterpret_cast<const float4 *>(gate) + 2u * v + 1u);
-            gv[0] = ga.x; gv[1] = ga.y; gv[2] = ga.z; gv[3] = ga.w;
-            gv[4] = gb.x; gv[5] = gb.y; gv[6] = gb.z; gv[7] = gb.w;
-        }
         uint32_t r = 0;                                              // current row of the chunk
         uint32_t next_end = __shfl_sync(0xFFFFFFFFu, my_seg, 1);      // first position after it
         if (nu == 1) next_end = P1;
-        float acc[8];
+        float acc[kStrips][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+        for (int k = 0; k < kStrips; ++k)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[k][j] = 0.0f;
         for (uint32_t p0 = P0; p0 < P1; p0 += 32u) {
             const uint32_t nb = min(32u, P1 - p0);
             const uint32_t my_tok = lane < nb ? __ldg(occ_tok + p0 + lane) : 0u;
-            for (uint32_t j0 = 0; j0 < nb; j0 += 8u) {
-                uint4 w[8], gw[8];
+            for (uint32_t j0 = 0; j0 < nb; j0 += kBatch) {
+                uint2 w[kBatch][kStrips][2], gw[kBatch][kStrips][2];
 #pragma unroll
-                for (uint32_t q = 0; q < 8; ++q) {
+                for (uint32_t q = 0; q < kBatch; ++q) {
                     const uint32_t tok = __shfl_sync(0xFFFFFFFFu, my_tok, (j0 + q) & 31u);
-                    if (j0 + q < nb && active) {
-                        const size_t off = static_cast<size_t>(tok) * d + v * 8u;
-                        w[q] = __ldg(reinterpret_cast<const uint4 *>(dy + off));
-                        if (kTokGate) gw[q] = __ldg(reinterpret_cast<const uint4 *>(gate_tok + off));
+                    if (j0 + q < nb) {
+                        const uint16_t *row = dy + static_cast<size_t>(tok) * d;
+                        const uint16_t *grow = gate_tok + static_cast<size_t>(tok) * d;
+#pragma unroll
+                        for (int k = 0; k < kStrips; ++k) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                if (act[k][h]) {
+                                    w[q][k][h] = __ldg(reinterpret_cast<const uint2 *>(row + c0[k] + h * 128u));
+                                    if (kTokGate)
+                                        gw[q][k][h] = __ldg(reinterpret_cast<const uint2 *>(grow + c0[k] + h * 128u));
+                                }
+                            }
+                        }
                     }
                 }
 #pragma unroll
-                for (uint32_t q = 0; q < 8; ++q) {
+                for (uint32_t q = 0; q < kBatch; ++q) {
                     if (j0 + q >= nb) break;                          // warp-uniform
-                    if (active) {
-                        const uint32_t ww[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
-                        if (kTokGate) {
-                            const uint32_t gg[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
 #pragma unroll
-                            for (int p = 0; p < 4; ++p) {
-                                acc[2 * p] = __fmaf_rn(bf16_lo(gg[p]), bf16_lo(ww[p]), acc[2 * p]);
-                                acc[2 * p + 1] = __fmaf_rn(bf16_hi(gg[p]), bf16_hi(ww[p]), acc[2 * p + 1]);
-                            }
-                        } else {
+                    for (int k = 0; k < kStrips; ++k) {
 #pragma unroll
-                            for (int p = 0; p < 4; ++p) {
-                                acc[2 * p] = __fadd_rn(acc[2 * p], bf16_lo(ww[p]));
-                                acc[2 * p + 1] = __fadd_rn(acc[2 * p + 1], bf16_hi(ww[p]));
+                        for (int h = 0; h < 2; ++h) {
+                            if (!act[k][h]) continue;
+                            const uint32_t ww[2] = {w[q][k][h].x, w[q][k][h].y};
+                            float *a = &acc[k][4 * h];
+                            if (kTokGate) {
+                                const uint32_t gg[2] = {gw[q][k][h].x, gw[q][k][h].y};
+#pragma unroll
+                                for (int p = 0; p < 2; ++p) {
+                                    a[2 * p] = __fmaf_rn(bf16_lo(gg[p]), bf16_lo(ww[p]), a[2 * p]);
+                                    a[2 * p + 1] = __fmaf_rn(bf16_hi(gg[p]), bf16_hi(ww[p]), a[2 * p + 1]);
+                                }
+                            } else {
+#pragma unroll
+                                for (int p = 0; p < 2; ++p) {
+                                    a[2 * p] = __fadd_rn(a[2 * p], bf16_lo(ww[p]));
+                                    a[2 * p + 1] = __fadd_rn(a[2 * p + 1], bf16_hi(ww[p]));
+                                }
                             }
                         }
                     }
                     if (p0 + j0 + q + 1u == next_end) {                // row u0 + r is complete
-                        if (active) {
-                            float o[8];
+                        float *row = grad + static_cast<size_t>(u0 + r) * d;
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) o[k] = kTokGate ? acc[k] : __fmul_rn(gv[k], acc[k]);
-                            float4 *dst = reinterpret_cast<float4 *>(grad + static_cast<size_t>(u0 + r) * d + v * 8u);
-                            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                        for (int k = 0; k < kStrips; ++k) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                if (act[k][h]) {
+                                    float o[4];
+                                    if (kTokGate) {
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j) o[j] = acc[k][4 * h + j];
+                                    } else {
+                                        const float4 gq = __ldg(reinterpret_cast<const float4 *>(gate + c0[k] + h * 128u));
+                                        o[0] = __fmul_rn(gq.x, acc[k][4 * h]);
+                                        o[1] = __fmul_rn(gq.y, acc[k][4 * h + 1]);
+                                        o[2] = __fmul_rn(gq.z, acc[k][4 * h + 2]);
+                                        o[3] = __fmul_rn(gq.w, acc[k][4 * h + 3]);
+                                    }
+                                    *reinterpret_cast<float4 *>(row + c0[k] + h * 128u) =
+                                        make_float4(o[0], o[1], o[2], o[3]);
+                                }
+                            }
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) acc[k][j] = 0.0f;
                         }
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
                         ++r;
                         const uint32_t e = __shfl_sync(0xFFFFFFFFu, my_seg, (r + 1u) & 31u);
                         next_end = (r + 1u < nu) ? e : P1;

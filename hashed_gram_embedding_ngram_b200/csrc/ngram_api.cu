@@ -25,7 +25,6 @@
 #include "gather_nvfp4.cuh"
 #include "gather_c8.cuh"
 #include "gather_staged.cuh"
-#include "gather_async.cuh"
 #include "gather_bulk.cuh"
 #include "dedup.cuh"
 #include "order.cuh"
@@ -41,12 +40,6 @@ using namespace ngram;
 #endif
 static bool use_c8(ngram_dtype t) { return t != NGRAM_BF16 && ((NGRAM_C8_FORMATS >> t) & 1u); }
 
-// NVFP4 rows gathered by k_gather_nvfp4_async (cp.async double buffer per warp) instead
-// of the register gather k_gather_nvfp4.
-#ifndef NGRAM_NVFP4_ASYNC
-#define NGRAM_NVFP4_ASYNC 0
-#endif
-static constexpr uint32_t kAsyncSmem = kAsyncWarps * kAsyncWarpBytes;
 
 // Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
 //   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
@@ -113,7 +106,6 @@ struct ngram_ctx {
     int gather_blocks_per_sm;
     int bulk_smem_set;
     int staged_smem_set;
-    int async_smem_set;
     uint32_t wait_ms;           // bound of every host-side wait
     uint32_t *d_err;            // 4 words
     float *d_gscale;            // NVFP4: device copy of the global scale
@@ -480,11 +472,6 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 template <bool kTok>
 void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
     const bool h16 = g.h.n_heads == 16;
-    if (NGRAM_NVFP4_ASYNC && t == NGRAM_NVFP4) {
-        if (h16) k_gather_nvfp4_async<16, kTok><<<nb, 256, kAsyncSmem, s>>>(g);
-        else k_gather_nvfp4_async<0, kTok><<<nb, 256, kAsyncSmem, s>>>(g);
-        return;
-    }
     if (use_c8(t)) {
         switch (t) {
             case NGRAM_INT8_ROWSCALE: launch_c8<Rows8bit<Int8Codes>, kTok>(g, nb, s, rb); break;
@@ -877,17 +864,7 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess) {
         int *bps = &c->gather_blocks_per_sm;
-        if (NGRAM_NVFP4_ASYNC && dtype == NGRAM_NVFP4) {
-            const void *fns[] = {reinterpret_cast<const void *>(k_gather_nvfp4_async<16, false>),
-                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<0, false>),
-                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<16, true>),
-                                 reinterpret_cast<const void *>(k_gather_nvfp4_async<0, true>)};
-            for (const void *f : fns)
-                if (e == cudaSuccess)
-                    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kAsyncSmem);
-            if (e == cudaSuccess)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_nvfp4_async<16, false>, 256, kAsyncSmem);
-        } else if (use_c8(dtype)) {
+        if (use_c8(dtype)) {
             if (dtype == NGRAM_NVFP4)
                 e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, RowsNvfp4, false>, 256, 0);
             else if (dtype == NGRAM_FP8_E4M3_ROWSCALE)
@@ -1293,7 +1270,7 @@ ngram_status ensure_backward_sort(ngram_ctx *c) {
     NG_CUDA(cudaMalloc(&c->bw_hist, L * 4), "backward scratch");
     NG_CUDA(cudaMalloc(&c->bw_tot, nb * 4), "backward scratch");
     NG_CUDA(cudaMalloc(&c->bw_seg, (M + 1) * 4), "backward scratch");
-    NG_CUDA(cudaMalloc(&c->bw_word, 4), "backward scratch");
+    NG_CUDA(cudaMalloc(&c->bw_word, 8), "backward scratch");     // scan total, item counter
     return NGRAM_OK;
 }
 
@@ -1379,16 +1356,20 @@ ngram_status ngram_backward_rows(ngram_ctx *c, const int32_t *tokens, const int3
     NG_CHECK(sort_occurrences(c, c->d_inv, M, s, &skeys, &stok));
     k_seg_starts<<<grid_for(c, M, 256), 256, 0, s>>>(skeys, M, c->bw_seg);
     const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
+    constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
     int per_sm = 0;
     NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, tok_gate ? k_rows_grad<true> : k_rows_grad<false>, 256, 0), "occupancy");
+                &per_sm, tok_gate ? k_rows_grad<true, kS> : k_rows_grad<false, kS>, 256, 0), "occupancy");
     const unsigned grid = static_cast<unsigned>(c->num_sms) * static_cast<unsigned>(std::max(1, per_sm));
+    NG_CUDA(cudaMemsetAsync(c->bw_word + 1, 0, 4, s), "cudaMemsetAsync");     // the item counter
     if (tok_gate)
-        k_rows_grad<true><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out, nullptr,
-                                               static_cast<const uint16_t *>(gate), c->d, grad_rows);
+        k_rows_grad<true, kS><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out, nullptr,
+                                                   static_cast<const uint16_t *>(gate), c->d, grad_rows,
+                                                   c->bw_word + 1);
     else
-        k_rows_grad<false><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out,
-                                                static_cast<const float *>(gate), nullptr, c->d, grad_rows);
+        k_rows_grad<false, kS><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out,
+                                                    static_cast<const float *>(gate), nullptr, c->d, grad_rows,
+                                                    c->bw_word + 1);
     NG_CUDA(cudaGetLastError(), "k_rows_grad launch");
     return NGRAM_OK;
 }
