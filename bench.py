@@ -315,8 +315,10 @@ def run_ours(args, w):
         scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
     ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
     flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING,
-             "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER}[args.variant]
-    grouped = args.variant == "sort" or (args.variant == "default" and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
+             "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER,
+             "token_gate": ng.NGRAM_FLAG_TOKEN_GATE}[args.variant]
+    grouped = args.variant == "sort" or (args.variant in ("default", "token_gate")
+                                         and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
     hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
 
@@ -334,6 +336,9 @@ def run_ours(args, w):
     residual = res_cpu.to(dev)
     out = torch.empty_like(residual)
     gate = torch.from_numpy(gate_h).to(dev)
+    if args.variant == "token_gate":       # one bf16 gate per token and column
+        gate = torch.from_numpy(np.random.default_rng(12).uniform(0, 1, (w.N, w.d)).astype(np.float32)
+                                ).to(torch.bfloat16).to(dev)
     stream = torch.cuda.current_stream()
 
     def step(i, s=None):
@@ -394,6 +399,7 @@ def run_ours(args, w):
     hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in host_hist]
     res_h = res_cpu.pin_memory()
     out_h = torch.empty_like(res_h).pin_memory()
+    gate_h_tok = gate.cpu().pin_memory() if args.variant == "token_gate" else None
     E = max(1, args.e2e_steps)
 
     def e2e_step(i):
@@ -406,6 +412,8 @@ def run_ours(args, w):
             if hist_h[b] is not None:
                 hist_d[b].copy_(hist_h[b], non_blocking=True)
             residual.copy_(res_h, non_blocking=True)
+            if gate_h_tok is not None:        # a per-token gate is an activation: it comes in too
+                gate.copy_(gate_h_tok, non_blocking=True)
             ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
             out_h.copy_(out, non_blocking=True)
 
@@ -421,7 +429,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    h2d = w.N * 4 + (w.n_seq * 8 if w.history else 0) + w.N * w.d * 2
+    h2d = w.N * 4 + (w.n_seq * 8 if w.history else 0) + w.N * w.d * 2 * (2 if args.variant == "token_gate" else 1)
     d2h = w.N * w.d * 2
 
     # ---- max over ranks
@@ -432,7 +440,7 @@ def run_ours(args, w):
         value = weak_scaling_tokens_per_s(world, w.N, K, elapsed_ms)
         e2e_value = weak_scaling_tokens_per_s(world, w.N, E, e2e_ms)
         peaks = measured_peaks()
-        bytes_launch = algorithmic_bytes(w)
+        bytes_launch = algorithmic_bytes(w) + (w.N * 2 * w.d if args.variant == "token_gate" else 0)
         achieved = bytes_launch / (kern_ms / 1e3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -899,7 +907,7 @@ def main():
     ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
                     help="eager launches, or 100-step CUDA graphs (auto: graph for N <= 1024)")
     ap.add_argument("--variant", default="default",
-                    choices=["default", "dedup", "tma", "sort", "batch_order", "shard"],
+                    choices=["default", "dedup", "tma", "sort", "batch_order", "shard", "token_gate"],
                     help="HBM path: library default (grouped order from 16,384 tokens), dedup + "
                          "staged gather, TMA staging, always grouped, always batch order; shard: "
                          "the table split by columns over the ranks (strong scaling)")

@@ -3,10 +3,11 @@
 // k_gather_fp8 / k_gather_nvfp4, so the same bits).
 //
 // A lane holds one 8-column fragment per head in flight (16 B of bf16, 8 B of int8 / FP8,
-// 4 B of E2M1 codes + a block-scale byte), half of what the 16-column gathers of the
-// 8- and 4-bit formats hold, so a CTA needs fewer registers and more CTAs fit on an SM;
-// which of the two layouts is faster for a format is a measured choice (the build switch
-// NGRAM_C8_FORMATS, bit t for ngram_dtype t).
+// 4 B of E2M1 codes + a block-scale byte), half of what the 16-column gathers of the 8- and
+// 4-bit formats hold, so a CTA needs fewer registers and more CTAs fit on an SM.  Over a
+// whole table the 16-column gathers measured faster on B200 (the 8-bit and 4-bit decode
+// wants the longer fragment); this kernel serves the column-sharded table, where one
+// layout for every format keeps the shard widths simple.
 //
 // kShard: the table holds a column shard (columns col0 .. col0 + d - 1 of a wider table, as
 // the per-rank shards of the SGLang TP4 setup on "Qwen Brought Back N-Grams. All 51 Billion

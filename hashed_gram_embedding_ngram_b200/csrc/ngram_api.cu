@@ -33,13 +33,6 @@
 
 using namespace ngram;
 
-// Row formats (bit t = ngram_dtype t) whose gather runs k_gather_c8 (8 columns per lane)
-// instead of the format's 16-column kernel.
-#ifndef NGRAM_C8_FORMATS
-#define NGRAM_C8_FORMATS 0u
-#endif
-static bool use_c8(ngram_dtype t) { return t != NGRAM_BF16 && ((NGRAM_C8_FORMATS >> t) & 1u); }
-
 
 // Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
 //   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
@@ -404,7 +397,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.N = N;
     g.tok_begin = 0;
     g.d = c->d;
-    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16 || use_c8(c->dtype)) ? 8u : 16u;
+    const uint32_t cols_per_lane = (c->dtype == NGRAM_BF16) ? 8u : 16u;   // 16: 8- and 4-bit rows
     g.n_strips = (c->d / cols_per_lane + 31) / 32;
     g.strips_per_item = g.n_strips;
     g.groups_per_token = 1;
@@ -448,12 +441,6 @@ ngram_status launch_bulk(ngram_ctx *c, GatherArgs &g, cudaStream_t s) {
 }
 
 template <class Rows, bool kTok>
-void launch_c8(const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
-    if (g.h.n_heads == 16) k_gather_c8<16, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
-    else k_gather_c8<0, Rows, kTok><<<nb, 256, 0, s>>>(g, rb);
-}
-
-template <class Rows, bool kTok>
 void launch_c8_shard(const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
     if (g.h.n_heads == 16) k_gather_c8<16, Rows, kTok, true><<<nb, 256, 0, s>>>(g, rb);
     else k_gather_c8<0, Rows, kTok, true><<<nb, 256, 0, s>>>(g, rb);
@@ -472,15 +459,6 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 template <bool kTok>
 void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
     const bool h16 = g.h.n_heads == 16;
-    if (use_c8(t)) {
-        switch (t) {
-            case NGRAM_INT8_ROWSCALE: launch_c8<Rows8bit<Int8Codes>, kTok>(g, nb, s, rb); break;
-            case NGRAM_FP8_E4M3_ROWSCALE: launch_c8<Rows8bit<E4m3Codes>, kTok>(g, nb, s, rb); break;
-            case NGRAM_NVFP4: launch_c8<RowsNvfp4, kTok>(g, nb, s, rb); break;
-            default: break;
-        }
-        return;
-    }
     switch (t) {
         case NGRAM_BF16:
             if (h16) k_gather_bf16<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_bf16<0, kTok><<<nb, 256, 0, s>>>(g);
@@ -864,14 +842,7 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
     if (e == cudaSuccess) {
         int *bps = &c->gather_blocks_per_sm;
-        if (use_c8(dtype)) {
-            if (dtype == NGRAM_NVFP4)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, RowsNvfp4, false>, 256, 0);
-            else if (dtype == NGRAM_FP8_E4M3_ROWSCALE)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, Rows8bit<E4m3Codes>, false>, 256, 0);
-            else
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_c8<16, Rows8bit<Int8Codes>, false>, 256, 0);
-        } else switch (dtype) {
+        switch (dtype) {
             case NGRAM_BF16: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_bf16<16>, 256, 0); break;
             case NGRAM_INT8_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_int8<16>, 256, 0); break;
             case NGRAM_FP8_E4M3_ROWSCALE: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, k_gather_fp8<16>, 256, 0); break;
