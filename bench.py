@@ -346,6 +346,11 @@ def run_ours(args, w):
         ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b],
                          stream=s if s is not None else stream)
 
+    # ---- distinct rows of the first batch (outside any timed region): U * row bytes is the
+    # least a lookup of this batch can read from the table, whatever the order or reuse
+    _, ucount, _ = ng.ngram_dedup_rows(ctx, tok_d[0], history=hist_d[0])
+    unique_rows = int(ucount.item())
+
     # ---- device-resident timing.  Eager: one launch per step, CUDA events around each
     # launch.  Graph: G steps captured once into a CUDA graph and replayed, events around
     # each replay (decode-sized launches are otherwise bound by the Python launch path).
@@ -456,6 +461,8 @@ def run_ours(args, w):
                                     else ("grouped order (3 kernels) + " if grouped else "")
                                     + KERNEL_NAME[w.dtype]),
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
+                         "unique_rows": unique_rows,
+                         "unique_row_bytes": unique_rows * row_bytes(w),
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E,
@@ -471,11 +478,14 @@ def run_ours(args, w):
             inp = {"tokens": host_tok[0], "history": host_hist[0], "residual": res_bits,
                    "gate": gate_h}
             v, n, dt = oracle_tokens_per_s(w, inp, args.cpu_seconds, threads)
+            v1, n1, dt1 = oracle_tokens_per_s(w, inp, min(3.0, args.cpu_seconds / 4), 1, seed=1)
             line["cpu_baseline"] = {
                 "value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                 "sample": "%d of %d tokens of this workload, %.1f s, rows regenerated from "
                           "the synthetic-table definition (the 95 GiB table is not on the host)"
-                          % (n, w.N, dt)}
+                          % (n, w.N, dt),
+                "single_thread": {"value": v1, "unit": UNIT, "cores": 1,
+                                  "sample": "%d tokens, %.1f s" % (n1, dt1)}}
         print(json.dumps(line), flush=True)
     ctx.close()
     if world > 1:
