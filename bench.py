@@ -348,7 +348,7 @@ def run_ours(args, w):
 
     # ---- distinct rows of the first batch (outside any timed region): U * row bytes is the
     # least a lookup of this batch can read from the table, whatever the order or reuse
-    _, ucount, _ = ng.ngram_dedup_rows(ctx, tok_d[0], history=hist_d[0])
+    _, _, ucount = ng.ngram_dedup_rows(ctx, tok_d[0], history=hist_d[0])
     unique_rows = int(ucount.item())
 
     # ---- device-resident timing.  Eager: one launch per step, CUDA events around each

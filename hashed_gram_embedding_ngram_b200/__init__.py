@@ -23,4 +23,5 @@ from ._binding import (  # noqa: F401
     ngram_auto_choice, ngram_dedup_rows, ngram_prefetch, ngram_forward_staged, ngram_row_bytes,
     ngram_backward_rows, ngram_backward_gate, ngram_fill_synthetic_cols, ngram_forward_shard,
     ngram_device_alloc, ngram_device_free, ngram_ipc_get_handle, ngram_ipc_open, ngram_ipc_close,
+    ngram_selftest_wait_timeout,
 )

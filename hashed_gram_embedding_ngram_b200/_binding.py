@@ -118,6 +118,8 @@ _lib.ngram_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(_P)]
 _lib.ngram_ipc_open.restype = _i32
 _lib.ngram_ipc_close.argtypes = [_P]
 _lib.ngram_ipc_close.restype = _i32
+_lib.ngram_selftest_wait_timeout.argtypes = [_P, _u32, _P]
+_lib.ngram_selftest_wait_timeout.restype = _i32
 
 
 def lib() -> ctypes.CDLL:
@@ -545,3 +547,8 @@ def ngram_ipc_open(handle: bytes) -> int:
 
 def ngram_ipc_close(ptr: int) -> None:
     _check(_lib.ngram_ipc_close(ptr))
+
+
+def ngram_selftest_wait_timeout(ctx: Context, limit_ms: int = 100, stream=None) -> None:
+    """Run one bounded wait that nothing ends; it must give up and set error code 2."""
+    _check(_lib.ngram_selftest_wait_timeout(ctx.handle, limit_ms, _stream(stream)))

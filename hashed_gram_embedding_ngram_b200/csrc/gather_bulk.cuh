@@ -57,9 +57,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of bar, giving up after the deadline.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t deadline = global_ns() + kWaitLimitNs;
+    const uint64_t deadline = global_ns() + limit_ns;
     while (!mbar_try_wait(bar, parity))
         if (global_ns() > deadline) return false;
     return true;
@@ -74,6 +75,19 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
             smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
+}
+
+// The error path of the bounded waits, on demand: one mbarrier that expects one arrival
+// which never comes, waited on with mbar_wait_bounded.  The wait must give up after
+// limit_ns, set the device error word (code 2) and return; nothing else runs.
+__global__ void __launch_bounds__(32) k_selftest_wait(uint32_t *err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicCAS(err, 0u, 2u);
 }
 
 struct BulkPlan {

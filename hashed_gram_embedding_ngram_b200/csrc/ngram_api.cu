@@ -1382,6 +1382,14 @@ ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int3
     return NGRAM_OK;
 }
 
+ngram_status ngram_selftest_wait_timeout(ngram_ctx *c, uint32_t limit_ms, ngram_stream_t stream) {
+    if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
+    if (limit_ms == 0 || limit_ms > 2000) return fail(NGRAM_EINVAL, "limit_ms must be in [1, 2000]");
+    k_selftest_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->d_err, limit_ms * 1000000ull);
+    NG_CUDA(cudaGetLastError(), "k_selftest_wait launch");
+    return NGRAM_OK;
+}
+
 ngram_status ngram_get_device_error(ngram_ctx *c, uint32_t info[4], int clear) {
     if (c == nullptr) return fail(NGRAM_EINVAL, "ctx is NULL");
     uint32_t h[4] = {0, 0, 0, 0};

@@ -401,6 +401,14 @@ NGRAM_API ngram_status ngram_ipc_get_handle(const void *dev_ptr, uint8_t handle[
 NGRAM_API ngram_status ngram_ipc_open(const uint8_t handle[64], void **dev_ptr);
 NGRAM_API ngram_status ngram_ipc_close(void *dev_ptr);
 
+/* Self-test of the kernels' bounded waits: launches one wait that nothing ends (an
+ * mbarrier expecting an arrival that never comes), through the same bounded-wait code the
+ * TMA-staged gathers use, with a limit of limit_ms (1 .. 2000) instead of their 1 s.  The
+ * wait gives up, the kernel sets the context's device error word to code 2 (as a staged
+ * gather whose copies never land would) and returns; the context stays usable.  For tests
+ * of the failure path; nothing faults or hangs.  Asynchronous on stream. */
+NGRAM_API ngram_status ngram_selftest_wait_timeout(ngram_ctx *ctx, uint32_t limit_ms, ngram_stream_t stream);
+
 /* Synchronise the context's device, read and optionally clear its error word.
  * info (may be NULL) receives {code, flat position, bad id, 0}.  Code 1: a token id was
  * out of range (a position with bit 31 set names history entry (position & 0x7FFFFFFF)

@@ -139,6 +139,11 @@ def test_fill_rejects_bad_arguments():
         ng.ngram_fill_synthetic(_T, 10, 48, ng.NGRAM_NVFP4, row_scale=_T, stream=0)
 
 
+def test_selftest_rejects_bad_arguments():
+    lib = ng.lib()
+    assert lib.ngram_selftest_wait_timeout(None, 100, None) == ng.NGRAM_EINVAL
+
+
 def test_backward_entry_points_reject_a_null_context():
     lib = ng.lib()
     assert lib.ngram_backward_rows(None, None, None, 1, 1, None, None, None, None, None, None) == ng.NGRAM_EINVAL

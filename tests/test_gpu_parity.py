@@ -440,3 +440,23 @@ def test_sort_flag_ragged_heads(cuda_device):
     got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
     r = assert_parity(got, _oracle(w, inp, n_bigram=3, n_trigram=5))
     assert r["exact"] == r["n"]
+
+
+def test_device_wait_gives_up_and_context_survives(cuda_device):
+    """The kernels' bounded wait, on an mbarrier nothing completes (the path a TMA-staged
+    gather would take if its copies never landed): it gives up after the limit, sets device
+    error code 2, and the context keeps working afterwards."""
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    ref = from_dev_bf16(_run(w, cuda_device, dv, ctx))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    ng.ngram_selftest_wait_timeout(ctx, 100)
+    t1.record()
+    st, info = ng.ngram_get_device_error(ctx, clear=True)
+    assert st == ng.NGRAM_EDEVICE and info[0] == 2
+    assert 90.0 <= t0.elapsed_time(t1) < 1000.0            # it waited about the limit, then left
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK   # cleared
+    assert np.array_equal(from_dev_bf16(_run(w, cuda_device, dv, ctx)), ref)
