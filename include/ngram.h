@@ -98,9 +98,12 @@ typedef enum {
  * inverse map.  Same results bit for bit.  Staging (max_tokens * H rows) and the dedup
  * scratch are allocated by the first call that needs them. */
 #define NGRAM_FLAG_DEDUP 0x1u
-/* Stage the bf16 rows through shared memory with TMA bulk copies (cp.async.bulk into
- * an mbarrier ring) instead of register loads.  Same results bit for bit; measured
- * slower on B200 (522-895 us vs 455 us on the full-size gather), kept for comparison. */
+/* Stage the rows through shared memory with TMA bulk copies (cp.async.bulk into an
+ * mbarrier ring) instead of register loads: bf16 rows in column chunks, the 8- and 4-bit
+ * formats as whole rows (a producer warp copies, consumer warps decode; HBM residency).
+ * Same results bit for bit; measured slower on B200 (bf16 522-895 us vs 455 us on the
+ * full-size gather; NVFP4 52-76 M vs 121 M tokens/s), kept for comparison.  Every wait is
+ * bounded (1 s; then device error code 2).  Not with NGRAM_FLAG_TOKEN_GATE. */
 #define NGRAM_FLAG_TMA_STAGING 0x2u
 /* Grouped order: before the gather, group the batch's tokens by bigram context
  * (counting sort on a 13-bit hash of (w_{t-1}, w_t): 3 small kernels and a memset, ~11 us)

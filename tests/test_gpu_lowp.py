@@ -266,6 +266,12 @@ def test_host_residency_bitidentical(cuda_device, fmt):
                                   row_scale=hs.tensor)
                 for _ in range(2):
                     assert np.array_equal(from_dev_bf16(_fwd(c, dv)), ref), (where, flags)
+                if where == ng.NGRAM_RES_HOST_UVA and flags == 0:
+                    # the gate gradient reads the host rows through UVA: the HBM result
+                    dy = dv["residual"]
+                    g_hbm = ng.ngram_backward_gate(hbm, dv["tokens"], dy, history=dv["history"])
+                    g_uva = ng.ngram_backward_gate(c, dv["tokens"], dy, history=dv["history"])
+                    assert torch.equal(g_hbm, g_uva)
                 c.close()
     finally:
         TABLES.drop()

@@ -610,3 +610,20 @@ def test_forward_per_token_gate():
     E = _bits_to_f64(oracle.fill_bf16(3, 0, R, d)).reshape(R, d)
     want = _bits_to_f64(res).reshape(N, d) + _bits_to_f64(G).reshape(N, d) * _one_hot_sum(idx, E)
     assert np.array_equal(y, want)
+
+
+def test_hash_rows_are_uniform():
+    """Sanity, not parity: 100,000 random contexts x 16 heads land in R = 1009 rows
+    uniformly (chi-square with 1008 degrees of freedom, p > 1e-4), and the heads of one
+    context are independent of one another (pairwise equal rows at the 1/R rate)."""
+    from scipy import stats
+    R, V = 1009, 151_936
+    rng = np.random.default_rng(123)
+    toks = rng.integers(0, V, (1000, 100)).astype(np.int32)
+    hist = rng.integers(0, V, (1000, 2)).astype(np.int32)
+    idx = oracle.indices(toks, hist, R=R, vocab_size=V).reshape(-1, 16)
+    counts = np.bincount(idx.ravel(), minlength=R)
+    chi2, p = stats.chisquare(counts)
+    assert p > 1e-4, (chi2, p)
+    same = np.mean(idx[:, 0] == idx[:, 8])                 # a bigram and a trigram head
+    assert abs(same - 1.0 / R) < 5 * np.sqrt(1.0 / R / idx.shape[0])
