@@ -428,10 +428,11 @@ int oracle_indices(const int32_t *tokens, const int32_t *history, uint32_t n_seq
  * ---------------------------------------------------------------------------------- */
 /* Element (row, col) of the table: bf16 value v (s = 1, unused), or the pair (q, s)
  * with value q * s (int8: q the integer, s the row scale; fp8: q the E4M3 value, s the
- * row scale; nvfp4: q the E2M1 value, s = fp32(E4M3 block scale * global scale)).
- * Returns the exact value q * s in double.  For fp8 / nvfp4 a materialised table is
- * passed as table_i8 (bytes) and the scales as `scale` (fp8: per row; nvfp4: the global
- * scale at scale[0], block scales inside the row bytes). */
+ * row scale; nvfp4: q the E2M1 value, s the E4M3 block scale -- the global scale gs is
+ * applied to the head sum, see head_sum).  Returns the exact value q * s (* gs for nvfp4)
+ * in double.  For fp8 / nvfp4 a materialised table is passed as table_i8 (bytes) and the
+ * scales as `scale` (fp8: per row; nvfp4: the global scale at scale[0], block scales
+ * inside the row bytes). */
 static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
                         const float *scale, uint64_t seed, uint64_t row, uint32_t col,
                         uint32_t d, float *v_or_q, float *s_out)
@@ -456,10 +457,10 @@ static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *tab
             bs = oracle_block_scale_fp4(seed, row, col / 16);
         }
         gs = scale ? scale[0] : ORACLE_FP4_GLOBAL_SCALE;
-        cs = (float)oracle_e4m3_value(bs) * gs;             /* rounded to fp32 */
+        cs = (float)oracle_e4m3_value(bs);                  /* exact */
         *v_or_q = (float)oracle_e2m1_value(code);           /* exact */
         *s_out = cs;
-        return (double)*v_or_q * (double)cs;
+        return (double)*v_or_q * (double)cs * (double)gs;  /* exact in double */
     }
     if (dtype == ORACLE_BF16) {
         uint16_t b = table_bf16 ? table_bf16[row * d + col] : oracle_table_bf16(seed, row, col);
@@ -480,7 +481,9 @@ static double row_value(int dtype, const uint16_t *table_bf16, const int8_t *tab
  *   acc64 the exact sum (fp64; exact for these operands),
  *   acc32 the fp32 sum in head order: bf16 rows acc = acc + v; scaled rows
  *         acc = fmaf(q, s, acc), one rounding per head (int8, fp8, nvfp4 alike; q exact
- *         in fp32 in every case),
+ *         in fp32 in every case); for nvfp4 s is the E4M3 block scale (q * s exact) and
+ *         the table's fp32 global scale multiplies the sum once at the end,
+ *         acc32 = fp32(gs * acc32),
  *   mag   sum_h |E_h| (error-bound scale). */
 static void head_sum(int dtype, const uint16_t *table_bf16, const int8_t *table_i8,
                      const float *row_scale, uint64_t table_seed, const uint32_t *idx,
@@ -499,6 +502,10 @@ static void head_sum(int dtype, const uint16_t *table_bf16, const int8_t *table_
         else
             a32 = fmaf(v, sc, a32);
         m += fabs(e64);
+    }
+    if (dtype == ORACLE_NVFP4) {
+        const float gs = row_scale ? row_scale[0] : ORACLE_FP4_GLOBAL_SCALE;
+        a32 = gs * a32;                                     /* rounded once */
     }
     *acc32 = a32;
     *acc64 = a64;

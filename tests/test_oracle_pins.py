@@ -484,7 +484,8 @@ def test_low_precision_brute_force_and_fp32_mode(dtype):
         rows = oracle.fill_fp4(21, 0, R, d)
         codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(R, d)
         e2 = np.array([oracle.e2m1_value(c) for c in range(16)])
-        cs = np.array([[np.float32(np.float32(oracle.e4m3_value(int(b))) * np.float32(oracle.FP4_GLOBAL_SCALE))
+        # value = e2m1 * e4m3(block scale) * global scale, exactly (the sum is scaled once)
+        cs = np.array([[oracle.e4m3_value(int(b)) * float(oracle.FP4_GLOBAL_SCALE)
                         for b in r[d // 2:d // 2 + d // 16]] for r in rows], dtype=np.float64)
         E = e2[codes] * np.repeat(cs, 16, axis=1)
         tab, sc = rows, np.array([oracle.FP4_GLOBAL_SCALE], dtype=np.float32)
@@ -627,3 +628,32 @@ def test_hash_rows_are_uniform():
     assert p > 1e-4, (chi2, p)
     same = np.mean(idx[:, 0] == idx[:, 8])                 # a bigram and a trigram head
     assert abs(same - 1.0 / R) < 5 * np.sqrt(1.0 / R / idx.shape[0])
+
+
+
+def test_nvfp4_fp32_mode_scales_the_head_sum_once():
+    """NVFP4 in fp32 mode: each head adds q * block scale (exact) with one rounding, and the
+    global scale multiplies the sum once.  With gs = 1, r = 0, g = 1 the output is the
+    bf16 of the fp32 fma chain over exact products; with gs = 2^k it is that times 2^k."""
+    R, d, V = 61, 32, 40
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    N = toks.size
+    rows = oracle.fill_fp4(9, 0, R, d)
+    idx = oracle.indices(toks, None, R=R, vocab_size=V).reshape(N, 16)
+    codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(R, d)
+    e2 = np.array([oracle.e2m1_value(c) for c in range(16)], dtype=np.float32)
+    bsv = np.array([[oracle.e4m3_value(int(b)) for b in r[d // 2:d // 2 + d // 16]] for r in rows],
+                   dtype=np.float32)
+    zero = np.zeros(N * d, dtype=np.uint16)
+    one = np.ones(d, dtype=np.float32)
+    for gs in (1.0, 0.25):
+        acc = np.zeros((N, d), dtype=np.float32)
+        for h in range(16):                  # fp32 fma chain: q * s exact, one rounding each
+            q = e2[codes[idx[:, h]]].astype(np.float64)
+            sc = np.repeat(bsv[idx[:, h]], 16, axis=1).astype(np.float64)
+            acc = (q * sc + acc.astype(np.float64)).astype(np.float32)
+        y = torch.from_numpy((np.float32(gs) * acc).ravel())           # fp32 multiply, rounded once
+        want = y.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        got = oracle.forward(toks, None, zero, one, R=R, d=d, dtype=oracle.NVFP4, table_i8=rows,
+                             row_scale=np.array([gs], np.float32), acc=oracle.ACC_F32, vocab_size=V)
+        assert np.array_equal(got.ravel(), want)
