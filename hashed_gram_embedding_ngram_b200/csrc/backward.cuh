@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(256, 2) k_gate_grad(const GatherArgs g, const 
 #pragma unroll
             for (int h = 0; h < 16; ++h)
                 if (kH || h < static_cast<int>(H)) Rows::add(acc, f[h], sc[h], gs);
+            Rows::finish(acc, gs);
             const float dv[8] = {bf16_lo(dw.x), bf16_hi(dw.x), bf16_lo(dw.y), bf16_hi(dw.y),
                                  bf16_lo(dw.z), bf16_hi(dw.z), bf16_lo(dw.w), bf16_hi(dw.w)};
             const float ev[8] = {acc[0].x, acc[0].y, acc[1].x, acc[1].y,

@@ -213,26 +213,30 @@ __device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float2 &c01, float2 
     c23 = half2_bits_to_float2(h23);
 }
 
-// One E4M3 code (the low byte of b) -> fp32.
-__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-    float f;
-    asm("{\n\t.reg .b16 x, lo, hi;\n\t.reg .b32 h;\n\tcvt.u16.u32 x, %1;\n\t"
-        "cvt.rn.f16x2.e4m3x2 h, x;\n\tmov.b32 {lo, hi}, h;\n\tcvt.f32.f16 %0, lo;\n\t}"
-        : "=f"(f) : "r"(b & 0xFFu));
-    return f;
+// One E4M3 code (the low byte of b) -> its f16 bits (exact), in the low 16 bits.
+__device__ __forceinline__ uint32_t e4m3_to_half_bits(uint32_t b) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 x, lo, hi;\n\t.reg .b32 t;\n\tcvt.u16.u32 x, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 t, x;\n\tmov.b32 {lo, hi}, t;\n\tcvt.u32.u16 %0, lo;\n\t}"
+        : "=r"(h) : "r"(b & 0xFFu));
+    return h;
 }
 
-// Eight E2M1 codes (nibble k = column k) -> columns (0, 1), (2, 3), (4, 5), (6, 7).
-__device__ __forceinline__ void e2m1x8_to_float(uint32_t w, float2 c[4]) {
+// Eight E2M1 codes (nibble k = column k), each times the f16 value s, added to fp32
+// accumulators: acc[j] (columns 2j, 2j+1) += q * s with one rounding (fma.rn.f32.f16: the
+// f16 operands enter exactly, q * s is exact for E2M1 x E4M3).
+__device__ __forceinline__ void e2m1x8_fma(uint32_t w, uint32_t s_half, float2 acc[4]) {
     uint32_t h0, h1, h2, h3;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
         "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
         "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
         : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3) : "r"(w));
-    c[0] = half2_bits_to_float2(h0);
-    c[1] = half2_bits_to_float2(h1);
-    c[2] = half2_bits_to_float2(h2);
-    c[3] = half2_bits_to_float2(h3);
+    const uint32_t hh[4] = {h0, h1, h2, h3};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        asm("{\n\t.reg .b16 lo, hi, s, u;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {s, u}, %3;\n\t"
+            "fma.rn.f32.f16 %0, lo, s, %0;\n\tfma.rn.f32.f16 %1, hi, s, %1;\n\t}"
+            : "+f"(acc[j].x), "+f"(acc[j].y) : "r"(hh[j]), "r"(s_half));
 }
 
 }  // namespace ngram

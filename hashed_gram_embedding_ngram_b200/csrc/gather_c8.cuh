@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256, NGRAM_C8_MIN_BLOCKS) k_gather_c8(const Ga
 #pragma unroll
             for (int h = 0; h < 16; ++h)
                 if (kH || h < static_cast<int>(H)) Rows::add(acc, f[h], sc[h], gs);
+            Rows::finish(acc, gs);
             float gv[8];
             load_gate8<kTokGate>(g, tok_off, v, gv);
             // y = r + (g * acc): the product is rounded on its own (scalar, never fused)

@@ -5,8 +5,10 @@
 // Heterogeneous Memory Prefetch" (its architecture figure: 51B parameters, ~25.5 GB at
 // FP4; "Qwen3.8-Flash-Next: A 125B MoE for the Local Stack?", section "Hardware math for
 // self-hosting", weighs 4-bit n-gram tables too).  Same operation as k_gather_bf16, with
-// row value  q * cs,  q the E2M1 value of the code and cs = fp32(E4M3 block scale *
-// global scale), summed per head in order with one fused multiply-add per head.
+// row value  q * bs * gs,  q the E2M1 value of the code, bs its E4M3 block scale and gs the
+// table's fp32 global scale: per head in order acc = fma(q, bs, acc) -- both as f16 into
+// one fp32 fma (fma.rn.f32.f16), q * bs exact, one rounding -- and the global scale
+// multiplies the sum once, e = fp32(gs * acc).
 //
 // Row layout (rb = d/2 + ceil16(d/16) bytes, a multiple of 16 for d % 32 == 0): d/2 code
 // bytes, column 2j in the low nibble of byte j; then d/16 block-scale bytes; then zero
@@ -69,17 +71,14 @@ __global__ void __launch_bounds__(256, NGRAM_NVFP4_MIN_BLOCKS) k_gather_nvfp4(co
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
                 if (kH || h < static_cast<int>(H)) {
-                    const float cs = __fmul_rn(e4m3_to_float(bs[h]), gs);
-                    const float2 s2 = make_float2(cs, cs);
-                    float2 q[4];
-                    e2m1x8_to_float(e[h].x, q);           // columns 0..7
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) acc[k] = fma2(q[k], s2, acc[k]);
-                    e2m1x8_to_float(e[h].y, q);           // columns 8..15
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) acc[4 + k] = fma2(q[k], s2, acc[4 + k]);
+                    const uint32_t s16 = e4m3_to_half_bits(bs[h]);
+                    e2m1x8_fma(e[h].x, s16, acc);         // columns 0..7
+                    e2m1x8_fma(e[h].y, s16, acc + 4);     // columns 8..15
                 }
             }
+            const float2 g2 = make_float2(gs, gs);       // the global scale, once per sum
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = mul2(acc[k], g2);
             store_gated16<kTokGate>(g, tok_off, v, r0, r1, acc);
         }
     }

@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(352, NGRAM_STAGED_MIN_BLOCKS) k_gather_staged(
                 for (int h = 0; h < 16; ++h)
                     if (kH || h < static_cast<int>(H))
                         Rows::add(acc, Rows::load_smem(base + h * plan.row_bytes, v, g.d), sc[h], gs);
+                Rows::finish(acc, gs);
                 const uint4 r = *reinterpret_cast<const uint4 *>(base + plan.res_off + v * 16u);
                 float gv[8];
                 load_gate8<false>(g, tok_off, v, gv);

@@ -2,9 +2,10 @@
 // columns 8v .. 8v+7, and add their values to fp32 accumulators in head order.
 //
 // Each policy decodes and accumulates exactly as the format's own gather does (bf16:
-// acc = acc + v; int8 / FP8: acc = fma(q, s_row, acc); NVFP4: acc = fma(q, cs, acc) with
-// cs = fp32(e4m3(block scale) * global scale)), so every kernel built on them computes
-// the head sum bit for bit as the forward does.  Formats: "Qwen Brought Back N-Grams. All
+// acc = acc + v; int8 / FP8: acc = fma(q, s_row, acc); NVFP4: acc = fma(q, block scale,
+// acc), then finish() multiplies the sum by the global scale once), so every kernel built
+// on them -- add() for each head in order, then finish() -- computes the head sum bit for
+// bit as the forward does.  Formats: "Qwen Brought Back N-Grams. All
 // 51 Billion Parameters of Them." (bf16 table, section "N-grams, of all things");
 // "Qwen3.8-Flash-Next: A 51B N-gram Embedding Table with Heterogeneous Memory Prefetch"
 // (INT8, Key point 3; FP4, architecture figure); "Qwen3.8-Flash-Next: A 125B MoE for the
@@ -37,6 +38,7 @@ struct RowsBf16 {
         acc[2] = add2(acc[2], bf16x2(f.z));
         acc[3] = add2(acc[3], bf16x2(f.w));
     }
+    static __device__ __forceinline__ void finish(float2 (&)[4], float) {}
 };
 
 template <class Codes>
@@ -59,6 +61,7 @@ struct Rows8bit {                       // int8 / FP8 E4M3 codes with a per-row 
         acc[2] = fma2(lo, s2, acc[2]);
         acc[3] = fma2(hi, s2, acc[3]);
     }
+    static __device__ __forceinline__ void finish(float2 (&)[4], float) {}
 };
 
 struct RowsNvfp4 {                      // E2M1 codes, E4M3 block scale, global scale gs
@@ -72,13 +75,13 @@ struct RowsNvfp4 {                      // E2M1 codes, E4M3 block scale, global 
     static __device__ __forceinline__ Frag load_smem(const uint8_t *row, uint32_t v, uint32_t d) {
         return Frag{*reinterpret_cast<const uint32_t *>(row + v * 4u), row[(d >> 1) + (v >> 1)]};
     }
-    static __device__ __forceinline__ void add(float2 (&acc)[4], const Frag &f, float, float gs) {
-        const float cs = __fmul_rn(e4m3_to_float(f.bs), gs);
-        const float2 s2 = make_float2(cs, cs);
-        float2 q[4];
-        e2m1x8_to_float(f.codes, q);
+    static __device__ __forceinline__ void add(float2 (&acc)[4], const Frag &f, float, float) {
+        e2m1x8_fma(f.codes, e4m3_to_half_bits(f.bs), acc);      // acc += q * bs, one rounding
+    }
+    static __device__ __forceinline__ void finish(float2 (&acc)[4], float gs) {
+        const float2 g2 = make_float2(gs, gs);                    // the global scale, once
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = fma2(q[k], s2, acc[k]);
+        for (int k = 0; k < 4; ++k) acc[k] = mul2(acc[k], g2);
     }
 };
 

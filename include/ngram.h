@@ -83,7 +83,10 @@ typedef enum {
                                   2, 3, 4, 6; column 2j in the low nibble of byte j), then one
                                   E4M3 scale byte per 16 columns, then zero padding to rb.
                                   row_scale points at ONE fp32 global scale gs.  value =
-                                  e2m1(q) * cs, cs = fp32(e4m3(block scale) * gs); d % 32 == 0 */
+                                  e2m1(q) * e4m3(block scale) * gs.  In the sum, each head
+                                  adds e2m1(q) * e4m3(bs) (exact) to an fp32 accumulator with
+                                  one rounding, and gs multiplies the 16-head sum once, in
+                                  fp32; d % 32 == 0 */
 } ngram_dtype;
 
 typedef enum {
