@@ -111,6 +111,26 @@ def read_stream_gbs(dev, nbytes=4 << 30, reps=5) -> float:
     return nbytes / (best / 1e3) / 1e9
 
 
+def write_stream_gbs(dev, nbytes=4 << 30, reps=5) -> float:
+    """A write-only HBM stream measured in this run (outside every timed region): the best
+    of `reps` fills of nbytes of int32 -- the denominator for kernels that mostly write."""
+    import torch
+    x = torch.empty(nbytes // 4, dtype=torch.int32, device=dev)
+    best = float("inf")
+    for i in range(reps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        x.fill_(i)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            best = min(best, e0.elapsed_time(e1))
+    del x
+    torch.cuda.empty_cache()
+    return nbytes / (best / 1e3) / 1e9
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -648,6 +668,7 @@ def run_host(args):
     gemm_ms = a.elapsed_time(b) / 200
     report = {}
     modes = {"uva": (ng.NGRAM_RES_HOST_UVA, 0), "uva_grouped": (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT),
+             "uva_dedup": (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP),
              "dma": (ng.NGRAM_RES_HOST_DMA, 0), "auto": (ng.NGRAM_RES_HOST_AUTO, 0)}
     for name in names:
         w = gen.WORKLOADS[name]
@@ -667,6 +688,9 @@ def run_host(args):
             for _ in range(3):
                 ng.ngram_forward(ctx, tok, res, gate, out=out, history=hist, stream=main_s)
             torch.cuda.synchronize()
+            # host-blocking modes count wall time: DMA, and AUTO once it has picked DMA
+            blocking = mname == "dma" or (where == ng.NGRAM_RES_HOST_AUTO and
+                                          ng.ngram_auto_choice(ctx, w.N) == ng.NGRAM_RES_HOST_DMA)
             got = out.clone()
             if ref is None:
                 ref = got
@@ -679,7 +703,7 @@ def run_host(args):
             e1.record(main_s)
             torch.cuda.synchronize()
             wall = (time.perf_counter() - w0) * 1e3 / K
-            ms = max(e0.elapsed_time(e1) / K, wall if mname in ("dma", "auto") else 0.0)
+            ms = max(e0.elapsed_time(e1) / K, wall if blocking else 0.0)
             # overlapped with the GEMM stand-in on the side stream
             n_gemm = max(1, int(ms * K / gemm_ms))
             ga, gb = time_gemms(n_gemm)
@@ -700,7 +724,8 @@ def run_host(args):
                 "bit_identical_to_uva": same, "device_error": st,
             }
             if where == ng.NGRAM_RES_HOST_AUTO:
-                entry[mname]["choice"] = {ng.NGRAM_RES_HOST_UVA: "uva", ng.NGRAM_RES_HOST_DMA: "dma"}.get(
+                entry[mname]["choice"] = {ng.NGRAM_RES_HOST_UVA: "uva", ng.NGRAM_RES_HOST_DMA: "dma",
+                                          ng.NGRAM_AUTO_UVA_DEDUP: "uva_dedup"}.get(
                     ng.ngram_auto_choice(ctx, w.N), "undecided")
             ctx.close()
         entry["prefetch"] = prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B)
@@ -906,6 +931,10 @@ def run_backward(args, w):
     # written; gate gradient = the forward's row reads + dy read (+ fp64 partials)
     rows_bytes = N * 2 * d + U * 4 * d + 4 * d
     gate_bytes = N * (HEADS * row_bytes(w) + 2 * d + 4) + 2 * 8 * d * ((N + 15) // 16) + 4 * d
+    # the table gradient mostly writes: its stream bound is the gradient rows at the
+    # measured write stream plus dy at the measured read stream
+    wr_gbs, rd_gbs = write_stream_gbs(dev), read_stream_gbs(dev)
+    rows_bound_ms = (U * 4 * d / wr_gbs + N * 2 * d / rd_gbs) / 1e6
     line = {
         "metric": "n-gram embed backward tokens/s (table + gate gradients), 1 B200",
         "value": N / (step_ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": args.warmup,
@@ -914,6 +943,8 @@ def run_backward(args, w):
         "backward_rows": {"ms": rows_ms, "algorithmic_bytes": rows_bytes,
                           "achieved_gbs": rows_bytes / rows_ms / 1e6,
                           "frac": rows_bytes / rows_ms / 1e6 / peaks["hbm_gbs"],
+                          "stream_bound_ms": rows_bound_ms, "frac_of_stream_bound": rows_bound_ms / rows_ms,
+                          "write_stream_gbs": wr_gbs, "read_stream_gbs": rd_gbs,
                           "kernels": "hash, dedup (5), radix sort (%d passes x 5), segments, k_rows_grad"
                                      % ((max(1, (N * H - 1).bit_length()) + 7) // 8)},
         "backward_gate": {"ms": gate_ms, "algorithmic_bytes": gate_bytes,

@@ -15,7 +15,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH, Context, HashParams, NgramError, lib,
     NGRAM_OK, NGRAM_EINVAL, NGRAM_ENOMEM, NGRAM_ECUDA, NGRAM_EUNSUPPORTED, NGRAM_ETIMEOUT,
     NGRAM_EDEVICE, NGRAM_BF16, NGRAM_INT8_ROWSCALE, NGRAM_FP8_E4M3_ROWSCALE, NGRAM_NVFP4, NGRAM_RES_HBM, NGRAM_RES_HOST_UVA,
-    NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO, NGRAM_FLAG_DEDUP, NGRAM_FLAG_TMA_STAGING, NGRAM_FLAG_SORT, NGRAM_FLAG_BATCH_ORDER, NGRAM_FLAG_TOKEN_GATE, NGRAM_SORT_MIN_TOKENS,
+    NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO, NGRAM_AUTO_UVA_DEDUP, NGRAM_FLAG_DEDUP, NGRAM_FLAG_TMA_STAGING, NGRAM_FLAG_SORT, NGRAM_FLAG_BATCH_ORDER, NGRAM_FLAG_TOKEN_GATE, NGRAM_SORT_MIN_TOKENS,
     NGRAM_STAGE_SLOTS, MAX_HEADS, DEFAULT_BASE_SEED, DEFAULT_PAD_ID,
     ngram_default_hash_params, ngram_init, ngram_forward, ngram_forward_host, ngram_hash_indices,
     ngram_fill_synthetic, ngram_get_device_error, ngram_last_error, ngram_status_string,

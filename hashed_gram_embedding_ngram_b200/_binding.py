@@ -30,6 +30,7 @@ NGRAM_EUNSUPPORTED, NGRAM_ETIMEOUT, NGRAM_EDEVICE = 4, 5, 6
 NGRAM_BF16, NGRAM_INT8_ROWSCALE, NGRAM_FP8_E4M3_ROWSCALE, NGRAM_NVFP4 = 0, 1, 2, 3
 # ngram_residency
 NGRAM_RES_HBM, NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA, NGRAM_RES_HOST_AUTO = 0, 1, 2, 3
+NGRAM_AUTO_UVA_DEDUP = 4      # ngram_auto_choice: HOST_UVA with NGRAM_FLAG_DEDUP
 
 NGRAM_FLAG_DEDUP = 0x1
 NGRAM_FLAG_TMA_STAGING = 0x2

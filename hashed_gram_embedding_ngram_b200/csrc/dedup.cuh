@@ -143,8 +143,14 @@ __global__ void __launch_bounds__(256) k_dedup_inverse(const uint32_t *__restric
         inv[i] = uid[slot_of[i]];
 }
 
-// Copy the U unique rows (and int8 row scales) of the table into a dense staging
-// buffer, one warp per row, 16-byte vectors.
+// Copy the U unique rows (and per-row scales) of the table into a dense staging buffer.
+// The copy is flat over the U * nv 16-byte vectors (vector f = row u, column vector v):
+// a warp owns 512 consecutive vectors at a time and a lane issues its 16 loads before its
+// first store, so every warp keeps 8 KB in flight whatever the row width.  Read from host
+// memory over PCIe, the link's throughput follows the bytes in flight (the latency grows
+// with the queue), so a few CTAs reach the link's rate only with this depth.
+constexpr uint32_t kCompactBatch = 16;
+
 __global__ void __launch_bounds__(256) k_compact_rows(const uint8_t *__restrict__ table,
                                                       const float *__restrict__ row_scale,
                                                       const uint32_t *__restrict__ uniq,
@@ -154,13 +160,32 @@ __global__ void __launch_bounds__(256) k_compact_rows(const uint8_t *__restrict_
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t U = *count;
     const uint32_t nv = row_bytes >> 4;
-    for (uint32_t u = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U;
-         u += (gridDim.x * blockDim.x) >> 5) {
-        const uint32_t r = uniq[u];
-        const uint4 *src = reinterpret_cast<const uint4 *>(table + static_cast<size_t>(r) * row_bytes);
-        uint4 *dst = reinterpret_cast<uint4 *>(stage + static_cast<size_t>(u) * row_bytes);
-        for (uint32_t v = lane; v < nv; v += 32u) dst[v] = ld_stream_v4(src + v);
-        if (lane == 0 && row_scale != nullptr) stage_scale[u] = row_scale[r];
+    const uint64_t total = static_cast<uint64_t>(U) * nv;
+    const uint64_t warp = (static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const uint64_t n_warps = (static_cast<uint64_t>(gridDim.x) * blockDim.x) >> 5;
+    uint4 *dst = reinterpret_cast<uint4 *>(stage);
+    for (uint64_t base = warp * 32u * kCompactBatch; base < total; base += n_warps * 32u * kCompactBatch) {
+        uint4 x[kCompactBatch];
+#pragma unroll
+        for (uint32_t j = 0; j < kCompactBatch; ++j) {
+            const uint64_t f = base + 32u * j + lane;
+            if (f < total) {
+                // 32-bit division whenever the vector index fits (every batch up to 2^32 vectors)
+                const uint32_t u = (total >> 32) ? static_cast<uint32_t>(f / nv)
+                                                 : static_cast<uint32_t>(f) / nv;
+                const uint32_t v = static_cast<uint32_t>(f - static_cast<uint64_t>(u) * nv);
+                x[j] = ld_stream_v4(table + static_cast<size_t>(uniq[u]) * row_bytes + 16u * v);
+            }
+        }
+#pragma unroll
+        for (uint32_t j = 0; j < kCompactBatch; ++j) {
+            const uint64_t f = base + 32u * j + lane;
+            if (f < total) dst[f] = x[j];
+        }
+    }
+    if (row_scale != nullptr) {
+        for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < U; u += gridDim.x * blockDim.x)
+            stage_scale[u] = row_scale[uniq[u]];
     }
 }
 

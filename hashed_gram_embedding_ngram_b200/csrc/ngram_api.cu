@@ -117,7 +117,8 @@ struct ngram_ctx {
     cudaEvent_t ev_stage_free;  // last H2D of the previous DMA call
     int stage_in_use;
     cudaEvent_t ev_t0, ev_t1;   // AUTO timing
-    int auto_choice[33];        // per ceil(log2 N): 0 undecided, else ngram_residency
+    int auto_choice[33];        // per ceil(log2 N): 0 undecided, else HOST_UVA, HOST_DMA or
+                                // NGRAM_AUTO_UVA_DEDUP
     // ngram_forward_host: device copies of the host inputs, double-buffered chunks
     int32_t *hp_tok, *hp_hist;
     uint16_t *hp_res[NGRAM_HOST_BUFFERS], *hp_out[NGRAM_HOST_BUFFERS];
@@ -592,13 +593,15 @@ ngram_status forward_direct(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
 }
 
 // hash -> dedup -> compact the unique rows into HBM staging -> gather from staging.
-ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
+// compact_grid: CTAs of the copy kernel (a full grid from HBM; NGRAM_UVA_CTAS from host
+// memory, where each distinct row then crosses PCIe once).
+ngram_status forward_dedup(ngram_ctx *c, const Call &k, unsigned compact_grid) {
     NG_CHECK(ensure_dedup_scratch(c));
     NG_CHECK(ensure_device_stage(c));
     const uint32_t M = k.N * c->H;
     NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
     NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
-    k_compact_rows<<<grid_for(c, M * 32ull, 256), 256, 0, k.s>>>(
+    k_compact_rows<<<compact_grid, 256, 0, k.s>>>(
         static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c), c->d_uniq, c->d_count,
         c->row_bytes, c->d_stage, c->d_stage_scale);
     NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
@@ -697,28 +700,51 @@ ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
     return launch_gather(c, g, k.s, max_blocks);
 }
 
-ngram_status forward_uva(ngram_ctx *c, const Call &k) {
+ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
+    return forward_dedup(c, k, grid_for(c, static_cast<uint64_t>(k.N) * c->H * 32ull, 256));
+}
+
+// UVA with dedup: each distinct row crosses PCIe once, read by the copy kernel.
+ngram_status forward_dedup_uva(ngram_ctx *c, const Call &k) {
+    return forward_dedup(c, k, static_cast<unsigned>(std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c))));
+}
+
+// UVA without dedup: the gather kernel reads the host rows itself, on a bounded grid.
+ngram_status forward_direct_uva(ngram_ctx *c, const Call &k) {
     const uint64_t blocks = std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c));
     if (c->hp.flags & NGRAM_FLAG_SORT) return forward_sorted(c, k, blocks);
     return forward_direct(c, k, blocks);
 }
 
-// AUTO: the first call of each batch-size bucket runs and times both host modes
-// (both write the same output), keeps the faster, and later calls use it.
+ngram_status forward_uva(ngram_ctx *c, const Call &k) {
+    if (c->hp.flags & NGRAM_FLAG_DEDUP) return forward_dedup_uva(c, k);
+    return forward_direct_uva(c, k);
+}
+
+// AUTO: the first call of each batch-size bucket runs and times the three host modes
+// (UVA, UVA with dedup, DMA; all write the same output), keeps the fastest, and later
+// calls use it.  auto_choice holds NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA or
+// NGRAM_AUTO_UVA_DEDUP.
 ngram_status forward_auto(ngram_ctx *c, const Call &k) {
     const uint32_t b = ceil_log2(k.N);
-    if (c->auto_choice[b] == NGRAM_RES_HOST_UVA) return forward_uva(c, k);
+    if (c->auto_choice[b] == NGRAM_RES_HOST_UVA) return forward_direct_uva(c, k);
+    if (c->auto_choice[b] == NGRAM_AUTO_UVA_DEDUP) return forward_dedup_uva(c, k);
     if (c->auto_choice[b] == NGRAM_RES_HOST_DMA) return forward_dma(c, k);
     if (!c->ev_t0) {
         NG_CUDA(cudaEventCreate(&c->ev_t0), "cudaEventCreate");
         NG_CUDA(cudaEventCreate(&c->ev_t1), "cudaEventCreate");
     }
-    float t_uva = 0.f, t_dma = 0.f;
+    float t_uva = 0.f, t_dedup = 0.f, t_dma = 0.f;
     NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
-    NG_CHECK(forward_uva(c, k));
+    NG_CHECK(forward_direct_uva(c, k));
     NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
     NG_CHECK(wait_event(c, c->ev_t1, "AUTO: UVA timing"));
     NG_CUDA(cudaEventElapsedTime(&t_uva, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
+    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
+    NG_CHECK(forward_dedup_uva(c, k));
+    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
+    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: UVA dedup timing"));
+    NG_CUDA(cudaEventElapsedTime(&t_dedup, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
     const auto h0 = std::chrono::steady_clock::now();
     NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
     NG_CHECK(forward_dma(c, k));
@@ -729,7 +755,11 @@ ngram_status forward_auto(ngram_ctx *c, const Call &k) {
         std::chrono::duration<float, std::milli>(std::chrono::steady_clock::now() - h0).count();
     NG_CUDA(cudaEventElapsedTime(&t_dma, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
     t_dma = std::max(t_dma, wall);
-    c->auto_choice[b] = (t_dma < t_uva) ? NGRAM_RES_HOST_DMA : NGRAM_RES_HOST_UVA;
+    int best = NGRAM_RES_HOST_UVA;
+    float t_best = t_uva;
+    if (t_dedup < t_best) { best = NGRAM_AUTO_UVA_DEDUP; t_best = t_dedup; }
+    if (t_dma < t_best) best = NGRAM_RES_HOST_DMA;
+    c->auto_choice[b] = best;
     return NGRAM_OK;
 }
 
@@ -807,8 +837,8 @@ ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_sca
     if (static_cast<uint64_t>(max_tokens) * n_strips > 0xFFFFFFFFull ||
         static_cast<uint64_t>(max_tokens) * NGRAM_MAX_HEADS > (1ull << 30))
         return fail(NGRAM_EINVAL, "max_tokens %u too large for d = %u", max_tokens, d);
-    if ((p.flags & NGRAM_FLAG_DEDUP) && where != NGRAM_RES_HBM)
-        return fail(NGRAM_EINVAL, "NGRAM_FLAG_DEDUP applies to HBM residency (host modes dedup on their own)");
+    if ((p.flags & NGRAM_FLAG_DEDUP) && where != NGRAM_RES_HBM && where != NGRAM_RES_HOST_UVA)
+        return fail(NGRAM_EINVAL, "NGRAM_FLAG_DEDUP applies to HBM and HOST_UVA residency (DMA always dedups, AUTO tries both)");
     if ((p.flags & NGRAM_FLAG_SORT) && where != NGRAM_RES_HBM && where != NGRAM_RES_HOST_UVA)
         return fail(NGRAM_EINVAL, "NGRAM_FLAG_SORT applies to HBM and HOST_UVA residency");
     if ((p.flags & NGRAM_FLAG_SORT) &&

@@ -93,13 +93,19 @@ typedef enum {
     NGRAM_RES_HBM = 0,         /* table in this GPU's memory */
     NGRAM_RES_HOST_UVA = 1,    /* table in pinned host memory, read by the kernel over PCIe */
     NGRAM_RES_HOST_DMA = 2,    /* table in pinned host memory, rows staged by copy engine */
-    NGRAM_RES_HOST_AUTO = 3    /* host-resident; the faster of UVA / DMA, chosen by timing */
+    NGRAM_RES_HOST_AUTO = 3    /* host-resident; the fastest of UVA / UVA with dedup / DMA,
+                                  chosen by timing */
 } ngram_residency;
 
-/* HBM residency only: dedup the batch's rows first (ngram_dedup_rows), copy each
+/* ngram_auto_choice's value for HOST_UVA with NGRAM_FLAG_DEDUP (not a residency). */
+#define NGRAM_AUTO_UVA_DEDUP 4
+
+/* HBM or HOST_UVA residency: dedup the batch's rows first (ngram_dedup_rows), copy each
  * distinct row once into an HBM staging buffer, and gather from staging through the
- * inverse map.  Same results bit for bit.  Staging (max_tokens * H rows) and the dedup
- * scratch are allocated by the first call that needs them. */
+ * inverse map.  Same results bit for bit.  With HOST_UVA the copy kernel reads each
+ * distinct row once over PCIe (a few CTAs), where the plain UVA gather reads every
+ * occurrence.  Staging (max_tokens * H rows in HBM) and the dedup scratch are allocated by
+ * the first call that needs them. */
 #define NGRAM_FLAG_DEDUP 0x1u
 /* Stage the rows through shared memory with TMA bulk copies (cp.async.bulk into an
  * mbarrier ring) instead of register loads: bf16 rows in column chunks, the 8- and 4-bit
@@ -182,8 +188,9 @@ NGRAM_API ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *
  *                        from HBM; the call blocks the host until the rows are staged
  *                        (bounded wait, see ngram_set_wait_timeout);
  *              HOST_AUTO the first call of each batch-size bucket (ceil(log2 N)) runs
- *                        and times both UVA and DMA (synchronously), later calls use
- *                        the faster (ngram_auto_choice reports it).
+ *                        and times UVA, UVA with dedup (NGRAM_FLAG_DEDUP) and DMA
+ *                        (synchronously); later calls use the fastest
+ *                        (ngram_auto_choice reports it).
  *   hp         hash parameters (NULL = defaults).
  *   max_tokens largest n_seq * T a later call may pass (>= 1).
  * The context owns a 16-byte device error word; dedup scratch and staging buffers are
@@ -274,7 +281,8 @@ NGRAM_API ngram_status ngram_backward_gate(ngram_ctx *ctx, const int32_t *tokens
 NGRAM_API ngram_status ngram_set_wait_timeout(ngram_ctx *ctx, uint32_t ms);
 
 /* Residency HOST_AUTO picked for batches of n_tokens (its ceil(log2) bucket):
- * NGRAM_RES_HOST_UVA or NGRAM_RES_HOST_DMA, or -1 while undecided. */
+ * NGRAM_RES_HOST_UVA, NGRAM_AUTO_UVA_DEDUP or NGRAM_RES_HOST_DMA, or -1 while
+ * undecided. */
 NGRAM_API ngram_status ngram_auto_choice(const ngram_ctx *ctx, uint32_t n_tokens, int *where_out);
 
 /* Per-batch row dedup (the optional dedup step): with idx the [N][H] row indices of

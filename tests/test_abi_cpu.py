@@ -170,11 +170,12 @@ def test_new_entry_points_reject_bad_arguments():
     assert lib.ngram_host_free(None) == ng.NGRAM_OK
 
 
-def test_dedup_flag_is_for_hbm_only():
+def test_dedup_flag_is_for_hbm_and_uva_only():
     hp = ng.ngram_default_hash_params(flags=ng.NGRAM_FLAG_DEDUP)
-    with pytest.raises(ng.NgramError) as ei:
-        ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, ng.NGRAM_RES_HOST_DMA, hp, 16)
-    assert ei.value.status == ng.NGRAM_EINVAL and "HBM" in str(ei.value)
+    for where in (ng.NGRAM_RES_HOST_DMA, ng.NGRAM_RES_HOST_AUTO):
+        with pytest.raises(ng.NgramError) as ei:
+            ng.ngram_init(_T, 1000, 256, ng.NGRAM_BF16, where, hp, 16)
+        assert ei.value.status == ng.NGRAM_EINVAL and "HOST_UVA" in str(ei.value)
 
 
 def test_sort_flag_combinations_rejected():

@@ -168,14 +168,16 @@ def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
     hbm = ng.ngram_init(dev_table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
     ref = from_dev_bf16(_forward(hbm, dv))
     for where, flags in ((ng.NGRAM_RES_HOST_UVA, 0), (ng.NGRAM_RES_HOST_DMA, 0),
-                         (ng.NGRAM_RES_HOST_AUTO, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT)):
+                         (ng.NGRAM_RES_HOST_AUTO, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT),
+                         (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP)):
         ctx = host_bf16.ctx(where, V, w.N, flags=flags)
         for _ in range(2):                       # second call reuses the staging buffers
             got = from_dev_bf16(_forward(ctx, dv))
             assert np.array_equal(got, ref), where
         assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
         if where == ng.NGRAM_RES_HOST_AUTO:
-            assert ng.ngram_auto_choice(ctx, w.N) in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA)
+            assert ng.ngram_auto_choice(ctx, w.N) in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA,
+                                                      ng.NGRAM_AUTO_UVA_DEDUP)
         if where == ng.NGRAM_RES_HOST_UVA and not flags:   # host table and host activations
             t = torch.from_numpy(inp["tokens"]).pin_memory()
             h = None if inp["history"] is None else torch.from_numpy(inp["history"]).pin_memory()
@@ -200,8 +202,9 @@ def test_host_int8_modes(cuda_device):
         want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R,
                               d=d, dtype=oracle.INT8, table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32,
                               n_threads=N_CPU, vocab_size=V)
-        for where in (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_RES_HOST_DMA):
-            ctx = f.ctx(where, V, w.N)
+        for where, flags in ((ng.NGRAM_RES_HOST_UVA, 0), (ng.NGRAM_RES_HOST_DMA, 0),
+                             (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP)):
+            ctx = f.ctx(where, V, w.N, flags=flags)    # the row scales cross PCIe too
             r = assert_parity(from_dev_bf16(_forward(ctx, dv)), want)
             assert r["exact"] == r["n"]
             ctx.close()
