@@ -276,8 +276,10 @@ __global__ void __launch_bounds__(256, 2) k_rows_grad(const uint32_t *__restrict
                                         o[2] = __fmul_rn(gq.z, acc[k][4 * h + 2]);
                                         o[3] = __fmul_rn(gq.w, acc[k][4 * h + 3]);
                                     }
-                                    *reinterpret_cast<float4 *>(row + c0[k] + h * 128u) =
-                                        make_float4(o[0], o[1], o[2], o[3]);
+                                    // streaming store: the gradient rows are written once,
+                                    // so they should not push dy out of L2
+                                    __stcs(reinterpret_cast<float4 *>(row + c0[k] + h * 128u),
+                                           make_float4(o[0], o[1], o[2], o[3]));
                                 }
                             }
 #pragma unroll

@@ -722,9 +722,27 @@ ngram_status forward_uva(ngram_ctx *c, const Call &k) {
 }
 
 // AUTO: the first call of each batch-size bucket runs and times the three host modes
-// (UVA, UVA with dedup, DMA; all write the same output), keeps the fastest, and later
-// calls use it.  auto_choice holds NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA or
+// (UVA, UVA with dedup, DMA; all write the same output) twice each, keeps the fastest by
+// the better of its two runs (the first run of a mode also allocates its staging), and
+// later calls use it.  auto_choice holds NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA or
 // NGRAM_AUTO_UVA_DEDUP.
+ngram_status time_mode(ngram_ctx *c, const Call &k, int mode, float *ms) {
+    const auto h0 = std::chrono::steady_clock::now();
+    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
+    if (mode == NGRAM_RES_HOST_UVA) NG_CHECK(forward_direct_uva(c, k));
+    else if (mode == NGRAM_AUTO_UVA_DEDUP) NG_CHECK(forward_dedup_uva(c, k));
+    else NG_CHECK(forward_dma(c, k));
+    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
+    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: timing"));
+    NG_CUDA(cudaEventElapsedTime(ms, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
+    if (mode == NGRAM_RES_HOST_DMA) {      // DMA blocks the host while it stages rows
+        const float wall =
+            std::chrono::duration<float, std::milli>(std::chrono::steady_clock::now() - h0).count();
+        *ms = std::max(*ms, wall);
+    }
+    return NGRAM_OK;
+}
+
 ngram_status forward_auto(ngram_ctx *c, const Call &k) {
     const uint32_t b = ceil_log2(k.N);
     if (c->auto_choice[b] == NGRAM_RES_HOST_UVA) return forward_direct_uva(c, k);
@@ -734,31 +752,16 @@ ngram_status forward_auto(ngram_ctx *c, const Call &k) {
         NG_CUDA(cudaEventCreate(&c->ev_t0), "cudaEventCreate");
         NG_CUDA(cudaEventCreate(&c->ev_t1), "cudaEventCreate");
     }
-    float t_uva = 0.f, t_dedup = 0.f, t_dma = 0.f;
-    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
-    NG_CHECK(forward_direct_uva(c, k));
-    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
-    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: UVA timing"));
-    NG_CUDA(cudaEventElapsedTime(&t_uva, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
-    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
-    NG_CHECK(forward_dedup_uva(c, k));
-    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
-    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: UVA dedup timing"));
-    NG_CUDA(cudaEventElapsedTime(&t_dedup, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
-    const auto h0 = std::chrono::steady_clock::now();
-    NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
-    NG_CHECK(forward_dma(c, k));
-    NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
-    NG_CHECK(wait_event(c, c->ev_t1, "AUTO: DMA timing"));
-    // the DMA path blocks the host while it stages rows: count wall time from its start
-    const float wall =
-        std::chrono::duration<float, std::milli>(std::chrono::steady_clock::now() - h0).count();
-    NG_CUDA(cudaEventElapsedTime(&t_dma, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
-    t_dma = std::max(t_dma, wall);
+    const int modes[3] = {NGRAM_RES_HOST_UVA, NGRAM_AUTO_UVA_DEDUP, NGRAM_RES_HOST_DMA};
     int best = NGRAM_RES_HOST_UVA;
-    float t_best = t_uva;
-    if (t_dedup < t_best) { best = NGRAM_AUTO_UVA_DEDUP; t_best = t_dedup; }
-    if (t_dma < t_best) best = NGRAM_RES_HOST_DMA;
+    float t_best = 0.f;
+    for (int m = 0; m < 3; ++m) {
+        float t0 = 0.f, t1 = 0.f;
+        NG_CHECK(time_mode(c, k, modes[m], &t0));
+        NG_CHECK(time_mode(c, k, modes[m], &t1));
+        const float t = std::min(t0, t1);
+        if (m == 0 || t < t_best) { best = modes[m]; t_best = t; }
+    }
     c->auto_choice[b] = best;
     return NGRAM_OK;
 }
