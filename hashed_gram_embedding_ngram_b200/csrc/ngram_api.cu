@@ -35,13 +35,17 @@ using namespace ngram;
 
 
 // Build-time tuning of the gathers (measured on B200, 20M x 2560 bf16, 32,768 tokens):
-//   NGRAM_SPI_ALWAYS_ONE = 1: every warp work item is one 32-vector strip, so the 10
-//     strips of a token run on 10 warps at once (455 us) instead of one warp walking
-//     them (470 us); the 16 hashes are recomputed per strip, which the issue slots absorb.
+//   NGRAM_SPI_ONE_FORMATS: bit t set = row format t always gives a warp one 32-vector strip
+//     per work item, so the strips of a token run on several warps at once and each
+//     recomputes the 16 hashes: bf16 (10 strips, 455 us against 470 us with one warp walking
+//     them) and NVFP4 (132.5 against 124.7 M tokens/s).  The row-scale formats (int8, FP8)
+//     walk a token's strips in one warp once the batch fills the GPU, so the hashes and the
+//     dependent row-scale loads run once per token: FP8 114.1 against 107.3 M tokens/s,
+//     int8 (uniform tokens) 110.4 against 104.8.
 //   The TMA-staged kernel (NGRAM_FLAG_TMA_STAGING) measured 522-895 us depending on
 //     chunk and ring depth; its tunables are below.
-#ifndef NGRAM_SPI_ALWAYS_ONE
-#define NGRAM_SPI_ALWAYS_ONE 1
+#ifndef NGRAM_SPI_ONE_FORMATS
+#define NGRAM_SPI_ONE_FORMATS ((1u << NGRAM_BF16) | (1u << NGRAM_NVFP4))
 #endif
 #ifndef NGRAM_BULK_CHUNK_COLS           // columns per work item of the bulk kernel
 #define NGRAM_BULK_CHUNK_COLS 1280
@@ -522,7 +526,7 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
         g.row_ids == nullptr && g.gate_tok == nullptr && g.tok_begin == 0)
         return launch_staged(c, g, s);
     const uint64_t resident_warps = max_blocks * 8u;
-    g.strips_per_item = (NGRAM_SPI_ALWAYS_ONE ||
+    g.strips_per_item = (((NGRAM_SPI_ONE_FORMATS >> c->dtype) & 1u) ||
                          static_cast<uint64_t>(g.N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
     g.groups_per_token = (g.n_strips + g.strips_per_item - 1) / g.strips_per_item;
     const uint64_t items = static_cast<uint64_t>(g.N) * g.groups_per_token;
