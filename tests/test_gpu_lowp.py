@@ -242,7 +242,7 @@ def test_flags_and_staging_bitidentical(cuda_device, fmt):
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
 def test_host_residency_bitidentical(cuda_device, fmt):
     """The table in pinned host memory (filled through its device alias): UVA, DMA, AUTO
-    and UVA grouped equal the HBM result bit for bit."""
+    UVA grouped and UVA + dedup equal the HBM result bit for bit."""
     R, d, V = 300_000, 2560, 151_936
     dt = ng_dtype(fmt)
     TABLES.drop()
@@ -261,7 +261,8 @@ def test_host_residency_bitidentical(cuda_device, fmt):
             hbm = ng.ngram_init(table, R, d, dt, ng.NGRAM_RES_HBM, _hp(V), w.N, row_scale=scale)
             ref = from_dev_bf16(_fwd(hbm, dv))
             for where, flags in ((ng.NGRAM_RES_HOST_UVA, 0), (ng.NGRAM_RES_HOST_DMA, 0),
-                                 (ng.NGRAM_RES_HOST_AUTO, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT)):
+                                 (ng.NGRAM_RES_HOST_AUTO, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT),
+                                 (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP)):
                 c = ng.ngram_init(host.tensor, R, d, dt, where, _hp(V, flags=flags), w.N,
                                   row_scale=hs.tensor)
                 for _ in range(2):
