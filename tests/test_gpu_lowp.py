@@ -241,7 +241,7 @@ def test_flags_and_staging_bitidentical(cuda_device, fmt):
 
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
 def test_host_residency_bitidentical(cuda_device, fmt):
-    """The table in pinned host memory (filled through its device alias): UVA, DMA, AUTO
+    """The table in pinned host memory (filled through its device alias): UVA, DMA, AUTO,
     UVA grouped and UVA + dedup equal the HBM result bit for bit."""
     R, d, V = 300_000, 2560, 151_936
     dt = ng_dtype(fmt)
