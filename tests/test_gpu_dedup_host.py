@@ -4,7 +4,8 @@ Dedup: the distinct rows (in order of first appearance) and the inverse map must
 the oracle's exactly.  Residency: HBM, HBM + dedup staging, host UVA, host DMA and
 host AUTO must give bit-identical outputs (the analogue of the offload on/off output
 check on the aibacon page, section "Which is why the offload matters more than the
-parameter count"), and those outputs must match the oracle.  The host waits of the DMA
+parameter count"), and those outputs must match the oracle, at full size too (the 20M-row
+table pinned in host memory, sampled tokens).  The host waits of the DMA
 mode are bounded: a stream kept busy past the bound makes the call return
 NGRAM_ETIMEOUT and leaves the context usable.
 """
@@ -300,3 +301,34 @@ def test_prefetch_int8_and_errors(cuda_device):
     with pytest.raises(ng.NgramError) as ei:
         ng.ngram_prefetch(ctx, 2, toks, hist)                # out of range
     assert ei.value.status == ng.NGRAM_EINVAL
+
+
+def test_host_full_size_sampled(cuda_device):
+    """The host-resident configuration at full size: the 20,000,000 x 2560 bf16 table
+    (95.4 GiB) pinned in host memory, the 8,192-token prefill and a 256-token decode batch.
+    UVA, UVA + dedup and DMA agree bit for bit, and sampled tokens equal the oracle."""
+    TABLES.drop()                                   # no device table is needed here
+    w0 = W["host_prefill"]
+    R, d, V = w0.R, w0.d, w0.vocab
+    host = ng.HostTable((R, d), torch.bfloat16)
+    try:
+        ng.ngram_fill_synthetic(host.tensor, R, d, ng.NGRAM_BF16, gen.TABLE_SEED)
+        torch.cuda.synchronize()
+        for name in ("host_prefill", "host_decode_256"):
+            w = W[name]
+            inp, dv = workload_on_device(w, cuda_device)
+            outs = []
+            for where, flags in ((ng.NGRAM_RES_HOST_UVA, 0), (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP),
+                                 (ng.NGRAM_RES_HOST_DMA, 0)):
+                ctx = ng.ngram_init(host.tensor, R, d, ng.NGRAM_BF16, where, _hp(V, flags=flags), w.N)
+                outs.append(from_dev_bf16(_forward(ctx, dv)))
+                assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+                ctx.close()
+            assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2]), name
+            sel = sample_tokens(w, 256)
+            want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
+                                  table_seed=gen.TABLE_SEED, sel=sel, acc=oracle.ACC_F32, n_threads=N_CPU,
+                                  vocab_size=V)
+            assert_parity(outs[0].reshape(w.N, d)[sel], want)
+    finally:
+        host.close()
