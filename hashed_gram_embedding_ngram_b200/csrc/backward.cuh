@@ -164,9 +164,18 @@ __global__ void __launch_bounds__(256) k_seg_starts(const uint32_t *__restrict__
 #ifndef NGRAM_ROWS_GRAD_STRIPS
 #define NGRAM_ROWS_GRAD_STRIPS 1
 #endif
+// Depth per warp beats warps per SM here (B200, full prefill, ngram_backward_rows):
+// 16 fragments at 2 CTAs/SM 1.077 ms; 8 at 3 CTAs 1.19 ms; 8 at 4 CTAs 1.22 ms; 12 at 3
+// CTAs 1.25 ms.
+#ifndef NGRAM_ROWS_GRAD_BATCH         // dy fragments in flight per lane (shared gate)
+#define NGRAM_ROWS_GRAD_BATCH 16
+#endif
+#ifndef NGRAM_ROWS_GRAD_MIN_BLOCKS    // resident CTAs per SM the register budget targets
+#define NGRAM_ROWS_GRAD_MIN_BLOCKS 2
+#endif
 
 template <bool kTokGate, int kStrips>
-__global__ void __launch_bounds__(256, 2) k_rows_grad(const uint32_t *__restrict__ count,
+__global__ void __launch_bounds__(256, NGRAM_ROWS_GRAD_MIN_BLOCKS) k_rows_grad(const uint32_t *__restrict__ count,
                                                       const uint32_t *__restrict__ seg,
                                                       const uint32_t *__restrict__ occ_tok,
                                                       const uint16_t *__restrict__ dy,
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(256, 2) k_rows_grad(const uint32_t *__restrict
                                                       const uint16_t *__restrict__ gate_tok,
                                                       uint32_t d, float *__restrict__ grad,
                                                       uint32_t *next_item) {
-    constexpr uint32_t kBatch = (kTokGate ? 8u : 16u) / kStrips;   // 16 (8) fragments in flight
+    constexpr uint32_t kBatch = (kTokGate ? NGRAM_ROWS_GRAD_BATCH / 2u : NGRAM_ROWS_GRAD_BATCH) / kStrips;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t n_strips = ((d >> 3) + 31u) >> 5;
     const uint32_t n_groups = (n_strips + kStrips - 1u) / kStrips;
