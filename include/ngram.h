@@ -210,9 +210,15 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  *             NGRAM_FLAG_TOKEN_GATE device bf16 [N][d] (one gate per token).
  *   out       device bf16 [N][d], 16-byte aligned; may equal residual (in place),
  *             must not otherwise overlap it.
- * One kernel launch on stream; N == 0 launches nothing.  EINVAL if N > max_tokens,
- * a pointer is NULL or misaligned.  Bad token ids are reported asynchronously through
- * ngram_get_device_error. */
+ * Launches on stream: the fused gather kernel.  A grouped batch (HBM: NGRAM_FLAG_SORT, or by
+ * default from NGRAM_SORT_MIN_TOKENS tokens) is preceded by the grouped-order step (a memset
+ * and 3 small kernels) and, for bf16 and NVFP4 tables from 4,096 tokens, by k_hash_indices,
+ * which hashes every token once (64 B per token) so that the gather's work items read row
+ * ids instead of hashing per column strip.  N == 0
+ * launches nothing.  The grouping and row-id scratch belong to the context: order the
+ * context's ngram_forward calls (one stream, or events); ngram_prefetch uses other scratch
+ * and may run beside them.  EINVAL if N > max_tokens, a pointer is NULL or misaligned.  Bad
+ * token ids are reported asynchronously through ngram_get_device_error. */
 NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
                            const void *gate, uint16_t *out, ngram_stream_t stream);
