@@ -360,7 +360,8 @@ def run_ours(args, w):
              "token_gate": ng.NGRAM_FLAG_TOKEN_GATE}[args.variant]
     grouped = args.variant == "sort" or (args.variant in ("default", "token_gate")
                                          and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
-    # grouped bf16 / NVFP4 batches of >= 4096 tokens hash every token once first (k_hash_indices)
+    # grouped bf16 / NVFP4 batches of >= 4096 tokens hash every token once, in the order
+    # step's count kernel, and the gather reads the row ids
     prehash = grouped and w.dtype in ("bf16", "nvfp4") and w.N >= 4096
     hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
@@ -502,8 +503,8 @@ def run_ours(args, w):
                          "traffic": profiled_traffic(w.name, w.dtype) if args.variant == "default" else None,
                          "kernel": ("hash + dedup + compact + gather (8 kernels)" if args.variant == "dedup"
                                     else "k_gather_bf16_bulk<16>" if args.variant == "tma"
-                                    else ("grouped order (3 kernels) + " if grouped else "")
-                                    + ("k_hash_indices + " if prehash else "")
+                                    else ("grouped order (3 kernels%s) + " % (
+                                        ", row ids hashed once" if prehash else "") if grouped else "")
                                     + KERNEL_NAME[w.dtype]),
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
                          "unique_rows": unique_rows,
@@ -518,7 +519,7 @@ def run_ours(args, w):
                     if args.variant == "default" else
                             "pinned host tokens + residual -> device, ngram_forward, out -> pinned host"},
             "clocks": clocks,
-            "gpu_launches": K * (8 if args.variant == "dedup" else (4 + prehash) if grouped else 1),
+            "gpu_launches": K * (8 if args.variant == "dedup" else 4 if grouped else 1),
         }
         if world == 1 and not args.no_cpu_baseline:
             threads = os.cpu_count() or 1

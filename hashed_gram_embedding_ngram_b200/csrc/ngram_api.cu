@@ -711,7 +711,8 @@ bool grouped_order(const ngram_ctx *c, uint32_t N) {
 // then the fused gather walks them in that order.  Same outputs; repeated rows run back
 // to back so L2 serves the repeats.
 // Grouped order of a batch's tokens into c->so_perm (3 kernels and a memset).
-ngram_status order_tokens(ngram_ctx *c, const Call &k) {
+// idx_out: also write every token's row ids [N][H] in the same pass, or null.
+ngram_status order_tokens(ngram_ctx *c, const Call &k, uint32_t *idx_out = nullptr) {
     if (!c->so_perm) {
         NG_CUDA(cudaMalloc(&c->so_bucket, c->max_tokens * 4ull), "order scratch");
         NG_CUDA(cudaMalloc(&c->so_hist, kOrderBuckets * 4ull), "order scratch");
@@ -720,7 +721,8 @@ ngram_status order_tokens(ngram_ctx *c, const Call &k) {
     const HashArgs a = hash_args(c);
     const unsigned gn = grid_for(c, k.N, 256);
     NG_CUDA(cudaMemsetAsync(c->so_hist, 0, kOrderBuckets * 4ull, k.s), "order clear");
-    k_order_count<<<gn, 256, 0, k.s>>>(k.tokens, k.history, k.T, k.N, a, c->d_err, c->so_bucket, c->so_hist);
+    k_order_count<<<gn, 256, 0, k.s>>>(k.tokens, k.history, k.T, k.N, a, c->d_err, c->so_bucket, c->so_hist,
+                                        idx_out);
     k_order_scan<<<1, 1024, 0, k.s>>>(c->so_hist);
     k_order_scatter<<<gn, 256, 0, k.s>>>(c->so_bucket, k.N, c->so_hist, c->so_perm);
     NG_CUDA(cudaGetLastError(), "order launch");
@@ -728,13 +730,13 @@ ngram_status order_tokens(ngram_ctx *c, const Call &k) {
 }
 
 // NGRAM_PREHASH_FORMATS bit t: on grouped batches of at least NGRAM_PREHASH_MIN_TOKENS
-// tokens in HBM, row format t hashes every token once into idx [N][H] (k_hash_indices, 64 B
-// per token) before the gather, which then reads the row ids instead of hashing in every
-// work item.  It pays for the formats whose work item is one strip of a token (bf16: 10
-// strips, NVFP4: 5), which otherwise hash each token once per strip: measured on B200,
-// NVFP4 prefill 133.4 -> 140.2 M tokens/s, bf16 prefill 75.6 -> 76.6 M.  int8 and FP8 walk
-// a token's strips in one warp and hash once anyway (with prehashing 110.6 -> 108.5 and
-// 114.0 -> 112.1 M: the extra kernel costs more than it saves).
+// tokens in HBM, row format t hashes every token once -- k_order_count writes its row ids
+// [N][H] (64 B per token) beside the bucket counts -- and the gather reads the row ids
+// instead of hashing in every work item.  It pays for the formats whose work item is one
+// strip of a token (bf16: 10 strips, NVFP4: 5), which otherwise hash each token once per
+// strip: measured on B200 with a separate hash kernel, NVFP4 prefill 133.4 -> 140.2 M
+// tokens/s, bf16 prefill 75.6 -> 76.6 M.  int8 and FP8 walk a token's strips in one warp
+// and hash once anyway (with the separate kernel 110.6 -> 108.5 and 114.0 -> 112.1 M).
 #ifndef NGRAM_PREHASH_FORMATS
 #define NGRAM_PREHASH_FORMATS ((1u << NGRAM_BF16) | (1u << NGRAM_NVFP4))
 #endif
@@ -742,21 +744,14 @@ ngram_status order_tokens(ngram_ctx *c, const Call &k) {
 #define NGRAM_PREHASH_MIN_TOKENS 4096u
 #endif
 
-ngram_status prehash(ngram_ctx *c, const Call &k, GatherArgs &g) {
-    if (!((NGRAM_PREHASH_FORMATS >> c->dtype) & 1u) || c->where != NGRAM_RES_HBM ||
-        k.N < NGRAM_PREHASH_MIN_TOKENS)
-        return NGRAM_OK;
-    if (!c->d_rowid) NG_CUDA(cudaMalloc(&c->d_rowid, c->dd_cap * 4ull), "row-id buffer");
-    NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_rowid, k.s));
-    g.row_ids = c->d_rowid;
-    return NGRAM_OK;
-}
-
 ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
-    NG_CHECK(order_tokens(c, k));
+    const bool prehash = ((NGRAM_PREHASH_FORMATS >> c->dtype) & 1u) && c->where == NGRAM_RES_HBM &&
+                         k.N >= NGRAM_PREHASH_MIN_TOKENS;
+    if (prehash && !c->d_rowid) NG_CUDA(cudaMalloc(&c->d_rowid, c->dd_cap * 4ull), "row-id buffer");
+    NG_CHECK(order_tokens(c, k, prehash ? c->d_rowid : nullptr));
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     g.perm = c->so_perm;
-    NG_CHECK(prehash(c, k, g));
+    if (prehash) g.row_ids = c->d_rowid;
     return launch_gather(c, g, k.s, max_blocks);
 }
 

@@ -21,24 +21,25 @@ namespace ngram {
 constexpr uint32_t kOrderBucketsLog2 = 13;
 constexpr uint32_t kOrderBuckets = 1u << kOrderBucketsLog2;
 
-__device__ __forceinline__ uint32_t bigram_bucket(const int32_t *tokens, const int32_t *history,
-                                                  uint32_t tok, uint32_t T, const HashArgs &a,
-                                                  uint32_t *err) {
-    uint32_t w0, w1, w2;
-    token_context(tokens, history, tok, T, a, err, w0, w1, w2);
-    const uint64_t k2 = (static_cast<uint64_t>(w1) << 21) | w0;
-    return static_cast<uint32_t>(splitmix64_step(k2) >> (64 - kOrderBucketsLog2));
-}
-
+// Bucket counts, one thread per token.  With idx_out, the same thread also writes the
+// token's row ids idx_out[t][h] = head_row(h, context) for h < H (the hash-once step of
+// the gather, folded into this pass over the contexts).
 __global__ void __launch_bounds__(256) k_order_count(const int32_t *__restrict__ tokens,
                                                      const int32_t *__restrict__ history,
                                                      uint32_t T, uint32_t N, const HashArgs a,
                                                      uint32_t *err, uint32_t *__restrict__ bucket_of,
-                                                     uint32_t *hist) {
+                                                     uint32_t *hist, uint32_t *__restrict__ idx_out) {
     for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x) {
-        const uint32_t b = bigram_bucket(tokens, history, t, T, a, err);
+        uint32_t w0, w1, w2;
+        token_context(tokens, history, t, T, a, err, w0, w1, w2);
+        const uint64_t k2 = (static_cast<uint64_t>(w1) << 21) | w0;
+        const uint32_t b = static_cast<uint32_t>(splitmix64_step(k2) >> (64 - kOrderBucketsLog2));
         bucket_of[t] = b;
         atomicAdd(hist + b, 1u);
+        if (idx_out != nullptr) {
+            uint32_t *dst = idx_out + static_cast<size_t>(t) * a.n_heads;
+            for (uint32_t h = 0; h < a.n_heads; ++h) dst[h] = head_row(h, w0, w1, w2, a);
+        }
     }
 }
 

@@ -212,9 +212,9 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  *             must not otherwise overlap it.
  * Launches on stream: the fused gather kernel.  A grouped batch (HBM: NGRAM_FLAG_SORT, or by
  * default from NGRAM_SORT_MIN_TOKENS tokens) is preceded by the grouped-order step (a memset
- * and 3 small kernels) and, for bf16 and NVFP4 tables from 4,096 tokens, by k_hash_indices,
- * which hashes every token once (64 B per token) so that the gather's work items read row
- * ids instead of hashing per column strip.  N == 0
+ * and 3 small kernels); for bf16 and NVFP4 tables from 4,096 tokens its first kernel also
+ * hashes every token once (64 B of row ids per token), so that the gather's work items read
+ * row ids instead of hashing per column strip.  N == 0
  * launches nothing.  The grouping and row-id scratch belong to the context: order the
  * context's ngram_forward calls (one stream, or events); ngram_prefetch uses other scratch
  * and may run beside them.  EINVAL if N > max_tokens, a pointer is NULL or misaligned.  Bad
