@@ -38,6 +38,32 @@ def test_library_exports_nothing_else():
     assert exported == _declared()
 
 
+def _header_constants():
+    """Integer constants of the header: #define NGRAM_X <literal> and enum entries."""
+    text = open(HEADER).read()
+    out = {}
+    for name, val in re.findall(r"#define\s+(NGRAM_\w+)\s+(0x[0-9A-Fa-f]+|\d+)[uUlL]*\b", text):
+        out[name] = int(val, 0)
+    for name, val in re.findall(r"^\s+(NGRAM_\w+)\s*=\s*(\d+)", text, flags=re.M):
+        out[name] = int(val)
+    return out
+
+
+def test_binding_constants_match_the_header():
+    consts = _header_constants()
+    assert {"NGRAM_FLAG_DEDUP", "NGRAM_AUTO_UVA_DEDUP", "NGRAM_NVFP4", "NGRAM_RES_HOST_AUTO",
+            "NGRAM_EDEVICE", "NGRAM_SORT_MIN_TOKENS", "NGRAM_STAGE_SLOTS"} <= set(consts)
+    aliases = {"NGRAM_MAX_HEADS": "MAX_HEADS", "NGRAM_DEFAULT_BASE_SEED": "DEFAULT_BASE_SEED",
+               "NGRAM_DEFAULT_PAD_ID": "DEFAULT_PAD_ID"}
+    checked = 0
+    for name, val in consts.items():
+        attr = aliases.get(name, name)
+        if hasattr(ng, attr):
+            assert getattr(ng, attr) == val, name
+            checked += 1
+    assert checked >= 20
+
+
 def test_status_strings():
     assert ng.ngram_status_string(ng.NGRAM_OK) == "NGRAM_OK"
     assert ng.ngram_status_string(ng.NGRAM_EDEVICE) == "NGRAM_EDEVICE"
