@@ -111,7 +111,8 @@ typedef enum {
  * mbarrier ring) instead of register loads: bf16 rows in column chunks, the 8- and 4-bit
  * formats as whole rows (a producer warp copies, consumer warps decode; HBM residency).
  * Same results bit for bit; measured slower on B200 (bf16 522-895 us vs 455 us on the
- * full-size gather; NVFP4 52-76 M vs 121 M tokens/s), kept for comparison.  Every wait is
+ * full-size gather; NVFP4 52-76 M vs 121 M tokens/s for the register gather of that time,
+ * 138 M now), kept for comparison.  Every wait is
  * bounded (1 s; then device error code 2).  Not with NGRAM_FLAG_TOKEN_GATE. */
 #define NGRAM_FLAG_TMA_STAGING 0x2u
 /* Grouped order: before the gather, group the batch's tokens by bigram context
