@@ -20,6 +20,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -140,17 +141,31 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_sha(dtype: str = "bf16") -> str:
+def code_only(text: str) -> str:
+    """A source file without its comments and blank lines: the hash below tracks the code,
+    so that editing a comment does not orphan a committed ncu summary."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
+def kernel_sha(dtype: str = "bf16", read=None) -> str:
+    """Hash of the code (comments stripped) of the sources a timed kernel is built from.
+    read(rel) -> text; default: the working tree."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[dtype]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel)) as f:
+                text = f.read()
+        else:
+            text = read(rel)
+        h.update(code_only(text).encode())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(workload: str, dtype: str = "bf16"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    kernel source as it is now (else None)."""
+    kernel code as it is now (its kernel_sha line, first word; else None)."""
     p = os.path.join(ROOT, "profiles", "gather_%s.txt" % workload)
     if not os.path.exists(p):
         return None
@@ -160,7 +175,7 @@ def profiled_traffic(workload: str, dtype: str = "bf16"):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("kernel_sha") != kernel_sha(dtype):
+    if (kv.get("kernel_sha", "").split() or [""])[0] != kernel_sha(dtype):
         return None
     try:
         return float(kv["traffic_bytes_per_launch"])

@@ -15,9 +15,10 @@
 //     before the first add, then sums in head order 0..H-1 in fp32 (packed pairs of
 //     columns, each rounded like a scalar add), applies y = r + g * acc with separately
 //     rounded multiply and add, and stores bf16.
-//   * Work items are dealt to a persistent grid (blocks = SMs x resident blocks);
-//     decode-sized batches split a token's strips across warps for latency, large
-//     batches keep all strips of a token in one warp so the hash is computed once.
+//   * Work items are dealt to a persistent grid (blocks = SMs x resident blocks).  For
+//     bf16 every item is one strip, so a token's strips run on several warps at once;
+//     on large grouped batches the order step has already written every token's 16 row
+//     ids (row_ids), which the hashing lanes then read instead of hashing per strip.
 #pragma once
 
 #include "device_common.cuh"
@@ -64,8 +65,9 @@ __device__ __forceinline__ uint4 ld_na_v4(const void *p) {
 }
 
 // Row indices of the warp's token, one head per lane (lanes >= H hold 0): hashed
-// from the context, or read from precomputed ids (dedup'ed / staged paths, where
-// `table` is the staging buffer and row_ids the inverse map).
+// from the context, or read from precomputed ids -- the table's own rows hashed once by
+// the order step, or, on the dedup'ed / staged paths, the inverse map into the staging
+// buffer that `table` then points to.
 __device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t tok,
                                                   uint32_t lane, uint32_t H) {
     uint32_t row = 0;
