@@ -492,7 +492,7 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 }
 
 template <bool kTok>
-void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, uint32_t rb) {
+void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s) {
     const bool h16 = g.h.n_heads == 16;
     switch (t) {
         case NGRAM_BF16:
@@ -563,8 +563,8 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
     uint64_t blocks = (items + 7) / 8;
     if (blocks > max_blocks) blocks = max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
-    if (g.gate_tok != nullptr) launch_gather_kernel<true>(c->dtype, g, nb, s, c->row_bytes);
-    else launch_gather_kernel<false>(c->dtype, g, nb, s, c->row_bytes);
+    if (g.gate_tok != nullptr) launch_gather_kernel<true>(c->dtype, g, nb, s);
+    else launch_gather_kernel<false>(c->dtype, g, nb, s);
     NG_CUDA(cudaGetLastError(), "gather kernel launch");
     return NGRAM_OK;
 }
