@@ -585,6 +585,52 @@ def test_backward_gate_matches_autograd(gate_tok):
         assert np.array_equal(part, dg32[sel])
 
 
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,            # OCP MX v1.0 FP4 E2M1
+                  -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+
+def _e4m3_torch(codes):
+    """E4M3 codes -> fp64 through torch's float8_e4m3fn (independent of the oracle)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("gate_tok", [False, True])
+def test_backward_gate_low_precision_matches_autograd(fmt, gate_tok):
+    """The gate gradient over FP8 and NVFP4 tables: fp64 autograd of sum(dy * out), with
+    out = r + G * (A E) and E the table decoded by torch's E4M3 and the OCP E2M1 table."""
+    R, d, V, n_seq, T, nb, nt = 61, 32, 40, 2, 13, 5, 3
+    toks, res, g = _tiny_case(seed=14, n_seq=n_seq, T=T, V=V, R=R, d=d, nb=nb, nt=nt)
+    N = n_seq * T
+    rng = np.random.default_rng(23)
+    dy = _bf16_bits(rng.normal(0, 1.0, (N, d)))
+    gt = _bf16_bits(rng.normal(0, 1.0, (N, d))) if gate_tok else None
+    if fmt == "fp8":
+        q, sc = oracle.fill_fp8(31, 0, R, d)
+        E = _e4m3_torch(q) * sc.astype(np.float64)[:, None]
+        dtype, tab = oracle.FP8, q
+    else:
+        rows = oracle.fill_fp4(31, 0, R, d)
+        codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(R, d)
+        bs = _e4m3_torch(rows[:, d // 2:d // 2 + d // 16])
+        gs = float.fromhex("0x1.4fp-9")
+        E = _E2M1[codes] * np.repeat(bs, 16, axis=1) * gs
+        sc = np.array([gs], dtype=np.float32)
+        dtype, tab = oracle.NVFP4, rows
+    idx = oracle.indices(toks, None, R=R, n_bigram=nb, n_trigram=nt, vocab_size=V).reshape(N, nb + nt)
+    Et = torch.tensor(E)
+    G = torch.tensor(_bits_to_f64(gt).reshape(N, d) if gate_tok else g.astype(np.float64),
+                     requires_grad=True)
+    e = torch.nn.functional.embedding_bag(torch.from_numpy(idx.astype(np.int64)), Et, mode="sum")
+    out = torch.tensor(_bits_to_f64(res).reshape(N, d)) + G * e
+    (torch.tensor(_bits_to_f64(dy).reshape(N, d)) * out).sum().backward()
+    dg = oracle.backward_gate(toks, None, dy, R=R, d=d, dtype=dtype, table_i8=tab, row_scale=sc,
+                              per_token=gate_tok, acc=oracle.ACC_F64, n_bigram=nb, n_trigram=nt,
+                              vocab_size=V)
+    assert np.allclose(dg, G.grad.numpy(), rtol=1e-12, atol=1e-15)
+
+
 def test_backward_gate_shared_is_the_sum_of_per_token():
     c = _autograd_case(13, False)
     kw = dict(R=c["R"], d=c["d"], dtype=oracle.BF16, table=c["Eb"].reshape(c["R"], c["d"]),
