@@ -659,6 +659,36 @@ def test_forward_per_token_gate():
     assert np.array_equal(y, want)
 
 
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_forward_per_token_gate_low_precision(fmt):
+    """FP8 / NVFP4 tables: a per-token gate whose rows all equal bf16(g) gives the shared-
+    gate result bit for bit (fp32 mode), and a general one matches r + G * (A E) in fp64
+    with E decoded by torch's float8_e4m3fn and the OCP E2M1 table."""
+    R, d, V = 97, 32, 50
+    toks, res, g = _tiny_case(R=R, d=d, V=V)
+    N = toks.size
+    gb = _bf16_bits(g)
+    if fmt == "fp8":
+        q, sc = oracle.fill_fp8(5, 0, R, d)
+        E = _e4m3_torch(q) * sc.astype(np.float64)[:, None]
+        kw = dict(R=R, d=d, dtype=oracle.FP8, table_i8=q, row_scale=sc, vocab_size=V)
+    else:
+        rows = oracle.fill_fp4(5, 0, R, d)
+        codes = np.stack([rows[:, :d // 2] & 15, rows[:, :d // 2] >> 4], axis=2).reshape(R, d)
+        gs = float.fromhex("0x1.4fp-9")
+        E = _E2M1[codes] * np.repeat(_e4m3_torch(rows[:, d // 2:d // 2 + d // 16]), 16, axis=1) * gs
+        kw = dict(R=R, d=d, dtype=oracle.NVFP4, table_i8=rows, row_scale=np.array([gs], np.float32),
+                  vocab_size=V)
+    a = oracle.forward(toks, None, res, _bits_to_f64(gb).astype(np.float32), **kw)
+    b = oracle.forward(toks, None, res, None, gate_tok=np.tile(gb, (N, 1)), **kw)
+    assert np.array_equal(a, b)
+    G = _bf16_bits(np.random.default_rng(4).normal(0, 1, (N, d)))
+    _, y, _, idx = oracle.forward(toks, None, res, None, gate_tok=G, acc=oracle.ACC_F64,
+                                  want_aux=True, **kw)
+    want = _bits_to_f64(res).reshape(N, d) + _bits_to_f64(G).reshape(N, d) * _one_hot_sum(idx, E)
+    assert np.allclose(y, want, rtol=1e-15, atol=0)
+
+
 def test_hash_rows_are_uniform():
     """Sanity, not parity: 100,000 random contexts x 16 heads land in R = 1009 rows
     uniformly (chi-square with 1008 degrees of freedom, p > 1e-4), and the heads of one
