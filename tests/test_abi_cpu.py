@@ -64,6 +64,32 @@ def test_binding_constants_match_the_header():
     assert checked >= 20
 
 
+def _prototypes():
+    """(name, parameter count) of every NGRAM_API prototype of the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"NGRAM_API\s+[\w\s\*]*?\b(ngram_\w+)\s*\(([^;]*?)\)\s*;", text,
+                                   flags=re.S):
+        p = params.strip()
+        out[name] = 0 if p in ("", "void") else len(p.split(","))
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every entry point the binding declares argtypes for takes as many arguments as its
+    prototype (an ABI drift would otherwise only show as a crash on the GPU)."""
+    protos = _prototypes()
+    assert set(protos) == set(_declared())
+    lib = ng.lib()
+    checked = 0
+    for name, n in protos.items():
+        at = getattr(lib, name).argtypes
+        if at is not None:
+            assert len(at) == n, (name, len(at), n)
+            checked += 1
+    assert checked >= len(protos) - 1          # ngram_dedup_rows_noalloc is bound by its test
+
+
 def test_status_strings():
     assert ng.ngram_status_string(ng.NGRAM_OK) == "NGRAM_OK"
     assert ng.ngram_status_string(ng.NGRAM_EDEVICE) == "NGRAM_EDEVICE"
