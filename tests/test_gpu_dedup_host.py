@@ -191,7 +191,8 @@ def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
     want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
                           table_seed=gen.TABLE_SEED, sel=sel, acc=oracle.ACC_F32, n_threads=N_CPU,
                           vocab_size=V)
-    assert_parity(ref.reshape(w.N, d)[sel], want)
+    r = assert_parity(ref.reshape(w.N, d)[sel], want)
+    assert r["exact"] == r["n"]
 
 
 def test_host_int8_modes(cuda_device):

@@ -137,7 +137,8 @@ def test_forward_full_prefill_sampled(cuda_device):
     sel = sample_tokens(w, 1024)
     want, _, mag, idx = _oracle(w, inp, sel=sel, acc=oracle.ACC_F64, want_aux=True)
     assert_parity(got[sel], want, mag)
-    assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    r = assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    assert r["exact"] == r["n"]              # same operations in the same order
     # the same sampled indices straight from the index step
     gi = ng.ngram_hash_indices(ctx, dv["tokens"]).cpu().numpy().view(np.uint32)
     assert np.array_equal(gi[sel], idx)
@@ -192,7 +193,8 @@ def test_forward_collisions_R2(cuda_device):
           "residual": to_dev_bf16(inp["residual"], cuda_device).view(w.N, d),
           "gate": torch.from_numpy(inp["gate"]).to(cuda_device)}
     got = from_dev_bf16(_run(w, cuda_device, dv, ctx))
-    assert_parity(got, _oracle(w, inp))
+    r = assert_parity(got, _oracle(w, inp))
+    assert r["exact"] == r["n"]
 
 
 def test_forward_large_batch_small_rows(cuda_device):
@@ -202,7 +204,8 @@ def test_forward_large_batch_small_rows(cuda_device):
     ctx = _ctx_for(w, cuda_device)
     got = from_dev_bf16(_run(w, cuda_device, dv, ctx)).reshape(w.N, w.d)
     sel = sample_tokens(w, 4096)
-    assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    r = assert_parity(got[sel], _oracle(w, inp, sel=sel))
+    assert r["exact"] == r["n"]
 
 
 def test_in_place_equals_out_of_place(cuda_device):
@@ -290,7 +293,8 @@ def test_bad_token_ids_flag_the_device_error_word(cuda_device):
     t2 = inp["tokens"].copy()
     t2.reshape(-1)[300] = oracle.DEFAULT_PAD_ID
     inp2 = dict(inp, tokens=t2)
-    assert_parity(from_dev_bf16(out), _oracle(w, inp2))
+    r = assert_parity(from_dev_bf16(out), _oracle(w, inp2))
+    assert r["exact"] == r["n"]
     assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK   # cleared
     hist = torch.full((w.n_seq, 2), -1, dtype=torch.int32, device=cuda_device)
     ng.ngram_forward(ctx, dv["tokens"], dv["residual"], dv["gate"], history=hist)
