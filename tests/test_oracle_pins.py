@@ -426,6 +426,62 @@ def test_int8_fp32_mode_within_tolerance_of_exact():
     assert np.all(np.abs(a - b) <= _bf16_ulp(b) + 2.0 ** -20 * mag)
 
 
+def _f32_of_exact_sum(p64, acc32):
+    """fp32 nearest (ties to even) to the exact p64 + acc32, where p64 is an exact fp64
+    product: the fp64 sum s plus its exact error (Knuth's TwoSum) is the exact value; s
+    rounds to the right fp32 unless s sits exactly halfway between two fp32 values, where
+    the sign of the error decides.  Written from IEEE 754 round-to-nearest, no fmaf."""
+    a = acc32.astype(np.float64)
+    s = p64 + a
+    bb = s - p64
+    err = (p64 - (s - bb)) + (a - bb)
+    f = s.astype(np.float32)
+    dlt = s - f.astype(np.float64)                          # exact: f is within an ulp of s
+    toward = np.where(dlt > 0, np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf)))
+    mid = (dlt != 0) & (2.0 * dlt == toward.astype(np.float64) - f.astype(np.float64))
+    return np.where(mid & (err != 0) & (np.sign(err) == np.sign(dlt)), toward, f)
+
+
+@pytest.mark.parametrize("fmt", ["int8", "fp8"])
+def test_scaled_rows_fp32_mode_is_one_rounding_per_head(fmt):
+    """The fp32 reference of the row-scale formats (int8, FP8 E4M3), restated without the
+    oracle's arithmetic: per head, the exact product q * s (q: the int8 value, or the E4M3
+    code decoded by torch's float8_e4m3fn; s: the fp32 row scale) is added to the fp32
+    accumulator with ONE rounding, in head order 0..15; then y = fp32(r + fp32(g * acc))
+    with numpy's fp32 multiply and add, and bf16 by torch.  The oracle's fp32 value y and
+    its bf16 output must equal this bit for bit.  The same chain with the product rounded
+    on its own first (two roundings per head) must differ somewhere, so this pin tells the
+    two readings apart (the bf16 output alone rarely can)."""
+    R, d, V = 211, 64, 90
+    toks, res, g = _tiny_case(seed=5, R=R, d=d, V=V, n_seq=4, T=40)
+    N = toks.size
+    if fmt == "int8":
+        q, s = oracle.fill_int8(23, 0, R, d)
+        qv, dt = q.astype(np.float64), oracle.INT8
+    else:
+        q, s = oracle.fill_fp8(23, 0, R, d)
+        qv, dt = _e4m3_torch(q), oracle.FP8
+    idx = oracle.indices(toks, None, R=R, vocab_size=V).reshape(N, 16)
+    acc1 = np.zeros((N, d), dtype=np.float32)                 # one rounding per head
+    acc2 = np.zeros((N, d), dtype=np.float32)                 # product rounded first
+    for h in range(16):
+        p = qv[idx[:, h]] * s[idx[:, h]].astype(np.float64)[:, None]     # exact in fp64
+        acc1 = _f32_of_exact_sum(p, acc1)
+        acc2 = (p.astype(np.float32) + acc2).astype(np.float32)
+    r32 = _bits_to_f64(res).reshape(N, d).astype(np.float32)
+    for rr, gg in ((np.zeros_like(r32), np.ones(d, np.float32)), (r32, g)):
+        y1 = (rr + (gg[None, :] * acc1).astype(np.float32)).astype(np.float32)
+        y2 = (rr + (gg[None, :] * acc2).astype(np.float32)).astype(np.float32)
+        rbits = torch.from_numpy(rr.ravel()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        want = torch.from_numpy(y1.ravel()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        for kw in (dict(table_i8=q, row_scale=s), dict(table_seed=23)):
+            out, y, _, _ = oracle.forward(toks, None, rbits, gg, R=R, d=d, dtype=dt,
+                                          acc=oracle.ACC_F32, vocab_size=V, want_aux=True, **kw)
+            assert np.array_equal(y.astype(np.float32).ravel().view(np.uint32), y1.ravel().view(np.uint32))
+            assert np.array_equal(out.ravel(), want)
+        assert np.any(y1 != y2)
+
+
 
 # --------------------------------------------------------------------------- low-precision rows
 def test_e4m3_decode_matches_torch_float8_e4m3fn():
