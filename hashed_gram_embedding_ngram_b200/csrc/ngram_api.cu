@@ -16,6 +16,7 @@
 #include <thread>
 #include <vector>
 
+#include <cuda.h>            // CUcontext / CUresult types for the driver entry points
 #include <cuda_runtime.h>
 
 #include "ngram.h"
@@ -776,17 +777,23 @@ ngram_status forward_uva(ngram_ctx *c, const Call &k) {
     return forward_direct_uva(c, k);
 }
 
-// AUTO: the first call of each batch-size bucket runs and times the three host modes
-// (UVA, UVA with dedup, DMA; all write the same output) twice each, keeps the fastest by
-// the better of its two runs (the first run of a mode also allocates its staging), and
-// later calls use it.  auto_choice holds NGRAM_RES_HOST_UVA, NGRAM_RES_HOST_DMA or
-// NGRAM_AUTO_UVA_DEDUP.
+// AUTO: the first call of each batch-size bucket runs the three host modes (UVA, UVA with
+// dedup, DMA; all write the same output), each once untimed (the first call of a mode
+// also allocates its staging) and then kNAutoTimed times timed, keeps the mode with the
+// lowest median time, and later calls use it.  auto_choice holds NGRAM_RES_HOST_UVA,
+// NGRAM_RES_HOST_DMA or NGRAM_AUTO_UVA_DEDUP.
+constexpr int kNAutoTimed = 3;
+
+ngram_status run_mode(ngram_ctx *c, const Call &k, int mode) {
+    if (mode == NGRAM_RES_HOST_UVA) return forward_direct_uva(c, k);
+    if (mode == NGRAM_AUTO_UVA_DEDUP) return forward_dedup_uva(c, k);
+    return forward_dma(c, k);
+}
+
 ngram_status time_mode(ngram_ctx *c, const Call &k, int mode, float *ms) {
     const auto h0 = std::chrono::steady_clock::now();
     NG_CUDA(cudaEventRecord(c->ev_t0, k.s), "cudaEventRecord");
-    if (mode == NGRAM_RES_HOST_UVA) NG_CHECK(forward_direct_uva(c, k));
-    else if (mode == NGRAM_AUTO_UVA_DEDUP) NG_CHECK(forward_dedup_uva(c, k));
-    else NG_CHECK(forward_dma(c, k));
+    NG_CHECK(run_mode(c, k, mode));
     NG_CUDA(cudaEventRecord(c->ev_t1, k.s), "cudaEventRecord");
     NG_CHECK(wait_event(c, c->ev_t1, "AUTO: timing"));
     NG_CUDA(cudaEventElapsedTime(ms, c->ev_t0, c->ev_t1), "cudaEventElapsedTime");
@@ -811,11 +818,12 @@ ngram_status forward_auto(ngram_ctx *c, const Call &k) {
     int best = NGRAM_RES_HOST_UVA;
     float t_best = 0.f;
     for (int m = 0; m < 3; ++m) {
-        float t0 = 0.f, t1 = 0.f;
-        NG_CHECK(time_mode(c, k, modes[m], &t0));
-        NG_CHECK(time_mode(c, k, modes[m], &t1));
-        const float t = std::min(t0, t1);
-        if (m == 0 || t < t_best) { best = modes[m]; t_best = t; }
+        NG_CHECK(run_mode(c, k, modes[m]));              // warm-up: staging, caches
+        float t[kNAutoTimed];
+        for (int r = 0; r < kNAutoTimed; ++r) NG_CHECK(time_mode(c, k, modes[m], &t[r]));
+        std::sort(t, t + kNAutoTimed);
+        const float med = t[kNAutoTimed / 2];
+        if (m == 0 || med < t_best) { best = modes[m]; t_best = med; }
     }
     c->auto_choice[b] = best;
     return NGRAM_OK;
@@ -1527,21 +1535,63 @@ constexpr size_t kNoAllocWords = 3ull * kNoAllocMaxEntries + 3ull * kNoAllocSlot
 
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocWords];
 
-// Device address of g_noalloc_scratch per device, looked up once per device.
+// Device address of g_noalloc_scratch per device, looked up once per device and again
+// whenever the device's current context is not the one the address was taken in (a
+// cudaDeviceReset destroys the primary context; the array of the next one may sit at
+// another address).  The context is identified by cuCtxGetId, reached through
+// cudaGetDriverEntryPoint (no link against libcuda); where that is unavailable, or no
+// context is current yet, the address is looked up again on that call.
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+struct NoallocAddr {
+    uint32_t *ptr = nullptr;
+    unsigned long long ctx_id = 0;   // 0: unknown
+};
+
 std::mutex g_noalloc_mu;
-uint32_t *g_noalloc_addr[256] = {nullptr};
+NoallocAddr g_noalloc_addr[256];
+PfnCtxGetCurrent g_ctx_get_current = nullptr;
+PfnCtxGetId g_ctx_get_id = nullptr;
+bool g_ctx_fns_tried = false;
+
+// Unique id of the calling thread's current context, or 0 when it cannot be had.
+unsigned long long current_ctx_id() {
+    if (!g_ctx_fns_tried) {
+        g_ctx_fns_tried = true;
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess && qb == cudaDriverEntryPointSuccess) {
+            g_ctx_get_current = reinterpret_cast<PfnCtxGetCurrent>(a);
+            g_ctx_get_id = reinterpret_cast<PfnCtxGetId>(b);
+        }
+        cudaGetLastError();                  // a failed query leaves no sticky error
+    }
+    if (g_ctx_get_current == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 ngram_status noalloc_scratch(uint32_t **out) {
     int dev = -1;
     NG_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 0 || dev >= 256) return fail(NGRAM_EUNSUPPORTED, "device ordinal %d out of range", dev);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
+    NoallocAddr &a = g_noalloc_addr[dev];
+    const unsigned long long id = current_ctx_id();
+    if (a.ptr == nullptr || id == 0 || id != a.ctx_id) {
+        a = NoallocAddr();
         void *p = nullptr;
         NG_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(noalloc scratch)");
-        g_noalloc_addr[dev] = static_cast<uint32_t *>(p);
+        a.ptr = static_cast<uint32_t *>(p);
+        a.ctx_id = current_ctx_id();         // the lookup above made the primary context current
     }
-    *out = g_noalloc_addr[dev];
+    *out = a.ptr;
     return NGRAM_OK;
 }
 
@@ -1559,7 +1609,7 @@ extern "C" ngram_status ngram_dedup_rows_noalloc(const ngram_hash_params *hp, ui
     if (count_out == nullptr) return fail(NGRAM_EINVAL, "count_out is NULL");
     const uint32_t H = p.n_bigram_heads + p.n_trigram_heads;
     const uint64_t N = static_cast<uint64_t>(n_seq) * T;
-    if (N * H > kNoAllocMaxEntries)
+    if (H == 0 || N > kNoAllocMaxEntries / H)          // N * H could wrap: compare by division
         return fail(NGRAM_EINVAL,
                     "ngram_dedup_rows_noalloc: %llu tokens x %u heads exceed its fixed scratch of %u "
                     "entries; use ngram_dedup_rows", static_cast<unsigned long long>(N), H,

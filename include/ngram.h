@@ -189,8 +189,9 @@ NGRAM_API ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *
  *                        from HBM; the call blocks the host until the rows are staged
  *                        (bounded wait, see ngram_set_wait_timeout);
  *              HOST_AUTO the first call of each batch-size bucket (ceil(log2 N)) runs
- *                        and times UVA, UVA with dedup (NGRAM_FLAG_DEDUP) and DMA
- *                        (synchronously); later calls use the fastest
+ *                        UVA, UVA with dedup (NGRAM_FLAG_DEDUP) and DMA, each once
+ *                        untimed and then three times timed (synchronously); later
+ *                        calls use the mode with the lowest median time
  *                        (ngram_auto_choice reports it).
  *   hp         hash parameters (NULL = defaults).
  *   max_tokens largest n_seq * T a later call may pass (>= 1).
@@ -320,7 +321,10 @@ NGRAM_API ngram_status ngram_dedup_rows(ngram_ctx *ctx, const int32_t *tokens,
  *   Limit: n_seq * T * heads <= 65,536 entries (4,096 tokens at 16 heads); larger
  *     batches return NGRAM_EINVAL with a message naming the limit.
  *   Set-up: the first call on each device looks the array's device address up (with
- *     that device current); make that first call before any stream capture.
+ *     that device current); make that first call before any stream capture.  The
+ *     address is kept per device together with the id of the context it was taken in;
+ *     a call that finds another context current (after cudaDeviceReset) looks it up
+ *     again, so make the first call after a reset before any stream capture too.
  *   Sharing: every call on a device uses the same array and leaves its contents
  *     behind; the call clears what must start empty.  Calls that overlap on the GPU
  *     (other streams, other host threads) race on the array: serialise them.

@@ -245,3 +245,19 @@ def test_prefetch_entry_points_reject_null_context():
     lib = ng.lib()
     assert lib.ngram_prefetch(None, 0, None, None, 1, 1, None) == ng.NGRAM_EINVAL
     assert lib.ngram_forward_staged(None, 0, None, None, None, None) == ng.NGRAM_EINVAL
+
+
+def test_noalloc_dedup_refuses_over_limit_batches_before_cuda():
+    """The limit check of ngram_dedup_rows_noalloc runs before any CUDA call, and a batch
+    whose n_seq * T * heads wraps in 64 bits (2^31 x 2^31 x 16 = 2^66) is refused too."""
+    lib = ng.lib()
+    P, u32, u64 = ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64
+    f = lib.ngram_dedup_rows_noalloc
+    f.argtypes = [P, u64, P, P, u32, u32, P, P, P, P]
+    f.restype = ctypes.c_int
+    hp = ng.ngram_default_hash_params(vocab_size=1000)
+    x = P(16)                                  # never dereferenced: refused first
+    for n_seq, T in ((1, 4097), (1 << 31, 1 << 31), (4096, 1 << 20)):
+        assert f(ctypes.byref(hp), 1000, x, None, n_seq, T, x, x, x, None) == ng.NGRAM_EINVAL
+        assert "65536" in ng.ngram_last_error()
+    assert f(ctypes.byref(hp), 0, x, None, 1, 1, x, x, x, None) == ng.NGRAM_EINVAL
