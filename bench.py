@@ -38,19 +38,13 @@ import ngram_inputs as gen  # noqa: E402
 METRIC = "n-gram embed tokens/s and gather GB/s (% of HBM or PCIe H2D roofline), 1 B200"
 UNIT = "tokens/s"
 HEADS = 16
-KERNEL_SOURCES = {   # the source files each timed kernel is built from
-    "bf16": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
-             "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
-    "int8": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
-             "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
-             "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
-    "fp8": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
-            "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
-            "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
-    "nvfp4": ["hashed_gram_embedding_ngram_b200/csrc/gather.cuh",
-              "hashed_gram_embedding_ngram_b200/csrc/gather_int8.cuh",
-              "hashed_gram_embedding_ngram_b200/csrc/gather_nvfp4.cuh",
-              "hashed_gram_embedding_ngram_b200/csrc/device_common.cuh"],
+_CS = "hashed_gram_embedding_ngram_b200/csrc/"
+KERNEL_SOURCES = {   # the source files each timed kernel and its processing order are built from
+    "bf16": [_CS + "gather.cuh", _CS + "device_common.cuh", _CS + "order.cuh"],
+    "int8": [_CS + "gather.cuh", _CS + "gather_int8.cuh", _CS + "device_common.cuh", _CS + "order.cuh"],
+    "fp8": [_CS + "gather.cuh", _CS + "gather_int8.cuh", _CS + "device_common.cuh", _CS + "order.cuh"],
+    "nvfp4": [_CS + "gather.cuh", _CS + "gather_int8.cuh", _CS + "gather_nvfp4.cuh",
+              _CS + "device_common.cuh", _CS + "order.cuh"],
 }
 KERNEL_NAME = {"bf16": "k_gather_bf16<16>", "int8": "k_gather_int8<16>",
                "fp8": "k_gather_fp8<16>", "nvfp4": "k_gather_nvfp4<16>"}
@@ -163,26 +157,6 @@ def kernel_sha(dtype: str = "bf16", read=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, dtype: str = "bf16"):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    kernel code as it is now (its kernel_sha line, first word; else None)."""
-    p = os.path.join(ROOT, "profiles", "gather_%s.txt" % workload)
-    if not os.path.exists(p):
-        return None
-    kv = {}
-    with open(p) as f:
-        for line in f:
-            if ":" in line and not line.startswith(" "):
-                k, v = line.split(":", 1)
-                kv[k.strip()] = v.strip()
-    if (kv.get("kernel_sha", "").split() or [""])[0] != kernel_sha(dtype):
-        return None
-    try:
-        return float(kv["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
-
-
 class ClockSampler:
     """nvidia-smi samples of SM clock, power and throttle reasons while running."""
 
@@ -267,14 +241,19 @@ def weak_scaling_tokens_per_s(world: int, tokens_per_rank: int, steps: int, elap
 
 
 # --------------------------------------------------------------------------- CPU oracle
-def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0):
-    """Time the oracle (test infrastructure; rows regenerated on the fly, the full table
-    cannot be materialised on the host) on a bounded sample of this workload's tokens."""
+def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0, table=None):
+    """Time the oracle (test infrastructure) on a bounded sample of this workload's tokens.
+    table: the materialised table (uint16 [R][d] bf16 bits, e.g. a view of pinned host
+    memory) the oracle reads its rows from; None: rows regenerated from the synthetic-table
+    definition (one Philox call per two elements).  Returns (tokens/s, tokens, seconds)."""
     import oracle
     rng = np.random.default_rng(seed)
-    kw = dict(R=w.R, d=w.d, dtype=oracle_dtype(w),
-              table_seed=gen.TABLE_SEED, acc=oracle.ACC_F32, n_threads=threads,
+    kw = dict(R=w.R, d=w.d, dtype=oracle_dtype(w), acc=oracle.ACC_F32, n_threads=threads,
               vocab_size=w.vocab)
+    if table is None:
+        kw["table_seed"] = gen.TABLE_SEED
+    else:
+        kw["table"] = table
     probe = rng.choice(w.N, size=min(w.N, 4 * threads), replace=False)
     t0 = time.perf_counter()
     oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=probe, **kw)
@@ -285,6 +264,31 @@ def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0):
     oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sel, **kw)
     dt = time.perf_counter() - t0
     return n / dt, n, dt
+
+
+def cpu_baseline_record(w, inp, budget_s: float, table=None, table_desc: str = "") -> dict:
+    """The oracle on all host cores and on one core, reading the materialised table when one
+    is given (the rows a CPU lookup would read), plus, as a secondary labelled figure, the
+    oracle regenerating its rows from their definition.  Tokens/s and the algorithmic GB/s."""
+    threads = os.cpu_count() or 1
+    per_tok = algorithmic_bytes(w) / w.N
+    src = "materialised" if table is not None else "regenerated"
+    v, n, dt = oracle_tokens_per_s(w, inp, budget_s, threads, table=table)
+    v1, n1, dt1 = oracle_tokens_per_s(w, inp, min(3.0, budget_s / 4), 1, seed=1, table=table)
+    rec = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "row_source": src,
+           "gbs": v * per_tok / 1e9,
+           "sample": "%d of %d tokens of this workload, %.1f s, rows read from %s" % (
+               n, w.N, dt, table_desc if table is not None else
+               "their synthetic-table definition (regenerated per element)"),
+           "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "gbs": v1 * per_tok / 1e9,
+                             "sample": "%d tokens, %.1f s" % (n1, dt1)}}
+    if table is not None:
+        vr, nr, dtr = oracle_tokens_per_s(w, inp, min(5.0, budget_s / 3), threads, seed=2)
+        rec["regenerated_rows"] = {"value": vr, "unit": UNIT, "cores": threads,
+                                   "gbs": vr * per_tok / 1e9,
+                                   "sample": "%d tokens, %.1f s, rows regenerated from their "
+                                             "definition (Philox-bound, secondary)" % (nr, dtr)}
+    return rec
 
 
 # --------------------------------------------------------------------------- arms
@@ -326,6 +330,11 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def resolved_launch(w, args) -> str:
+    """eager launches, or CUDA graphs of 100 steps (auto: graphs for N <= 1024 tokens)."""
+    return args.launch if args.launch != "auto" else ("graph" if w.N <= 1024 else "eager")
+
+
 def config_for(w, args) -> dict:
     return {
         "workload": w.name, "R": w.R, "d": w.d, "table_dtype": w.dtype,
@@ -336,33 +345,13 @@ def config_for(w, args) -> dict:
         "l2": "inputs larger than L2: %.2f GB moved per step vs 126 MB L2; %d token batches "
               "alternate" % (algorithmic_bytes(w) / 1e9, args.batches),
         "parallelism": "replicas x%d (tokens sharded, table replicated)" % args.gpus,
-        "launch": args.launch,
+        "launch": resolved_launch(w, args),
     }
 
 
-def run_ours(args, w):
-    import datetime
-
+def make_table(ng, w, dev):
+    """The workload's synthetic table in HBM (set-up, untimed): (dtype, table, scale)."""
     import torch
-    import torch.distributed as dist
-
-    import hashed_gram_embedding_ngram_b200 as ng
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    # ---- table (set-up, untimed): a replica of the whole table on every GPU
     dtype = {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
              "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[w.dtype]
     table = torch.empty((w.R, ng.ngram_row_bytes(dtype, w.d)), dtype=torch.uint8, device=dev)
@@ -370,56 +359,55 @@ def run_ours(args, w):
     if dtype != ng.NGRAM_BF16:     # per-row scales, or the one NVFP4 global scale
         scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
     ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
-    flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING,
-             "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER,
-             "token_gate": ng.NGRAM_FLAG_TOKEN_GATE}[args.variant]
-    grouped = args.variant == "sort" or (args.variant in ("default", "token_gate")
-                                         and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
-    # grouped bf16 / NVFP4 batches of >= 4096 tokens hash every token once, in the order
-    # step's count kernel, and the gather reads the row ids
-    prehash = grouped and w.dtype in ("bf16", "nvfp4") and w.N >= 4096
-    hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
-    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
+    return dtype, table, scale
 
-    # ---- inputs: this rank's token batches (distinct seeds per rank and batch)
-    host_tok, host_hist = [], []
-    for b in range(args.batches):
-        ts, hs = rank_seeds(rank, b)
-        host_tok.append(gen.tokens_for(w, ts))
-        host_hist.append(gen.history_for(w, hs))
-    res_bits = gen.residual_bf16_bits(w.N, w.d, gen.RESIDUAL_SEED + rank)
-    gate_h = gen.gate_f32(w.d)
-    tok_d = [torch.from_numpy(t).to(dev) for t in host_tok]
-    hist_d = [None if h is None else torch.from_numpy(h).to(dev) for h in host_hist]
-    res_cpu = torch.from_numpy(res_bits.view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
-    residual = res_cpu.to(dev)
-    out = torch.empty_like(residual)
-    gate = torch.from_numpy(gate_h).to(dev)
-    if args.variant == "token_gate":       # one bf16 gate per token and column
-        gate = torch.from_numpy(np.random.default_rng(12).uniform(0, 1, (w.N, w.d)).astype(np.float32)
-                                ).to(torch.bfloat16).to(dev)
-    stream = torch.cuda.current_stream()
+
+class Batches:
+    """One rank's token batches (distinct seeds per rank and batch) and the activations of
+    a workload, on the host and on the device."""
+
+    def __init__(self, w, dev, rank=0, batches=2, token_gate=False):
+        import torch
+        self.host_tok, self.host_hist = [], []
+        for b in range(batches):
+            ts, hs = rank_seeds(rank, b)
+            self.host_tok.append(gen.tokens_for(w, ts))
+            self.host_hist.append(gen.history_for(w, hs))
+        self.res_bits = gen.residual_bf16_bits(w.N, w.d, gen.RESIDUAL_SEED + rank)
+        self.gate_h = gen.gate_f32(w.d)
+        self.tok_d = [torch.from_numpy(t).to(dev) for t in self.host_tok]
+        self.hist_d = [None if h is None else torch.from_numpy(h).to(dev) for h in self.host_hist]
+        self.res_cpu = torch.from_numpy(self.res_bits.view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
+        self.residual = self.res_cpu.to(dev)
+        self.out = torch.empty_like(self.residual)
+        self.gate = torch.from_numpy(self.gate_h).to(dev)
+        if token_gate:                      # one bf16 gate per token and column
+            g = np.random.default_rng(12).uniform(0, 1, (w.N, w.d)).astype(np.float32)
+            self.gate = torch.from_numpy(g).to(torch.bfloat16).to(dev)
+        self.n = batches
+
+    def inputs(self, b=0):
+        return {"tokens": self.host_tok[b], "history": self.host_hist[b], "residual": self.res_bits,
+                "gate": self.gate_h}
+
+
+def time_forward(ng, ctx, bt, stream, steps, warmup, launch, dev, barrier=lambda: None, G=100):
+    """W untimed warm-up steps, then K timed steps bracketed by a barrier and a
+    synchronize.  Eager: one ngram_forward per step, CUDA events around each launch.
+    Graph: G steps captured once into a CUDA graph and replayed, events around each replay
+    (decode-sized launches are otherwise bound by the Python launch path).  Returns
+    (elapsed_ms, kernel ms per step, K, clock summary)."""
+    import torch
 
     def step(i, s=None):
-        b = i % args.batches
-        ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b],
+        b = i % bt.n
+        ng.ngram_forward(ctx, bt.tok_d[b], bt.residual, bt.gate, out=bt.out, history=bt.hist_d[b],
                          stream=s if s is not None else stream)
 
-    # ---- distinct rows of the first batch (outside any timed region): U * row bytes is the
-    # least a lookup of this batch can read from the table, whatever the order or reuse
-    _, _, ucount = ng.ngram_dedup_rows(ctx, tok_d[0], history=hist_d[0])
-    unique_rows = int(ucount.item())
-    read_gbs = read_stream_gbs(dev)
-
-    # ---- device-resident timing.  Eager: one launch per step, CUDA events around each
-    # launch.  Graph: G steps captured once into a CUDA graph and replayed, events around
-    # each replay (decode-sized launches are otherwise bound by the Python launch path).
-    launch = args.launch if args.launch != "auto" else ("graph" if w.N <= 1024 else "eager")
-    G = 100
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    K = args.steps
+    K = steps
     graph = None
     if launch == "graph":
         K = max(G, (K + G - 1) // G * G)
@@ -453,6 +441,260 @@ def run_ours(args, w):
     if graph is not None:
         kern_ms /= G                          # per step inside the graph (kernel + gap)
         del graph
+    return elapsed_ms, kern_ms, K, clk.summary()
+
+
+def distinct_bytes(w, unique_rows: int) -> int:
+    """The least DRAM traffic of one launch whatever the order or reuse: every distinct row
+    once, the residual read and output write per token, the token ids and the gate."""
+    return unique_rows * row_bytes(w) + w.N * (2 * 2 * w.d + 4) + 4 * w.d
+
+
+PROFILE_FOR = {"full_prefill": "gather_bf16_prefill", "int8_uniform": "gather_int8_uniform",
+               "fp8_prefill": "gather_fp8_prefill", "nvfp4_prefill": "gather_nvfp4_prefill"}
+
+
+def profiled_traffic(workload: str, dtype: str, distinct: int):
+    """DRAM bytes per launch, estimated from the committed ncu summary of a small case of the
+    same kernel in the same launch configuration (profiles/<kernel>_<workload>.txt), if it was
+    taken on the kernel code as it is now (its kernel_sha line, first word).  The small case's
+    DRAM bytes over its own distinct bytes (the excess of re-reads over the least traffic)
+    times this launch's distinct bytes.  Returns (bytes, source) or (None, reason)."""
+    name = PROFILE_FOR.get(workload)
+    if name is None:
+        return None, "no small-case profile for this workload"
+    p = os.path.join(ROOT, "profiles", name + ".txt")
+    if not os.path.exists(p):
+        return None, "profiles/%s.txt missing" % name
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith(" "):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if (kv.get("kernel_sha", "").split() or [""])[0] != kernel_sha(dtype):
+        return None, "profiles/%s.txt was taken on other kernel code" % name
+    try:
+        dram = float(kv["small_dram_bytes_per_launch"].split()[0])
+        small = float(kv["small_distinct_bytes_per_launch"].split()[0])
+    except (KeyError, ValueError, IndexError):
+        return None, "profiles/%s.txt lacks the small-case figures" % name
+    return dram / small * distinct, ("ncu DRAM bytes of %s (%s) over its distinct bytes = %.4f, "
+                                     "times this launch's distinct bytes" % (
+                                         kv.get("small_workload", "?").split(" ")[0], name, dram / small))
+
+
+def hbm_record(ng, dev, w, dtype, table, scale, steps, launch, read_gbs=None, flags=0) -> dict:
+    """One workload on an HBM-resident table, timed like the headline (bounded steps), as a
+    sub-record of the bench line: tokens/s, the roofline against the measured copy peak,
+    the clocks sampled during its timed region and the device error word."""
+    import torch
+    hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
+    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
+    bt = Batches(w, dev)
+    stream = torch.cuda.current_stream()
+    elapsed_ms, kern_ms, K, clocks = time_forward(ng, ctx, bt, stream, steps, 5, launch, dev)
+    st, info = ng.ngram_get_device_error(ctx)
+    _, _, ucount = ng.ngram_dedup_rows(ctx, bt.tok_d[0], history=bt.hist_d[0])
+    U = int(ucount.item())
+    ctx.close()
+    peaks = measured_peaks()
+    nbytes = algorithmic_bytes(w)
+    dist_b = distinct_bytes(w, U)
+    achieved = nbytes / (kern_ms / 1e3) / 1e9
+    traffic, tsrc = profiled_traffic(w.name, w.dtype, dist_b)
+    rec = {
+        "workload": w.name,
+        "config": {"R": w.R, "d": w.d, "table_dtype": w.dtype, "n_seq": w.n_seq, "T": w.T,
+                   "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
+                   "history": w.history, "residency": "hbm", "launch": launch,
+                   "table_gib": round(w.R * stored_row_bytes(w) / 2**30, 2)},
+        "value": w.N * K / (elapsed_ms / 1e3), "unit": UNIT, "ms_per_step": elapsed_ms / K,
+        "kernel_ms": kern_ms, "steps": K,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "traffic_source": tsrc,
+                     "algorithmic_bytes_per_launch": nbytes, "unique_rows": U,
+                     "unique_row_bytes": U * row_bytes(w), "distinct_bytes_per_launch": dist_b,
+                     "frac_on_distinct_bytes": dist_b / (kern_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
+        "clocks": clocks,
+        "device_error": "ok" if st == ng.NGRAM_OK else str(info),
+    }
+    if read_gbs:
+        rec["roofline"]["frac_of_read_stream"] = achieved / read_gbs
+    if launch == "graph":
+        rec["us_per_step"] = kern_ms * 1e3
+        if clocks.get("sm_mhz"):
+            rec["kcycles_per_step"] = kern_ms * clocks["sm_mhz"]      # us x MHz / 1000
+    return rec
+
+
+def host_mem_available() -> int:
+    """MemAvailable of this host in bytes (0 if unknown)."""
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return int(line.split()[1]) * 1024
+    except OSError:
+        pass
+    return 0
+
+
+def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
+    """The other configurations on one GPU, each a sub-record of the bench line (bounded:
+    fixed step counts, tables filled once).  Called after the headline with the full bf16
+    table still resident; ends with the CPU baseline on the materialised host table, the
+    host-resident configuration, and the 8- and 4-bit tables."""
+    import gc
+
+    import torch
+    os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+    t_start = time.perf_counter()
+    W = gen.WORKLOADS
+    extra = []
+    dtype, table, scale = full
+    full.clear()
+    # ---- mid (its own 9.5 GiB table), the decode batches and the backward on the full table
+    mid = W["mid"]
+    mdt, mtab, msc = make_table(ng, mid, dev)
+    extra.append(hbm_record(ng, dev, mid, mdt, mtab, msc, 400, "eager", read_gbs))
+    del mtab, msc
+    gc.collect()
+    torch.cuda.empty_cache()
+    for n in (1, 16, 64, 256):
+        extra.append(hbm_record(ng, dev, W["full_decode_%d" % n], dtype, table, scale, 20_000, "graph"))
+    fw = W["full_prefill"]
+    ctx = ng.ngram_init(table, fw.R, fw.d, dtype, ng.NGRAM_RES_HBM,
+                        ng.ngram_default_hash_params(vocab_size=fw.vocab), fw.N)
+    bw = backward_record(ng, dev, fw, ctx, 2, 100, 5)
+    ctx.close()
+    del ctx
+    bw.update(workload="full_prefill_backward",
+              config={"R": fw.R, "d": fw.d, "table_dtype": "bf16", "n_seq": fw.n_seq, "T": fw.T,
+                      "mode": "backward: table gradient + shared-gate gradient"})
+    extra.append(bw)
+    # ---- CPU baseline on the materialised host table, then the host-resident configuration
+    host_bytes = fw.R * fw.d * 2
+    avail = host_mem_available()
+    ht = None
+    if avail >= host_bytes + (24 << 30):
+        t0 = time.perf_counter()
+        ht = ng.HostTable((fw.R, fw.d), torch.bfloat16)
+        pin_s = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ng.ngram_fill_synthetic(ht.tensor, fw.R, fw.d, ng.NGRAM_BF16, gen.TABLE_SEED)
+        torch.cuda.synchronize()
+        fill_s = time.perf_counter() - t0
+    else:
+        pin_s = fill_s = None
+    if not args.no_cpu_baseline:
+        tab = None if ht is None else ht.tensor.view(torch.int16).numpy().view(np.uint16)
+        line["cpu_baseline"] = cpu_baseline_record(
+            fw, bt_full.inputs(0), args.cpu_seconds, table=tab,
+            table_desc="the materialised 20,000,000 x 2560 bf16 table (95.4 GiB, pinned host memory)")
+        if ht is None:
+            line["cpu_baseline"]["note"] = ("host RAM too small for the 95.4 GiB table (%.1f GiB "
+                                            "available): rows regenerated" % (avail / 2**30))
+    if ht is not None:
+        with ClockSampler(gpu_id_for(dev)) as clk:
+            report, h2d, gemm_ms, gemm_tflops = host_modes(
+                ng, ht, fw.R, fw.d, ["host_decode_256", "host_prefill"], dev, 200,
+                modes=("uva", "uva_dedup", "dma", "auto"))
+        clocks = clk.summary()
+        for name, entry in report.items():
+            hw = W[name]
+            best = entry["auto"]
+            extra.append({
+                "workload": name,
+                "config": {"R": fw.R, "d": fw.d, "table_dtype": "bf16", "n_seq": hw.n_seq, "T": hw.T,
+                           "residency": "host (pinned, mapped)", "pin_s": pin_s, "fill_s": fill_s,
+                           "stand_in": "bf16 [4096x2560]x[2560x2560] GEMM looped on a second stream"},
+                "value": best["tokens_per_s"], "unit": UNIT, "ms_per_step": best["ms"],
+                "steps": entry["steps"], "mode": "auto (chose %s)" % best.get("choice"),
+                "roofline": {"bound": "pcie_h2d", "achieved": best["nominal_row_gbs"], "peak": h2d,
+                             "unit": "GB/s", "frac": best["nominal_row_gbs"] / h2d,
+                             "nominal_bytes": "16 x 5120 B per token, every mode",
+                             "peak_source": "measured in this run: pinned 1 GiB cudaMemcpyAsync, best of 10"},
+                "modes": {m: entry[m] for m in ("uva", "uva_dedup", "dma", "auto")},
+                "overlap": {"gemm_alone_tflops": gemm_tflops, "gemm_alone_ms": gemm_ms,
+                            "per_mode": {m: {"lookup_alone_ms": entry[m]["ms"],
+                                             "lookup_overlapped_ms": entry[m]["overlapped_ms"],
+                                             "gemm_tflops_overlapped": entry[m]["gemm_tflops_overlapped"]}
+                                         for m in ("uva", "uva_dedup", "dma", "auto")}},
+                "prefetch": entry.get("prefetch"),
+                "clocks": clocks,
+                "device_error": "ok" if all(entry[m]["device_error"] == ng.NGRAM_OK
+                                            for m in ("uva", "uva_dedup", "dma", "auto")) else "set",
+            })
+        ht.close()
+    else:
+        extra.append({"workload": "host_prefill", "skipped": "host RAM: %.1f GiB available, the table "
+                                                             "needs 95.4 GiB + 24 GiB margin" % (avail / 2**30)})
+    # ---- the 8- and 4-bit tables (the bf16 table is released first)
+    del table, scale
+    gc.collect()
+    torch.cuda.empty_cache()
+    for name in ("int8_uniform", "fp8_prefill", "nvfp4_prefill"):
+        lw = W[name]
+        ldt, ltab, lsc = make_table(ng, lw, dev)
+        extra.append(hbm_record(ng, dev, lw, ldt, ltab, lsc, 200, "eager"))
+        del ltab, lsc
+        gc.collect()
+        torch.cuda.empty_cache()
+    line["extra"] = extra
+    line["extra_wall_s"] = time.perf_counter() - t_start
+
+
+def run_ours(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_ngram_b200 as ng
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- table (set-up, untimed): a replica of the whole table on every GPU
+    dtype, table, scale = make_table(ng, w, dev)
+    flags = {"default": 0, "dedup": ng.NGRAM_FLAG_DEDUP, "tma": ng.NGRAM_FLAG_TMA_STAGING,
+             "sort": ng.NGRAM_FLAG_SORT, "batch_order": ng.NGRAM_FLAG_BATCH_ORDER,
+             "token_gate": ng.NGRAM_FLAG_TOKEN_GATE}[args.variant]
+    grouped = args.variant == "sort" or (args.variant in ("default", "token_gate")
+                                         and w.N >= ng.NGRAM_SORT_MIN_TOKENS)
+    # grouped bf16 / NVFP4 batches of >= 4096 tokens hash every token once, in the order
+    # step's count kernel, and the gather reads the row ids
+    prehash = grouped and w.dtype in ("bf16", "nvfp4") and w.N >= 4096
+    hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
+    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
+
+    # ---- inputs: this rank's token batches (distinct seeds per rank and batch)
+    bt = Batches(w, dev, rank, args.batches, token_gate=args.variant == "token_gate")
+    stream = torch.cuda.current_stream()
+
+    # ---- distinct rows of the first batch (outside any timed region): U * row bytes is the
+    # least a lookup of this batch can read from the table, whatever the order or reuse
+    _, _, ucount = ng.ngram_dedup_rows(ctx, bt.tok_d[0], history=bt.hist_d[0])
+    unique_rows = int(ucount.item())
+    read_gbs = read_stream_gbs(dev)
+
+    # ---- device-resident timing
+    launch = resolved_launch(w, args)
+    elapsed_ms, kern_ms, K, clocks = time_forward(ng, ctx, bt, stream, args.steps, args.warmup,
+                                                  launch, dev, barrier)
     st, info = ng.ngram_get_device_error(ctx)
     if st != ng.NGRAM_OK:
         raise SystemExit("device error word set: %s" % info)
@@ -460,27 +702,28 @@ def run_ours(args, w):
     # ---- end to end through the host-buffer call: every step moves its tokens and
     # residual from pinned host memory to the device and its output back to the host
     # (ngram_forward_host pipelines the copies with the gather in ~8 MB chunks)
-    tok_h = [torch.from_numpy(t).pin_memory() for t in host_tok]
-    hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in host_hist]
-    res_h = res_cpu.pin_memory()
+    tok_h = [torch.from_numpy(t).pin_memory() for t in bt.host_tok]
+    hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in bt.host_hist]
+    res_h = bt.res_cpu.pin_memory()
     out_h = torch.empty_like(res_h).pin_memory()
-    gate_h_tok = gate.cpu().pin_memory() if args.variant == "token_gate" else None
+    gate_h_tok = bt.gate.cpu().pin_memory() if args.variant == "token_gate" else None
     E = max(1, args.e2e_steps)
 
     def e2e_step(i):
         b = i % args.batches
         if args.variant == "default":
-            ng.ngram_forward_host(ctx, tok_h[b], res_h, gate, out=out_h, history=hist_h[b],
+            ng.ngram_forward_host(ctx, tok_h[b], res_h, bt.gate, out=out_h, history=hist_h[b],
                                   stream=stream)
         else:                                 # staged variants: copy in, forward, copy out
-            tok_d[b].copy_(tok_h[b], non_blocking=True)
+            bt.tok_d[b].copy_(tok_h[b], non_blocking=True)
             if hist_h[b] is not None:
-                hist_d[b].copy_(hist_h[b], non_blocking=True)
-            residual.copy_(res_h, non_blocking=True)
+                bt.hist_d[b].copy_(hist_h[b], non_blocking=True)
+            bt.residual.copy_(res_h, non_blocking=True)
             if gate_h_tok is not None:        # a per-token gate is an activation: it comes in too
-                gate.copy_(gate_h_tok, non_blocking=True)
-            ng.ngram_forward(ctx, tok_d[b], residual, gate, out=out, history=hist_d[b], stream=stream)
-            out_h.copy_(out, non_blocking=True)
+                bt.gate.copy_(gate_h_tok, non_blocking=True)
+            ng.ngram_forward(ctx, bt.tok_d[b], bt.residual, bt.gate, out=bt.out, history=bt.hist_d[b],
+                             stream=stream)
+            out_h.copy_(bt.out, non_blocking=True)
 
     for i in range(min(3, E)):
         e2e_step(i)
@@ -499,7 +742,6 @@ def run_ours(args, w):
 
     # ---- max over ranks
     elapsed_ms, kern_ms, e2e_ms = max_over_ranks([elapsed_ms, kern_ms, e2e_ms], world, dev)
-    clocks = clk.summary()
 
     if rank == 0:
         value = weak_scaling_tokens_per_s(world, w.N, K, elapsed_ms)
@@ -507,15 +749,18 @@ def run_ours(args, w):
         peaks = measured_peaks()
         bytes_launch = algorithmic_bytes(w) + (w.N * 2 * w.d if args.variant == "token_gate" else 0)
         achieved = bytes_launch / (kern_ms / 1e3) / 1e9
+        dist_b = distinct_bytes(w, unique_rows)
+        traffic, tsrc = (profiled_traffic(w.name, w.dtype, dist_b) if args.variant == "default"
+                         else (None, "variant %s: not profiled" % args.variant))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": dict(config_for(w, args), launch=launch),
+            "config": config_for(w, args),
             "gather_gbs": bytes_launch * world * K / (elapsed_ms / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic(w.name, w.dtype) if args.variant == "default" else None,
+                         "traffic": traffic, "traffic_source": tsrc,
                          "kernel": ("hash + dedup + compact + gather (8 kernels)" if args.variant == "dedup"
                                     else "k_gather_bf16_bulk<16>" if args.variant == "tma"
                                     else ("grouped order (3 kernels%s) + " % (
@@ -524,6 +769,8 @@ def run_ours(args, w):
                          "kernel_ms": kern_ms, "algorithmic_bytes_per_launch": bytes_launch,
                          "unique_rows": unique_rows,
                          "unique_row_bytes": unique_rows * row_bytes(w),
+                         "distinct_bytes_per_launch": dist_b,
+                         "frac_on_distinct_bytes": dist_b / (kern_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                          "read_stream_gbs": read_gbs, "frac_of_read_stream": achieved / read_gbs,
                          "frac_of_8tbs_nominal": achieved / 8000.0,
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
@@ -536,21 +783,19 @@ def run_ours(args, w):
             "clocks": clocks,
             "gpu_launches": K * (8 if args.variant == "dedup" else 4 if grouped else 1),
         }
-        if world == 1 and not args.no_cpu_baseline:
-            threads = os.cpu_count() or 1
-            inp = {"tokens": host_tok[0], "history": host_hist[0], "residual": res_bits,
-                   "gate": gate_h}
-            v, n, dt = oracle_tokens_per_s(w, inp, args.cpu_seconds, threads)
-            v1, n1, dt1 = oracle_tokens_per_s(w, inp, min(3.0, args.cpu_seconds / 4), 1, seed=1)
-            line["cpu_baseline"] = {
-                "value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                "sample": "%d of %d tokens of this workload, %.1f s, rows regenerated from "
-                          "the synthetic-table definition (the 95 GiB table is not on the host)"
-                          % (n, w.N, dt),
-                "single_thread": {"value": v1, "unit": UNIT, "cores": 1,
-                                  "sample": "%d tokens, %.1f s" % (n1, dt1)}}
+        extras = (world == 1 and not args.no_extra and args.variant == "default"
+                  and w.name == "full_prefill")
+        ctx.close()
+        ctx = None                            # the context object holds the table too
+        if extras:
+            full = [dtype, table, scale]      # run_extras releases the bf16 table midway
+            del table, scale
+            run_extras(args, ng, dev, full, bt, read_gbs, line)
+        elif world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_record(w, bt.inputs(0), args.cpu_seconds)
         print(json.dumps(line), flush=True)
-    ctx.close()
+    else:
+        ctx.close()
     if world > 1:
         dist.destroy_process_group()
 
@@ -638,30 +883,16 @@ def prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B):
             "lookup_on_critical_path_ms": piped_ms - comp_ms}
 
 
-def run_host(args):
-    """Host-resident table: the 20M x 2560 bf16 table pinned in host memory, each host
-    workload timed in UVA, DMA and AUTO residency, alone and overlapped with a stand-in
-    bf16 [4096 x 2560] x [2560 x 2560] GEMM looped on a second stream."""
-    # the DMA mode gathers rows with OpenMP threads; let them sleep between calls so they
-    # do not spin on the cores the launching thread needs during the other modes
-    os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+HOST_MODES = ("uva", "uva_grouped", "uva_dedup", "dma", "auto")
+
+
+def host_modes(ng, ht, R, d, names, dev, host_steps, modes=HOST_MODES, prefetch=True):
+    """Each host workload in each residency mode: time alone (K calls, CUDA events; wall
+    time for the host-blocking DMA mode), time again while a stand-in bf16
+    [4096 x 2560] x [2560 x 2560] GEMM loops on a second stream, check bit-identity with
+    the first mode and the device error word; then the prefetch pattern.  Returns
+    (report, h2d GB/s, GEMM ms alone, GEMM TFLOP/s alone)."""
     import torch
-
-    import hashed_gram_embedding_ngram_b200 as ng
-
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    names = args.host_workloads.split(",")
-    R, d = gen.WORKLOADS[names[0]].R, gen.WORKLOADS[names[0]].d
-    if args.host_rows:
-        R = args.host_rows
-    t0 = time.perf_counter()
-    ht = ng.HostTable((R, d), torch.bfloat16)
-    pin_s = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    ng.ngram_fill_synthetic(ht.tensor, R, d, ng.NGRAM_BF16, gen.TABLE_SEED)
-    torch.cuda.synchronize()
-    fill_s = time.perf_counter() - t0
     h2d = measure_h2d_gbs(dev)
     main_s = torch.cuda.current_stream()
     side = torch.cuda.Stream()
@@ -686,7 +917,7 @@ def run_host(args):
     torch.cuda.synchronize()
     gemm_ms = a.elapsed_time(b) / 200
     report = {}
-    modes = {"uva": (ng.NGRAM_RES_HOST_UVA, 0), "uva_grouped": (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT),
+    table = {"uva": (ng.NGRAM_RES_HOST_UVA, 0), "uva_grouped": (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_SORT),
              "uva_dedup": (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP),
              "dma": (ng.NGRAM_RES_HOST_DMA, 0), "auto": (ng.NGRAM_RES_HOST_AUTO, 0)}
     for name in names:
@@ -697,11 +928,12 @@ def run_host(args):
         res = torch.from_numpy(inp["residual"].view(np.int16)).view(torch.bfloat16).view(w.N, w.d).to(dev)
         gate = torch.from_numpy(inp["gate"]).to(dev)
         out = torch.empty_like(res)
-        K = max(5, min(args.host_steps, int(2e5 / w.N)))
+        K = max(5, min(host_steps, int(2e5 / w.N)))
         row_bytes = HEADS * 2 * w.d * w.N               # nominal row bytes per call
         entry = {"N": w.N, "steps": K}
         ref = None
-        for mname, (where, flags) in modes.items():
+        for mname in modes:
+            where, flags = table[mname]
             hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
             ctx = ng.ngram_init(ht.tensor, R, d, ng.NGRAM_BF16, where, hp, w.N)
             for _ in range(3):
@@ -740,15 +972,45 @@ def run_host(args):
                 "nominal_row_gbs": row_bytes / (ms / 1e3) / 1e9,
                 "frac_of_h2d": row_bytes / (ms / 1e3) / 1e9 / h2d,
                 "overlapped_ms": ms_ov, "gemm_tflops_overlapped": gemm_flop / (gemm_ov_ms / 1e3) / 1e12,
-                "bit_identical_to_uva": same, "device_error": st,
+                "bit_identical_to_%s" % modes[0]: same, "device_error": st,
             }
             if where == ng.NGRAM_RES_HOST_AUTO:
                 entry[mname]["choice"] = {ng.NGRAM_RES_HOST_UVA: "uva", ng.NGRAM_RES_HOST_DMA: "dma",
                                           ng.NGRAM_AUTO_UVA_DEDUP: "uva_dedup"}.get(
                     ng.ngram_auto_choice(ctx, w.N), "undecided")
             ctx.close()
-        entry["prefetch"] = prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B)
+        if prefetch:
+            entry["prefetch"] = prefetch_pipeline(ng, ht, R, d, w, gemm_ms, time_gemms, main_s, dev, A, B)
         report[name] = entry
+    return report, h2d, gemm_ms, gemm_flop / (gemm_ms / 1e3) / 1e12
+
+
+def run_host(args):
+    """Host-resident table: the 20M x 2560 bf16 table pinned in host memory, each host
+    workload timed in UVA, DMA and AUTO residency, alone and overlapped with a stand-in
+    bf16 [4096 x 2560] x [2560 x 2560] GEMM looped on a second stream."""
+    # the DMA mode gathers rows with OpenMP threads; let them sleep between calls so they
+    # do not spin on the cores the launching thread needs during the other modes
+    os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+    import torch
+
+    import hashed_gram_embedding_ngram_b200 as ng
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    names = args.host_workloads.split(",")
+    R, d = gen.WORKLOADS[names[0]].R, gen.WORKLOADS[names[0]].d
+    if args.host_rows:
+        R = args.host_rows
+    t0 = time.perf_counter()
+    ht = ng.HostTable((R, d), torch.bfloat16)
+    pin_s = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    ng.ngram_fill_synthetic(ht.tensor, R, d, ng.NGRAM_BF16, gen.TABLE_SEED)
+    torch.cuda.synchronize()
+    fill_s = time.perf_counter() - t0
+    with ClockSampler(gpu_id_for(dev)) as clk:
+        report, h2d, gemm_ms, gemm_tflops = host_modes(ng, ht, R, d, names, dev, args.host_steps)
     head = names[-1]
     best = report[head]["auto"]
     line = {
@@ -762,8 +1024,9 @@ def run_host(args):
         "roofline": {"bound": "pcie_h2d", "achieved": best["nominal_row_gbs"], "peak": h2d,
                      "unit": "GB/s", "frac": best["nominal_row_gbs"] / h2d, "traffic": None,
                      "peak_source": "measured in this run: pinned 1 GiB cudaMemcpyAsync, best of 10"},
-        "gemm_alone_tflops": gemm_flop / (gemm_ms / 1e3) / 1e12,
+        "gemm_alone_tflops": gemm_tflops,
         "host_modes": report,
+        "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
     ht.close()
@@ -879,31 +1142,15 @@ def run_shard(args, w):
         dist.destroy_process_group()
 
 
-def run_backward(args, w):
-    """The backward pass of the lookup, timed like the forward: one step = the table
-    gradient (ngram_backward_rows) + the shared-gate gradient (ngram_backward_gate) of one
-    batch, on one GPU.  CUDA events around each call give the per-kernel-group times."""
+def backward_record(ng, dev, w, ctx, batches, steps, warmup) -> dict:
+    """The backward pass of the lookup on one batch: the table gradient
+    (ngram_backward_rows) then the shared-gate gradient (ngram_backward_gate), CUDA events
+    around each call; their algorithmic bytes and stream bounds."""
     import torch
-
-    import hashed_gram_embedding_ngram_b200 as ng
-
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
-    dtype = {"bf16": ng.NGRAM_BF16, "int8": ng.NGRAM_INT8_ROWSCALE,
-             "fp8": ng.NGRAM_FP8_E4M3_ROWSCALE, "nvfp4": ng.NGRAM_NVFP4}[w.dtype]
-    table = torch.empty((w.R, ng.ngram_row_bytes(dtype, w.d)), dtype=torch.uint8, device=dev)
-    scale = None
-    if dtype != ng.NGRAM_BF16:
-        scale = torch.empty((1 if dtype == ng.NGRAM_NVFP4 else w.R,), dtype=torch.float32, device=dev)
-    ng.ngram_fill_synthetic(table, w.R, w.d, dtype, gen.TABLE_SEED, row_scale=scale)
-    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM,
-                        ng.ngram_default_hash_params(vocab_size=w.vocab), w.N, row_scale=scale)
     N, d, H = w.N, w.d, HEADS
-    toks = [torch.from_numpy(gen.tokens_for(w, gen.TOKEN_SEED + b)).to(dev) for b in range(args.batches)]
+    toks = [torch.from_numpy(gen.tokens_for(w, gen.TOKEN_SEED + b)).to(dev) for b in range(batches)]
     hists = [None if not w.history else torch.from_numpy(gen.history_for(w, gen.HISTORY_SEED + b)).to(dev)
-             for b in range(args.batches)]
+             for b in range(batches)]
     rng = np.random.default_rng(11)
     dy = torch.from_numpy(rng.standard_normal((N, d), dtype=np.float32)).to(torch.bfloat16).to(dev)
     gate = torch.from_numpy(gen.gate_f32(d)).to(dev)
@@ -914,19 +1161,19 @@ def run_backward(args, w):
     stream = torch.cuda.current_stream()
 
     def rows(i):
-        b = i % args.batches
+        b = i % batches
         ng.ngram_backward_rows(ctx, toks[b], dy, gate, history=hists[b], uniq_out=uniq,
                                count_out=count, grad_rows=grad_rows, stream=stream)
 
     def gate_grad(i):
-        b = i % args.batches
+        b = i % batches
         ng.ngram_backward_gate(ctx, toks[b], dy, history=hists[b], out=grad_gate, stream=stream)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         rows(i)
         gate_grad(i)
     torch.cuda.synchronize()
-    K = args.steps
+    K = steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     Us = []
     with ClockSampler(gpu_id_for(dev)) as clk:
@@ -938,9 +1185,10 @@ def run_backward(args, w):
             gate_grad(i)
             ev[i][2].record(stream)
         torch.cuda.synchronize()
-    for b in range(args.batches):          # distinct rows of each batch (outside the timing)
+    for b in range(batches):               # distinct rows of each batch (outside the timing)
         rows(b)
         Us.append(int(count.item()))
+    st, info = ng.ngram_get_device_error(ctx)
     rows_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
     gate_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
     step_ms = statistics.fmean(e[0].elapsed_time(e[2]) for e in ev)
@@ -954,11 +1202,10 @@ def run_backward(args, w):
     # measured write stream plus dy at the measured read stream
     wr_gbs, rd_gbs = write_stream_gbs(dev), read_stream_gbs(dev)
     rows_bound_ms = (U * 4 * d / wr_gbs + N * 2 * d / rd_gbs) / 1e6
-    line = {
-        "metric": "n-gram embed backward tokens/s (table + gate gradients), 1 B200",
-        "value": N / (step_ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": args.warmup,
-        "ms_per_step": step_ms, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
-        "config": dict(config_for(w, args), mode="backward", distinct_rows_per_batch=U),
+    del grad_rows
+    return {
+        "value": N / (step_ms / 1e3), "unit": UNIT, "steps": K, "warmup": warmup,
+        "ms_per_step": step_ms, "distinct_rows_per_batch": U,
         "backward_rows": {"ms": rows_ms, "algorithmic_bytes": rows_bytes,
                           "achieved_gbs": rows_bytes / rows_ms / 1e6,
                           "frac": rows_bytes / rows_ms / 1e6 / peaks["hbm_gbs"],
@@ -972,8 +1219,34 @@ def run_backward(args, w):
                           "kernels": "k_gate_grad + k_gate_reduce"},
         "peak": {"hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"]},
         "clocks": clk.summary(),
+        "device_error": "ok" if st == ng.NGRAM_OK else str(info),
     }
+
+
+def run_backward(args, w):
+    """The backward pass of the lookup, timed like the forward: one step = the table
+    gradient + the shared-gate gradient of one batch, on one GPU."""
+    import torch
+
+    import hashed_gram_embedding_ngram_b200 as ng
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the lookup has no CPU path)")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    dtype, table, scale = make_table(ng, w, dev)
+    ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM,
+                        ng.ngram_default_hash_params(vocab_size=w.vocab), w.N, row_scale=scale)
+    rec = backward_record(ng, dev, w, ctx, args.batches, args.steps, args.warmup)
+    line = {
+        "metric": "n-gram embed backward tokens/s (table + gate gradients), 1 B200",
+        "n_gpus": 1, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(config_for(w, args), mode="backward",
+                       distinct_rows_per_batch=rec.pop("distinct_rows_per_batch")),
+    }
+    line.update(rec)
     print(json.dumps(line), flush=True)
+    ctx.close()
 
 
 def main():
@@ -988,6 +1261,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations (mid, decode, backward, host-resident, "
+                         "int8 / FP8 / NVFP4) that the default full_prefill run adds as sub-records")
     ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
                     help="eager launches, or 100-step CUDA graphs (auto: graph for N <= 1024)")
     ap.add_argument("--variant", default="default",

@@ -85,14 +85,36 @@ __device__ __forceinline__ void token_context(const int32_t *__restrict__ tokens
                   : ((t == 1) ? h_new : h_old);
 }
 
-// Row index of head h for context (w0, w1, w2).
-__device__ __forceinline__ uint32_t head_row(uint32_t h, uint32_t w0, uint32_t w1,
-                                             uint32_t w2, const HashArgs &a) {
-    // seed_h = (h+1)-th splitmix64 output from base_seed
-    const uint64_t seed = splitmix64_step(a.base_seed + static_cast<uint64_t>(h) * kGolden);
+// seed_h = (h+1)-th splitmix64 output from base_seed.
+__device__ __forceinline__ uint64_t head_seed(uint32_t h, const HashArgs &a) {
+    return splitmix64_step(a.base_seed + static_cast<uint64_t>(h) * kGolden);
+}
+
+// Row index of head h for context (w0, w1, w2), given seed = head_seed(h).
+__device__ __forceinline__ uint32_t head_row_seeded(uint32_t h, uint64_t seed, uint32_t w0, uint32_t w1,
+                                                    uint32_t w2, const HashArgs &a) {
     const uint64_t k2 = (static_cast<uint64_t>(w1) << 21) | w0;
     const uint64_t key = (h < a.n_bigram) ? k2 : ((static_cast<uint64_t>(w2) << 42) | k2);
     return mod_rows(splitmix64_step(key ^ seed), a.R, a.barrett_m);
+}
+
+// Row index of head h for context (w0, w1, w2).
+__device__ __forceinline__ uint32_t head_row(uint32_t h, uint32_t w0, uint32_t w1,
+                                             uint32_t w2, const HashArgs &a) {
+    return head_row_seeded(h, head_seed(h, a), w0, w1, w2, a);
+}
+
+// Programmatic dependent launch (sm_90+).  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still running;
+// grid_dependency_wait() returns once every prerequisite grid has completed and its
+// memory operations are visible, so a kernel calls it before its first global memory
+// access and keeps plain stream-order semantics.  allow_dependents() lets the next such
+// kernel of the stream be scheduled early (it waits the same way before touching memory).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Philox4x32-10 (Salmon, Moraes, Dror & Shaw, SC'11): ten rounds of two 32x32->64
@@ -127,6 +149,12 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
         : "l"(p));
 #endif
     return r;
+}
+
+// Bulk prefetch of [p, p + bytes) from global memory into L2 (sm_90+; p and bytes multiples
+// of 16).  No registers, no completion to wait for: later loads of the range hit L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
 }
 
 // 8-byte and 1-byte forms of the same load (the NVFP4 rows: 8 code bytes and one block

@@ -52,6 +52,9 @@ struct GatherArgs {
     uint32_t ld;
     uint32_t n_outs;
     uint16_t *outs[8];
+    // 1: when a warp walks several strips of a token, its hashing lanes first prefetch the
+    // rest of their rows into L2 (the table is in device memory)
+    uint32_t prefetch_rows;
 };
 
 // 16-byte load through L2 without L1 allocation; coherent (the residual may be the
@@ -67,9 +70,10 @@ __device__ __forceinline__ uint4 ld_na_v4(const void *p) {
 // Row indices of the warp's token, one head per lane (lanes >= H hold 0): hashed
 // from the context, or read from precomputed ids -- the table's own rows hashed once by
 // the order step, or, on the dedup'ed / staged paths, the inverse map into the staging
-// buffer that `table` then points to.
+// buffer that `table` then points to.  seed: head_seed(lane) (the caller computes it once
+// per lane, outside its item loop).
 __device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t tok,
-                                                  uint32_t lane, uint32_t H) {
+                                                  uint32_t lane, uint32_t H, uint64_t seed) {
     uint32_t row = 0;
     if (lane < H) {
         const uint32_t flat = g.tok_begin + tok;
@@ -78,10 +82,15 @@ __device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t 
         } else {
             uint32_t w0, w1, w2;
             token_context(g.tokens, g.history, flat, g.T, g.h, g.err, w0, w1, w2);
-            row = head_row(lane, w0, w1, w2, g.h);
+            row = head_row_seeded(lane, seed, w0, w1, w2, g.h);
         }
     }
     return row;
+}
+
+__device__ __forceinline__ uint32_t warp_head_row(const GatherArgs &g, uint32_t tok,
+                                                  uint32_t lane, uint32_t H) {
+    return warp_head_row(g, tok, lane, H, head_seed(lane, g.h));
 }
 
 // The gate of columns 8v .. 8v+7 of one token: the shared fp32 gate, or (kTokGate) the
@@ -109,9 +118,11 @@ __device__ __forceinline__ void load_gate8(const GatherArgs &g, size_t tok_off, 
 #endif
 
 // kH: compile-time head count (16), or 0: runtime g.h.n_heads <= 16.  kTokGate: the gate
-// is g.gate_tok (per token) instead of g.gate.
-template <int kH, bool kTokGate = false>
-__global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const GatherArgs g) {
+// is g.gate_tok (per token) instead of g.gate.  kMinBlocks: resident CTAs per SM the
+// register budget targets (2 by default; 3 for batches whose work items fit one wave of
+// 3 CTAs per SM but not of 2, the decode batches of a few hundred tokens).
+template <int kH, bool kTokGate = false, int kMinBlocks = NGRAM_LDG_MIN_BLOCKS>
+__global__ void __launch_bounds__(256, kMinBlocks) k_gather_bf16(const GatherArgs g) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
@@ -119,12 +130,15 @@ __global__ void __launch_bounds__(256, NGRAM_LDG_MIN_BLOCKS) k_gather_bf16(const
     const uint32_t nvec = g.d >> 3;
     const uint32_t n_items = g.N * g.groups_per_token;
     const uint16_t *__restrict__ table = static_cast<const uint16_t *>(g.table);
+    const uint64_t seed = head_seed(lane, g.h);           // arithmetic only: before the wait
+    allow_dependents();
+    grid_dependency_wait();
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {
         const uint32_t pos = item / g.groups_per_token;
         const uint32_t grp = item - pos * g.groups_per_token;
         const uint32_t tok = g.perm ? __ldg(g.perm + pos) : pos;
-        const uint32_t my_row = warp_head_row(g, tok, lane, H);
+        const uint32_t my_row = warp_head_row(g, tok, lane, H, seed);
         uint32_t rows[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) rows[h] = __shfl_sync(0xFFFFFFFFu, my_row, h);

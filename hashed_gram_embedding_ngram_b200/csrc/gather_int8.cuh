@@ -71,12 +71,15 @@ __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
     const uint32_t nvec = g.d >> 4;
     const uint32_t n_items = g.N * g.groups_per_token;
     const uint8_t *__restrict__ table = static_cast<const uint8_t *>(g.table);
+    const uint64_t seed = head_seed(lane, g.h);           // arithmetic only: before the wait
+    allow_dependents();
+    grid_dependency_wait();
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {
         const uint32_t pos = item / g.groups_per_token;
         const uint32_t grp = item - pos * g.groups_per_token;
         const uint32_t tok = g.perm ? __ldg(g.perm + pos) : pos;
-        const uint32_t my_row = warp_head_row(g, tok, lane, H);
+        const uint32_t my_row = warp_head_row(g, tok, lane, H, seed);
         // the scale load is issued here but first used after the row loads are in flight
         const float my_scale = (lane < H) ? __ldg(g.row_scale + my_row) : 0.0f;
         uint32_t rows[16];
@@ -85,6 +88,12 @@ __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
         const uint32_t s_begin = grp * g.strips_per_item;
         const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
         const size_t tok_off = static_cast<size_t>(tok) * g.d;
+        // one warp walks several strips: the strips after the first are prefetched into L2
+        // now, so their loads wait for L2 rather than DRAM
+        if (g.prefetch_rows && s_end - s_begin > 1 && lane < H) {
+            const uint32_t b0 = (s_begin + 1) * 512u, b1 = min(s_end * 512u, g.d);
+            if (b1 > b0) prefetch_l2_bulk(table + static_cast<size_t>(my_row) * g.d + b0, b1 - b0);
+        }
         for (uint32_t s = s_begin; s < s_end; ++s) {
             const uint32_t v = s * 32u + lane;
             const bool active = v < nvec;             // the last strip may be ragged

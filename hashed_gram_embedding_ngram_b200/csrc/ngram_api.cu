@@ -49,6 +49,15 @@ using namespace ngram;
 #ifndef NGRAM_SPI_ONE_FORMATS
 #define NGRAM_SPI_ONE_FORMATS ((1u << NGRAM_BF16) | (1u << NGRAM_NVFP4))
 #endif
+#ifndef NGRAM_L2_PREFETCH_FORMATS       // bit t: row format t prefetches a token's later strips into L2
+#define NGRAM_L2_PREFETCH_FORMATS 0u
+#endif
+#ifndef NGRAM_PDL                        // 1: gathers and order kernels launch as programmatic dependents
+#define NGRAM_PDL 1
+#endif
+#ifndef NGRAM_THREE_CTA_DECODE           // 1: bf16 batches that fit one wave of 3 CTAs/SM use them
+#define NGRAM_THREE_CTA_DECODE 1
+#endif
 #ifndef NGRAM_BULK_CHUNK_COLS           // columns per work item of the bulk kernel
 #define NGRAM_BULK_CHUNK_COLS 1280
 #endif
@@ -440,6 +449,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.ld = c->d;
     g.n_outs = 0;
     for (uint16_t *&o : g.outs) o = nullptr;
+    g.prefetch_rows = (c->where == NGRAM_RES_HBM && ((NGRAM_L2_PREFETCH_FORMATS >> c->dtype) & 1u)) ? 1u : 0u;
     return g;
 }
 
@@ -492,23 +502,48 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
     }
 }
 
-template <bool kTok>
-void launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s) {
+// Launch with programmatic stream serialization: the kernel may be scheduled while the
+// previous kernel of the stream is still running, and waits for it (griddepcontrol.wait)
+// before its first global memory access -- the launch latency overlaps the previous
+// kernel's tail, the results are those of plain stream order.  Only kernels that call
+// grid_dependency_wait() first are launched this way.
+template <typename... KArgs>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
+                             const KArgs &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = NGRAM_PDL ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// kThree: the bf16 gather compiled for 3 resident CTAs per SM (see k_gather_bf16).
+template <bool kTok, bool kThree = false>
+cudaError_t launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s) {
     const bool h16 = g.h.n_heads == 16;
     switch (t) {
         case NGRAM_BF16:
-            if (h16) k_gather_bf16<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_bf16<0, kTok><<<nb, 256, 0, s>>>(g);
-            break;
+            if (kThree) return h16 ? launch_dependent(k_gather_bf16<16, kTok, 3>, nb, 256, s, g)
+                                   : launch_dependent(k_gather_bf16<0, kTok, 3>, nb, 256, s, g);
+            return h16 ? launch_dependent(k_gather_bf16<16, kTok>, nb, 256, s, g)
+                       : launch_dependent(k_gather_bf16<0, kTok>, nb, 256, s, g);
         case NGRAM_INT8_ROWSCALE:
-            if (h16) k_gather_int8<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_int8<0, kTok><<<nb, 256, 0, s>>>(g);
-            break;
+            return h16 ? launch_dependent(k_gather_int8<16, kTok>, nb, 256, s, g)
+                       : launch_dependent(k_gather_int8<0, kTok>, nb, 256, s, g);
         case NGRAM_FP8_E4M3_ROWSCALE:
-            if (h16) k_gather_fp8<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_fp8<0, kTok><<<nb, 256, 0, s>>>(g);
-            break;
+            return h16 ? launch_dependent(k_gather_fp8<16, kTok>, nb, 256, s, g)
+                       : launch_dependent(k_gather_fp8<0, kTok>, nb, 256, s, g);
         case NGRAM_NVFP4:
-            if (h16) k_gather_nvfp4<16, kTok><<<nb, 256, 0, s>>>(g); else k_gather_nvfp4<0, kTok><<<nb, 256, 0, s>>>(g);
-            break;
+            return h16 ? launch_dependent(k_gather_nvfp4<16, kTok>, nb, 256, s, g)
+                       : launch_dependent(k_gather_nvfp4<0, kTok>, nb, 256, s, g);
     }
+    return cudaErrorInvalidValue;
 }
 
 // The TMA-staged gather of the 8- and 4-bit formats: whole rows through a shared-memory
@@ -551,6 +586,8 @@ ngram_status launch_staged(ngram_ctx *c, const GatherArgs &g, cudaStream_t s) {
     }
 }
 
+uint64_t full_grid(const ngram_ctx *c);
+
 // The register gather (every row format); max_blocks bounds the persistent grid.
 ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t max_blocks) {
     if ((c->hp.flags & NGRAM_FLAG_TMA_STAGING) && c->dtype != NGRAM_BF16 && c->where == NGRAM_RES_HBM &&
@@ -561,12 +598,22 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
                          static_cast<uint64_t>(g.N) * g.n_strips <= 2ull * resident_warps) ? 1u : g.n_strips;
     g.groups_per_token = (g.n_strips + g.strips_per_item - 1) / g.strips_per_item;
     const uint64_t items = static_cast<uint64_t>(g.N) * g.groups_per_token;
+    // a bf16 batch whose items overflow one wave of the full grid but fit one wave at 3
+    // CTAs per SM (decode batches of ~240..350 tokens at d = 2560) runs the 3-CTA build:
+    // otherwise the items beyond the first wave pay a second round of load latency
+    const uint64_t three = static_cast<uint64_t>(c->num_sms) * 3u;
+    const bool use_three = NGRAM_THREE_CTA_DECODE && c->dtype == NGRAM_BF16 &&
+                           max_blocks == full_grid(c) && c->gather_blocks_per_sm < 3 &&
+                           items > max_blocks * 8u && items <= three * 8u;
     uint64_t blocks = (items + 7) / 8;
-    if (blocks > max_blocks) blocks = max_blocks;
+    if (blocks > (use_three ? three : max_blocks)) blocks = use_three ? three : max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
-    if (g.gate_tok != nullptr) launch_gather_kernel<true>(c->dtype, g, nb, s);
-    else launch_gather_kernel<false>(c->dtype, g, nb, s);
-    NG_CUDA(cudaGetLastError(), "gather kernel launch");
+    cudaError_t e;
+    if (g.gate_tok != nullptr) e = use_three ? launch_gather_kernel<true, true>(c->dtype, g, nb, s)
+                                             : launch_gather_kernel<true>(c->dtype, g, nb, s);
+    else e = use_three ? launch_gather_kernel<false, true>(c->dtype, g, nb, s)
+                       : launch_gather_kernel<false>(c->dtype, g, nb, s);
+    NG_CUDA(e, "gather kernel launch");
     return NGRAM_OK;
 }
 
@@ -722,11 +769,14 @@ ngram_status order_tokens(ngram_ctx *c, const Call &k, uint32_t *idx_out = nullp
     const HashArgs a = hash_args(c);
     const unsigned gn = grid_for(c, k.N, 256);
     NG_CUDA(cudaMemsetAsync(c->so_hist, 0, kOrderBuckets * 4ull, k.s), "order clear");
-    k_order_count<<<gn, 256, 0, k.s>>>(k.tokens, k.history, k.T, k.N, a, c->d_err, c->so_bucket, c->so_hist,
-                                        idx_out);
-    k_order_scan<<<1, 1024, 0, k.s>>>(c->so_hist);
-    k_order_scatter<<<gn, 256, 0, k.s>>>(c->so_bucket, k.N, c->so_hist, c->so_perm);
-    NG_CUDA(cudaGetLastError(), "order launch");
+    const int32_t *tokens = k.tokens, *history = k.history;
+    const uint32_t T = k.T, N = k.N;
+    uint32_t *err = c->d_err, *bucket = c->so_bucket, *hist = c->so_hist, *perm = c->so_perm;
+    const uint32_t *bucket_c = bucket;
+    NG_CUDA(launch_dependent(k_order_count, gn, 256, k.s, tokens, history, T, N, a, err, bucket, hist,
+                             idx_out), "k_order_count launch");
+    NG_CUDA(launch_dependent(k_order_scan, 1, 1024, k.s, hist), "k_order_scan launch");
+    NG_CUDA(launch_dependent(k_order_scatter, gn, 256, k.s, bucket_c, N, hist, perm), "k_order_scatter launch");
     return NGRAM_OK;
 }
 

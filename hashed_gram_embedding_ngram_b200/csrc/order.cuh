@@ -11,7 +11,8 @@
 // histogram, one exclusive scan over the 8,192 buckets (in shared memory), and a
 // scatter with per-bucket atomic cursors.  The order inside a bucket depends on timing,
 // which is harmless: every token's output is computed and written the same way in any
-// order.
+// order.  Each kernel waits for the previous grid of its stream before touching memory
+// (grid_dependency_wait), so the three may be launched as programmatic dependents.
 #pragma once
 
 #include "device_common.cuh"
@@ -29,6 +30,8 @@ __global__ void __launch_bounds__(256) k_order_count(const int32_t *__restrict__
                                                      uint32_t T, uint32_t N, const HashArgs a,
                                                      uint32_t *err, uint32_t *__restrict__ bucket_of,
                                                      uint32_t *hist, uint32_t *__restrict__ idx_out) {
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x) {
         uint32_t w0, w1, w2;
         token_context(tokens, history, t, T, a, err, w0, w1, w2);
@@ -50,6 +53,8 @@ __global__ void __launch_bounds__(1024) k_order_scan(uint32_t *hist) {
     __shared__ uint32_t sh[kOrderBuckets];
     __shared__ uint32_t warp_tot[32];
     constexpr uint32_t kPer = kOrderBuckets / 1024;
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t i = threadIdx.x; i < kOrderBuckets; i += 1024) sh[i] = hist[i];
     __syncthreads();
     const uint32_t base = threadIdx.x * kPer;
@@ -80,6 +85,8 @@ __global__ void __launch_bounds__(1024) k_order_scan(uint32_t *hist) {
 __global__ void __launch_bounds__(256) k_order_scatter(const uint32_t *__restrict__ bucket_of,
                                                        uint32_t N, uint32_t *cursor,
                                                        uint32_t *__restrict__ perm) {
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x)
         perm[atomicAdd(cursor + bucket_of[t], 1u)] = t;
 }

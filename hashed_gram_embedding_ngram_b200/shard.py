@@ -100,7 +100,8 @@ def complete(group=None) -> None:
         flag = torch.zeros(1, dtype=torch.int32, device=torch.cuda.current_device())
         dist.all_reduce(flag, group=group)
     else:
-        torch.cuda.current_stream().synchronize()
+        if torch.cuda.is_available():
+            torch.cuda.current_stream().synchronize()
         dist.barrier(group=group)
 
 
@@ -114,7 +115,7 @@ def forward_shard(ctx, peers: PeerOutputs, tokens: torch.Tensor, residual: torch
     if N > peers.max_tokens:
         raise ValueError("N = %d exceeds the buffers' %d tokens" % (N, peers.max_tokens))
     complete(group)
-    _b.ngram_forward_shard(ctx, tokens, residual, gate, peers.ptrs, peers.d_full, col0,
-                           history=history)
+    peers.lib.ngram_forward_shard(ctx, tokens, residual, gate, peers.ptrs, peers.d_full, col0,
+                                  history=history)
     complete(group)
-    return peers.out[:N]
+    return None if peers.out is None else peers.out[:N]

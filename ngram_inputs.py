@@ -79,6 +79,12 @@ WORKLOADS = {
     # profiling cases: 1M x 2560 fp8 (2.4 GiB) and 2M x 2560 nvfp4 (2.7 GiB), 16 x 1024 uniform
     "profile_fp8": Workload("profile_fp8", 1_000_000, 2560, "fp8", 151_936, 16, 1024, tokens="uniform"),
     "profile_nvfp4": Workload("profile_nvfp4", 2_000_000, 2560, "nvfp4", 151_936, 16, 1024, tokens="uniform"),
+    # small cases of the prefill launch configuration (one 32,768-token Zipf(1.1) batch,
+    # grouped order) for ncu counter captures: 400k x 2560 bf16 (2.0 GB), 1M x 2560 FP8
+    # (2.6 GB), 2M x 2560 NVFP4 (2.9 GB)
+    "profile_prefill": Workload("profile_prefill", 400_000, 2560, "bf16", 151_936, 1, 32_768),
+    "profile_fp8_prefill": Workload("profile_fp8_prefill", 1_000_000, 2560, "fp8", 151_936, 1, 32_768),
+    "profile_nvfp4_prefill": Workload("profile_nvfp4_prefill", 2_000_000, 2560, "nvfp4", 151_936, 1, 32_768),
 }
 
 

@@ -9,6 +9,8 @@ table pinned in host memory, sampled tokens).  The host waits of the DMA
 mode are bounded: a stream kept busy past the bound makes the call return
 NGRAM_ETIMEOUT and leaves the context usable.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -195,6 +197,53 @@ def test_host_modes_bitidentical_to_hbm(cuda_device, host_bf16, n_seq, T, hist):
     assert r["exact"] == r["n"]
 
 
+def _median_ms(fn, reps=7, warm=2):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.perf_counter()
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        # the DMA mode blocks the host while it stages rows: count the wall time too
+        ts.append(max(a.elapsed_time(b), (time.perf_counter() - w0) * 1e3))
+    return float(np.median(ts))
+
+
+def test_auto_picks_a_mode_within_10_percent_of_the_best(cuda_device, host_bf16):
+    """HOST_AUTO on a 256-token decode batch: the mode it keeps (lowest median of three
+    timed calls after a warm-up call per mode) runs within 10% of the fastest of UVA,
+    UVA + dedup and DMA, each timed in its own context by the median of 7 calls.  Timing
+    noise gets three attempts."""
+    R, d, V = host_bf16.R, host_bf16.d, 151_936
+    w = gen.Workload("host_auto", R, d, "bf16", V, 256, 1, history=True)
+    inp, dv = workload_on_device(w, cuda_device, token_seed=333)
+    modes = {ng.NGRAM_RES_HOST_UVA: (ng.NGRAM_RES_HOST_UVA, 0),
+             ng.NGRAM_AUTO_UVA_DEDUP: (ng.NGRAM_RES_HOST_UVA, ng.NGRAM_FLAG_DEDUP),
+             ng.NGRAM_RES_HOST_DMA: (ng.NGRAM_RES_HOST_DMA, 0)}
+    ctxs = {m: host_bf16.ctx(where, V, w.N, flags=fl) for m, (where, fl) in modes.items()}
+    auto = host_bf16.ctx(ng.NGRAM_RES_HOST_AUTO, V, w.N)
+    try:
+        ref = from_dev_bf16(_forward(ctxs[ng.NGRAM_RES_HOST_UVA], dv))
+        assert np.array_equal(from_dev_bf16(_forward(auto, dv)), ref)
+        choice = ng.ngram_auto_choice(auto, w.N)
+        assert choice in modes
+        for attempt in range(3):
+            t = {m: _median_ms(lambda c=c: _forward(c, dv)) for m, c in ctxs.items()}
+            if t[choice] <= 1.10 * min(t.values()):
+                break
+        assert t[choice] <= 1.10 * min(t.values()), (choice, t)
+        assert np.array_equal(from_dev_bf16(_forward(auto, dv)), ref)
+    finally:
+        auto.close()
+        for c in ctxs.values():
+            c.close()
+
+
 def test_host_int8_modes(cuda_device):
     R, d, V = 50_000, 512, 9000
     f = _HostFixture(cuda_device, R, d, ng.NGRAM_INT8_ROWSCALE)
@@ -330,6 +379,12 @@ def test_host_full_size_sampled(cuda_device):
             want = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R, d=d,
                                   table_seed=gen.TABLE_SEED, sel=sel, acc=oracle.ACC_F32, n_threads=N_CPU,
                                   vocab_size=V)
-            assert_parity(outs[0].reshape(w.N, d)[sel], want)
+            r = assert_parity(outs[0].reshape(w.N, d)[sel], want)
+            assert r["exact"] == r["n"]
+            want64, _, mag, _ = oracle.forward(inp["tokens"], inp["history"], inp["residual"],
+                                               inp["gate"], R=R, d=d, table_seed=gen.TABLE_SEED,
+                                               sel=sel, acc=oracle.ACC_F64, n_threads=N_CPU,
+                                               vocab_size=V, want_aux=True)
+            assert_parity(outs[0].reshape(w.N, d)[sel], want64, mag)
     finally:
         host.close()

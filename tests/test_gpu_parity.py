@@ -218,6 +218,53 @@ def test_in_place_equals_out_of_place(cuda_device):
     assert np.array_equal(from_dev_bf16(buf), ref)
 
 
+@pytest.mark.parametrize("fmt,n_seq,T", [("bf16", 256, 1), ("bf16", 1, 20_000), ("bf16", 3, 300),
+                                          ("int8", 64, 1), ("fp8", 2, 500), ("nvfp4", 1, 20_000)])
+def test_back_to_back_in_place_calls_keep_stream_order(cuda_device, fmt, n_seq, T):
+    """The gathers (and the grouped-order kernels) are launched as programmatic dependents:
+    each may be scheduled while the previous kernel of the stream still runs and waits for
+    it before touching memory.  Six in-place calls in a row, each reading the residual the
+    previous one wrote, with no host synchronisation between them -- eagerly and replayed
+    from a CUDA graph -- must equal the same calls with a synchronisation after each."""
+    R, d, V = 65_536, 2560, 151_936
+    w = gen.Workload("chain", R, d, fmt, V, n_seq, T, history=T == 1)
+    dt = ng_dtype(fmt)
+    table, scale = TABLES.get(R, d, dt, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, dt, ng.NGRAM_RES_HBM, _hp(V), w.N, row_scale=scale)
+    batches = [gen.make_inputs(w, token_seed=700 + i) for i in range(6)]
+    toks = [torch.from_numpy(b["tokens"]).to(cuda_device) for b in batches]
+    hist = [None if b["history"] is None else torch.from_numpy(b["history"]).to(cuda_device) for b in batches]
+    res0 = torch.from_numpy(batches[0]["residual"].view(np.int16)).view(torch.bfloat16).view(w.N, d).to(cuda_device)
+    gate = torch.from_numpy(batches[0]["gate"]).to(cuda_device)
+    ref = res0.clone()
+    for i in range(6):
+        ng.ngram_forward(ctx, toks[i], ref, gate, out=ref, history=hist[i])
+        torch.cuda.synchronize()
+    buf = res0.clone()
+    for i in range(6):
+        ng.ngram_forward(ctx, toks[i], buf, gate, out=buf, history=hist[i])
+    torch.cuda.synchronize()
+    assert torch.equal(buf.view(torch.int16), ref.view(torch.int16))
+    g = torch.cuda.CUDAGraph()
+    gbuf = res0.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):                          # warm the capture stream
+        ng.ngram_forward(ctx, toks[0], gbuf.clone(), gate, history=hist[0], stream=s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        cs = torch.cuda.current_stream()
+        for i in range(6):
+            ng.ngram_forward(ctx, toks[i], gbuf, gate, out=gbuf, history=hist[i], stream=cs)
+    gbuf.copy_(res0)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(gbuf.view(torch.int16), ref.view(torch.int16))
+    del g
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
 def test_zero_gate_returns_residual_bitwise(cuda_device):
     w = W["tiny"]
     inp, dv = workload_on_device(w, cuda_device)

@@ -3,9 +3,12 @@
 - The shard fill equals the oracle's table restricted to the shard's columns, bit for bit.
 - P shards, each its own context over its [R][d_full/P] table, calling
   ngram_forward_shard into one or two full-width buffers, give ngram_forward over the
-  whole table bit for bit (every format, per-token gate, grouped order).
+  whole table bit for bit (every format, per-token gate, grouped order), and the
+  assembled output equals the CPU oracle on sampled tokens (bit for bit against its fp32
+  mode, within the stated bar of its exact mode).
 - Two processes on this GPU, each holding one shard, write into each other's output
-  buffer through CUDA IPC (ngram_ipc_*) and end with the full output.  The two processes'
+  buffer through CUDA IPC (ngram_ipc_*) and end with the full output, equal to the
+  unsharded lookup and to the CPU oracle on sampled tokens.  The two processes'
   kernels never wait on each other (a host barrier orders them), so sharing one GPU is
   safe; the same code runs one process per GPU over NVLink.
 """
@@ -21,7 +24,8 @@ import ngram_inputs as gen
 import oracle
 import hashed_gram_embedding_ngram_b200 as ng
 from hashed_gram_embedding_ngram_b200 import shard
-from parity_helpers import TABLES, from_dev_bf16, ng_dtype, to_dev_bf16, to_dev_tokens
+from parity_helpers import (N_CPU, TABLES, assert_parity, from_dev_bf16, ng_dtype, oracle_dtype,
+                            sample_tokens, to_dev_bf16, to_dev_tokens)
 
 pytestmark = pytest.mark.gpu
 FMTS = ["bf16", "int8", "fp8", "nvfp4"]
@@ -106,6 +110,19 @@ def test_virtual_shards_equal_the_full_lookup(cuda_device, case):
     torch.cuda.synchronize()
     for o in outs:
         assert np.array_equal(from_dev_bf16(o), want)
+    # the assembled full-width output against the CPU oracle (sampled tokens)
+    sel = sample_tokens(w, 256)
+    kw = dict(R=R, d=d_full, dtype=oracle_dtype(fmt), table_seed=gen.TABLE_SEED, sel=sel,
+              n_threads=N_CPU, vocab_size=V)
+    gt = from_dev_bf16(gate).reshape(N, d_full) if tg else None
+    g = None if tg else inp["gate"]
+    got = from_dev_bf16(outs[-1]).reshape(N, d_full)[sel]
+    r = assert_parity(got, oracle.forward(inp["tokens"], inp["history"], inp["residual"], g,
+                                          gate_tok=gt, acc=oracle.ACC_F32, **kw))
+    assert r["exact"] == r["n"]
+    want64, _, mag, _ = oracle.forward(inp["tokens"], inp["history"], inp["residual"], g,
+                                       gate_tok=gt, acc=oracle.ACC_F64, want_aux=True, **kw)
+    assert_parity(got, want64, mag)
 
 
 def test_shard_arguments(cuda_device):
@@ -162,7 +179,13 @@ def _ipc_rank(rank, world, port, q):
         ng.ngram_fill_synthetic(full_t, R, d_full, ng.NGRAM_BF16, gen.TABLE_SEED)
         full = ng.ngram_init(full_t, R, d_full, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), N)
         want = from_dev_bf16(ng.ngram_forward(full, tok, res, gate, history=hst))
-        q.put((rank, bool(np.array_equal(got, want)), None))
+        # and the assembled output against the CPU oracle on sampled tokens
+        sel = sample_tokens(w, 128)
+        ref = oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], R=R,
+                             d=d_full, table_seed=gen.TABLE_SEED, sel=sel, acc=oracle.ACC_F32,
+                             n_threads=4, vocab_size=V)
+        same_oracle = bool(np.array_equal(got.reshape(N, d_full)[sel], ref))
+        q.put((rank, bool(np.array_equal(got, want)) and same_oracle, None))
         dist.barrier()                                   # nobody unmaps while a peer still writes
     except Exception as e:                               # report, never hang the other rank
         q.put((rank, False, repr(e)))
