@@ -29,6 +29,10 @@ import time
 
 import numpy as np
 
+# the DMA host mode copies rows with OpenMP threads: let them sleep between calls instead of
+# spinning on the cores the launching thread needs (read by libgomp when it loads)
+os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -342,8 +346,9 @@ def config_for(w, args) -> dict:
         "tokens_per_step_per_gpu": w.N, "heads": "8 bigram + 8 trigram",
         "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
         "accumulate": "fp32, head order", "residency": "hbm", "variant": args.variant,
-        "l2": "inputs larger than L2: %.2f GB moved per step vs 126 MB L2; %d token batches "
-              "alternate" % (algorithmic_bytes(w) / 1e9, args.batches),
+        "l2": "inputs larger than L2: %.2f GB moved per step, %d token batches cycle (their rows "
+              "span %.0f MB) vs 126 MB L2" % (algorithmic_bytes(w) / 1e9, max(args.batches, batches_for(w)),
+                                              max(args.batches, batches_for(w)) * w.N * HEADS * row_bytes(w) / 1e6),
         "parallelism": "replicas x%d (tokens sharded, table replicated)" % args.gpus,
         "launch": resolved_launch(w, args),
     }
@@ -362,11 +367,24 @@ def make_table(ng, w, dev):
     return dtype, table, scale
 
 
+L2_BYTES = 126 * 10**6          # B200 L2
+
+
+def batches_for(w, minimum: int = 2) -> int:
+    """Token batches a timed loop cycles through: enough that the rows they read (16 per
+    token) span twice the L2, so that no batch finds its rows left in L2 by its previous
+    turn (decode batches are small: 82 KB of rows for one token)."""
+    per = w.N * HEADS * row_bytes(w)
+    return max(minimum, -(-2 * L2_BYTES // per))
+
+
 class Batches:
     """One rank's token batches (distinct seeds per rank and batch) and the activations of
-    a workload, on the host and on the device."""
+    a workload, on the host and on the device.  per_batch: every batch has its own residual
+    and output rows too (used when many small batches cycle, so that the activations do not
+    stay in L2 either); else one residual and one output serve every batch."""
 
-    def __init__(self, w, dev, rank=0, batches=2, token_gate=False):
+    def __init__(self, w, dev, rank=0, batches=2, token_gate=False, per_batch=False):
         import torch
         self.host_tok, self.host_hist = [], []
         for b in range(batches):
@@ -375,11 +393,25 @@ class Batches:
             self.host_hist.append(gen.history_for(w, hs))
         self.res_bits = gen.residual_bf16_bits(w.N, w.d, gen.RESIDUAL_SEED + rank)
         self.gate_h = gen.gate_f32(w.d)
-        self.tok_d = [torch.from_numpy(t).to(dev) for t in self.host_tok]
-        self.hist_d = [None if h is None else torch.from_numpy(h).to(dev) for h in self.host_hist]
+        tok_all = torch.from_numpy(np.stack(self.host_tok)).to(dev)
+        self.tok_d = [tok_all[b] for b in range(batches)]
+        if w.history:
+            hist_all = torch.from_numpy(np.stack(self.host_hist)).to(dev)
+            self.hist_d = [hist_all[b] for b in range(batches)]
+        else:
+            self.hist_d = [None] * batches
         self.res_cpu = torch.from_numpy(self.res_bits.view(np.int16)).view(torch.bfloat16).view(w.N, w.d)
         self.residual = self.res_cpu.to(dev)
         self.out = torch.empty_like(self.residual)
+        n_act = batches if per_batch else 1
+        if per_batch:
+            bits = gen.residual_bf16_bits(n_act * w.N, w.d, gen.RESIDUAL_SEED + 1000 + rank)
+            res_all = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).view(n_act, w.N, w.d).to(dev)
+            out_all = torch.empty_like(res_all)
+            self.res_b = [res_all[b] for b in range(n_act)]
+            self.out_b = [out_all[b] for b in range(n_act)]
+        else:
+            self.res_b, self.out_b = [self.residual], [self.out]
         self.gate = torch.from_numpy(self.gate_h).to(dev)
         if token_gate:                      # one bf16 gate per token and column
             g = np.random.default_rng(12).uniform(0, 1, (w.N, w.d)).astype(np.float32)
@@ -393,32 +425,38 @@ class Batches:
 
 def time_forward(ng, ctx, bt, stream, steps, warmup, launch, dev, barrier=lambda: None, G=100):
     """W untimed warm-up steps, then K timed steps bracketed by a barrier and a
-    synchronize.  Eager: one ngram_forward per step, CUDA events around each launch.
-    Graph: G steps captured once into a CUDA graph and replayed, events around each replay
-    (decode-sized launches are otherwise bound by the Python launch path).  Returns
-    (elapsed_ms, kernel ms per step, K, clock summary)."""
+    synchronize; step i uses token batch i % B (and its own activations when bt has them).
+    Eager: one ngram_forward per step, CUDA events around each launch.  Graph: the steps
+    are captured in CUDA graphs of G steps (ceil(B / G) graphs, so every batch is used) and
+    replayed in turn, events around each replay (decode-sized launches are otherwise bound
+    by the Python launch path).  Returns (elapsed_ms, kernel ms per step, K, clocks)."""
     import torch
 
     def step(i, s=None):
         b = i % bt.n
-        ng.ngram_forward(ctx, bt.tok_d[b], bt.residual, bt.gate, out=bt.out, history=bt.hist_d[b],
+        a = b % len(bt.res_b)
+        ng.ngram_forward(ctx, bt.tok_d[b], bt.res_b[a], bt.gate, out=bt.out_b[a], history=bt.hist_d[b],
                          stream=s if s is not None else stream)
 
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     K = steps
-    graph = None
+    graphs = []
     if launch == "graph":
-        K = max(G, (K + G - 1) // G * G)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            cap = torch.cuda.current_stream()
-            for i in range(G):
-                step(i, cap)
-        graph.replay()
+        n_graphs = -(-bt.n // G)
+        K = max(G * n_graphs, -(-K // (G * n_graphs)) * G * n_graphs)
+        for j in range(n_graphs):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                cap = torch.cuda.current_stream()
+                for i in range(G):
+                    step(j * G + i, cap)
+            graphs.append(gr)
+        for gr in graphs:
+            gr.replay()
         torch.cuda.synchronize()
-    n_ev = K if graph is None else K // G
+    n_ev = K if not graphs else K // G
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -428,19 +466,19 @@ def time_forward(ng, ctx, bt, stream, steps, warmup, launch, dev, barrier=lambda
         t0.record(stream)
         for i in range(n_ev):
             ev_s[i].record(stream)
-            if graph is None:
+            if not graphs:
                 step(i)
             else:
-                graph.replay()
+                graphs[i % len(graphs)].replay()
             ev_e[i].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = t0.elapsed_time(t1)
     kern_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(n_ev))
-    if graph is not None:
+    if graphs:
         kern_ms /= G                          # per step inside the graph (kernel + gap)
-        del graph
+        del graphs
     return elapsed_ms, kern_ms, K, clk.summary()
 
 
@@ -454,12 +492,17 @@ PROFILE_FOR = {"full_prefill": "gather_bf16_prefill", "int8_uniform": "gather_in
                "fp8_prefill": "gather_fp8_prefill", "nvfp4_prefill": "gather_nvfp4_prefill"}
 
 
-def profiled_traffic(workload: str, dtype: str, distinct: int):
+def profiled_traffic(workload: str, dtype: str, distinct: int, n_tokens: int):
     """DRAM bytes per launch, estimated from the committed ncu summary of a small case of the
     same kernel in the same launch configuration (profiles/<kernel>_<workload>.txt), if it was
-    taken on the kernel code as it is now (its kernel_sha line, first word).  The small case's
-    DRAM bytes over its own distinct bytes (the excess of re-reads over the least traffic)
-    times this launch's distinct bytes.  Returns (bytes, source) or (None, reason)."""
+    taken on the kernel code as it is now (its kernel_sha line, first word).  The summary
+    names its scaling:
+      per_token       the small case is the same token batch on a smaller table: its DRAM
+                      bytes per token times this launch's tokens;
+      distinct_ratio  the small case has fewer tokens (uniform ids: row reuse comes only from
+                      hash collisions): its DRAM bytes over its distinct bytes, times this
+                      launch's distinct bytes.
+    Returns (bytes, source) or (None, reason)."""
     name = PROFILE_FOR.get(workload)
     if name is None:
         return None, "no small-case profile for this workload"
@@ -476,12 +519,21 @@ def profiled_traffic(workload: str, dtype: str, distinct: int):
         return None, "profiles/%s.txt was taken on other kernel code" % name
     try:
         dram = float(kv["small_dram_bytes_per_launch"].split()[0])
-        small = float(kv["small_distinct_bytes_per_launch"].split()[0])
+        small_distinct = float(kv["small_distinct_bytes_per_launch"].split()[0])
+        small_tokens = float(kv["small_tokens"].split()[0])
+        scaling = kv["scaling"].split()[0]
     except (KeyError, ValueError, IndexError):
         return None, "profiles/%s.txt lacks the small-case figures" % name
-    return dram / small * distinct, ("ncu DRAM bytes of %s (%s) over its distinct bytes = %.4f, "
-                                     "times this launch's distinct bytes" % (
-                                         kv.get("small_workload", "?").split(" ")[0], name, dram / small))
+    small = kv.get("small_workload", "?").split(" ")[0]
+    if scaling == "per_token":
+        return dram / small_tokens * n_tokens, (
+            "ncu DRAM bytes of %s (%s): %.0f per token, times this launch's %d tokens" % (
+                small, name, dram / small_tokens, n_tokens))
+    if scaling == "distinct_ratio":
+        return dram / small_distinct * distinct, (
+            "ncu DRAM bytes of %s (%s) over its distinct bytes = %.4f, times this launch's "
+            "distinct bytes" % (small, name, dram / small_distinct))
+    return None, "profiles/%s.txt names an unknown scaling %r" % (name, scaling)
 
 
 def hbm_record(ng, dev, w, dtype, table, scale, steps, launch, read_gbs=None, flags=0) -> dict:
@@ -491,7 +543,8 @@ def hbm_record(ng, dev, w, dtype, table, scale, steps, launch, read_gbs=None, fl
     import torch
     hp = ng.ngram_default_hash_params(vocab_size=w.vocab, flags=flags)
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
-    bt = Batches(w, dev)
+    nb = batches_for(w)
+    bt = Batches(w, dev, batches=nb, per_batch=nb > 2)
     stream = torch.cuda.current_stream()
     elapsed_ms, kern_ms, K, clocks = time_forward(ng, ctx, bt, stream, steps, 5, launch, dev)
     st, info = ng.ngram_get_device_error(ctx)
@@ -502,13 +555,16 @@ def hbm_record(ng, dev, w, dtype, table, scale, steps, launch, read_gbs=None, fl
     nbytes = algorithmic_bytes(w)
     dist_b = distinct_bytes(w, U)
     achieved = nbytes / (kern_ms / 1e3) / 1e9
-    traffic, tsrc = profiled_traffic(w.name, w.dtype, dist_b)
+    traffic, tsrc = profiled_traffic(w.name, w.dtype, dist_b, w.N)
     rec = {
         "workload": w.name,
         "config": {"R": w.R, "d": w.d, "table_dtype": w.dtype, "n_seq": w.n_seq, "T": w.T,
                    "tokens": "%s over vocab %d" % ("Zipf(1.1)" if w.tokens == "zipf" else "uniform", w.vocab),
                    "history": w.history, "residency": "hbm", "launch": launch,
-                   "table_gib": round(w.R * stored_row_bytes(w) / 2**30, 2)},
+                   "table_gib": round(w.R * stored_row_bytes(w) / 2**30, 2),
+                   "l2": "%d token batches cycle%s: their rows span %.0f MB, over twice the 126 MB L2" % (
+                       nb, " (each with its own residual and output rows)" if nb > 2 else "",
+                       nb * w.N * HEADS * row_bytes(w) / 1e6)},
         "value": w.N * K / (elapsed_ms / 1e3), "unit": UNIT, "ms_per_step": elapsed_ms / K,
         "kernel_ms": kern_ms, "steps": K,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -549,7 +605,6 @@ def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
     import gc
 
     import torch
-    os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
     t_start = time.perf_counter()
     W = gen.WORKLOADS
     extra = []
@@ -574,7 +629,7 @@ def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
               config={"R": fw.R, "d": fw.d, "table_dtype": "bf16", "n_seq": fw.n_seq, "T": fw.T,
                       "mode": "backward: table gradient + shared-gate gradient"})
     extra.append(bw)
-    # ---- CPU baseline on the materialised host table, then the host-resident configuration
+    # ---- the host-resident configuration, then the CPU baseline on the same materialised table
     host_bytes = fw.R * fw.d * 2
     avail = host_mem_available()
     ht = None
@@ -588,14 +643,6 @@ def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
         fill_s = time.perf_counter() - t0
     else:
         pin_s = fill_s = None
-    if not args.no_cpu_baseline:
-        tab = None if ht is None else ht.tensor.view(torch.int16).numpy().view(np.uint16)
-        line["cpu_baseline"] = cpu_baseline_record(
-            fw, bt_full.inputs(0), args.cpu_seconds, table=tab,
-            table_desc="the materialised 20,000,000 x 2560 bf16 table (95.4 GiB, pinned host memory)")
-        if ht is None:
-            line["cpu_baseline"]["note"] = ("host RAM too small for the 95.4 GiB table (%.1f GiB "
-                                            "available): rows regenerated" % (avail / 2**30))
     if ht is not None:
         with ClockSampler(gpu_id_for(dev)) as clk:
             report, h2d, gemm_ms, gemm_tflops = host_modes(
@@ -627,6 +674,18 @@ def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
                 "device_error": "ok" if all(entry[m]["device_error"] == ng.NGRAM_OK
                                             for m in ("uva", "uva_dedup", "dma", "auto")) else "set",
             })
+    # the oracle reads the materialised table after the host-resident timings: rows it leaves in
+    # the CPU caches would slow the GPU's reads of them over PCIe
+    if not args.no_cpu_baseline:
+        tab = None if ht is None else ht.tensor.view(torch.int16).numpy().view(np.uint16)
+        line["cpu_baseline"] = cpu_baseline_record(
+            fw, bt_full.inputs(0), args.cpu_seconds, table=tab,
+            table_desc="the materialised 20,000,000 x 2560 bf16 table (95.4 GiB, pinned host memory)")
+        if ht is None:
+            line["cpu_baseline"]["note"] = ("host RAM too small for the 95.4 GiB table (%.1f GiB "
+                                            "available): rows regenerated" % (avail / 2**30))
+        del tab                               # a view of the pinned table: gone before close()
+    if ht is not None:
         ht.close()
     else:
         extra.append({"workload": "host_prefill", "skipped": "host RAM: %.1f GiB available, the table "
@@ -682,7 +741,8 @@ def run_ours(args, w):
     ctx = ng.ngram_init(table, w.R, w.d, dtype, ng.NGRAM_RES_HBM, hp, w.N, row_scale=scale)
 
     # ---- inputs: this rank's token batches (distinct seeds per rank and batch)
-    bt = Batches(w, dev, rank, args.batches, token_gate=args.variant == "token_gate")
+    nb = max(args.batches, batches_for(w))
+    bt = Batches(w, dev, rank, nb, token_gate=args.variant == "token_gate", per_batch=nb > args.batches)
     stream = torch.cuda.current_stream()
 
     # ---- distinct rows of the first batch (outside any timed region): U * row bytes is the
@@ -702,15 +762,15 @@ def run_ours(args, w):
     # ---- end to end through the host-buffer call: every step moves its tokens and
     # residual from pinned host memory to the device and its output back to the host
     # (ngram_forward_host pipelines the copies with the gather in ~8 MB chunks)
-    tok_h = [torch.from_numpy(t).pin_memory() for t in bt.host_tok]
-    hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in bt.host_hist]
+    tok_h = [torch.from_numpy(t).pin_memory() for t in bt.host_tok[:64]]
+    hist_h = [None if h is None else torch.from_numpy(h).pin_memory() for h in bt.host_hist[:64]]
     res_h = bt.res_cpu.pin_memory()
     out_h = torch.empty_like(res_h).pin_memory()
     gate_h_tok = bt.gate.cpu().pin_memory() if args.variant == "token_gate" else None
     E = max(1, args.e2e_steps)
 
     def e2e_step(i):
-        b = i % args.batches
+        b = i % len(tok_h)
         if args.variant == "default":
             ng.ngram_forward_host(ctx, tok_h[b], res_h, bt.gate, out=out_h, history=hist_h[b],
                                   stream=stream)
@@ -750,7 +810,7 @@ def run_ours(args, w):
         bytes_launch = algorithmic_bytes(w) + (w.N * 2 * w.d if args.variant == "token_gate" else 0)
         achieved = bytes_launch / (kern_ms / 1e3) / 1e9
         dist_b = distinct_bytes(w, unique_rows)
-        traffic, tsrc = (profiled_traffic(w.name, w.dtype, dist_b) if args.variant == "default"
+        traffic, tsrc = (profiled_traffic(w.name, w.dtype, dist_b, w.N) if args.variant == "default"
                          else (None, "variant %s: not profiled" % args.variant))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -989,9 +1049,6 @@ def run_host(args):
     """Host-resident table: the 20M x 2560 bf16 table pinned in host memory, each host
     workload timed in UVA, DMA and AUTO residency, alone and overlapped with a stand-in
     bf16 [4096 x 2560] x [2560 x 2560] GEMM looped on a second stream."""
-    # the DMA mode gathers rows with OpenMP threads; let them sleep between calls so they
-    # do not spin on the cores the launching thread needs during the other modes
-    os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
     import torch
 
     import hashed_gram_embedding_ngram_b200 as ng

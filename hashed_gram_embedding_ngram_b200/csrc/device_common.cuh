@@ -151,12 +151,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     return r;
 }
 
-// Bulk prefetch of [p, p + bytes) from global memory into L2 (sm_90+; p and bytes multiples
-// of 16).  No registers, no completion to wait for: later loads of the range hit L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
-}
-
 // 8-byte and 1-byte forms of the same load (the NVFP4 rows: 8 code bytes and one block
 // scale per 16 columns).
 __device__ __forceinline__ uint2 ld_stream_v2(const void *p) {

@@ -52,9 +52,6 @@ struct GatherArgs {
     uint32_t ld;
     uint32_t n_outs;
     uint16_t *outs[8];
-    // 1: when a warp walks several strips of a token, its hashing lanes first prefetch the
-    // rest of their rows into L2 (the table is in device memory)
-    uint32_t prefetch_rows;
 };
 
 // 16-byte load through L2 without L1 allocation; coherent (the residual may be the

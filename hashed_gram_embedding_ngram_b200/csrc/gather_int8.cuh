@@ -88,12 +88,6 @@ __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
         const uint32_t s_begin = grp * g.strips_per_item;
         const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
         const size_t tok_off = static_cast<size_t>(tok) * g.d;
-        // one warp walks several strips: the strips after the first are prefetched into L2
-        // now, so their loads wait for L2 rather than DRAM
-        if (g.prefetch_rows && s_end - s_begin > 1 && lane < H) {
-            const uint32_t b0 = (s_begin + 1) * 512u, b1 = min(s_end * 512u, g.d);
-            if (b1 > b0) prefetch_l2_bulk(table + static_cast<size_t>(my_row) * g.d + b0, b1 - b0);
-        }
         for (uint32_t s = s_begin; s < s_end; ++s) {
             const uint32_t v = s * 32u + lane;
             const bool active = v < nvec;             // the last strip may be ragged

@@ -51,14 +51,6 @@ __global__ void __launch_bounds__(256, NGRAM_NVFP4_MIN_BLOCKS) k_gather_nvfp4(co
         const uint32_t s_begin = grp * g.strips_per_item;
         const uint32_t s_end = min(s_begin + g.strips_per_item, g.n_strips);
         const size_t tok_off = static_cast<size_t>(tok) * g.d;
-        // one warp walks several strips: the codes of the strips after the first, and the
-        // block scales, are prefetched into L2 now (256 code bytes and 32 scale bytes a strip)
-        if (g.prefetch_rows && s_end - s_begin > 1 && lane < H) {
-            const uint8_t *row = table + static_cast<size_t>(my_row) * rb;
-            const uint32_t c0 = (s_begin + 1) * 256u, c1 = min(s_end * 256u, code_bytes);
-            if (c1 > c0) prefetch_l2_bulk(row + c0, c1 - c0);
-            prefetch_l2_bulk(row + code_bytes, static_cast<uint32_t>(rb) - code_bytes);
-        }
         for (uint32_t s = s_begin; s < s_end; ++s) {
             const uint32_t v = s * 32u + lane;
             if (v >= nvec) continue;                      // the last strip may be ragged

@@ -16,6 +16,10 @@
 #include <thread>
 #include <vector>
 
+#if defined(__x86_64__)
+#include <immintrin.h>
+#endif
+
 #include <cuda.h>            // CUcontext / CUresult types for the driver entry points
 #include <cuda_runtime.h>
 
@@ -48,9 +52,6 @@ using namespace ngram;
 //     chunk and ring depth; its tunables are below.
 #ifndef NGRAM_SPI_ONE_FORMATS
 #define NGRAM_SPI_ONE_FORMATS ((1u << NGRAM_BF16) | (1u << NGRAM_NVFP4))
-#endif
-#ifndef NGRAM_L2_PREFETCH_FORMATS       // bit t: row format t prefetches a token's later strips into L2
-#define NGRAM_L2_PREFETCH_FORMATS 0u
 #endif
 #ifndef NGRAM_PDL                        // 1: gathers and order kernels launch as programmatic dependents
 #define NGRAM_PDL 1
@@ -449,7 +450,6 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.ld = c->d;
     g.n_outs = 0;
     for (uint16_t *&o : g.outs) o = nullptr;
-    g.prefetch_rows = (c->where == NGRAM_RES_HBM && ((NGRAM_L2_PREFETCH_FORMATS >> c->dtype) & 1u)) ? 1u : 0u;
     return g;
 }
 
@@ -694,6 +694,47 @@ ngram_status forward_dedup(ngram_ctx *c, const Call &k, unsigned compact_grid) {
     return launch_gather(c, g, k.s, full_grid(c));
 }
 
+// One table row into pinned staging by a host thread.  NGRAM_DMA_NONTEMPORAL (x86-64):
+//   0  memcpy;
+//   1  the source lines are read after a non-temporal prefetch and the staging lines are
+//      written with streaming stores;
+//   2  as 1, and every source line is then flushed from the caches (clflushopt, where the
+//      CPU has it), so no table row stays in the private caches of the copying cores.
+// Rows left in those caches (worker threads that then go idle) made every later GPU read of
+// them over PCIe (UVA, or UVA + dedup) 2.4x slower until the cores slept deeper.  bytes and
+// both addresses are multiples of 16.
+#ifndef NGRAM_DMA_NONTEMPORAL
+#define NGRAM_DMA_NONTEMPORAL 2
+#endif
+#if defined(__x86_64__)
+#include <cpuid.h>
+bool cpu_has_clflushopt() {
+    unsigned a = 0, b = 0, c = 0, d = 0;
+    if (!__get_cpuid_count(7, 0, &a, &b, &c, &d)) return false;
+    return (b >> 23) & 1u;                     // CPUID.(EAX=7, ECX=0):EBX[23]
+}
+const bool g_clflushopt = cpu_has_clflushopt();
+
+// Every 64-byte line that [p, p + bytes) touches, the partial lines at both ends included.
+__attribute__((target("clflushopt"))) void flush_lines(const uint8_t *p, uint32_t bytes) {
+    const uintptr_t end = reinterpret_cast<uintptr_t>(p) + bytes;
+    for (uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(63); a < end; a += 64)
+        _mm_clflushopt(reinterpret_cast<void *>(a));
+}
+#endif
+inline void copy_row_to_staging(uint8_t *dst, const uint8_t *src, uint32_t bytes) {
+#if defined(__x86_64__) && NGRAM_DMA_NONTEMPORAL
+    for (uint32_t o = 0; o < bytes; o += 64)
+        _mm_prefetch(reinterpret_cast<const char *>(src + o), _MM_HINT_NTA);
+    for (uint32_t o = 0; o < bytes; o += 16)
+        _mm_stream_si128(reinterpret_cast<__m128i *>(dst + o),
+                         _mm_load_si128(reinterpret_cast<const __m128i *>(src + o)));
+    if (NGRAM_DMA_NONTEMPORAL >= 2 && g_clflushopt) flush_lines(src, bytes);
+#else
+    memcpy(dst, src, bytes);
+#endif
+}
+
 // Host-resident, copy-engine path: the unique rows are compacted by host threads
 // into pinned staging and moved to HBM by cudaMemcpyAsync in chunks (the copy of
 // chunk i overlaps the host gather of chunk i+1), then gathered from HBM.
@@ -719,11 +760,17 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
     const uint32_t chunk_rows = std::max<uint32_t>(1u, NGRAM_DMA_CHUNK_BYTES / rb);
     for (uint32_t r0 = 0; r0 < U; r0 += chunk_rows) {
         const uint32_t r1 = std::min(U, r0 + chunk_rows);
-#pragma omp parallel for schedule(static) if (r1 - r0 >= 256)
-        for (int64_t u = r0; u < static_cast<int64_t>(r1); ++u) {
-            memcpy(c->h_stage + static_cast<size_t>(u) * rb,
-                   table + static_cast<size_t>(c->h_uniq[u]) * rb, rb);
-            if (c->h_stage_scale) c->h_stage_scale[u] = c->row_scale[c->h_uniq[u]];
+#pragma omp parallel if (r1 - r0 >= 256)
+        {
+#pragma omp for schedule(static)
+            for (int64_t u = r0; u < static_cast<int64_t>(r1); ++u) {
+                copy_row_to_staging(c->h_stage + static_cast<size_t>(u) * rb,
+                                    table + static_cast<size_t>(c->h_uniq[u]) * rb, rb);
+                if (c->h_stage_scale) c->h_stage_scale[u] = c->row_scale[c->h_uniq[u]];
+            }
+#if defined(__x86_64__) && NGRAM_DMA_NONTEMPORAL
+            _mm_sfence();                     // this thread's streaming stores are visible
+#endif
         }
         NG_CUDA(cudaMemcpyAsync(c->d_stage + static_cast<size_t>(r0) * rb,
                                 c->h_stage + static_cast<size_t>(r0) * rb,
@@ -829,8 +876,8 @@ ngram_status forward_uva(ngram_ctx *c, const Call &k) {
 
 // AUTO: the first call of each batch-size bucket runs the three host modes (UVA, UVA with
 // dedup, DMA; all write the same output), each once untimed (the first call of a mode
-// also allocates its staging) and then kNAutoTimed times timed, keeps the mode with the
-// lowest median time, and later calls use it.  auto_choice holds NGRAM_RES_HOST_UVA,
+// also allocates its staging) and then kNAutoTimed times timed in interleaved rounds,
+// keeps the mode with the lowest median time, and later calls use it.  auto_choice holds NGRAM_RES_HOST_UVA,
 // NGRAM_RES_HOST_DMA or NGRAM_AUTO_UVA_DEDUP.
 constexpr int kNAutoTimed = 3;
 
@@ -865,14 +912,17 @@ ngram_status forward_auto(ngram_ctx *c, const Call &k) {
         NG_CUDA(cudaEventCreate(&c->ev_t1), "cudaEventCreate");
     }
     const int modes[3] = {NGRAM_RES_HOST_UVA, NGRAM_AUTO_UVA_DEDUP, NGRAM_RES_HOST_DMA};
+    for (int m = 0; m < 3; ++m) NG_CHECK(run_mode(c, k, modes[m]));    // warm-up: staging, caches
+    // timed rounds interleave the modes, so a slow spell of the host or the link costs
+    // every mode alike instead of the one that happened to run then
+    float t[3][kNAutoTimed];
+    for (int r = 0; r < kNAutoTimed; ++r)
+        for (int m = 0; m < 3; ++m) NG_CHECK(time_mode(c, k, modes[m], &t[m][r]));
     int best = NGRAM_RES_HOST_UVA;
     float t_best = 0.f;
     for (int m = 0; m < 3; ++m) {
-        NG_CHECK(run_mode(c, k, modes[m]));              // warm-up: staging, caches
-        float t[kNAutoTimed];
-        for (int r = 0; r < kNAutoTimed; ++r) NG_CHECK(time_mode(c, k, modes[m], &t[r]));
-        std::sort(t, t + kNAutoTimed);
-        const float med = t[kNAutoTimed / 2];
+        std::sort(t[m], t[m] + kNAutoTimed);
+        const float med = t[m][kNAutoTimed / 2];
         if (m == 0 || med < t_best) { best = modes[m]; t_best = med; }
     }
     c->auto_choice[b] = best;

@@ -190,8 +190,9 @@ NGRAM_API ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *
  *                        (bounded wait, see ngram_set_wait_timeout);
  *              HOST_AUTO the first call of each batch-size bucket (ceil(log2 N)) runs
  *                        UVA, UVA with dedup (NGRAM_FLAG_DEDUP) and DMA, each once
- *                        untimed and then three times timed (synchronously); later
- *                        calls use the mode with the lowest median time
+ *                        untimed and then three times timed in interleaved rounds
+ *                        (synchronously); later calls use the mode with the lowest
+ *                        median time
  *                        (ngram_auto_choice reports it).
  *   hp         hash parameters (NULL = defaults).
  *   max_tokens largest n_seq * T a later call may pass (>= 1).
