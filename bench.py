@@ -267,6 +267,13 @@ def oracle_tokens_per_s(w, inp, budget_s: float, threads: int, seed: int = 0, ta
     t0 = time.perf_counter()
     oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sel, **kw)
     dt = time.perf_counter() - t0
+    if dt < budget_s / 2:                 # the whole batch took less than the budget: repeat it
+        reps = int(min(100, budget_s / max(dt, 1e-9)))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.forward(inp["tokens"], inp["history"], inp["residual"], inp["gate"], sel=sel, **kw)
+        dt = time.perf_counter() - t0
+        n *= reps
     return n / dt, n, dt
 
 
@@ -281,7 +288,8 @@ def cpu_baseline_record(w, inp, budget_s: float, table=None, table_desc: str = "
     v1, n1, dt1 = oracle_tokens_per_s(w, inp, min(3.0, budget_s / 4), 1, seed=1, table=table)
     rec = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "row_source": src,
            "gbs": v * per_tok / 1e9,
-           "sample": "%d of %d tokens of this workload, %.1f s, rows read from %s" % (
+           "sample": "%d tokens of this %d-token workload (repeated passes when one pass is short), "
+                     "%.1f s, rows read from %s" % (
                n, w.N, dt, table_desc if table is not None else
                "their synthetic-table definition (regenerated per element)"),
            "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "gbs": v1 * per_tok / 1e9,
@@ -600,8 +608,9 @@ def host_mem_available() -> int:
 def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
     """The other configurations on one GPU, each a sub-record of the bench line (bounded:
     fixed step counts, tables filled once).  Called after the headline with the full bf16
-    table still resident; ends with the CPU baseline on the materialised host table, the
-    host-resident configuration, and the 8- and 4-bit tables."""
+    table still resident: mid, the decode batches and the backward; then the host-resident
+    configuration and the CPU baseline on the same materialised host table; then the 8- and
+    4-bit tables, after the bf16 table is released."""
     import gc
 
     import torch
@@ -614,6 +623,12 @@ def run_extras(args, ng, dev, full, bt_full, read_gbs, line):
     mid = W["mid"]
     mdt, mtab, msc = make_table(ng, mid, dev)
     extra.append(hbm_record(ng, dev, mid, mdt, mtab, msc, 400, "eager", read_gbs))
+    if not args.no_cpu_baseline:        # the oracle on a host copy of mid's 9.5 GiB table
+        host_mid = mtab.view(torch.int16).cpu().numpy().view(np.uint16).reshape(mid.R, mid.d)
+        extra[-1]["cpu_baseline"] = cpu_baseline_record(
+            mid, gen.make_inputs(mid), min(args.cpu_seconds, 8.0), table=host_mid,
+            table_desc="a host copy of the 2,000,000 x 2560 bf16 table (9.5 GiB)")
+        del host_mid
     del mtab, msc
     gc.collect()
     torch.cuda.empty_cache()
@@ -799,6 +814,7 @@ def run_ours(args, w):
     e2e_ms = e0.elapsed_time(e1)
     h2d = w.N * 4 + (w.n_seq * 8 if w.history else 0) + w.N * w.d * 2 * (2 if args.variant == "token_gate" else 1)
     d2h = w.N * w.d * 2
+    bidir = measure_bidir_gbs(dev) if rank == 0 else (0.0, 0.0)
 
     # ---- max over ranks
     elapsed_ms, kern_ms, e2e_ms = max_over_ranks([elapsed_ms, kern_ms, e2e_ms], world, dev)
@@ -806,6 +822,9 @@ def run_ours(args, w):
     if rank == 0:
         value = weak_scaling_tokens_per_s(world, w.N, K, elapsed_ms)
         e2e_value = weak_scaling_tokens_per_s(world, w.N, E, e2e_ms)
+        # the PCIe bound of a call: its input and output bytes at the rates measured with both
+        # directions busy at once (one GPU's link; every rank has its own)
+        bound_ms = max(h2d / bidir[0], d2h / bidir[1]) / 1e6 if min(bidir) > 0 else None
         peaks = measured_peaks()
         bytes_launch = algorithmic_bytes(w) + (w.N * 2 * w.d if args.variant == "token_gate" else 0)
         achieved = bytes_launch / (kern_ms / 1e3) / 1e9
@@ -836,6 +855,9 @@ def run_ours(args, w):
                          "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E,
+                    "pcie_both_directions_gbs": {"h2d": bidir[0], "d2h": bidir[1]},
+                    "pcie_bound_tokens_per_s": (w.N * world / (bound_ms / 1e3)) if bound_ms else None,
+                    "frac_of_pcie_bound": (bound_ms / (e2e_ms / E)) if bound_ms else None,
                     "path": ("ngram_forward_host: pinned host tokens + residual in, bf16 out "
                              "back to pinned host, chunked H2D / gather / D2H on 3 streams")
                     if args.variant == "default" else
@@ -858,6 +880,40 @@ def run_ours(args, w):
         ctx.close()
     if world > 1:
         dist.destroy_process_group()
+
+
+def measure_bidir_gbs(dev, nbytes=1 << 30, reps=5):
+    """Best-of-N pinned copies in both directions at once (H2D on one stream, D2H on
+    another, from a common start): (H2D GB/s, D2H GB/s) -- the PCIe bound of a call that
+    moves its inputs in and its outputs out."""
+    import torch
+    src_h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst_h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    a_d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    b_d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    best = (0.0, 0.0)
+    for _ in range(reps):
+        start = torch.cuda.Event(enable_timing=True)
+        e1, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record()
+        s1.wait_event(start)
+        s2.wait_event(start)
+        with torch.cuda.stream(s1):
+            a_d.copy_(src_h, non_blocking=True)
+            e1.record(s1)
+        with torch.cuda.stream(s2):
+            dst_h.copy_(b_d, non_blocking=True)
+            e2.record(s2)
+        torch.cuda.synchronize()
+        h2d = nbytes / (start.elapsed_time(e1) / 1e3) / 1e9
+        d2h = nbytes / (start.elapsed_time(e2) / 1e3) / 1e9
+        if min(h2d, d2h) > min(best):
+            best = (h2d, d2h)
+    del src_h, dst_h, a_d, b_d
+    torch.cuda.empty_cache()
+    return best
 
 
 def measure_h2d_gbs(dev, nbytes=1 << 30, reps=10) -> float:

@@ -17,6 +17,7 @@
 #include <vector>
 
 #if defined(__x86_64__)
+#include <cpuid.h>
 #include <immintrin.h>
 #endif
 
@@ -707,7 +708,6 @@ ngram_status forward_dedup(ngram_ctx *c, const Call &k, unsigned compact_grid) {
 #define NGRAM_DMA_NONTEMPORAL 2
 #endif
 #if defined(__x86_64__)
-#include <cpuid.h>
 bool cpu_has_clflushopt() {
     unsigned a = 0, b = 0, c = 0, d = 0;
     if (!__get_cpuid_count(7, 0, &a, &b, &c, &d)) return false;
