@@ -96,6 +96,37 @@ def test_indices_exact_remainder_edge_R(cuda_device, R):
     assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
 
 
+def test_largest_vocabulary_uses_every_key_bit(cuda_device):
+    """Token ids up to 2^21 - 2 with vocab_size = 2^21 - 1 (the largest the 21-bit packing
+    allows): the trigram key fills 63 bits.  Indices (R = 2^32 - 1, and R = 20M in the
+    forward), the grouped-order path that hashes every token once (20,000 tokens) and the
+    forward itself equal the oracle; ids at the top of the range appear on purpose."""
+    V = (1 << 21) - 1
+    rng = np.random.default_rng(31)
+    toks = rng.integers(0, V, (2, 10_000)).astype(np.int32)
+    toks[0, :64] = V - 1 - np.arange(64)            # the largest ids, consecutive
+    hist = rng.integers(V - 8, V, (2, 2)).astype(np.int32)
+    ctx = _dummy_ctx(cuda_device, 4_294_967_295, vocab=V, max_tokens=toks.size)
+    got = ng.ngram_hash_indices(ctx, to_dev_tokens(toks, cuda_device), to_dev_tokens(hist, cuda_device))
+    want = oracle.indices(toks, hist, 4_294_967_295, vocab_size=V)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+    R, d = 20_000_000, 64
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    w = gen.Workload("vmax", R, d, "bf16", V, 2, 10_000, history=True)
+    fctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    res = gen.residual_bf16_bits(w.N, d, 32)
+    gate = gen.gate_f32(d, 33)
+    out = ng.ngram_forward(fctx, to_dev_tokens(toks, cuda_device), to_dev_bf16(res, cuda_device).view(w.N, d),
+                           torch.from_numpy(gate).to(cuda_device), history=to_dev_tokens(hist, cuda_device))
+    sel = sample_tokens(w, 512)
+    ref = oracle.forward(toks, hist, res, gate, R=R, d=d, table_seed=gen.TABLE_SEED, sel=sel,
+                         acc=oracle.ACC_F32, n_threads=N_CPU, vocab_size=V)
+    r = assert_parity(from_dev_bf16(out).reshape(w.N, d)[sel], ref)
+    assert r["exact"] == r["n"]
+    assert ng.ngram_get_device_error(fctx)[0] == ng.NGRAM_OK
+
+
 @pytest.mark.parametrize("nb,nt", [(1, 0), (0, 1), (3, 5), (16, 0), (0, 16), (7, 9)])
 def test_indices_head_counts(cuda_device, nb, nt):
     toks = gen.zipf_tokens(3, 50, 32_000, seed=23)
