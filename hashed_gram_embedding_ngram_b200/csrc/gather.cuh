@@ -52,6 +52,10 @@ struct GatherArgs {
     uint32_t ld;
     uint32_t n_outs;
     uint16_t *outs[8];
+    // 1: the kernel lets the next programmatic-dependent kernel of its stream be scheduled as
+    // soon as it starts (full-grid launches); 0: only when it ends (a bounded grid that runs
+    // long beside other work, whose successor would otherwise sit resident and waiting)
+    uint32_t trigger_early;
 };
 
 // 16-byte load through L2 without L1 allocation; coherent (the residual may be the
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(256, kMinBlocks) k_gather_bf16(const GatherArg
     const uint32_t n_items = g.N * g.groups_per_token;
     const uint16_t *__restrict__ table = static_cast<const uint16_t *>(g.table);
     const uint64_t seed = head_seed(lane, g.h);           // arithmetic only: before the wait
-    allow_dependents();
+    if (g.trigger_early) allow_dependents();
     grid_dependency_wait();
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {

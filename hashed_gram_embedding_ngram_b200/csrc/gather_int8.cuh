@@ -72,7 +72,7 @@ __device__ __forceinline__ void gather_rowscale(const GatherArgs &g) {
     const uint32_t n_items = g.N * g.groups_per_token;
     const uint8_t *__restrict__ table = static_cast<const uint8_t *>(g.table);
     const uint64_t seed = head_seed(lane, g.h);           // arithmetic only: before the wait
-    allow_dependents();
+    if (g.trigger_early) allow_dependents();
     grid_dependency_wait();
 
     for (uint32_t item = warp; item < n_items; item += n_warps) {

@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(256, NGRAM_NVFP4_MIN_BLOCKS) k_gather_nvfp4(co
     const uint32_t n_items = g.N * g.groups_per_token;
     const uint8_t *__restrict__ table = static_cast<const uint8_t *>(g.table);
     const uint64_t seed = head_seed(lane, g.h);           // arithmetic only: before the wait
-    allow_dependents();
+    if (g.trigger_early) allow_dependents();
     grid_dependency_wait();
     const float gs = __ldg(g.row_scale);                  // the global scale
 

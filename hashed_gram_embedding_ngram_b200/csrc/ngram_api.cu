@@ -451,6 +451,7 @@ GatherArgs gather_args(const ngram_ctx *c, const int32_t *tokens, const int32_t 
     g.ld = c->d;
     g.n_outs = 0;
     for (uint16_t *&o : g.outs) o = nullptr;
+    g.trigger_early = 1;
     return g;
 }
 
@@ -507,10 +508,13 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 // previous kernel of the stream is still running, and waits for it (griddepcontrol.wait)
 // before its first global memory access -- the launch latency overlaps the previous
 // kernel's tail, the results are those of plain stream order.  Only kernels that call
-// grid_dependency_wait() first are launched this way.
+// grid_dependency_wait() first are launched this way.  dependent = false launches plainly
+// (grid_dependency_wait() then returns at once): the bounded-grid lookups that run beside
+// other work on the GPU, whose early resident-but-waiting CTAs would hold SM slots that work
+// could use.
 template <typename... KArgs>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
-                             const KArgs &...args) {
+cudaError_t launch_maybe_dependent(bool dependent, void (*kernel)(KArgs...), unsigned grid, unsigned block,
+                                   cudaStream_t s, const KArgs &...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
@@ -520,29 +524,35 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned b
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = NGRAM_PDL ? 1 : 0;
+    cfg.numAttrs = (NGRAM_PDL && dependent) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename... KArgs>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
+                             const KArgs &...args) {
+    return launch_maybe_dependent(true, kernel, grid, block, s, args...);
 }
 
 // kThree: the bf16 gather compiled for 3 resident CTAs per SM (see k_gather_bf16).
 template <bool kTok, bool kThree = false>
-cudaError_t launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s) {
+cudaError_t launch_gather_kernel(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t s, bool dep) {
     const bool h16 = g.h.n_heads == 16;
     switch (t) {
         case NGRAM_BF16:
-            if (kThree) return h16 ? launch_dependent(k_gather_bf16<16, kTok, 3>, nb, 256, s, g)
-                                   : launch_dependent(k_gather_bf16<0, kTok, 3>, nb, 256, s, g);
-            return h16 ? launch_dependent(k_gather_bf16<16, kTok>, nb, 256, s, g)
-                       : launch_dependent(k_gather_bf16<0, kTok>, nb, 256, s, g);
+            if (kThree) return h16 ? launch_maybe_dependent(dep, k_gather_bf16<16, kTok, 3>, nb, 256, s, g)
+                                   : launch_maybe_dependent(dep, k_gather_bf16<0, kTok, 3>, nb, 256, s, g);
+            return h16 ? launch_maybe_dependent(dep, k_gather_bf16<16, kTok>, nb, 256, s, g)
+                       : launch_maybe_dependent(dep, k_gather_bf16<0, kTok>, nb, 256, s, g);
         case NGRAM_INT8_ROWSCALE:
-            return h16 ? launch_dependent(k_gather_int8<16, kTok>, nb, 256, s, g)
-                       : launch_dependent(k_gather_int8<0, kTok>, nb, 256, s, g);
+            return h16 ? launch_maybe_dependent(dep, k_gather_int8<16, kTok>, nb, 256, s, g)
+                       : launch_maybe_dependent(dep, k_gather_int8<0, kTok>, nb, 256, s, g);
         case NGRAM_FP8_E4M3_ROWSCALE:
-            return h16 ? launch_dependent(k_gather_fp8<16, kTok>, nb, 256, s, g)
-                       : launch_dependent(k_gather_fp8<0, kTok>, nb, 256, s, g);
+            return h16 ? launch_maybe_dependent(dep, k_gather_fp8<16, kTok>, nb, 256, s, g)
+                       : launch_maybe_dependent(dep, k_gather_fp8<0, kTok>, nb, 256, s, g);
         case NGRAM_NVFP4:
-            return h16 ? launch_dependent(k_gather_nvfp4<16, kTok>, nb, 256, s, g)
-                       : launch_dependent(k_gather_nvfp4<0, kTok>, nb, 256, s, g);
+            return h16 ? launch_maybe_dependent(dep, k_gather_nvfp4<16, kTok>, nb, 256, s, g)
+                       : launch_maybe_dependent(dep, k_gather_nvfp4<0, kTok>, nb, 256, s, g);
     }
     return cudaErrorInvalidValue;
 }
@@ -609,11 +619,15 @@ ngram_status launch_gather(ngram_ctx *c, GatherArgs &g, cudaStream_t s, uint64_t
     uint64_t blocks = (items + 7) / 8;
     if (blocks > (use_three ? three : max_blocks)) blocks = use_three ? three : max_blocks;
     const unsigned nb = static_cast<unsigned>(blocks);
+    // a full-grid gather launches as a programmatic dependent; a bounded grid (the
+    // host-resident lookup that runs beside other work) launches plainly
+    const bool dep = max_blocks == full_grid(c);
+    g.trigger_early = dep ? 1u : 0u;
     cudaError_t e;
-    if (g.gate_tok != nullptr) e = use_three ? launch_gather_kernel<true, true>(c->dtype, g, nb, s)
-                                             : launch_gather_kernel<true>(c->dtype, g, nb, s);
-    else e = use_three ? launch_gather_kernel<false, true>(c->dtype, g, nb, s)
-                       : launch_gather_kernel<false>(c->dtype, g, nb, s);
+    if (g.gate_tok != nullptr) e = use_three ? launch_gather_kernel<true, true>(c->dtype, g, nb, s, dep)
+                                             : launch_gather_kernel<true>(c->dtype, g, nb, s, dep);
+    else e = use_three ? launch_gather_kernel<false, true>(c->dtype, g, nb, s, dep)
+                       : launch_gather_kernel<false>(c->dtype, g, nb, s, dep);
     NG_CUDA(e, "gather kernel launch");
     return NGRAM_OK;
 }
