@@ -221,7 +221,12 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  * launches nothing.  The grouping and row-id scratch belong to the context: order the
  * context's ngram_forward calls (one stream, or events); ngram_prefetch uses other scratch
  * and may run beside them.  EINVAL if N > max_tokens, a pointer is NULL or misaligned.  Bad
- * token ids are reported asynchronously through ngram_get_device_error. */
+ * token ids are reported asynchronously through ngram_get_device_error.
+ *   Stream order: the gather and the order kernels of an HBM lookup are launched as
+ *   programmatic dependents (the launch may overlap the previous kernel of the stream; each
+ *   waits for that kernel to complete before touching memory), and they let the next such
+ *   kernel be scheduled as soon as they start.  Results are those of plain stream order.
+ *   The host-resident lookups on a bounded grid launch plainly. */
 NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
                            const void *gate, uint16_t *out, ngram_stream_t stream);
