@@ -75,12 +75,20 @@ using namespace ngram;
 #ifndef NGRAM_BULK_CTAS_PER_SM
 #define NGRAM_BULK_CTAS_PER_SM 2
 #endif
-// NGRAM_UVA_CTAS: CTAs of the host-resident (UVA) gather.  8 CTAs (512 KB of row loads
-//   in flight) already saturate PCIe (51.4 GB/s, 0.93 of measured H2D, for the same
-//   8192-token prefill as 296 CTAs) and leave 140 SMs to the work beside the lookup: a
-//   bf16 4096x2560x2560 GEMM on another stream keeps 1166 TFLOP/s vs 667 with 296 CTAs.
+// NGRAM_UVA_CTAS: CTAs of the host-resident (UVA) gather.  4 CTAs (256 KB of row loads in
+//   flight) keep PCIe as busy as 8 or 296 (decode-256 0.416 against 0.414 ms at 8; prefill
+//   8192 13.05 ms at both, 0.92 of measured H2D) and leave the most SMs to the work beside
+//   the lookup: a bf16 4096x2560x2560 GEMM on another stream keeps 1222-1236 TFLOP/s beside
+//   the decode-256 lookup at 4 CTAs, 1061-1063 at 8, 667 at 296; at 2 CTAs the lookup slows
+//   to 0.49 ms.
+// NGRAM_UVA_COPY_CTAS: CTAs of the copy kernel that moves each distinct host row once into
+//   HBM staging (UVA + dedup, prefetch).  Its flat copy needs 8: at 4 the 8192-token copy
+//   took 14.1 against 11.4 ms.
 #ifndef NGRAM_UVA_CTAS
-#define NGRAM_UVA_CTAS 8
+#define NGRAM_UVA_CTAS 4
+#endif
+#ifndef NGRAM_UVA_COPY_CTAS
+#define NGRAM_UVA_COPY_CTAS 8
 #endif
 #ifndef NGRAM_DMA_CHUNK_BYTES           // host gather -> H2D pipelining granularity
 #define NGRAM_DMA_CHUNK_BYTES (8u << 20)
@@ -690,7 +698,7 @@ ngram_status forward_direct(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
 }
 
 // hash -> dedup -> compact the unique rows into HBM staging -> gather from staging.
-// compact_grid: CTAs of the copy kernel (a full grid from HBM; NGRAM_UVA_CTAS from host
+// compact_grid: CTAs of the copy kernel (a full grid from HBM; NGRAM_UVA_COPY_CTAS from host
 // memory, where each distinct row then crosses PCIe once).
 ngram_status forward_dedup(ngram_ctx *c, const Call &k, unsigned compact_grid) {
     NG_CHECK(ensure_dedup_scratch(c));
@@ -873,7 +881,7 @@ ngram_status forward_dedup_hbm(ngram_ctx *c, const Call &k) {
 
 // UVA with dedup: each distinct row crosses PCIe once, read by the copy kernel.
 ngram_status forward_dedup_uva(ngram_ctx *c, const Call &k) {
-    return forward_dedup(c, k, static_cast<unsigned>(std::min<uint64_t>(NGRAM_UVA_CTAS, full_grid(c))));
+    return forward_dedup(c, k, static_cast<unsigned>(std::min<uint64_t>(NGRAM_UVA_COPY_CTAS, full_grid(c))));
 }
 
 // UVA without dedup: the gather kernel reads the host rows itself, on a bounded grid.
@@ -1223,7 +1231,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, sl.inv, c->d_count, s));
     // each distinct row crosses once; from host memory a few CTAs keep PCIe busy
     const unsigned grid = (c->where == NGRAM_RES_HBM) ? grid_for(c, M * 32ull, 256)
-                                                      : static_cast<unsigned>(NGRAM_UVA_CTAS);
+                                                      : static_cast<unsigned>(NGRAM_UVA_COPY_CTAS);
     k_compact_rows<<<grid, 256, 0, s>>>(static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c),
                                         c->d_uniq, c->d_count, c->row_bytes, sl.stage, sl.stage_scale);
     NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
