@@ -174,22 +174,6 @@ __global__ void __launch_bounds__(256) k_seg_starts(const uint32_t *__restrict__
 #define NGRAM_ROWS_GRAD_MIN_BLOCKS 2
 #endif
 
-#ifndef NGRAM_ROWS_GRAD_DY_KEEP          // 1: dy loads ask L2 to keep the lines (evict_last)
-#define NGRAM_ROWS_GRAD_DY_KEEP 0
-#endif
-__device__ __forceinline__ uint2 ld_dy_v2(const void *p, uint64_t policy) {
-#if NGRAM_ROWS_GRAD_DY_KEEP
-    uint2 r;
-    asm("ld.global.nc.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
-        : "=r"(r.x), "=r"(r.y)
-        : "l"(p), "l"(policy));
-    return r;
-#else
-    (void)policy;
-    return __ldg(reinterpret_cast<const uint2 *>(p));
-#endif
-}
-
 template <bool kTokGate, int kStrips>
 __global__ void __launch_bounds__(256, NGRAM_ROWS_GRAD_MIN_BLOCKS) k_rows_grad(const uint32_t *__restrict__ count,
                                                       const uint32_t *__restrict__ seg,
@@ -205,10 +189,6 @@ __global__ void __launch_bounds__(256, NGRAM_ROWS_GRAD_MIN_BLOCKS) k_rows_grad(c
     const uint32_t n_groups = (n_strips + kStrips - 1u) / kStrips;
     const uint32_t U = *count;
     const uint32_t n_items = ((U + 31u) >> 5) * n_groups;
-    uint64_t keep = 0;
-#if NGRAM_ROWS_GRAD_DY_KEEP
-    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
-#endif
     for (;;) {
         uint32_t item = 0;
         if (lane == 0) item = atomicAdd(next_item, 1u);
@@ -253,9 +233,9 @@ __global__ void __launch_bounds__(256, NGRAM_ROWS_GRAD_MIN_BLOCKS) k_rows_grad(c
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
                                 if (act[k][h]) {
-                                    w[q][k][h] = ld_dy_v2(row + c0[k] + h * 128u, keep);
+                                    w[q][k][h] = __ldg(reinterpret_cast<const uint2 *>(row + c0[k] + h * 128u));
                                     if (kTokGate)
-                                        gw[q][k][h] = ld_dy_v2(grow + c0[k] + h * 128u, keep);
+                                        gw[q][k][h] = __ldg(reinterpret_cast<const uint2 *>(grow + c0[k] + h * 128u));
                                 }
                             }
                         }
