@@ -21,6 +21,9 @@
 // The gate-gradient kernel recomputes e with the row-format policies of rows.cuh, which
 // decode and sum exactly as the forward gathers do (same operations in the same head
 // order), so e is bit-identical to the forward's.  A lane owns 8 columns here.
+//
+// Every kernel here opens with allow_dependents(); grid_dependency_wait(), so the steps of
+// a backward call may be launched as programmatic dependents of one another.
 #pragma once
 
 #include "rows.cuh"
@@ -37,6 +40,8 @@ template <int kH, class Rows, bool kPerToken>
 __global__ void __launch_bounds__(256, 2) k_gate_grad(const GatherArgs g, const uint16_t *__restrict__ dy,
                                                       float *__restrict__ dg_tok,
                                                       double *__restrict__ partial, uint32_t row_bytes) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
@@ -119,6 +124,8 @@ constexpr uint32_t kGateGroup = 32;
 __global__ void __launch_bounds__(256) k_gate_reduce_groups(const double *__restrict__ partial,
                                                             uint32_t n_chunks, uint32_t d,
                                                             double *__restrict__ group) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t c = blockIdx.x * blockDim.x + threadIdx.x;
     const uint32_t gi = blockIdx.y;
     if (c >= d) return;
@@ -131,6 +138,8 @@ __global__ void __launch_bounds__(256) k_gate_reduce_groups(const double *__rest
 
 __global__ void __launch_bounds__(256) k_gate_reduce(const double *__restrict__ group, uint32_t n_groups,
                                                      uint32_t d, float *__restrict__ dg) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= d) return;
     double s = 0.0;
@@ -142,6 +151,8 @@ __global__ void __launch_bounds__(256) k_gate_reduce(const double *__restrict__ 
 // seg[u] = first position of row u in the sorted occurrence list; seg[U] = M.
 __global__ void __launch_bounds__(256) k_seg_starts(const uint32_t *__restrict__ skeys, uint32_t M,
                                                     uint32_t *__restrict__ seg) {
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t p = blockIdx.x * blockDim.x + threadIdx.x; p < M; p += gridDim.x * blockDim.x) {
         const uint32_t u = skeys[p];
         if (p == 0 || skeys[p - 1] != u) seg[u] = p;
@@ -183,6 +194,8 @@ __global__ void __launch_bounds__(256, NGRAM_ROWS_GRAD_MIN_BLOCKS) k_rows_grad(c
                                                       const uint16_t *__restrict__ gate_tok,
                                                       uint32_t d, float *__restrict__ grad,
                                                       uint32_t *next_item) {
+    allow_dependents();
+    grid_dependency_wait();
     constexpr uint32_t kBatch = (kTokGate ? NGRAM_ROWS_GRAD_BATCH / 2u : NGRAM_ROWS_GRAD_BATCH) / kStrips;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t n_strips = ((d >> 3) + 31u) >> 5;

@@ -22,6 +22,8 @@
 //   4. emit: each first occurrence i takes u = its global rank: uniq[u] = idx[i],
 //      uid[slot[i]] = u;
 //   5. inverse: inv[i] = uid[slot[i]].
+// Steps 1-5 open with allow_dependents(); grid_dependency_wait(): each may be launched as a
+// programmatic dependent of the step before and waits for it before touching memory.
 #pragma once
 
 #include "device_common.cuh"
@@ -38,6 +40,8 @@ __device__ __forceinline__ uint32_t dedup_home(uint32_t row, uint32_t log2p) {
 __global__ void __launch_bounds__(256) k_dedup_insert(const uint32_t *__restrict__ idx, uint32_t M,
                                                       uint32_t *keys, uint32_t *first,
                                                       uint32_t *__restrict__ slot_of, uint32_t log2p) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t mask = (1u << log2p) - 1u;
     for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < M; i += gridDim.x * blockDim.x) {
         const uint32_t row = idx[i];
@@ -58,6 +62,8 @@ __global__ void __launch_bounds__(256) k_dedup_scan_local(const uint32_t *__rest
                                                           const uint32_t *__restrict__ first,
                                                           uint32_t M, uint32_t *__restrict__ pos,
                                                           uint32_t *__restrict__ block_sum) {
+    allow_dependents();
+    grid_dependency_wait();
     __shared__ uint32_t warp_tot[8];
     const uint32_t base = blockIdx.x * kScanBlock + threadIdx.x * 4u;
     uint32_t f[4], run = 0;
@@ -92,6 +98,8 @@ __global__ void __launch_bounds__(256) k_dedup_scan_local(const uint32_t *__rest
 // Exclusive scan of the block totals by one CTA; writes U to *count.
 __global__ void __launch_bounds__(1024) k_dedup_scan_blocks(uint32_t *block_sum, uint32_t nb,
                                                             uint32_t *count) {
+    allow_dependents();
+    grid_dependency_wait();
     __shared__ uint32_t warp_tot[32];
     __shared__ uint32_t carry;
     if (threadIdx.x == 0) carry = 0;
@@ -126,6 +134,8 @@ __global__ void __launch_bounds__(256) k_dedup_emit(const uint32_t *__restrict__
                                                     const uint32_t *__restrict__ block_off, uint32_t M,
                                                     uint32_t *__restrict__ uniq,
                                                     uint32_t *__restrict__ uid) {
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < M; i += gridDim.x * blockDim.x) {
         const uint32_t s = slot_of[i];
         if (first[s] == i) {
@@ -139,6 +149,8 @@ __global__ void __launch_bounds__(256) k_dedup_emit(const uint32_t *__restrict__
 __global__ void __launch_bounds__(256) k_dedup_inverse(const uint32_t *__restrict__ slot_of,
                                                        const uint32_t *__restrict__ uid, uint32_t M,
                                                        uint32_t *__restrict__ inv) {
+    allow_dependents();
+    grid_dependency_wait();
     for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < M; i += gridDim.x * blockDim.x)
         inv[i] = uid[slot_of[i]];
 }

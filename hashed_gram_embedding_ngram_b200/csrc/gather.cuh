@@ -194,6 +194,8 @@ __global__ void __launch_bounds__(256) k_hash_indices(const HashArgs a,
                                                       const int32_t *__restrict__ history,
                                                       uint32_t T, uint32_t N, uint32_t *err,
                                                       uint32_t *__restrict__ idx_out) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t H = a.n_heads;
     const uint32_t total = N * H;
     for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total;

@@ -14,6 +14,7 @@
 #include <mutex>
 #include <string>
 #include <thread>
+#include <utility>
 #include <vector>
 
 #if defined(__x86_64__)
@@ -520,11 +521,11 @@ void launch_shard(ngram_dtype t, const GatherArgs &g, unsigned nb, cudaStream_t 
 // (grid_dependency_wait() then returns at once): the bounded-grid lookups that run beside
 // other work on the GPU, whose early resident-but-waiting CTAs would hold SM slots that work
 // could use.
-template <typename... KArgs>
-cudaError_t launch_maybe_dependent(bool dependent, void (*kernel)(KArgs...), unsigned grid, unsigned block,
-                                   cudaStream_t s, const KArgs &...args) {
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_dependent(bool dependent, void (*kernel)(KArgs...), dim3 grid, unsigned block,
+                                   cudaStream_t s, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
@@ -533,13 +534,13 @@ cudaError_t launch_maybe_dependent(bool dependent, void (*kernel)(KArgs...), uns
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (NGRAM_PDL && dependent) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <typename... KArgs>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
-                             const KArgs &...args) {
-    return launch_maybe_dependent(true, kernel, grid, block, s, args...);
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, unsigned block, cudaStream_t s,
+                             Args &&...args) {
+    return launch_maybe_dependent(true, kernel, grid, block, s, std::forward<Args>(args)...);
 }
 
 // kThree: the bf16 gather compiled for 3 resident CTAs per SM (see k_gather_bf16).
@@ -651,9 +652,9 @@ unsigned grid_for(const ngram_ctx *c, uint64_t work, uint32_t per_block) {
 ngram_status launch_hash(ngram_ctx *c, const int32_t *tokens, const int32_t *history, uint32_t T,
                          uint32_t N, uint32_t *idx_out, cudaStream_t s) {
     const HashArgs a = hash_args(c);
-    k_hash_indices<<<grid_for(c, static_cast<uint64_t>(N) * a.n_heads, 256), 256, 0, s>>>(
-        a, tokens, history, T, N, c->d_err, idx_out);
-    NG_CUDA(cudaGetLastError(), "k_hash_indices launch");
+    NG_CUDA(launch_dependent(k_hash_indices, grid_for(c, static_cast<uint64_t>(N) * a.n_heads, 256), 256, s,
+                             a, tokens, history, T, N, c->d_err, idx_out),
+            "k_hash_indices launch");
     return NGRAM_OK;
 }
 
@@ -661,18 +662,38 @@ ngram_status launch_hash(ngram_ctx *c, const int32_t *tokens, const int32_t *his
 ngram_status launch_dedup(ngram_ctx *c, const uint32_t *idx, uint32_t M, uint32_t *uniq,
                           uint32_t *inv, uint32_t *count, cudaStream_t s) {
     const uint32_t log2p = std::max<uint32_t>(10u, ceil_log2(2ull * M));
-    const uint32_t P = 1u << log2p;
     const uint32_t NB = (M + kScanBlock - 1) / kScanBlock;
+    const unsigned gm = grid_for(c, M, 256);
+    NG_CUDA(launch_dependent(k_dedup_insert, gm, 256, s, idx, M, c->d_keys, c->d_first, c->d_slot, log2p),
+            "dedup launch");
+    NG_CUDA(launch_dependent(k_dedup_scan_local, NB, 256, s, c->d_slot, c->d_first, M, c->d_pos, c->d_bsum),
+            "dedup launch");
+    NG_CUDA(launch_dependent(k_dedup_scan_blocks, 1, 1024, s, c->d_bsum, NB, count), "dedup launch");
+    NG_CUDA(launch_dependent(k_dedup_emit, gm, 256, s, idx, c->d_slot, c->d_first, c->d_pos, c->d_bsum, M,
+                             uniq, c->d_uid),
+            "dedup launch");
+    NG_CUDA(launch_dependent(k_dedup_inverse, gm, 256, s, c->d_slot, c->d_uid, M, inv), "dedup launch");
+    return NGRAM_OK;
+}
+
+// The two tables the dedup of M indices starts from, cleared (every slot empty).  Issued
+// before the hash kernel, so that the hash and dedup kernels follow one another directly
+// and each may be launched as a programmatic dependent of the one before.
+ngram_status dedup_clear(ngram_ctx *c, uint32_t M, cudaStream_t s) {
+    const uint32_t log2p = std::max<uint32_t>(10u, ceil_log2(2ull * M));
+    const uint64_t P = 1ull << log2p;
     NG_CUDA(cudaMemsetAsync(c->d_keys, 0xFF, P * 4ull, s), "dedup clear");
     NG_CUDA(cudaMemsetAsync(c->d_first, 0xFF, P * 4ull, s), "dedup clear");
-    const unsigned gm = grid_for(c, M, 256);
-    k_dedup_insert<<<gm, 256, 0, s>>>(idx, M, c->d_keys, c->d_first, c->d_slot, log2p);
-    k_dedup_scan_local<<<NB, 256, 0, s>>>(c->d_slot, c->d_first, M, c->d_pos, c->d_bsum);
-    k_dedup_scan_blocks<<<1, 1024, 0, s>>>(c->d_bsum, NB, count);
-    k_dedup_emit<<<gm, 256, 0, s>>>(idx, c->d_slot, c->d_first, c->d_pos, c->d_bsum, M, uniq, c->d_uid);
-    k_dedup_inverse<<<gm, 256, 0, s>>>(c->d_slot, c->d_uid, M, inv);
-    NG_CUDA(cudaGetLastError(), "dedup launch");
     return NGRAM_OK;
+}
+
+// Hash the N tokens' M = N * H row indices into c->d_idx, then dedup them.
+ngram_status launch_hash_dedup(ngram_ctx *c, const int32_t *tokens, const int32_t *history, uint32_t T,
+                               uint32_t N, uint32_t *uniq, uint32_t *inv, uint32_t *count, cudaStream_t s) {
+    const uint32_t M = N * c->H;
+    NG_CHECK(dedup_clear(c, M, s));
+    NG_CHECK(launch_hash(c, tokens, history, T, N, c->d_idx, s));
+    return launch_dedup(c, c->d_idx, M, uniq, inv, count, s);
 }
 
 // ---------------------------------------------------------------- forward paths
@@ -703,9 +724,7 @@ ngram_status forward_direct(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
 ngram_status forward_dedup(ngram_ctx *c, const Call &k, unsigned compact_grid) {
     NG_CHECK(ensure_dedup_scratch(c));
     NG_CHECK(ensure_device_stage(c));
-    const uint32_t M = k.N * c->H;
-    NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
-    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
+    NG_CHECK(launch_hash_dedup(c, k.tokens, k.history, k.T, k.N, c->d_uniq, c->d_inv, c->d_count, k.s));
     k_compact_rows<<<compact_grid, 256, 0, k.s>>>(
         static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c), c->d_uniq, c->d_count,
         c->row_bytes, c->d_stage, c->d_stage_scale);
@@ -764,8 +783,7 @@ ngram_status forward_dma(ngram_ctx *c, const Call &k) {
     NG_CHECK(ensure_dedup_scratch(c));
     NG_CHECK(ensure_host_stage(c));
     const uint32_t M = k.N * c->H;
-    NG_CHECK(launch_hash(c, k.tokens, k.history, k.T, k.N, c->d_idx, k.s));
-    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, c->d_inv, c->d_count, k.s));
+    NG_CHECK(launch_hash_dedup(c, k.tokens, k.history, k.T, k.N, c->d_uniq, c->d_inv, c->d_count, k.s));
     if (c->stage_in_use) NG_CHECK(wait_event(c, c->ev_stage_free, "DMA: previous staging copy"));
     NG_CUDA(cudaMemcpyAsync(c->h_count, c->d_count, 4, cudaMemcpyDeviceToHost, k.s), "D2H count");
     NG_CUDA(cudaMemcpyAsync(c->h_uniq, c->d_uniq, M * 4ull, cudaMemcpyDeviceToHost, k.s), "D2H rows");
@@ -1227,8 +1245,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint32_t M = static_cast<uint32_t>(N) * c->H;
-    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
-    NG_CHECK(launch_dedup(c, c->d_idx, M, c->d_uniq, sl.inv, c->d_count, s));
+    NG_CHECK(launch_hash_dedup(c, tokens, history, T, static_cast<uint32_t>(N), c->d_uniq, sl.inv, c->d_count, s));
     // each distinct row crosses once; from host memory a few CTAs keep PCIe busy
     const unsigned grid = (c->where == NGRAM_RES_HBM) ? grid_for(c, M * 32ull, 256)
                                                       : static_cast<unsigned>(NGRAM_UVA_COPY_CTAS);
@@ -1297,9 +1314,7 @@ ngram_status ngram_dedup_rows(ngram_ctx *c, const int32_t *tokens, const int32_t
     if (uniq_out == nullptr || inv_out == nullptr)
         return fail(NGRAM_EINVAL, "uniq_out and inv_out must be non-NULL");
     NG_CHECK(ensure_dedup_scratch(c));
-    const uint32_t M = static_cast<uint32_t>(N) * c->H;
-    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
-    return launch_dedup(c, c->d_idx, M, uniq_out, inv_out, count_out, s);
+    return launch_hash_dedup(c, tokens, history, T, static_cast<uint32_t>(N), uniq_out, inv_out, count_out, s);
 }
 
 ngram_status ngram_fill_synthetic(void *table, float *row_scale, uint64_t R, uint32_t d,
@@ -1468,10 +1483,9 @@ ngram_status ensure_backward_sort(ngram_ctx *c) {
 // Exclusive scan of a[0..n) in place.
 ngram_status scan_exclusive(ngram_ctx *c, uint32_t *a, uint32_t n, cudaStream_t s) {
     const uint32_t nb = (n + kScanChunk - 1) / kScanChunk;
-    k_scan_local<<<nb, 256, 0, s>>>(a, n, a, c->bw_tot);
-    k_dedup_scan_blocks<<<1, 1024, 0, s>>>(c->bw_tot, nb, c->bw_word);
-    k_scan_add<<<(n + 255) / 256, 256, 0, s>>>(a, n, c->bw_tot);
-    NG_CUDA(cudaGetLastError(), "scan launch");
+    NG_CUDA(launch_dependent(k_scan_local, nb, 256, s, a, n, a, c->bw_tot), "scan launch");
+    NG_CUDA(launch_dependent(k_dedup_scan_blocks, 1, 1024, s, c->bw_tot, nb, c->bw_word), "scan launch");
+    NG_CUDA(launch_dependent(k_scan_add, (n + 255) / 256, 256, s, a, n, c->bw_tot), "scan launch");
     return NGRAM_OK;
 }
 
@@ -1486,12 +1500,13 @@ ngram_status sort_occurrences(ngram_ctx *c, const uint32_t *keys, uint32_t M, cu
     const uint32_t *kin = keys, *vin = nullptr;
     for (uint32_t pass = 0; pass < passes; ++pass) {
         const uint32_t shift = 8 * pass;
-        k_radix_hist<<<grid, 256, 0, s>>>(kin, M, shift, n_tiles, c->bw_hist);
+        NG_CUDA(launch_dependent(k_radix_hist, grid, 256, s, kin, M, shift, n_tiles, c->bw_hist),
+                "radix sort launch");
         NG_CHECK(scan_exclusive(c, c->bw_hist, kSortRadix * n_tiles, s));
         const int o = static_cast<int>(pass & 1u);
-        k_radix_scatter<<<grid, 256, 0, s>>>(kin, vin, c->H, M, shift, n_tiles, c->bw_hist,
-                                             c->bw_k[o], c->bw_v[o]);
-        NG_CUDA(cudaGetLastError(), "radix sort launch");
+        NG_CUDA(launch_dependent(k_radix_scatter, grid, 256, s, kin, vin, c->H, M, shift, n_tiles, c->bw_hist,
+                                 c->bw_k[o], c->bw_v[o]),
+                "radix sort launch");
         kin = c->bw_k[o];
         vin = c->bw_v[o];
     }
@@ -1501,21 +1516,22 @@ ngram_status sort_occurrences(ngram_ctx *c, const uint32_t *keys, uint32_t M, cu
 }
 
 template <class Rows, bool kTok>
-void launch_gate_grad_fmt(const GatherArgs &g, unsigned grid, cudaStream_t s, const uint16_t *dy,
-                          float *dg, double *part, uint32_t rb) {
-    if (g.h.n_heads == 16) k_gate_grad<16, Rows, kTok><<<grid, 256, 0, s>>>(g, dy, dg, part, rb);
-    else k_gate_grad<0, Rows, kTok><<<grid, 256, 0, s>>>(g, dy, dg, part, rb);
+cudaError_t launch_gate_grad_fmt(const GatherArgs &g, unsigned grid, cudaStream_t s, const uint16_t *dy,
+                                 float *dg, double *part, uint32_t rb) {
+    if (g.h.n_heads == 16) return launch_dependent(k_gate_grad<16, Rows, kTok>, grid, 256, s, g, dy, dg, part, rb);
+    return launch_dependent(k_gate_grad<0, Rows, kTok>, grid, 256, s, g, dy, dg, part, rb);
 }
 
 template <bool kTok>
-void launch_gate_grad(ngram_dtype t, const GatherArgs &g, unsigned grid, cudaStream_t s,
-                      const uint16_t *dy, float *dg, double *part, uint32_t rb) {
+cudaError_t launch_gate_grad(ngram_dtype t, const GatherArgs &g, unsigned grid, cudaStream_t s,
+                             const uint16_t *dy, float *dg, double *part, uint32_t rb) {
     switch (t) {
-        case NGRAM_BF16: launch_gate_grad_fmt<RowsBf16, kTok>(g, grid, s, dy, dg, part, rb); break;
-        case NGRAM_INT8_ROWSCALE: launch_gate_grad_fmt<Rows8bit<Int8Codes>, kTok>(g, grid, s, dy, dg, part, rb); break;
-        case NGRAM_FP8_E4M3_ROWSCALE: launch_gate_grad_fmt<Rows8bit<E4m3Codes>, kTok>(g, grid, s, dy, dg, part, rb); break;
-        case NGRAM_NVFP4: launch_gate_grad_fmt<RowsNvfp4, kTok>(g, grid, s, dy, dg, part, rb); break;
+        case NGRAM_BF16: return launch_gate_grad_fmt<RowsBf16, kTok>(g, grid, s, dy, dg, part, rb);
+        case NGRAM_INT8_ROWSCALE: return launch_gate_grad_fmt<Rows8bit<Int8Codes>, kTok>(g, grid, s, dy, dg, part, rb);
+        case NGRAM_FP8_E4M3_ROWSCALE: return launch_gate_grad_fmt<Rows8bit<E4m3Codes>, kTok>(g, grid, s, dy, dg, part, rb);
+        case NGRAM_NVFP4: return launch_gate_grad_fmt<RowsNvfp4, kTok>(g, grid, s, dy, dg, part, rb);
     }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -1541,27 +1557,25 @@ ngram_status ngram_backward_rows(ngram_ctx *c, const int32_t *tokens, const int3
     NG_CHECK(ensure_dedup_scratch(c));
     NG_CHECK(ensure_backward_sort(c));
     const uint32_t M = static_cast<uint32_t>(N) * c->H;
-    NG_CHECK(launch_hash(c, tokens, history, T, static_cast<uint32_t>(N), c->d_idx, s));
-    NG_CHECK(launch_dedup(c, c->d_idx, M, uniq_out, c->d_inv, count_out, s));
+    NG_CUDA(cudaMemsetAsync(c->bw_word + 1, 0, 4, s), "cudaMemsetAsync");     // k_rows_grad's item counter
+    NG_CHECK(launch_hash_dedup(c, tokens, history, T, static_cast<uint32_t>(N), uniq_out, c->d_inv, count_out, s));
     const uint32_t *skeys = nullptr, *stok = nullptr;
     NG_CHECK(sort_occurrences(c, c->d_inv, M, s, &skeys, &stok));
-    k_seg_starts<<<grid_for(c, M, 256), 256, 0, s>>>(skeys, M, c->bw_seg);
+    NG_CUDA(launch_dependent(k_seg_starts, grid_for(c, M, 256), 256, s, skeys, M, c->bw_seg), "k_seg_starts launch");
     const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
     constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
     int per_sm = 0;
     NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                 &per_sm, tok_gate ? k_rows_grad<true, kS> : k_rows_grad<false, kS>, 256, 0), "occupancy");
     const unsigned grid = static_cast<unsigned>(c->num_sms) * static_cast<unsigned>(std::max(1, per_sm));
-    NG_CUDA(cudaMemsetAsync(c->bw_word + 1, 0, 4, s), "cudaMemsetAsync");     // the item counter
     if (tok_gate)
-        k_rows_grad<true, kS><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out, nullptr,
-                                                   static_cast<const uint16_t *>(gate), c->d, grad_rows,
-                                                   c->bw_word + 1);
+        NG_CUDA(launch_dependent(k_rows_grad<true, kS>, grid, 256, s, count_out, c->bw_seg, stok, grad_out,
+                                 nullptr, static_cast<const uint16_t *>(gate), c->d, grad_rows, c->bw_word + 1),
+                "k_rows_grad launch");
     else
-        k_rows_grad<false, kS><<<grid, 256, 0, s>>>(count_out, c->bw_seg, stok, grad_out,
-                                                    static_cast<const float *>(gate), nullptr, c->d, grad_rows,
-                                                    c->bw_word + 1);
-    NG_CUDA(cudaGetLastError(), "k_rows_grad launch");
+        NG_CUDA(launch_dependent(k_rows_grad<false, kS>, grid, 256, s, count_out, c->bw_seg, stok, grad_out,
+                                 static_cast<const float *>(gate), nullptr, c->d, grad_rows, c->bw_word + 1),
+                "k_rows_grad launch");
     return NGRAM_OK;
 }
 
@@ -1585,7 +1599,8 @@ ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int3
     const GatherArgs g = gather_args(c, tokens, history, T, static_cast<uint32_t>(N), nullptr, nullptr, nullptr);
     const unsigned grid = static_cast<unsigned>(c->num_sms) * 2u;
     if (tok_gate) {
-        launch_gate_grad<true>(c->dtype, g, grid, s, grad_out, grad_gate, nullptr, c->row_bytes);
+        NG_CUDA(launch_gate_grad<true>(c->dtype, g, grid, s, grad_out, grad_gate, nullptr, c->row_bytes),
+                "k_gate_grad launch");
     } else {
         const uint64_t max_chunks = (c->max_tokens + kGateChunk - 1) / kGateChunk;
         const uint64_t max_groups = (max_chunks + kGateGroup - 1) / kGateGroup;
@@ -1594,9 +1609,13 @@ ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int3
         const uint32_t n_chunks = static_cast<uint32_t>((N + kGateChunk - 1) / kGateChunk);
         const uint32_t n_groups = (n_chunks + kGateGroup - 1) / kGateGroup;
         double *groups = c->bw_part + max_chunks * c->d;
-        launch_gate_grad<false>(c->dtype, g, grid, s, grad_out, nullptr, c->bw_part, c->row_bytes);
-        k_gate_reduce_groups<<<dim3((c->d + 255) / 256, n_groups), 256, 0, s>>>(c->bw_part, n_chunks, c->d, groups);
-        k_gate_reduce<<<(c->d + 255) / 256, 256, 0, s>>>(groups, n_groups, c->d, grad_gate);
+        NG_CUDA(launch_gate_grad<false>(c->dtype, g, grid, s, grad_out, nullptr, c->bw_part, c->row_bytes),
+                "k_gate_grad launch");
+        NG_CUDA(launch_dependent(k_gate_reduce_groups, dim3((c->d + 255) / 256, n_groups), 256, s,
+                                 c->bw_part, n_chunks, c->d, groups),
+                "k_gate_reduce launch");
+        NG_CUDA(launch_dependent(k_gate_reduce, (c->d + 255) / 256, 256, s, groups, n_groups, c->d, grad_gate),
+                "k_gate_reduce launch");
     }
     NG_CUDA(cudaGetLastError(), "k_gate_grad launch");
     return NGRAM_OK;

@@ -18,9 +18,13 @@
 //            shared memory, and a key's position is the tile's offset for its digit +
 //            the keys of that digit in earlier rounds + in earlier warps of this round +
 //            its rank in the warp.  Stable by construction.
+// Every kernel opens with allow_dependents(); grid_dependency_wait(), so the passes may be
+// launched as programmatic dependents of one another.
 #pragma once
 
 #include <cstdint>
+
+#include "device_common.cuh"
 
 namespace ngram {
 
@@ -31,6 +35,8 @@ constexpr uint32_t kScanChunk = 1024;     // entries per block of the generic sc
 __global__ void __launch_bounds__(256) k_radix_hist(const uint32_t *__restrict__ keys, uint32_t M,
                                                     uint32_t shift, uint32_t n_tiles,
                                                     uint32_t *__restrict__ hist) {
+    allow_dependents();
+    grid_dependency_wait();
     __shared__ uint32_t h[kSortRadix];
     for (uint32_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         h[threadIdx.x] = 0;
@@ -56,6 +62,8 @@ __global__ void __launch_bounds__(256) k_radix_scatter(const uint32_t *__restric
                                                        const uint32_t *__restrict__ offsets,
                                                        uint32_t *__restrict__ keys_out,
                                                        uint32_t *__restrict__ vals_out) {
+    allow_dependents();
+    grid_dependency_wait();
     __shared__ uint32_t run[kSortRadix];          // keys of each digit placed so far + offset
     __shared__ uint16_t wcnt[8][kSortRadix];      // this round's count per (warp, digit)
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
@@ -97,6 +105,8 @@ __global__ void __launch_bounds__(256) k_radix_scatter(const uint32_t *__restric
 // (k_dedup_scan_blocks); k_scan_add adds them back.
 __global__ void __launch_bounds__(256) k_scan_local(const uint32_t *in, uint32_t n, uint32_t *out,
                                                     uint32_t *__restrict__ block_total) {
+    allow_dependents();
+    grid_dependency_wait();
     __shared__ uint32_t warp_tot[8];
     const uint32_t base = blockIdx.x * kScanChunk + threadIdx.x * 4u;
     uint32_t v[4], run = 0;
@@ -126,6 +136,8 @@ __global__ void __launch_bounds__(256) k_scan_local(const uint32_t *in, uint32_t
 
 __global__ void __launch_bounds__(256) k_scan_add(uint32_t *out, uint32_t n,
                                                   const uint32_t *__restrict__ block_off) {
+    allow_dependents();
+    grid_dependency_wait();
     const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) out[i] += block_off[i / kScanChunk];
 }

@@ -226,7 +226,9 @@ NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const floa
  *   programmatic dependents (the launch may overlap the previous kernel of the stream; each
  *   waits for that kernel to complete before touching memory), and they let the next such
  *   kernel be scheduled as soon as they start.  Results are those of plain stream order.
- *   The host-resident lookups on a bounded grid launch plainly. */
+ *   The hash, dedup, radix-sort and backward kernels of the other entry points are
+ *   launched the same way.  The host-resident lookups on a bounded grid, and the copy of
+ *   host rows into staging, launch plainly. */
 NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, const int32_t *history,
                            uint32_t n_seq, uint32_t T, const uint16_t *residual,
                            const void *gate, uint16_t *out, ngram_stream_t stream);

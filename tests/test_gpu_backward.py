@@ -143,6 +143,51 @@ def test_backward_rows_empty_and_errors(cuda_device):
                                torch.zeros(64, device=cuda_device))
 
 
+def test_back_to_back_calls_keep_stream_order(cuda_device):
+    """The hash, dedup, radix-sort and backward kernels are launched as programmatic
+    dependents: each may be scheduled while the previous kernel of the stream still runs and
+    waits for it before touching memory.  Three batches' dedup, table gradient, gate
+    gradient and staged forward, issued back to back on one stream with no host
+    synchronisation (the calls share the context's scratch), must equal the same calls with
+    a synchronisation after each."""
+    R, d, V = 65_536, 264, 7000
+    w = gen.Workload("bwchain", R, d, "bf16", V, 2, 150, history=True)
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    ins = [gen.make_inputs(w, token_seed=900 + i) for i in range(3)]
+    toks = [to_dev_tokens(x["tokens"], cuda_device) for x in ins]
+    hsts = [to_dev_tokens(x["history"], cuda_device) for x in ins]
+    dys = [to_dev_bf16(_dy(w.N, d, 30 + i), cuda_device).view(w.N, d) for i in range(3)]
+    res = [to_dev_bf16(x["residual"], cuda_device).view(w.N, d) for x in ins]
+    gate = torch.from_numpy(ins[0]["gate"]).to(cuda_device)
+
+    def run(sync):
+        outs = []
+        for i in range(3):
+            uu, inv, cc = ng.ngram_dedup_rows(ctx, toks[i], history=hsts[i])
+            u, c, g = ng.ngram_backward_rows(ctx, toks[i], dys[i], gate, history=hsts[i])
+            gg = ng.ngram_backward_gate(ctx, toks[i], dys[i], history=hsts[i])
+            ng.ngram_prefetch(ctx, i % 2, toks[i], history=hsts[i])
+            y = ng.ngram_forward_staged(ctx, i % 2, res[i], gate)
+            if sync:
+                torch.cuda.synchronize()
+            outs.append((uu, inv, cc, u, c, g, gg, y))
+        torch.cuda.synchronize()
+        return outs
+
+    ref = run(True)
+    got = run(False)
+    for a, b in zip(ref, got):
+        n_u = int(a[2].item())
+        assert int(b[2].item()) == n_u and int(b[4].item()) == n_u
+        assert torch.equal(a[0][:n_u], b[0][:n_u]) and torch.equal(a[1], b[1])
+        assert torch.equal(a[3][:n_u], b[3][:n_u])
+        assert torch.equal(a[5][:n_u].view(torch.int32), b[5][:n_u].view(torch.int32))
+        assert torch.equal(a[6].view(torch.int32), b[6].view(torch.int32))
+        assert torch.equal(a[7].view(torch.int16), b[7].view(torch.int16))
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
 # --------------------------------------------------------------------------- gate gradient
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("tg", [False, True])
