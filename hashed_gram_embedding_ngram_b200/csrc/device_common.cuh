@@ -244,9 +244,19 @@ __device__ __forceinline__ uint32_t e4m3_to_half_bits(uint32_t b) {
     return h;
 }
 
+// Two E4M3 codes (the low bytes of a and b) -> their f16 bits, a in the low half (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_half2_bits(uint32_t a, uint32_t b) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 x;\n\tcvt.u16.u32 x, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, x;\n\t}"
+        : "=r"(h) : "r"((a & 0xFFu) | ((b & 0xFFu) << 8)));
+    return h;
+}
+
 // Eight E2M1 codes (nibble k = column k), each times the f16 value s, added to fp32
 // accumulators: acc[j] (columns 2j, 2j+1) += q * s with one rounding (fma.rn.f32.f16: the
 // f16 operands enter exactly, q * s is exact for E2M1 x E4M3).
+// kHi: s is the high half of s_half (else the low half).
+template <bool kHi = false>
 __device__ __forceinline__ void e2m1x8_fma(uint32_t w, uint32_t s_half, float2 acc[4]) {
     uint32_t h0, h1, h2, h3;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
@@ -256,9 +266,14 @@ __device__ __forceinline__ void e2m1x8_fma(uint32_t w, uint32_t s_half, float2 a
     const uint32_t hh[4] = {h0, h1, h2, h3};
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-        asm("{\n\t.reg .b16 lo, hi, s, u;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {s, u}, %3;\n\t"
-            "fma.rn.f32.f16 %0, lo, s, %0;\n\tfma.rn.f32.f16 %1, hi, s, %1;\n\t}"
-            : "+f"(acc[j].x), "+f"(acc[j].y) : "r"(hh[j]), "r"(s_half));
+        if (kHi)
+            asm("{\n\t.reg .b16 lo, hi, s, u;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {u, s}, %3;\n\t"
+                "fma.rn.f32.f16 %0, lo, s, %0;\n\tfma.rn.f32.f16 %1, hi, s, %1;\n\t}"
+                : "+f"(acc[j].x), "+f"(acc[j].y) : "r"(hh[j]), "r"(s_half));
+        else
+            asm("{\n\t.reg .b16 lo, hi, s, u;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {s, u}, %3;\n\t"
+                "fma.rn.f32.f16 %0, lo, s, %0;\n\tfma.rn.f32.f16 %1, hi, s, %1;\n\t}"
+                : "+f"(acc[j].x), "+f"(acc[j].y) : "r"(hh[j]), "r"(s_half));
 }
 
 }  // namespace ngram
