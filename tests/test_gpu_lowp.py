@@ -122,12 +122,15 @@ SHAPES = {
             (272, 3, 5, 2, 45, True),      # 17 vectors: ragged strip
             (528, 16, 0, 1, 70, True),     # 33 vectors
             (2560, 8, 8, 2, 60, True),     # the pages' width
-            (2576, 0, 16, 3, 11, False)],  # 161 vectors: ragged tail
+            (2576, 0, 16, 3, 11, False),   # 161 vectors: ragged tail
+            (272, 3, 4, 2, 45, True)],     # 7 heads
     "nvfp4": [(32, 8, 8, 3, 37, False),    # two scale blocks, 14 pad bytes
               (288, 3, 5, 2, 45, True),    # 18 blocks
               (544, 16, 0, 1, 70, True),   # 34 blocks
               (2560, 8, 8, 2, 60, True),
-              (2592, 0, 16, 3, 11, False)],  # 162 blocks: ragged tail
+              (2592, 0, 16, 3, 11, False),   # 162 blocks: ragged tail
+              (288, 3, 4, 2, 45, True),    # 7 heads: the last block scale converted alone
+              (32, 1, 0, 2, 9, False)],    # a single head
 }
 
 

@@ -387,6 +387,7 @@ def test_bad_token_ids_flag_the_device_error_word(cuda_device):
     (528, 16, 0, 1, 70, True),     # 33 vectors
     (2560, 8, 8, 2, 60, True),     # the pages' width
     (2576, 0, 16, 3, 11, False),   # 161 vectors: ragged tail
+    (272, 3, 4, 2, 45, True),      # 7 heads
 ])
 def test_forward_int8_every_token(cuda_device, d, nb, nt, n_seq, T, hist):
     R, V = 5003, 7000
