@@ -160,6 +160,7 @@ struct ngram_ctx {
     // backward: radix-sort buffers (keys, values, twice), digit counts, scan totals,
     // segment starts; the shared-gate gradient's fp64 partials
     uint32_t *bw_k[2], *bw_v[2], *bw_hist, *bw_tot, *bw_seg, *bw_word;
+    int bw_rows_per_sm[2];      // resident k_rows_grad CTAs per SM (shared gate, per-token gate)
     double *bw_part;
     // ngram_prefetch / ngram_forward_staged: a ring of staged batches in HBM
     struct Slot {
@@ -1477,6 +1478,12 @@ ngram_status ensure_backward_sort(ngram_ctx *c) {
     NG_CUDA(cudaMalloc(&c->bw_tot, nb * 4), "backward scratch");
     NG_CUDA(cudaMalloc(&c->bw_seg, (M + 1) * 4), "backward scratch");
     NG_CUDA(cudaMalloc(&c->bw_word, 8), "backward scratch");     // scan total, item counter
+    // queried once here, not per call, so that a call may be captured in a CUDA graph
+    constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
+    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[0], k_rows_grad<false, kS>, 256, 0),
+            "occupancy");
+    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[1], k_rows_grad<true, kS>, 256, 0),
+            "occupancy");
     return NGRAM_OK;
 }
 
@@ -1564,9 +1571,7 @@ ngram_status ngram_backward_rows(ngram_ctx *c, const int32_t *tokens, const int3
     NG_CUDA(launch_dependent(k_seg_starts, grid_for(c, M, 256), 256, s, skeys, M, c->bw_seg), "k_seg_starts launch");
     const bool tok_gate = (c->hp.flags & NGRAM_FLAG_TOKEN_GATE) != 0;
     constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
-    int per_sm = 0;
-    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, tok_gate ? k_rows_grad<true, kS> : k_rows_grad<false, kS>, 256, 0), "occupancy");
+    const int per_sm = c->bw_rows_per_sm[tok_gate ? 1 : 0];
     const unsigned grid = static_cast<unsigned>(c->num_sms) * static_cast<unsigned>(std::max(1, per_sm));
     if (tok_gate)
         NG_CUDA(launch_dependent(k_rows_grad<true, kS>, grid, 256, s, count_out, c->bw_seg, stok, grad_out,

@@ -188,6 +188,51 @@ def test_back_to_back_calls_keep_stream_order(cuda_device):
     assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
 
 
+def test_backward_replays_from_a_cuda_graph(cuda_device):
+    """The table and gate gradients captured in a CUDA graph (their memsets and programmatic
+    dependent launches become graph nodes and edges) and replayed on new inputs copied into
+    the captured buffers equal the same calls run eagerly."""
+    R, d, V = 65_536, 264, 7000
+    w = gen.Workload("bwgraph", R, d, "bf16", V, 2, 150, history=True)
+    table, _ = TABLES.get(R, d, ng.NGRAM_BF16, gen.TABLE_SEED, cuda_device)
+    ctx = ng.ngram_init(table, R, d, ng.NGRAM_BF16, ng.NGRAM_RES_HBM, _hp(V), w.N)
+    ins = [gen.make_inputs(w, token_seed=950 + i) for i in range(2)]
+    toks = [to_dev_tokens(x["tokens"], cuda_device) for x in ins]
+    hsts = [to_dev_tokens(x["history"], cuda_device) for x in ins]
+    dys = [to_dev_bf16(_dy(w.N, d, 40 + i), cuda_device).view(w.N, d) for i in range(2)]
+    gate = torch.from_numpy(ins[0]["gate"]).to(cuda_device)
+    want = []
+    for i in range(2):                       # eager; the first call also allocates the scratch
+        u, c, g = ng.ngram_backward_rows(ctx, toks[i], dys[i], gate, history=hsts[i])
+        gg = ng.ngram_backward_gate(ctx, toks[i], dys[i], history=hsts[i])
+        want.append((u.clone(), int(c.item()), g.clone(), gg.clone()))
+    tok_b, hst_b, dy_b = toks[0].clone(), hsts[0].clone(), dys[0].clone()
+    uniq = torch.empty(w.N * 16, dtype=torch.int32, device=cuda_device)
+    count = torch.empty(1, dtype=torch.int32, device=cuda_device)
+    grad = torch.empty((w.N * 16, d), dtype=torch.float32, device=cuda_device)
+    ggate = torch.empty(d, dtype=torch.float32, device=cuda_device)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream()
+        ng.ngram_backward_rows(ctx, tok_b, dy_b, gate, history=hst_b, uniq_out=uniq, count_out=count,
+                               grad_rows=grad, stream=cs)
+        ng.ngram_backward_gate(ctx, tok_b, dy_b, history=hst_b, out=ggate, stream=cs)
+    for i in (1, 0):
+        tok_b.copy_(toks[i])
+        hst_b.copy_(hsts[i])
+        dy_b.copy_(dys[i])
+        graph.replay()
+        torch.cuda.synchronize()
+        u, n_u, g, gg = want[i]
+        assert int(count.item()) == n_u
+        assert torch.equal(uniq[:n_u], u[:n_u])
+        assert torch.equal(grad[:n_u].view(torch.int32), g[:n_u].view(torch.int32))
+        assert torch.equal(ggate.view(torch.int32), gg.view(torch.int32))
+    del graph
+    assert ng.ngram_get_device_error(ctx)[0] == ng.NGRAM_OK
+
+
 # --------------------------------------------------------------------------- gate gradient
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("tg", [False, True])
