@@ -30,7 +30,9 @@
  * the table in the host-resident modes, a pinned host pointer).  The caller owns
  * every buffer it passes.  bf16 arrays are passed as uint16_t bit patterns.
  * Streams: all compute calls are asynchronous on the stream given (NULL = legacy
- * default stream); the library creates no cross-stream dependency of its own.
+ * default stream).  The only other streams are ngram_forward_host's internal copy
+ * streams, which start after the given stream and which the given stream waits for;
+ * no call makes the given stream wait on anything else.
  * Errors: every call returns an ngram_status; invalid arguments are reported before
  * any CUDA work is issued, and nothing aborts the process.  ngram_last_error() gives
  * the text of the last failure on the calling thread.
