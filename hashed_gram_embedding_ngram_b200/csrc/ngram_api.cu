@@ -206,6 +206,31 @@ ngram_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Lazily made scratch: each buffer, event or stream is made only while its handle is still
+// NULL, so a call that failed part-way (ENOMEM) leaves the context consistent, and a later
+// call makes what is missing instead of running with a NULL buffer.
+template <class T>
+ngram_status dev_alloc(T **p, size_t bytes, const char *what) {
+    if (*p != nullptr) return NGRAM_OK;
+    void *q = nullptr;
+    NG_CUDA(cudaMalloc(&q, bytes), what);
+    *p = static_cast<T *>(q);
+    return NGRAM_OK;
+}
+template <class T>
+ngram_status pinned_alloc(T **p, size_t bytes, const char *what) {
+    if (*p != nullptr) return NGRAM_OK;
+    void *q = nullptr;
+    NG_CUDA(cudaHostAlloc(&q, bytes, cudaHostAllocPortable), what);
+    *p = static_cast<T *>(q);
+    return NGRAM_OK;
+}
+ngram_status event_once(cudaEvent_t *ev, unsigned flags) {
+    if (*ev != nullptr) return NGRAM_OK;
+    NG_CUDA(cudaEventCreateWithFlags(ev, flags), "cudaEventCreate");
+    return NGRAM_OK;
+}
+
 // Row formats.  Per-row scales (int8, fp8) travel with the rows through every staging
 // path; the NVFP4 block scales sit inside the row bytes and its global scale stays put.
 bool scale_per_row(ngram_dtype t) { return t == NGRAM_INT8_ROWSCALE || t == NGRAM_FP8_E4M3_ROWSCALE; }
@@ -335,41 +360,34 @@ void free_all(ngram_ctx *c) {
 
 // ---------------------------------------------------------------- scratch on first use
 ngram_status ensure_dedup_scratch(ngram_ctx *c) {
-    if (c->d_idx) return NGRAM_OK;
     const uint32_t M = c->dd_cap, P = c->dd_pcap, NB = (M + kScanBlock - 1) / kScanBlock;
-    NG_CUDA(cudaMalloc(&c->d_idx, M * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_slot, M * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_pos, M * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_inv, M * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_uniq, M * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_keys, P * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_first, P * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_uid, P * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_bsum, NB * 4ull), "dedup scratch");
-    NG_CUDA(cudaMalloc(&c->d_count, 4), "dedup scratch");
+    NG_CHECK(dev_alloc(&c->d_idx, M * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_slot, M * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_pos, M * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_inv, M * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_uniq, M * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_keys, P * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_first, P * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_uid, P * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_bsum, NB * 4ull, "dedup scratch"));
+    NG_CHECK(dev_alloc(&c->d_count, 4, "dedup scratch"));
     return NGRAM_OK;
 }
 
 ngram_status ensure_device_stage(ngram_ctx *c) {
-    if (c->d_stage) return NGRAM_OK;
-    NG_CUDA(cudaMalloc(&c->d_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging");
-    if (scale_per_row(c->dtype))
-        NG_CUDA(cudaMalloc(&c->d_stage_scale, c->dd_cap * 4ull), "staging");
+    NG_CHECK(dev_alloc(&c->d_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes, "staging"));
+    if (scale_per_row(c->dtype)) NG_CHECK(dev_alloc(&c->d_stage_scale, c->dd_cap * 4ull, "staging"));
     return NGRAM_OK;
 }
 
 ngram_status ensure_host_stage(ngram_ctx *c) {
-    if (c->h_stage) return NGRAM_OK;
     NG_CHECK(ensure_device_stage(c));
-    NG_CUDA(cudaHostAlloc(&c->h_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes,
-                          cudaHostAllocPortable), "pinned staging");
-    if (scale_per_row(c->dtype))
-        NG_CUDA(cudaHostAlloc(&c->h_stage_scale, c->dd_cap * 4ull, cudaHostAllocPortable),
-                "pinned staging");
-    NG_CUDA(cudaHostAlloc(&c->h_uniq, c->dd_cap * 4ull, cudaHostAllocPortable), "pinned staging");
-    NG_CUDA(cudaHostAlloc(&c->h_count, 4, cudaHostAllocPortable), "pinned staging");
-    NG_CUDA(cudaEventCreateWithFlags(&c->ev_sync, cudaEventDisableTiming), "cudaEventCreate");
-    NG_CUDA(cudaEventCreateWithFlags(&c->ev_stage_free, cudaEventDisableTiming), "cudaEventCreate");
+    NG_CHECK(pinned_alloc(&c->h_stage, static_cast<size_t>(c->dd_cap) * c->row_bytes, "pinned staging"));
+    if (scale_per_row(c->dtype)) NG_CHECK(pinned_alloc(&c->h_stage_scale, c->dd_cap * 4ull, "pinned staging"));
+    NG_CHECK(pinned_alloc(&c->h_uniq, c->dd_cap * 4ull, "pinned staging"));
+    NG_CHECK(pinned_alloc(&c->h_count, 4, "pinned staging"));
+    NG_CHECK(event_once(&c->ev_sync, cudaEventDisableTiming));
+    NG_CHECK(event_once(&c->ev_stage_free, cudaEventDisableTiming));
     return NGRAM_OK;
 }
 
@@ -405,23 +423,23 @@ void host_chunks(uint64_t N, uint64_t C, std::vector<uint32_t> &out) {
 }
 
 ngram_status ensure_host_path(ngram_ctx *c) {
-    if (c->hp_tok) return NGRAM_OK;
     const uint64_t row = 2ull * c->d;
     uint64_t chunk = NGRAM_HOST_CHUNK_BYTES / row;
     if (chunk < 1) chunk = 1;
     if (chunk > c->max_tokens) chunk = c->max_tokens;
     c->hp_chunk = static_cast<uint32_t>(chunk);
-    NG_CUDA(cudaMalloc(&c->hp_tok, c->max_tokens * 4ull), "host-path buffers");
-    NG_CUDA(cudaMalloc(&c->hp_hist, c->max_tokens * 8ull), "host-path buffers");
+    NG_CHECK(dev_alloc(&c->hp_tok, c->max_tokens * 4ull, "host-path buffers"));
+    NG_CHECK(dev_alloc(&c->hp_hist, c->max_tokens * 8ull, "host-path buffers"));
     for (int b = 0; b < NGRAM_HOST_BUFFERS; ++b) {
-        NG_CUDA(cudaMalloc(&c->hp_res[b], chunk * row), "host-path buffers");
-        NG_CUDA(cudaMalloc(&c->hp_out[b], chunk * row), "host-path buffers");
-        NG_CUDA(cudaEventCreateWithFlags(&c->hp_h2d[b], cudaEventDisableTiming), "cudaEventCreate");
-        NG_CUDA(cudaEventCreateWithFlags(&c->hp_d2h[b], cudaEventDisableTiming), "cudaEventCreate");
+        NG_CHECK(dev_alloc(&c->hp_res[b], chunk * row, "host-path buffers"));
+        NG_CHECK(dev_alloc(&c->hp_out[b], chunk * row, "host-path buffers"));
+        NG_CHECK(event_once(&c->hp_h2d[b], cudaEventDisableTiming));
+        NG_CHECK(event_once(&c->hp_d2h[b], cudaEventDisableTiming));
     }
-    NG_CUDA(cudaEventCreateWithFlags(&c->hp_entry, cudaEventDisableTiming), "cudaEventCreate");
+    NG_CHECK(event_once(&c->hp_entry, cudaEventDisableTiming));
     for (int i = 0; i < NGRAM_HOST_BUFFERS; ++i)
-        NG_CUDA(cudaStreamCreateWithFlags(&c->hp_s[i], cudaStreamNonBlocking), "cudaStreamCreate");
+        if (c->hp_s[i] == nullptr)
+            NG_CUDA(cudaStreamCreateWithFlags(&c->hp_s[i], cudaStreamNonBlocking), "cudaStreamCreate");
     return NGRAM_OK;
 }
 
@@ -849,11 +867,9 @@ bool grouped_order(const ngram_ctx *c, uint32_t N) {
 // Grouped order of a batch's tokens into c->so_perm (3 kernels and a memset).
 // idx_out: also write every token's row ids [N][H] in the same pass, or null.
 ngram_status order_tokens(ngram_ctx *c, const Call &k, uint32_t *idx_out = nullptr) {
-    if (!c->so_perm) {
-        NG_CUDA(cudaMalloc(&c->so_bucket, c->max_tokens * 4ull), "order scratch");
-        NG_CUDA(cudaMalloc(&c->so_hist, kOrderBuckets * 4ull), "order scratch");
-        NG_CUDA(cudaMalloc(&c->so_perm, c->max_tokens * 4ull), "order scratch");
-    }
+    NG_CHECK(dev_alloc(&c->so_bucket, c->max_tokens * 4ull, "order scratch"));
+    NG_CHECK(dev_alloc(&c->so_hist, kOrderBuckets * 4ull, "order scratch"));
+    NG_CHECK(dev_alloc(&c->so_perm, c->max_tokens * 4ull, "order scratch"));
     const HashArgs a = hash_args(c);
     const unsigned gn = grid_for(c, k.N, 256);
     NG_CUDA(cudaMemsetAsync(c->so_hist, 0, kOrderBuckets * 4ull, k.s), "order clear");
@@ -886,7 +902,7 @@ ngram_status order_tokens(ngram_ctx *c, const Call &k, uint32_t *idx_out = nullp
 ngram_status forward_sorted(ngram_ctx *c, const Call &k, uint64_t max_blocks) {
     const bool prehash = ((NGRAM_PREHASH_FORMATS >> c->dtype) & 1u) && c->where == NGRAM_RES_HBM &&
                          k.N >= NGRAM_PREHASH_MIN_TOKENS;
-    if (prehash && !c->d_rowid) NG_CUDA(cudaMalloc(&c->d_rowid, c->dd_cap * 4ull), "row-id buffer");
+    if (prehash) NG_CHECK(dev_alloc(&c->d_rowid, c->dd_cap * 4ull, "row-id buffer"));
     NG_CHECK(order_tokens(c, k, prehash ? c->d_rowid : nullptr));
     GatherArgs g = gather_args(c, k.tokens, k.history, k.T, k.N, k.residual, k.gate, k.out);
     g.perm = c->so_perm;
@@ -948,10 +964,8 @@ ngram_status forward_auto(ngram_ctx *c, const Call &k) {
     if (c->auto_choice[b] == NGRAM_RES_HOST_UVA) return forward_direct_uva(c, k);
     if (c->auto_choice[b] == NGRAM_AUTO_UVA_DEDUP) return forward_dedup_uva(c, k);
     if (c->auto_choice[b] == NGRAM_RES_HOST_DMA) return forward_dma(c, k);
-    if (!c->ev_t0) {
-        NG_CUDA(cudaEventCreate(&c->ev_t0), "cudaEventCreate");
-        NG_CUDA(cudaEventCreate(&c->ev_t1), "cudaEventCreate");
-    }
+    NG_CHECK(event_once(&c->ev_t0, cudaEventDefault));
+    NG_CHECK(event_once(&c->ev_t1, cudaEventDefault));
     const int modes[3] = {NGRAM_RES_HOST_UVA, NGRAM_AUTO_UVA_DEDUP, NGRAM_RES_HOST_DMA};
     for (int m = 0; m < 3; ++m) NG_CHECK(run_mode(c, k, modes[m]));    // warm-up: staging, caches
     // timed rounds interleave the modes, so a slow spell of the host or the link costs
@@ -1238,12 +1252,9 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     sl.epoch = ++c->prefetch_epoch;
     if (N == 0) return NGRAM_OK;
     NG_CHECK(ensure_dedup_scratch(c));
-    if (!sl.inv) {
-        NG_CUDA(cudaMalloc(&sl.inv, c->dd_cap * 4ull), "staging slot");
-        NG_CUDA(cudaMalloc(&sl.stage, static_cast<size_t>(c->dd_cap) * c->row_bytes), "staging slot");
-        if (scale_per_row(c->dtype))
-            NG_CUDA(cudaMalloc(&sl.stage_scale, c->dd_cap * 4ull), "staging slot");
-    }
+    NG_CHECK(dev_alloc(&sl.inv, c->dd_cap * 4ull, "staging slot"));
+    NG_CHECK(dev_alloc(&sl.stage, static_cast<size_t>(c->dd_cap) * c->row_bytes, "staging slot"));
+    if (scale_per_row(c->dtype)) NG_CHECK(dev_alloc(&sl.stage_scale, c->dd_cap * 4ull, "staging slot"));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint32_t M = static_cast<uint32_t>(N) * c->H;
     NG_CHECK(launch_hash_dedup(c, tokens, history, T, static_cast<uint32_t>(N), c->d_uniq, sl.inv, c->d_count, s));
@@ -1465,25 +1476,26 @@ ngram_status ngram_ipc_close(void *dev_ptr) {
 namespace {
 
 ngram_status ensure_backward_sort(ngram_ctx *c) {
-    if (c->bw_k[0]) return NGRAM_OK;
     const uint64_t M = c->dd_cap;
     const uint64_t n_tiles = (M + kSortTile - 1) / kSortTile;
     const uint64_t L = kSortRadix * n_tiles;
     const uint64_t nb = (L + kScanChunk - 1) / kScanChunk;
     for (int b = 0; b < 2; ++b) {
-        NG_CUDA(cudaMalloc(&c->bw_k[b], M * 4), "backward scratch");
-        NG_CUDA(cudaMalloc(&c->bw_v[b], M * 4), "backward scratch");
+        NG_CHECK(dev_alloc(&c->bw_k[b], M * 4, "backward scratch"));
+        NG_CHECK(dev_alloc(&c->bw_v[b], M * 4, "backward scratch"));
     }
-    NG_CUDA(cudaMalloc(&c->bw_hist, L * 4), "backward scratch");
-    NG_CUDA(cudaMalloc(&c->bw_tot, nb * 4), "backward scratch");
-    NG_CUDA(cudaMalloc(&c->bw_seg, (M + 1) * 4), "backward scratch");
-    NG_CUDA(cudaMalloc(&c->bw_word, 8), "backward scratch");     // scan total, item counter
-    // queried once here, not per call, so that a call may be captured in a CUDA graph
-    constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
-    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[0], k_rows_grad<false, kS>, 256, 0),
-            "occupancy");
-    NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[1], k_rows_grad<true, kS>, 256, 0),
-            "occupancy");
+    NG_CHECK(dev_alloc(&c->bw_hist, L * 4, "backward scratch"));
+    NG_CHECK(dev_alloc(&c->bw_tot, nb * 4, "backward scratch"));
+    NG_CHECK(dev_alloc(&c->bw_seg, (M + 1) * 4, "backward scratch"));
+    NG_CHECK(dev_alloc(&c->bw_word, 8, "backward scratch"));     // scan total, item counter
+    // queried once, not per call, so that a call may be captured in a CUDA graph
+    if (c->bw_rows_per_sm[0] == 0) {
+        constexpr int kS = NGRAM_ROWS_GRAD_STRIPS;
+        NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[1], k_rows_grad<true, kS>, 256, 0),
+                "occupancy");
+        NG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->bw_rows_per_sm[0], k_rows_grad<false, kS>, 256, 0),
+                "occupancy");
+    }
     return NGRAM_OK;
 }
 
@@ -1609,8 +1621,8 @@ ngram_status ngram_backward_gate(ngram_ctx *c, const int32_t *tokens, const int3
     } else {
         const uint64_t max_chunks = (c->max_tokens + kGateChunk - 1) / kGateChunk;
         const uint64_t max_groups = (max_chunks + kGateGroup - 1) / kGateGroup;
-        if (!c->bw_part)      // chunk partials, then group partials
-            NG_CUDA(cudaMalloc(&c->bw_part, (max_chunks + max_groups) * 8ull * c->d), "backward scratch");
+        // chunk partials, then group partials
+        NG_CHECK(dev_alloc(&c->bw_part, (max_chunks + max_groups) * 8ull * c->d, "backward scratch"));
         const uint32_t n_chunks = static_cast<uint32_t>((N + kGateChunk - 1) / kGateChunk);
         const uint32_t n_groups = (n_chunks + kGateGroup - 1) / kGateGroup;
         double *groups = c->bw_part + max_chunks * c->d;
