@@ -199,7 +199,8 @@ NGRAM_API ngram_status ngram_row_bytes(ngram_dtype dtype, uint32_t d, uint32_t *
  *   hp         hash parameters (NULL = defaults).
  *   max_tokens largest n_seq * T a later call may pass (>= 1).
  * The context owns a 16-byte device error word; dedup scratch and staging buffers are
- * allocated by the first call that needs them.  EINVAL on bad arguments (checked
+ * allocated by the first call that needs them (a call that returns NGRAM_ENOMEM keeps what
+ * it allocated and launches nothing that needs the rest; a later call allocates the rest).  EINVAL on bad arguments (checked
  * before any CUDA call, except the memory-kind checks of host residency),
  * ECUDA/ENOMEM on CUDA failures.  On failure *out is set to NULL. */
 NGRAM_API ngram_status ngram_init(ngram_ctx **out, const void *table, const float *row_scale,
