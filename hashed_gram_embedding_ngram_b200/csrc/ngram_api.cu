@@ -1247,10 +1247,13 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     if (c->where == NGRAM_RES_HOST_DMA)
         return fail(NGRAM_EUNSUPPORTED, "ngram_prefetch reads the table from the GPU: HBM, HOST_UVA or HOST_AUTO");
     auto &sl = c->slot[slot];
+    sl.epoch = 0;                    // the slot holds no batch until this call has issued its work
     sl.n_seq = n_seq;
     sl.T = T;
-    sl.epoch = ++c->prefetch_epoch;
-    if (N == 0) return NGRAM_OK;
+    if (N == 0) {
+        sl.epoch = ++c->prefetch_epoch;
+        return NGRAM_OK;
+    }
     NG_CHECK(ensure_dedup_scratch(c));
     NG_CHECK(dev_alloc(&sl.inv, c->dd_cap * 4ull, "staging slot"));
     NG_CHECK(dev_alloc(&sl.stage, static_cast<size_t>(c->dd_cap) * c->row_bytes, "staging slot"));
@@ -1264,6 +1267,7 @@ ngram_status ngram_prefetch(ngram_ctx *c, uint32_t slot, const int32_t *tokens, 
     k_compact_rows<<<grid, 256, 0, s>>>(static_cast<const uint8_t *>(c->table_dev), staged_scale_src(c),
                                         c->d_uniq, c->d_count, c->row_bytes, sl.stage, sl.stage_scale);
     NG_CUDA(cudaGetLastError(), "k_compact_rows launch");
+    sl.epoch = ++c->prefetch_epoch;
     return NGRAM_OK;
 }
 

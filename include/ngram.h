@@ -251,7 +251,11 @@ NGRAM_API ngram_status ngram_forward(ngram_ctx *ctx, const int32_t *tokens, cons
  * The slots and the dedup scratch belong to the context: prefetches on one context must
  * be ordered with each other, and a slot must not be refilled while a staged forward
  * still reads it.  Each slot holds max_tokens * H rows (allocated by its first
- * prefetch).  HOST_DMA residency: NGRAM_EUNSUPPORTED. */
+ * prefetch).  A slot that no prefetch has filled, or whose last prefetch failed to
+ * allocate or launch its work, holds no batch: ngram_forward_staged on it returns
+ * NGRAM_EINVAL (a prefetch refused for its arguments leaves the slot as it was).  HOST_DMA
+ * residency:
+ * NGRAM_EUNSUPPORTED. */
 #define NGRAM_STAGE_SLOTS 2u
 NGRAM_API ngram_status ngram_prefetch(ngram_ctx *ctx, uint32_t slot, const int32_t *tokens,
                                       const int32_t *history, uint32_t n_seq, uint32_t T,
