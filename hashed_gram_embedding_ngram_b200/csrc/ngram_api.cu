@@ -1186,6 +1186,11 @@ ngram_status ngram_forward_host(ngram_ctx *c, const int32_t *tokens_h, const int
     if (residual_h == nullptr || gate == nullptr || out_h == nullptr)
         return fail(NGRAM_EINVAL, "residual, gate and out must be non-NULL");
     if (!aligned16(gate)) return fail(NGRAM_EINVAL, "gate must be 16-byte aligned");
+    {   // the chunks' copies in and out may run in any order across streams
+        const uint64_t bytes = N * c->d * 2ull;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(out_h), b = reinterpret_cast<uintptr_t>(residual_h);
+        if (a < b + bytes && b < a + bytes) return fail(NGRAM_EINVAL, "out overlaps residual");
+    }
     if ((c->hp.flags & (NGRAM_FLAG_DEDUP | NGRAM_FLAG_TMA_STAGING | NGRAM_FLAG_SORT |
                         NGRAM_FLAG_TOKEN_GATE)) ||  // chunks keep batch order
         (c->where != NGRAM_RES_HBM && c->where != NGRAM_RES_HOST_UVA))

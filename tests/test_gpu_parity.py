@@ -491,6 +491,24 @@ def test_forward_host_rejects_staged_modes(cuda_device):
     assert ei.value.status == ng.NGRAM_EUNSUPPORTED
 
 
+def test_forward_host_rejects_overlapping_buffers(cuda_device):
+    """Output chunks are copied back while other chunks' inputs are still being read, on
+    other streams: the host output must not overlap the host residual, in place included."""
+    w = W["tiny"]
+    inp, dv = workload_on_device(w, cuda_device)
+    ctx = _ctx_for(w, cuda_device)
+    t, h, r = _host_inputs(inp, w)
+    with pytest.raises(ng.NgramError) as ei:                       # in place
+        ng.ngram_forward_host(ctx, t, r, dv["gate"], out=r, history=h)
+    assert ei.value.status == ng.NGRAM_EINVAL
+    big = torch.empty(r.numel() + w.d, dtype=torch.bfloat16).pin_memory()
+    res, out = big[:r.numel()].view_as(r), big[w.d:].view_as(r)     # one row apart
+    res.copy_(r)
+    with pytest.raises(ng.NgramError) as ei:
+        ng.ngram_forward_host(ctx, t, res, dv["gate"], out=out, history=h)
+    assert ei.value.status == ng.NGRAM_EINVAL
+
+
 # --------------------------------------------------------------------------- grouped order
 @pytest.mark.parametrize("name", ["tiny", "mid", "full_prefill", "full_decode_1",
                                   "full_decode_256", "int8_uniform"])
